@@ -1,0 +1,498 @@
+"""Benchmark of the PM-KVQ hot path on B200.
+
+Workload (one step): a decode step of a DeepSeek-R1-Distill-Qwen-7B-shaped
+model -- 28 blocks, 28 query / 4 KV heads, head_dim 128, batch 16, about
+32768 cached tokens per sequence, Fbit 4 for block 0 and the last 8 blocks and
+2 elsewhere.  Per block: quantize-on-append of the new token's K/V (with the
+budget-triggered shrink check) and GQA decode attention over the packed cache.
+Inputs are synthetic (seeded Gaussian K/V/Q with RoPE and x20 outlier Key
+channels); the cache (~5.4 GB) is far larger than L2, and every block's read
+(151-285 MB) exceeds L2, so no flush is needed between steps.
+
+Printed: one JSON line.  `value` is the step's algorithmic HBM bytes
+(attention reads of codes + meta + Q/O, append reads/writes) divided by the
+device time of the step.  `roofline` reports the decode-attention kernel
+alone; `shrink` the Equivalent-Right-Shift kernel on a full 128K-token block
+of a Llama-70B-shaped layer (4 -> 2 bits) and on the 7B progressive-stream
+events; `cpu_baseline` the CPU oracle on a bounded sample.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kvq_synth as S  # noqa: E402
+
+METRIC = "decode-attn HBM GB/s & % of B200 peak over packed mixed-bit KV; shrink GB/s"
+HEAD_DIM = 128
+SEED = 0
+
+# 7B decode workload
+L7, HQ7, HKV7, B7, T7 = 28, 28, 4, 16, 32768
+FBIT7 = [4 if (l == 0 or l >= L7 - 8) else 2 for l in range(L7)]
+ROOM = 4096  # tokens of head-room for the appended decode tokens
+WORKLOAD = ("DeepSeek-R1-Distill-Qwen-7B-shape decode: 28 layers, 28 Q / 4 KV heads, head_dim 128, "
+            "batch 16, context 32768, Fbit 4 for layer 0 and the last 8 layers else 2; one decode step "
+            "= append + attention per layer")
+
+
+def per_token_bytes(batch, kv_heads, fbit):
+    return batch * kv_heads * 2 * sum(16 * f + 4 for f in fbit)
+
+
+def decode_bytes(batch, kv_heads, q_heads, tokens, bits):
+    """Algorithmic bytes of one decode-attention call: every cached code and
+    meta word once, Q (bf16) in, O (fp32) out."""
+    return (batch * kv_heads * tokens * 2 * (16 * bits + 4)
+            + batch * q_heads * HEAD_DIM * (2 + 4))
+
+
+def append_bytes(batch, kv_heads, n, bits):
+    """bf16 K/V in, codes + meta out."""
+    return batch * kv_heads * n * 2 * (HEAD_DIM * 2 + 16 * bits + 4)
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def calib_lambda(k):
+    """Migration factor from the first chunk of a block's keys (the note's
+    calibration rule lambda_i = (max_m |K_m,i|)^alpha, alpha = 1/2)."""
+    return k.float().abs().amax(dim=(0, 1)).clamp_min(1e-6).pow(0.5)
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = max(mx, float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def build_cache(kvq, dev, layers, batch, kv_heads, fbit, tokens, n_f, seed, n_out, chunk=4096):
+    budget = n_f * per_token_bytes(batch, kv_heads, fbit)
+    cache = kvq.KVQCache(layers, batch, kv_heads, budget, fbit, device=dev)
+    assert cache.max_tokens == n_f, (cache.max_tokens, n_f)
+    for l in range(layers):
+        pos = 0
+        while pos < tokens:
+            n = min(chunk, tokens - pos)
+            k, v = S.keys_values(seed, l, batch, n, kv_heads, pos, n_out, dtype=torch.bfloat16, device=dev)
+            if pos == 0:
+                cache.set_lambda(l, calib_lambda(k))
+            cache.append(l, k, v)
+            pos += n
+    torch.cuda.synchronize(dev)
+    return cache
+
+
+def flush_l2(buf):
+    buf.add_(1)
+
+
+def measure_shrink(kvq, dev, flush_buf, reps=3):
+    """Equivalent Right Shift kernel GB/s (algorithmic: whole region read,
+    half written).  (a) Llama-70B-shape layer (batch 8, 8 KV heads), Fbit 2,
+    a block full with 131072 tokens at 4 bits shrinking to 2 bits.  (b) the
+    7B progressive stream (batch 8, 4 KV heads, 32768 tokens at Fbit 2):
+    events 16->8 at 4096, 8->4 at 8192, 4->2 at 16384 tokens."""
+    res = {}
+
+    def one(batch, kv_heads, n_f, fbit, fill_tokens, tag):
+        times = []
+        nbytes = None
+        for r in range(reps):
+            cache = build_cache(kvq, dev, 1, batch, kv_heads, [fbit], fill_tokens, n_f, SEED + 17 + r, 10,
+                                chunk=8192)
+            st = cache.query(0)
+            assert st["tokens"] == st["capacity"], st
+            region = batch * kv_heads * 2 * n_f * 16 * fbit  # code bytes of the block
+            nbytes = region + region // 2
+            flush_l2(flush_buf)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            cache.shrink(0)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            cache.device_status()
+            times.append(e0.elapsed_time(e1) / 1e3)
+            bits_from = st["bits"]
+            cache.free()
+            del cache
+        t = statistics.median(times)
+        res[tag] = {"gbs": nbytes / t / 1e9, "us": t * 1e6, "bytes": nbytes, "bits": f"{bits_from}->{bits_from // 2}",
+                    "reps": reps}
+
+    one(8, 8, 262144, 2, 131072, "llama70b_128k_4to2")
+    for tokens, tag in ((4096, "qwen7b_16to8"), (8192, "qwen7b_8to4"), (16384, "qwen7b_4to2")):
+        one(8, 4, 32768, 2, tokens, tag)
+    return res
+
+
+def measure_append_chunk(kvq, dev, flush_buf, reps=3):
+    """Chunked append of 4096 tokens (7B shape, batch 8) at 2 bits."""
+    batch, kv_heads, n_f = 8, 4, 65536
+    # past the 4 -> 2 shrink at 32768 tokens, with room for the timed chunks
+    cache = build_cache(kvq, dev, 1, batch, kv_heads, [2], 40960, n_f, SEED + 5, 5, chunk=8192)
+    st = cache.query(0)
+    k, v = S.keys_values(SEED, 99, batch, 4096, kv_heads, 0, 5, dtype=torch.bfloat16, device=dev)
+    times = []
+    for r in range(reps):
+        flush_l2(flush_buf)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        cache.append(0, k, v)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        times.append(e0.elapsed_time(e1) / 1e3)
+    bits = cache.query(0)["bits"]
+    assert bits == st["bits"]
+    cache.free()
+    nb = append_bytes(batch, kv_heads, 4096, bits)
+    t = statistics.median(times)
+    return {"gbs": nb / t / 1e9, "us": t * 1e6, "bytes": nb, "bits": bits, "tokens": 4096, "batch": batch}
+
+
+def run_gpu(args, rank, world):
+    from mixed_precision_kv_kvq_b200 import build as kbuild
+
+    kbuild.build()
+    import mixed_precision_kv_kvq_b200 as kvq
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    layers = args.layers
+    fbit = FBIT7 if layers == L7 else [4 if l % 2 == 1 else 2 for l in range(layers)]
+    K, W = args.steps, args.warmup
+    if K + W > ROOM:
+        raise SystemExit(f"--steps + --warmup must be <= {ROOM}")
+    n_f = T7 + ROOM
+    n_out = S.outliers_for(HKV7)
+    seed = SEED + 1000 * rank
+    cache = build_cache(kvq, dev, layers, B7, HKV7, fbit, T7, n_f, seed, n_out)
+    sm_scale = HEAD_DIM ** -0.5
+
+    # per-step inputs, generated up front on the device
+    nsteps = K + W
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed + 7)
+    kin = torch.randn((nsteps, layers, B7, 1, HKV7, HEAD_DIM), generator=g, device=dev).to(torch.bfloat16)
+    vin = torch.randn((nsteps, layers, B7, 1, HKV7, HEAD_DIM), generator=g, device=dev).to(torch.bfloat16)
+    qin = torch.randn((nsteps, layers, B7, HQ7, HEAD_DIM), generator=g, device=dev).to(torch.bfloat16)
+    out = torch.empty((layers, B7, HQ7, HEAD_DIM), dtype=torch.float32, device=dev)
+    ws = [cache.workspace(l, HQ7) for l in range(layers)]
+    stream = torch.cuda.current_stream(dev)
+
+    # Raw C-ABI calls with pre-built arguments keep the host well ahead of the GPU.
+    import ctypes as C
+    lib = kvq.load()
+    sp = C.c_void_p(stream.cuda_stream)
+    h = cache.handle
+    kp = [[C.c_void_p(kin[i, l].data_ptr()) for l in range(layers)] for i in range(nsteps)]
+    vp = [[C.c_void_p(vin[i, l].data_ptr()) for l in range(layers)] for i in range(nsteps)]
+    qp = [[C.c_void_p(qin[i, l].data_ptr()) for l in range(layers)] for i in range(nsteps)]
+    op = [C.c_void_p(out[l].data_ptr()) for l in range(layers)]
+    wp = [(C.c_void_p(w.data_ptr()), w.numel() * 4) for w in ws]
+    scale_c = C.c_float(sm_scale)
+
+    def step(i, ev=None):
+        for l in range(layers):
+            st = lib.kvq_append(h, l, kp[i][l], vp[i][l], kvq.KVQ_DTYPE_BF16, 1, sp)
+            if st:
+                kvq.check(st)
+            if ev is not None:
+                ev[l][0].record(stream)
+            st = lib.kvq_decode_attn(h, l, qp[i][l], HQ7, scale_c, op[l], wp[l][0], wp[l][1], sp)
+            if st:
+                kvq.check(st)
+            if ev is not None:
+                ev[l][1].record(stream)
+
+    def bytes_of_step(t_before):
+        """Algorithmic bytes of one step given the token count before it."""
+        tot, dec = 0, 0
+        for l in range(layers):
+            bits = fbit[l]
+            a = append_bytes(B7, HKV7, 1, bits)
+            d = decode_bytes(B7, HKV7, HQ7, t_before + 1, bits)
+            tot += a + d
+            dec += d
+        return tot, dec
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize(dev)
+    for l in range(layers):
+        st = cache.query(l)
+        assert st["bits"] == fbit[l], (l, st)
+    t0_tokens = cache.query(0)["tokens"]
+
+    # ---- timed region (device-only inputs) ----
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(layers)] for _ in range(K)]
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        torch.cuda.nvtx.range_push("timed")
+        e_start.record(stream)
+        for i in range(K):
+            step(W + i, evs[i])
+        e_end.record(stream)
+        torch.cuda.synchronize(dev)
+        torch.cuda.nvtx.range_pop()
+    cache.device_status()
+    total_ms = e_start.elapsed_time(e_end)
+    dec_ms = sum(evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(K) for l in range(layers))
+    tot_bytes, dec_bytes = 0, 0
+    for i in range(K):
+        tb, db = bytes_of_step(t0_tokens + i)
+        tot_bytes += tb
+        dec_bytes += db
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * tot_bytes / (total_ms / 1e3) / 1e9
+    launches = K * layers * 2
+
+    # ---- e2e: the same step through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        kh = kin.cpu().pin_memory()
+        vh = vin.cpu().pin_memory()
+        qh = qin.cpu().pin_memory()
+        oh = torch.empty((layers, B7, HQ7, HEAD_DIM), dtype=torch.float32).pin_memory()
+        E = min(K, ROOM - K - W)
+        if E > 0:
+            torch.cuda.synchronize(dev)
+            if world > 1:
+                torch.distributed.barrier()
+            f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            for i in range(E):
+                for l in range(layers):
+                    cache.append(l, kh[i, l], vh[i, l])       # H2D of this step's K/V inside the call
+                    o = cache.decode_attn(l, qh[i, l], sm_scale, out=out[l])  # H2D of q
+                    oh[l].copy_(o, non_blocking=True)        # D2H of the result
+            f1.record(stream)
+            torch.cuda.synchronize(dev)
+            e2e_ms = f0.elapsed_time(f1)
+            if world > 1:
+                t = torch.tensor([e2e_ms], device=dev)
+                torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+                e2e_ms = float(t.item())
+            eb = 0
+            t1 = cache.query(0)["tokens"] - E
+            for i in range(E):
+                eb += bytes_of_step(t1 + i)[0]
+            e2e = {"value": world * eb / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+                   "h2d_bytes_per_step": layers * (kin[0, 0].numel() * 2 * 2 + qin[0, 0].numel() * 2),
+                   "d2h_bytes_per_step": layers * out[0].numel() * 4, "steps": E}
+
+    # ---- roofline of the decode kernel ----
+    peak, peak_kind = peaks()
+    achieved = dec_bytes / (dec_ms / 1e3) / 1e9
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs (copy)",
+            "traffic": None, "kernel": "decode_kernel (kvq_decode_attn)",
+            "avg_launch_us": round(dec_ms * 1e3 / (K * layers), 2),
+            "bytes_per_launch": int(dec_bytes / (K * layers))}
+
+    extra = {}
+    if not args.no_shrink and rank == 0:
+        flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        cache.free()
+        del cache, kin, vin, qin
+        torch.cuda.empty_cache()
+        extra["shrink"] = measure_shrink(kvq, dev, flush)
+        extra["shrink"]["unit"] = "GB/s"
+        extra["append_chunk"] = measure_append_chunk(kvq, dev, flush)
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(total_ms / K, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "layers": layers, "batch": B7, "q_heads": HQ7, "kv_heads": HKV7,
+                   "head_dim": HEAD_DIM, "context": T7, "fbit": fbit, "parallelism": f"replicas x{world}",
+                   "l2": "no flush: every block's cache read (151-285 MB) exceeds the 126 MB L2",
+                   "decode_ms_share": round(dec_ms / total_ms, 3)},
+        "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
+        **extra,
+    }
+    return res
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_sample(tokens, fbit=2, g=HQ7 // HKV7, seed=SEED):
+    """One (sequence, KV head) stream of a 7B-shape block, replayed through
+    the oracle's progressive cache; returns (layer, q, lam)."""
+    from oracle import oracle as orc
+
+    # a block sized for exactly `tokens` (a multiple of 512) ends full at its Fbit
+    tokens = (tokens + 511) // 512 * 512
+    L = orc.Layer(1, 1, tokens, fbit)
+    lam = None
+    pos = 0
+    while pos < tokens:
+        n = min(4096, tokens - pos)
+        k, v = S.keys_values(seed, 1, 1, n, 1, pos, S.outliers_for(HKV7), dtype=torch.bfloat16)
+        if lam is None:
+            lam = calib_lambda(k).numpy().reshape(1, HEAD_DIM).astype(np.float32)
+        assert L.append(k.float().numpy(), v.float().numpy(), lam) == 0
+        pos += n
+    q = S.queries(seed, 1, 0, 1, g, tokens, dtype=torch.bfloat16).float().numpy()
+    return L, q, lam
+
+
+def cpu_baseline(budget_s=15.0):
+    """The oracle's fp64 attention over sampled streams of a 7B 2-bit block
+    at the full context, timed single-threaded on this host."""
+    L, q, lam = oracle_sample(T7)
+    nb = decode_bytes(1, 1, HQ7 // HKV7, T7, L.bits)
+    t_start = time.perf_counter()
+    n = 0
+    while True:
+        L.attention(q, lam, HEAD_DIM ** -0.5)
+        n += 1
+        if time.perf_counter() - t_start > budget_s:
+            break
+    dt = time.perf_counter() - t_start
+    return {"value": round(n * nb / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} x one (sequence, KV head) stream of a 2-bit 7B-shape block, {T7} tokens, "
+                      f"{HQ7 // HKV7} query heads, fp64 attention; {dt:.1f} s"}
+
+
+def run_reference(args):
+    K, W = args.steps, args.warmup
+    tokens = T7 if K + W <= 20 else max(1024, (T7 * 20 // (K + W)) // 512 * 512)
+    L, q, lam = oracle_sample(tokens)
+    nb = decode_bytes(1, 1, HQ7 // HKV7, tokens, L.bits)
+    for _ in range(W):
+        L.attention(q, lam, HEAD_DIM ** -0.5)
+    t0 = time.perf_counter()
+    for _ in range(K):
+        L.attention(q, lam, HEAD_DIM ** -0.5)
+    dt = time.perf_counter() - t0
+    v = K * nb / dt / 1e9
+    sample = (f"each step: one (sequence, KV head) stream of a 2-bit 7B-shape block, {tokens} tokens, "
+              f"{HQ7 // HKV7} query heads, fp64 attention in the CPU oracle")
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 5), "unit": "GB/s", "n_gpus": 1,
+            "steps": K, "warmup": W, "ms_per_step": round(dt * 1e3 / K, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "layers": L7, "batch": B7, "q_heads": HQ7, "kv_heads": HKV7,
+                       "head_dim": HEAD_DIM, "context": T7, "fbit": FBIT7},
+            "cpu_baseline": {"value": round(v, 5), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(v, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
+    ap.add_argument("--layers", type=int, default=L7, help="blocks of the 7B shape to run (profiling cases)")
+    ap.add_argument("--no-shrink", action="store_true", help="skip the separate shrink/append measurements")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "kvq":
+        print("note: warm-up raised to 3", file=sys.stderr)
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_gpu(args, rank, world)
+        if rank == 0:
+            if world == 1 and not args.no_cpu:
+                res["cpu_baseline"] = cpu_baseline()
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,152 @@
+/*
+ * kvq.h -- C ABI of libkvq, a B200 (sm_100a) implementation of the online hot
+ * path of PM-KVQ's progressive mixed-precision KV cache.
+ *
+ * Method source: "PM-KVQ: Progressive Mixed-Precision KV Cache Quantization
+ * for Long-CoT LLMs" (papernotes.org note on the ICLR 2026 paper):
+ *   - key design 1, progressive quantization: every transformer block keeps
+ *     its KV cache at 16 bits until the block's memory budget is full, then
+ *     shrinks the whole block one level 16 -> 8 -> 4 -> 2 with the Equivalent
+ *     Right Shift  X_b = ((2^{2b} - 2^b + 1)(X_{2b} + 2^{b-1})) >> 3b,
+ *     Z_b = Z_{2b}, S_b = (2^b + 1) S_{2b}, stopping at the block's Fbit;
+ *   - key design 2: each block has its own Fbit (chosen offline; an input);
+ *   - key design 3: Key outliers move to the Query per channel (K / lambda,
+ *     Q * lambda; lambda is calibrated offline and is an input here);
+ *   - training strategy: asymmetric quantization with groups of 128.
+ *
+ * Conventions for every call:
+ *   - head_dim is 128; one quantization group is one token's 128 channels of
+ *     one KV head.  Codes are unsigned; x^ = Z + q * R / (2^b - 1) with R and
+ *     Z binary16 per group.
+ *   - "device" pointers are CUDA global-memory addresses on the device that
+ *     was current when the cache was created; "host" pointers are ordinary
+ *     CPU memory.  The caller owns every buffer it passes (inputs, outputs,
+ *     workspace, the optional pool).  The library owns the cache's host state
+ *     and, when it allocated it, the device pool.
+ *   - stream: a cudaStream_t (NULL = legacy default stream).  Calls that take
+ *     a stream enqueue work on it and return without waiting, unless stated.
+ *   - A call that returns an error other than KVQ_ERR_CUDA has changed
+ *     nothing.  kvq_last_error() describes the last failure on the calling
+ *     thread.
+ *   - Calls on one cache are not thread-safe; serialise them.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct kvq_cache kvq_cache; /* opaque, host-owned */
+typedef struct CUstream_st* kvq_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID = 1,   /* bad argument (null pointer, range, shape) */
+  KVQ_ERR_BUDGET = 2,    /* the block is full at its Fbit: the tokens do not fit */
+  KVQ_ERR_STATE = 3,     /* the call is not allowed in the block's current state */
+  KVQ_ERR_OOM = 4,       /* device allocation failed */
+  KVQ_ERR_CUDA = 5,      /* a CUDA call or kernel launch failed */
+  KVQ_ERR_WORKSPACE = 6, /* workspace missing or smaller than kvq_decode_workspace() */
+  KVQ_ERR_TIMEOUT = 7    /* a kernel gave up waiting on one of its own copies */
+} kvq_status;
+
+enum { KVQ_DTYPE_BF16 = 0, KVQ_DTYPE_F32 = 1 };
+
+/* Size in bytes of the device pool a cache with these parameters needs, or 0
+ * if the parameters are invalid.  Pure host computation.
+ *
+ * Budget split (key designs 1 and 2): every block can hold the same number of
+ * tokens N at its own Fbit, the largest multiple of 512 with
+ *   batch * kv_heads * 2 * N * sum_l (16 * fbit[l] + 4)  <=  budget_bytes
+ * (16*F bytes of codes and 4 bytes of binary16 (R, Z) per token, head and
+ * K-or-V).  The pool is exactly that many bytes plus a few KiB of per-layer
+ * lambda tables and counters. */
+size_t kvq_pool_bytes(int layers, int batch, int kv_heads, int head_dim, size_t budget_bytes,
+                      const int* fbit /* host [layers], each 2, 4, 8 or 16 */);
+
+/* Create a cache.  fbit: host [layers].  dev_pool: a device buffer of at least
+ * kvq_pool_bytes(...) bytes, owned by the caller and kept alive until
+ * kvq_free; or NULL, and the library cudaMallocs the pool itself.  With a
+ * caller pool this call makes no CUDA call.  Every block starts empty at 16
+ * bits.  Errors: INVALID (shape, fbit, head_dim != 128), BUDGET (budget
+ * smaller than 512 tokens), OOM. */
+kvq_status kvq_alloc(kvq_cache** out, int layers, int batch, int kv_heads, int head_dim,
+                     size_t budget_bytes, const int* fbit, void* dev_pool, size_t pool_bytes);
+
+/* Per-channel migration factor of one block (key design 3).  lambda_host:
+ * host float [kv_heads][128], every value finite and > 0.  Stored Keys become
+ * fp32(k * fp32(1/lambda)) and queries are multiplied by lambda inside the
+ * attention kernel.  Until it is called a block uses lambda = 1.  Copies
+ * synchronously; must not be called while kernels on this block are in
+ * flight. */
+kvq_status kvq_set_lambda(kvq_cache* c, int layer, const float* lambda_host);
+
+/* Quantize-on-append (key design 1): append n_tokens tokens to every
+ * sequence of the batch.  k, v: device [batch][n_tokens][kv_heads][128],
+ * dtype KVQ_DTYPE_BF16 or KVQ_DTYPE_F32, 16-byte aligned.  Each token is
+ * quantized at the block's current width; when the block is full the block
+ * is first shrunk one level (never below its Fbit).  n tokens behave exactly
+ * like n single-token appends.  Errors: BUDGET when the block cannot hold
+ * them at its Fbit (nothing is written), INVALID, CUDA. */
+kvq_status kvq_append(kvq_cache* c, int layer, const void* k, const void* v, int dtype,
+                      int n_tokens, kvq_stream_t stream);
+
+/* Shrink a full block one level now (the step its next append would take):
+ * every stored code goes through the Equivalent Right Shift, in place.  Meta
+ * is not touched: with R = (2^b - 1) S, S_b = (2^b + 1) S_{2b} leaves R
+ * unchanged.  Errors: STATE if the block is not full at its current width or
+ * is already at its Fbit. */
+kvq_status kvq_shrink(kvq_cache* c, int layer, kvq_stream_t stream);
+
+/* Bytes of device workspace kvq_decode_attn needs for this block and number
+ * of query heads (any token count).  0 on invalid arguments. */
+size_t kvq_decode_workspace(const kvq_cache* c, int layer, int q_heads);
+
+/* GQA decode attention over the block's quantized cache:
+ *   out[b][h] = sum_t softmax_t(sm_scale * (q[b][h] * lambda) . k^_t) v^_t
+ * over every cached token, query head h reading KV head h / (q_heads /
+ * kv_heads).  q: device bf16 [batch][q_heads][128]; out: device fp32
+ * [batch][q_heads][128]; workspace: device buffer of at least
+ * kvq_decode_workspace(c, layer, q_heads) bytes (contents need no
+ * initialisation; the call owns it until it completes on the stream).
+ * q_heads must be a multiple of kv_heads with at most 8 query heads per KV
+ * head.  Errors: STATE if the block is empty, WORKSPACE, INVALID, CUDA. */
+kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, float sm_scale,
+                           float* out, void* workspace, size_t ws_bytes, kvq_stream_t stream);
+
+/* Host-side state of one block.  Any output pointer may be NULL.
+ * capacity: tokens that fit at the current width. */
+kvq_status kvq_query(const kvq_cache* c, int layer, int* tokens, int* bits, int* capacity,
+                     int* n_shrinks);
+
+/* Tokens every block can hold at its Fbit (N in kvq_pool_bytes). */
+int kvq_max_tokens(const kvq_cache* c);
+
+/* Copy one (sequence b, KV head j) stream of a block to host memory in
+ * logical token order (the order tokens were appended):
+ *   k_codes, v_codes: host uint16 [tokens][128] (codes at the current width)
+ *   k_meta,  v_meta : host uint16 [tokens][2]   (binary16 bits of R, Z)
+ * Any of the four may be NULL.  Synchronous: waits for the stream. */
+kvq_status kvq_export(const kvq_cache* c, int layer, int b, int j, uint16_t* k_codes,
+                      uint16_t* v_codes, uint16_t* k_meta, uint16_t* v_meta,
+                      kvq_stream_t stream);
+
+/* Wait for the stream and report whether a kernel of this cache gave up on a
+ * bounded wait (KVQ_ERR_TIMEOUT) since the last check; clears the flag. */
+kvq_status kvq_device_status(kvq_cache* c, kvq_stream_t stream);
+
+/* Message of the last failed call on this thread ("" if none). */
+const char* kvq_last_error(void);
+
+/* Release the cache (and the pool if the library allocated it).  Waits for
+ * the device.  NULL is ignored. */
+void kvq_free(kvq_cache* c);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVQ_H */

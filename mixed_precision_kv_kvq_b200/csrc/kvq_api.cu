@@ -1,0 +1,482 @@
+// kvq_api.cu -- the C ABI of libkvq (include/kvq.h): cache allocation, the
+// budget-triggered shrink scheduler, the slot map, export and error state.
+//
+// Scheduler (PM-KVQ note, key design 1): a block starts at 16 bits; a token
+// that arrives while the block holds cap(b) = N * Fbit / b tokens first
+// shrinks the whole block one level (16 -> 8 -> 4 -> 2, never below Fbit).
+// The host keeps every counter, so deciding to shrink never reads device
+// memory and nothing synchronises.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/kvq.h"
+#include "kvq_internal.cuh"
+
+using namespace kvq;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+kvq_status fail(kvq_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+kvq_status fail(kvq_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+kvq_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(KVQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr size_t kAlign = 256;
+constexpr int kTokenRound = 512;  // tokens per tile at 2 bits: a multiple for every width
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool valid_fbit(int f) { return f == 2 || f == 4 || f == 8 || f == 16; }
+
+struct LayerState {
+  int fbit;
+  int bits;
+  long long n;
+  int n_shrinks;
+  int nt;  // tiles per stream
+  int pf;  // meta slots per tile
+  bool counters_zeroed;
+  size_t off_lam, off_lam_inv, off_counters, off_codes, off_meta;
+  bool lambda_set;
+};
+
+struct Plan {
+  long long n_f;
+  size_t bytes;
+  std::vector<LayerState> layers;
+};
+
+// Budget split: every block holds the same N tokens at its own Fbit.
+bool make_plan(int layers, int batch, int kv_heads, int head_dim, size_t budget, const int* fbit, Plan& p,
+               kvq_status* why) {
+  *why = KVQ_ERR_INVALID;
+  if (layers < 1 || batch < 1 || kv_heads < 1 || head_dim != kHeadDim || !fbit) return false;
+  unsigned long long per_token = 0;  // bytes per token over all blocks
+  const unsigned long long streams = (unsigned long long)batch * kv_heads * 2;
+  for (int l = 0; l < layers; l++) {
+    if (!valid_fbit(fbit[l])) return false;
+    per_token += streams * (16ull * fbit[l] + 4ull);
+  }
+  const unsigned long long n_raw = budget / per_token;
+  const long long n_f = (long long)(n_raw / kTokenRound) * kTokenRound;
+  if (n_f < kTokenRound || n_f > (1ll << 30)) {
+    *why = KVQ_ERR_BUDGET;
+    return false;
+  }
+  p.n_f = n_f;
+  p.layers.assign(layers, LayerState{});
+  size_t off = kAlign;  // [0, 256): device error flag
+  const size_t n_streams = (size_t)batch * kv_heads;
+  for (int l = 0; l < layers; l++) {
+    LayerState& L = p.layers[l];
+    L.fbit = fbit[l];
+    L.bits = 16;
+    L.n = 0;
+    L.n_shrinks = 0;
+    L.pf = slots_per_tile(L.fbit);
+    L.nt = (int)(n_f / L.pf);
+    L.counters_zeroed = false;
+    L.lambda_set = false;
+    L.off_lam = off;
+    off += align_up((size_t)kv_heads * kHeadDim * 4);
+    L.off_lam_inv = off;
+    off += align_up((size_t)kv_heads * kHeadDim * 4);
+    L.off_counters = off;
+    off += align_up(n_streams * 4);
+    L.off_codes = off;
+    off += align_up(n_streams * 2 * (size_t)L.nt * kTileBytes);
+    L.off_meta = off;
+    off += align_up(n_streams * 2 * (size_t)L.nt * L.pf * 4);
+  }
+  p.bytes = off;
+  *why = KVQ_OK;
+  return true;
+}
+
+long long capacity(const LayerState& L, long long n_f, int bits) { return n_f * L.fbit / bits; }
+
+}  // namespace
+
+struct kvq_cache {
+  int layers, batch, kv_heads;
+  long long n_f;
+  uint8_t* pool;
+  size_t pool_bytes;
+  bool owns_pool;
+  int num_sms;
+  bool err_zeroed;
+  std::vector<LayerState> L;
+
+  // The error flag lives in the pool; clear it once, stream-ordered, before
+  // the first kernel of this cache can set it.
+  cudaError_t ensure_err(cudaStream_t s) {
+    if (err_zeroed) return cudaSuccess;
+    cudaError_t e = cudaMemsetAsync(pool, 0, 4, s);
+    if (e == cudaSuccess) err_zeroed = true;
+    return e;
+  }
+
+  int sms() {
+    if (num_sms <= 0) {
+      int dev = 0, n = 0;
+      if (cudaGetDevice(&dev) == cudaSuccess &&
+          cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) {
+        num_sms = n;
+      } else {
+        cudaGetLastError();
+        num_sms = 148;  // B200
+      }
+    }
+    return num_sms;
+  }
+  uint8_t* codes(int l) { return pool + L[l].off_codes; }
+  uint32_t* meta(int l) { return reinterpret_cast<uint32_t*>(pool + L[l].off_meta); }
+  float* lam(int l) { return reinterpret_cast<float*>(pool + L[l].off_lam); }
+  float* lam_inv(int l) { return reinterpret_cast<float*>(pool + L[l].off_lam_inv); }
+  int* counters(int l) { return reinterpret_cast<int*>(pool + L[l].off_counters); }
+  int* err() { return reinterpret_cast<int*>(pool); }
+};
+
+namespace {
+
+kvq_status check_layer(const kvq_cache* c, int layer) {
+  if (!c) return fail(KVQ_ERR_INVALID, "cache is NULL");
+  if (layer < 0 || layer >= c->layers) return fail(KVQ_ERR_INVALID, "layer %d out of range [0, %d)", layer, c->layers);
+  return KVQ_OK;
+}
+
+// Slot of logical token i: the epoch it was appended in fixes its tile/slot.
+void slot_of(const LayerState& L, long long i, int* tile, int* slot) {
+  int e = 0;
+  int bits = 16;
+  while (e < L.n_shrinks) {
+    const long long end = (long long)L.nt * slots_per_tile(bits);  // cap at this width
+    if (i < end) break;
+    bits >>= 1;
+    e++;
+  }
+  const int p = slots_per_tile(bits);
+  const int h = e > 0 ? p / 2 : 0;
+  const int ee = p - h;
+  const long long m = i - (long long)L.nt * h;
+  *tile = (int)(m / ee);
+  *slot = h + (int)(m % ee);
+}
+
+uint32_t rd32(const uint8_t* p) {
+  uint32_t w;
+  memcpy(&w, p, 4);
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kvq_pool_bytes(int layers, int batch, int kv_heads, int head_dim, size_t budget_bytes, const int* fbit) {
+  Plan p;
+  kvq_status why;
+  if (!make_plan(layers, batch, kv_heads, head_dim, budget_bytes, fbit, p, &why)) return 0;
+  return p.bytes;
+}
+
+kvq_status kvq_alloc(kvq_cache** out, int layers, int batch, int kv_heads, int head_dim, size_t budget_bytes,
+                     const int* fbit, void* dev_pool, size_t pool_bytes) {
+  if (!out) return fail(KVQ_ERR_INVALID, "out is NULL");
+  *out = nullptr;
+  Plan p;
+  kvq_status why;
+  if (!make_plan(layers, batch, kv_heads, head_dim, budget_bytes, fbit, p, &why)) {
+    if (why == KVQ_ERR_BUDGET) return fail(why, "budget of %zu bytes holds fewer than %d tokens per block", budget_bytes, kTokenRound);
+    return fail(why, "invalid shape or fbit (layers=%d batch=%d kv_heads=%d head_dim=%d; fbit must be 2/4/8/16, head_dim 128)",
+                layers, batch, kv_heads, head_dim);
+  }
+  if (dev_pool && pool_bytes < p.bytes)
+    return fail(KVQ_ERR_INVALID, "pool of %zu bytes is smaller than the %zu bytes needed", pool_bytes, p.bytes);
+  if (dev_pool && (reinterpret_cast<uintptr_t>(dev_pool) % kAlign))
+    return fail(KVQ_ERR_INVALID, "pool must be %zu-byte aligned", kAlign);
+  kvq_cache* c = new (std::nothrow) kvq_cache();
+  if (!c) return fail(KVQ_ERR_OOM, "host allocation failed");
+  c->layers = layers;
+  c->batch = batch;
+  c->kv_heads = kv_heads;
+  c->n_f = p.n_f;
+  c->L = p.layers;
+  c->num_sms = 0;
+  c->err_zeroed = false;
+  if (dev_pool) {
+    c->pool = static_cast<uint8_t*>(dev_pool);
+    c->owns_pool = false;
+  } else {
+    void* ptr = nullptr;
+    cudaError_t e = cudaMalloc(&ptr, p.bytes);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      delete c;
+      return fail(KVQ_ERR_OOM, "cudaMalloc(%zu): %s", p.bytes, cudaGetErrorString(e));
+    }
+    c->pool = static_cast<uint8_t*>(ptr);
+    c->owns_pool = true;
+  }
+  c->pool_bytes = p.bytes;
+  *out = c;
+  return KVQ_OK;
+}
+
+kvq_status kvq_set_lambda(kvq_cache* c, int layer, const float* lambda_host) {
+  if (kvq_status s = check_layer(c, layer)) return s;
+  if (!lambda_host) return fail(KVQ_ERR_INVALID, "lambda is NULL");
+  const size_t n = (size_t)c->kv_heads * kHeadDim;
+  std::vector<float> inv(n);
+  for (size_t i = 0; i < n; i++) {
+    const float v = lambda_host[i];
+    if (!(v > 0.0f) || !std::isfinite(v)) return fail(KVQ_ERR_INVALID, "lambda[%zu] = %g is not finite and > 0", i, (double)v);
+    inv[i] = (float)(1.0 / (double)v);
+  }
+  cudaError_t e = cudaMemcpy(c->lam(layer), lambda_host, n * 4, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(c->lam_inv(layer), inv.data(), n * 4, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "lambda upload");
+  c->L[layer].lambda_set = true;
+  return KVQ_OK;
+}
+
+kvq_status kvq_append(kvq_cache* c, int layer, const void* k, const void* v, int dtype, int n_tokens,
+                      kvq_stream_t stream) {
+  if (kvq_status s = check_layer(c, layer)) return s;
+  if (n_tokens < 0) return fail(KVQ_ERR_INVALID, "n_tokens %d < 0", n_tokens);
+  if (n_tokens == 0) return KVQ_OK;
+  if (!k || !v) return fail(KVQ_ERR_INVALID, "k or v is NULL");
+  if (dtype != KVQ_DTYPE_BF16 && dtype != KVQ_DTYPE_F32) return fail(KVQ_ERR_INVALID, "dtype %d unknown", dtype);
+  if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) % 16)
+    return fail(KVQ_ERR_INVALID, "k and v must be 16-byte aligned");
+  LayerState& L = c->L[layer];
+  if (L.n + n_tokens > c->n_f)
+    return fail(KVQ_ERR_BUDGET, "layer %d holds %lld of %lld tokens at Fbit %d; %d more do not fit", layer, L.n, c->n_f,
+                L.fbit, n_tokens);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaError_t e = c->ensure_err(s)) return cuda_fail(e, "error flag reset");
+  int off = 0;
+  while (off < n_tokens) {
+    const long long cap = capacity(L, c->n_f, L.bits);
+    if (L.n == cap) {  // full: shrink one level first (bits > fbit is implied by the budget check)
+      ShrinkArgs sa{c->codes(layer), (long long)c->batch * c->kv_heads * 2 * L.nt, L.bits / 2};
+      cudaError_t e = launch_shrink(sa, s);
+      if (e != cudaSuccess) return cuda_fail(e, "shrink launch");
+      L.bits /= 2;
+      L.n_shrinks++;
+      continue;
+    }
+    const int cnt = (int)std::min<long long>(n_tokens - off, cap - L.n);
+    AppendArgs a{};
+    a.k = k;
+    a.v = v;
+    a.dtype = dtype;
+    a.n_call = n_tokens;
+    a.tok_off = off;
+    a.cnt = cnt;
+    a.n0 = L.n;
+    a.bits = L.bits;
+    const int p = slots_per_tile(L.bits);
+    a.h = L.n_shrinks > 0 ? p / 2 : 0;
+    a.e = p - a.h;
+    a.nt = L.nt;
+    a.pf = L.pf;
+    a.batch = c->batch;
+    a.kv_heads = c->kv_heads;
+    a.codes = c->codes(layer);
+    a.meta = c->meta(layer);
+    a.lam_inv = L.lambda_set ? c->lam_inv(layer) : nullptr;
+    cudaError_t e = launch_append(a, s);
+    if (e != cudaSuccess) return cuda_fail(e, "append launch");
+    L.n += cnt;
+    off += cnt;
+  }
+  return KVQ_OK;
+}
+
+kvq_status kvq_shrink(kvq_cache* c, int layer, kvq_stream_t stream) {
+  if (kvq_status s = check_layer(c, layer)) return s;
+  LayerState& L = c->L[layer];
+  if (L.bits <= L.fbit) return fail(KVQ_ERR_STATE, "layer %d is at its Fbit %d", layer, L.fbit);
+  const long long cap = capacity(L, c->n_f, L.bits);
+  if (L.n != cap)
+    return fail(KVQ_ERR_STATE, "layer %d holds %lld tokens; a shrink needs the block full (%lld at %d bits)", layer, L.n, cap,
+                L.bits);
+  ShrinkArgs sa{c->codes(layer), (long long)c->batch * c->kv_heads * 2 * L.nt, L.bits / 2};
+  cudaError_t e = launch_shrink(sa, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "shrink launch");
+  L.bits /= 2;
+  L.n_shrinks++;
+  return KVQ_OK;
+}
+
+size_t kvq_decode_workspace(const kvq_cache* c, int layer, int q_heads) {
+  if (!c || layer < 0 || layer >= c->layers || q_heads <= 0 || q_heads % c->kv_heads) return 0;
+  const int G = q_heads / c->kv_heads;
+  if (G > 8) return 0;
+  kvq_cache* m = const_cast<kvq_cache*>(c);
+  return decode_parts_bytes(decode_grid(m->sms()), c->batch * c->kv_heads, G);
+}
+
+kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, float sm_scale, float* out,
+                           void* workspace, size_t ws_bytes, kvq_stream_t stream) {
+  if (kvq_status s = check_layer(c, layer)) return s;
+  if (!q || !out) return fail(KVQ_ERR_INVALID, "q or out is NULL");
+  if (q_heads <= 0 || q_heads % c->kv_heads)
+    return fail(KVQ_ERR_INVALID, "q_heads %d is not a positive multiple of kv_heads %d", q_heads, c->kv_heads);
+  const int G = q_heads / c->kv_heads;
+  if (G > 8) return fail(KVQ_ERR_INVALID, "%d query heads per KV head; at most 8 are supported", G);
+  if (!std::isfinite(sm_scale)) return fail(KVQ_ERR_INVALID, "sm_scale is not finite");
+  if ((reinterpret_cast<uintptr_t>(q) % 4) || (reinterpret_cast<uintptr_t>(out) % 4))
+    return fail(KVQ_ERR_INVALID, "q and out must be 4-byte aligned");
+  LayerState& L = c->L[layer];
+  if (L.n <= 0) return fail(KVQ_ERR_STATE, "layer %d is empty", layer);
+  const int n_streams = c->batch * c->kv_heads;
+  const int max_grid = decode_grid(c->sms());
+  const size_t need = decode_parts_bytes(max_grid, n_streams, G);
+  if (!workspace || ws_bytes < need)
+    return fail(KVQ_ERR_WORKSPACE, "workspace of %zu bytes; %zu needed", workspace ? ws_bytes : (size_t)0, need);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaError_t e = c->ensure_err(s)) return cuda_fail(e, "error flag reset");
+  if (!L.counters_zeroed) {
+    cudaError_t e = cudaMemsetAsync(c->counters(layer), 0, (size_t)n_streams * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "counter reset");
+    L.counters_zeroed = true;
+  }
+  DecodeArgs a{};
+  a.codes = c->codes(layer);
+  a.meta = c->meta(layer);
+  a.q = q;
+  a.lam = L.lambda_set ? c->lam(layer) : nullptr;
+  a.out = out;
+  a.parts = static_cast<float*>(workspace);
+  a.counters = c->counters(layer);
+  a.err = c->err();
+  a.fill = make_fill(L.bits, L.nt, L.pf, L.n_shrinks, L.n);
+  a.batch = c->batch;
+  a.kv_heads = c->kv_heads;
+  a.q_heads = q_heads;
+  a.group = G;
+  a.qscale = sm_scale * 1.4426950408889634f;
+  const long long tot = (long long)n_streams * a.fill.gps;
+  a.grid = (int)std::min<long long>(max_grid, tot);
+  cudaError_t e = launch_decode(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return KVQ_OK;
+}
+
+kvq_status kvq_query(const kvq_cache* c, int layer, int* tokens, int* bits, int* cap, int* n_shrinks) {
+  if (kvq_status s = check_layer(c, layer)) return s;
+  const LayerState& L = c->L[layer];
+  if (tokens) *tokens = (int)L.n;
+  if (bits) *bits = L.bits;
+  if (cap) *cap = (int)capacity(L, c->n_f, L.bits);
+  if (n_shrinks) *n_shrinks = L.n_shrinks;
+  return KVQ_OK;
+}
+
+int kvq_max_tokens(const kvq_cache* c) { return c ? (int)c->n_f : 0; }
+
+kvq_status kvq_export(const kvq_cache* c, int layer, int b, int j, uint16_t* k_codes, uint16_t* v_codes,
+                      uint16_t* k_meta, uint16_t* v_meta, kvq_stream_t stream) {
+  if (kvq_status s = check_layer(c, layer)) return s;
+  if (b < 0 || b >= c->batch || j < 0 || j >= c->kv_heads)
+    return fail(KVQ_ERR_INVALID, "stream (%d, %d) out of range", b, j);
+  const LayerState& L = c->L[layer];
+  kvq_cache* m = const_cast<kvq_cache*>(c);
+  const size_t code_bytes = (size_t)L.nt * kTileBytes, meta_words = (size_t)L.nt * L.pf;
+  const size_t sk = ((size_t)b * c->kv_heads + j) * 2, sv = sk + 1;
+  std::vector<uint8_t> kc(code_bytes), vc(code_bytes);
+  std::vector<uint32_t> km(meta_words), vm(meta_words);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(kc.data(), m->codes(layer) + sk * code_bytes, code_bytes, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(vc.data(), m->codes(layer) + sv * code_bytes, code_bytes, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(km.data(), m->meta(layer) + sk * meta_words, meta_words * 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(vm.data(), m->meta(layer) + sv * meta_words, meta_words * 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "export copy");
+  const int bits = L.bits, ppw = 16 / bits;
+  const uint32_t mask = bits == 16 ? 0xffffu : ((1u << bits) - 1u);
+  for (long long i = 0; i < L.n; i++) {
+    int tile, slot;
+    slot_of(L, i, &tile, &slot);
+    const int grp = slot >> 4, tok = slot & 15;
+    const size_t gbase = (size_t)tile * kTileBytes + (size_t)grp * group_bytes(bits);
+    if (k_codes) {
+      const int g = tok & 7, x = tok >> 3;
+      for (int ch = 0; ch < kHeadDim; ch++) {
+        const int sb = ch >> 4, rem = ch & 15, r = rem >> 3, t = (rem & 7) >> 1, mb = rem & 1;
+        const int p = 2 * sb + r, word = x * bits + p / ppw, pos = p % ppw;
+        const uint32_t w = rd32(&kc[gbase + (size_t)(4 * g + t) * unit_bytes(bits) + 4 * word]);
+        k_codes[i * kHeadDim + ch] = (uint16_t)((w >> (16 * mb + bits * pos)) & mask);
+      }
+    }
+    if (v_codes) {
+      const int t = (tok & 7) >> 1, mb = tok & 1, u = tok >> 3;
+      for (int ch = 0; ch < kHeadDim; ch++) {
+        const int sb = ch >> 4, rem = ch & 15, r = rem >> 3, g = rem & 7;
+        const int p = 2 * sb + r, word = u * bits + p / ppw, pos = p % ppw;
+        const uint32_t w = rd32(&vc[gbase + (size_t)(4 * g + t) * unit_bytes(bits) + 4 * word]);
+        v_codes[i * kHeadDim + ch] = (uint16_t)((w >> (16 * mb + bits * pos)) & mask);
+      }
+    }
+    const size_t mi = (size_t)tile * L.pf + slot;
+    if (k_meta) {
+      k_meta[2 * i] = (uint16_t)(km[mi] & 0xffffu);
+      k_meta[2 * i + 1] = (uint16_t)(km[mi] >> 16);
+    }
+    if (v_meta) {
+      v_meta[2 * i] = (uint16_t)(vm[mi] & 0xffffu);
+      v_meta[2 * i + 1] = (uint16_t)(vm[mi] >> 16);
+    }
+  }
+  return KVQ_OK;
+}
+
+kvq_status kvq_device_status(kvq_cache* c, kvq_stream_t stream) {
+  if (!c) return fail(KVQ_ERR_INVALID, "cache is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaError_t e = c->ensure_err(s)) return cuda_fail(e, "error flag reset");
+  int flag = 0;
+  cudaError_t e = cudaMemcpyAsync(&flag, c->err(), 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "device status");
+  if (flag) {
+    const int zero = 0;
+    e = cudaMemcpy(c->err(), &zero, 4, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "device status reset");
+    return fail(KVQ_ERR_TIMEOUT, "a kernel gave up waiting on its own bulk copies");
+  }
+  return KVQ_OK;
+}
+
+const char* kvq_last_error(void) { return g_last_error.c_str(); }
+
+void kvq_free(kvq_cache* c) {
+  if (!c) return;
+  if (c->owns_pool && c->pool) {
+    cudaDeviceSynchronize();
+    cudaFree(c->pool);
+  }
+  delete c;
+}
+
+}  // extern "C"

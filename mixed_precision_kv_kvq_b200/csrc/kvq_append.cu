@@ -1,0 +1,159 @@
+// kvq_append.cu -- quantize-on-append (PM-KVQ note, key design 1: each new
+// token is stored at the block's current width; key design 3: Keys are
+// divided by the per-channel migration factor lambda first; training
+// strategy: asymmetric groups of 128).
+//
+// One warp quantizes one group = one token's 128 channels of one KV head, K
+// or V.  Per group, with every step a single IEEE fp32 round-to-nearest
+// operation (no contraction):
+//   x_c = k_c * lambda_inv_c            (K only)
+//   Z   = binary16 round-down(min x)    R = binary16 round-up(max x - Z)
+//   q_c = clamp(floor((x_c - Z) * ((2^b - 1) / R) + 1/2), 0, 2^b - 1)
+// (R = 0: all codes 0), then scatters the codes into the group's lane units
+// (see kvq_internal.cuh) and writes (R, Z) to the slot's meta word.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kWarpsPerBlock = 8;
+
+__device__ __forceinline__ float warp_min(float x) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+__global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs a) {
+  __shared__ uint16_t codes_sh[kWarpsPerBlock][kHeadDim];
+  const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
+  const long long w = (long long)blockIdx.x * kWarpsPerBlock + wib;
+  const long long total = (long long)a.batch * a.cnt * a.kv_heads * 2;
+  if (w >= total) return;  // warp-uniform
+
+  const int kv = (int)(w & 1);
+  long long rest = w >> 1;
+  const int j = (int)(rest % a.kv_heads);
+  rest /= a.kv_heads;
+  const int tkn = (int)(rest % a.cnt);
+  const int b = (int)(rest / a.cnt);
+
+  // ---- load 4 channels per lane, migrate Keys ----
+  const size_t in_off =
+      (((size_t)b * a.n_call + (size_t)(a.tok_off + tkn)) * a.kv_heads + j) * kHeadDim + 4 * lane;
+  const void* src = kv ? a.v : a.k;
+  float x[4];
+  if (a.dtype == 1) {
+    float4 f = *reinterpret_cast<const float4*>(static_cast<const float*>(src) + in_off);
+    x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+  } else {
+    uint2 raw = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(src) + in_off);
+    __nv_bfloat162 p0 = *reinterpret_cast<__nv_bfloat162*>(&raw.x);
+    __nv_bfloat162 p1 = *reinterpret_cast<__nv_bfloat162*>(&raw.y);
+    x[0] = __low2float(p0); x[1] = __high2float(p0);
+    x[2] = __low2float(p1); x[3] = __high2float(p1);
+  }
+  if (kv == 0 && a.lam_inv) {
+    float4 li = *reinterpret_cast<const float4*>(a.lam_inv + (size_t)j * kHeadDim + 4 * lane);
+    x[0] = __fmul_rn(x[0], li.x); x[1] = __fmul_rn(x[1], li.y);
+    x[2] = __fmul_rn(x[2], li.z); x[3] = __fmul_rn(x[3], li.w);
+  }
+
+  // ---- group meta ----
+  float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
+  float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+  mn = warp_min(mn);
+  mx = warp_max(mx);
+  const __half zh = __float2half_rd(mn);
+  const float z = __half2float(zh);
+  const __half rh = __float2half_ru(__fsub_rn(mx, z));
+  const float r = __half2float(rh);
+  const int bits = a.bits;
+  const float qmax = (float)((1u << bits) - 1u);
+  uint16_t* sc = codes_sh[wib];
+  if (r == 0.0f) {
+#pragma unroll
+    for (int i = 0; i < 4; i++) sc[4 * lane + i] = 0;
+  } else {
+    const float inv = __fdiv_rn(qmax, r);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      float t = __fmul_rn(__fsub_rn(x[i], z), inv);
+      float f = floorf(__fadd_rn(t, 0.5f));
+      f = fminf(fmaxf(f, 0.0f), qmax);
+      sc[4 * lane + i] = (uint16_t)f;
+    }
+  }
+  __syncwarp();
+
+  // ---- slot of this token ----
+  const long long li = a.n0 + tkn;
+  const long long m = li - (long long)a.nt * a.h;
+  const int tile = (int)(m / a.e);
+  const int slot = a.h + (int)(m - (long long)tile * a.e);
+  const int grp = slot >> 4;
+  const int tok = slot & 15;
+  const size_t stream_kv = ((size_t)b * a.kv_heads + j) * 2 + kv;
+  uint8_t* gbase = a.codes + (stream_kv * a.nt + tile) * (size_t)kTileBytes + (size_t)grp * group_bytes(bits);
+  const int ppw = 16 / bits;  // pairs per 32-bit word (per 16-bit half)
+
+  if (kv == 0) {
+    // Token tok: g = tok % 8, x = tok / 8.  Lane units 4g + t (t = 0..3) each
+    // get `bits` words: unit word x*bits + jw holds pairs P = 16x + jw*ppw + kk.
+    const int g = tok & 7, xs = tok >> 3;
+    for (int wi = lane; wi < 4 * bits; wi += 32) {
+      const int t = wi / bits, jw = wi - t * bits;
+      uint32_t word = 0;
+      for (int kk = 0; kk < ppw; kk++) {
+        const int p = jw * ppw + kk;  // pair within the token's half: p = 2s + rr
+        const int ch0 = 16 * (p >> 1) + 2 * t + 8 * (p & 1);
+        word |= (uint32_t)sc[ch0] << (bits * kk);
+        word |= (uint32_t)sc[ch0 + 1] << (16 + bits * kk);
+      }
+      uint32_t* dst = reinterpret_cast<uint32_t*>(gbase + (4 * g + t) * unit_bytes(bits)) + xs * bits + jw;
+      *dst = word;
+    }
+  } else {
+    // Token tok: t = (tok % 8) / 2, member mb = tok % 2, pair set u = tok / 8.
+    // Units 4g + t (g = 0..7): word u*bits + jw, half mb, pairs p = 2s + rr of
+    // channel 16s + g + 8rr.
+    const int t = (tok & 7) >> 1, mb = tok & 1, u = tok >> 3;
+    for (int hw = lane; hw < 8 * bits; hw += 32) {
+      const int g = hw / bits, jw = hw - g * bits;
+      uint32_t half = 0;
+      for (int kk = 0; kk < ppw; kk++) {
+        const int p = jw * ppw + kk;
+        const int ch = 16 * (p >> 1) + g + 8 * (p & 1);
+        half |= (uint32_t)sc[ch] << (bits * kk);
+      }
+      uint16_t* dst = reinterpret_cast<uint16_t*>(gbase + (4 * g + t) * unit_bytes(bits)) +
+                      2 * (u * bits + jw) + mb;
+      *dst = (uint16_t)half;
+    }
+  }
+  if (lane == 0) {
+    const uint32_t mw = (uint32_t)__half_as_ushort(rh) | ((uint32_t)__half_as_ushort(zh) << 16);
+    a.meta[(stream_kv * a.nt + tile) * (size_t)a.pf + slot] = mw;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
+  const long long warps = (long long)a.batch * a.cnt * a.kv_heads * 2;
+  if (warps <= 0) return cudaSuccess;
+  const long long blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  append_kernel<<<(unsigned)blocks, kWarpsPerBlock * 32, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

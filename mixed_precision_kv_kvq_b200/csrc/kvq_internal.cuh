@@ -1,0 +1,171 @@
+// kvq_internal.cuh -- packed layout, block fill pattern and launch interfaces
+// shared by the libkvq kernels and the host scheduler.
+//
+// Packed layout (one "stream" = one (layer, sequence, KV head, K-or-V)):
+//   The stream is a region of NT tiles of 16 KiB.  At b bits a tile holds
+//   P_b = 1024 / b token slots (64 at 16 bits ... 512 at 2 bits), grouped in
+//   16-token groups of 256*b bytes.  A group is 32 "lane units" of 8*b bytes;
+//   unit L holds exactly the 64 codes that lane L of a warp needs as its
+//   mma.sync.m16n8k16 A-fragment registers:
+//     K (QK^T, A = K[token][channel]):  with L = 4g + t, tokens g and g+8 of
+//       the group, channels 16s + 2t + {0,1} + 8r  (s = 0..7, r = 0..1).
+//     V (P V,  A = V^T[channel][token]): channels 16s + g + 8r, tokens
+//       2t + {0,1} + 8u (u = 0..1).
+//   Codes come in pairs that fill one half2 register: for K a pair is two
+//   adjacent channels of one token, for V the same channel of tokens 2t+8u and
+//   2t+8u+1.  A unit holds 32 pairs; pair index P = 16*x + 2*s + r, where x
+//   selects the token (K: g or g+8) or token pair (V: u).  At b bits pair P
+//   lives in 32-bit word P / (16/b) of the unit at field position
+//   k = P % (16/b): the first member at bits [b*k, b*k+b), the second at
+//   bits [16 + b*k, 16 + b*k + b).  So each 16-bit half-word packs 16/b codes.
+//   Because this order is the same at every width, the shift 2b -> b maps
+//   input words (2J, 2J+1) of a tile to output word J of the same tile, with
+//   no data moving between tiles: a shrink compacts every tile into its first
+//   half in place and token slots keep their indices.
+//
+// Fill pattern of a block (the slot map): before the first shrink tokens
+// fill tile 0, tile 1, ... (P_16 each).  A shrink happens only when every
+// tile is full, so afterwards every tile is exactly half full (h = P_b / 2)
+// and new tokens fill the free halves tile by tile.  At any time the block is
+// therefore: tiles < k full, tile k holding h + r, tiles > k holding h.
+// Attention does not depend on token order, so nothing is ever reordered.
+//
+// Meta: one 32-bit word per (stream, tile, slot) = binary16 R (low half) and
+// binary16 Z (high half), sized for P_F slots per tile (F = the block's Fbit,
+// the widest a tile ever gets).  A shrink never touches it.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace kvq {
+
+constexpr int kHeadDim = 128;
+constexpr int kTileBytes = 16384;
+constexpr int kGroupTokens = 16;
+
+__host__ __device__ constexpr int slots_per_tile(int bits) { return 1024 / bits; }
+__host__ __device__ constexpr int group_bytes(int bits) { return 256 * bits; }
+__host__ __device__ constexpr int unit_bytes(int bits) { return 8 * bits; }
+
+// Fill pattern of one block at its current width (identical for every stream
+// of the block, since all sequences of a batch have the same length).
+struct Fill {
+  int bits;  // current width
+  int nt;    // tiles per stream
+  int pf;    // meta slots per tile (P at Fbit)
+  int p;     // slots per tile at `bits`
+  int h;     // base valid slots of every tile (0 before the first shrink)
+  int e;     // free slots per tile in this epoch (p - h)
+  int k;     // tiles completely full
+  int r;     // extra valid slots in tile k (beyond h)
+  int gpt;   // groups in a full tile
+  int gk;    // groups in tile k (0 if k == nt)
+  int gh;    // groups in a tile holding h
+  long long gps;  // groups per stream
+};
+
+inline Fill make_fill(int bits, int nt, int pf, int n_shrinks, long long n_tokens) {
+  Fill f;
+  f.bits = bits;
+  f.nt = nt;
+  f.pf = pf;
+  f.p = slots_per_tile(bits);
+  f.h = n_shrinks > 0 ? f.p / 2 : 0;
+  f.e = f.p - f.h;
+  long long m = n_tokens - (long long)nt * f.h;
+  f.k = (int)(m / f.e);
+  f.r = (int)(m % f.e);
+  f.gpt = f.p / kGroupTokens;
+  f.gh = f.h / kGroupTokens;
+  if (f.k >= nt) {
+    f.k = nt;
+    f.r = 0;
+    f.gk = 0;
+  } else {
+    f.gk = (f.h + f.r + kGroupTokens - 1) / kGroupTokens;
+  }
+  f.gps = (long long)f.k * f.gpt + (f.k < nt ? (long long)f.gk + (long long)(nt - f.k - 1) * f.gh : 0);
+  return f;
+}
+
+// vgroup index within a stream -> tile, group in tile, valid tokens, groups
+// in that tile.
+struct GroupLoc {
+  int tile, grp, valid, tile_groups;
+};
+
+__host__ __device__ inline GroupLoc locate_group(const Fill& f, long long v) {
+  GroupLoc g;
+  long long full = (long long)f.k * f.gpt;
+  if (v < full) {
+    g.tile = (int)(v / f.gpt);
+    g.grp = (int)(v - (long long)g.tile * f.gpt);
+    g.valid = kGroupTokens;
+    g.tile_groups = f.gpt;
+    return g;
+  }
+  v -= full;
+  if (v < f.gk) {
+    g.tile = f.k;
+    g.grp = (int)v;
+    int rem = f.h + f.r - kGroupTokens * g.grp;
+    g.valid = rem < kGroupTokens ? rem : kGroupTokens;
+    g.tile_groups = f.gk;
+    return g;
+  }
+  v -= f.gk;
+  long long t = v / f.gh;
+  g.tile = f.k + 1 + (int)t;
+  g.grp = (int)(v - t * f.gh);
+  g.valid = kGroupTokens;
+  g.tile_groups = f.gh;
+  return g;
+}
+
+// ---------------------------------------------------------------- launches
+
+struct AppendArgs {
+  const void* k;
+  const void* v;
+  int dtype;          // 0 bf16, 1 f32
+  int n_call;         // tokens in the caller's k/v arrays (batch stride)
+  int tok_off;        // first token of this launch within the call
+  int cnt;            // tokens in this launch (all in one epoch)
+  long long n0;       // logical index of the first token of this launch
+  int bits, h, e, nt, pf;
+  int batch, kv_heads;
+  uint8_t* codes;     // layer base: [batch][kv_heads][2][nt][16 KiB]
+  uint32_t* meta;     // layer base: [batch][kv_heads][2][nt][pf]
+  const float* lam_inv;  // [kv_heads][128] or null
+};
+
+struct ShrinkArgs {
+  uint8_t* codes;     // layer base
+  long long n_tiles;  // batch * kv_heads * 2 * nt
+  int bits_to;        // 8, 4 or 2
+};
+
+struct DecodeArgs {
+  const uint8_t* codes;
+  const uint32_t* meta;
+  const void* q;        // bf16 [batch][q_heads][128]
+  const float* lam;     // [kv_heads][128] or null
+  float* out;           // fp32 [batch][q_heads][128]
+  float* parts;         // workspace partials
+  int* counters;        // [batch*kv_heads] ticket counters (zero between calls)
+  int* err;             // device error flag
+  Fill fill;
+  int batch, kv_heads, q_heads, group;
+  float qscale;         // sm_scale * log2(e)
+  int grid;             // CTAs launched
+};
+
+int decode_grid(int num_sms);
+size_t decode_parts_bytes(int grid, int n_streams, int group);
+
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
+cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+
+}  // namespace kvq

@@ -1,0 +1,171 @@
+"""GPU parity: libkvq (through its C ABI) against the CPU oracle on the same
+seeded inputs.  Codes and meta must be bit-exact; attention output must be
+within a max relative error of 2e-3 per (sequence, query head):
+    max_c |o - o*| / max_c |o*|  <=  2e-3
+(the oracle attends over its own codes, which equal the GPU's)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import kvq_synth as S
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from mixed_precision_kv_kvq_b200 import build
+
+    build.build()
+    import mixed_precision_kv_kvq_b200 as m
+
+    m.load()
+    return m
+
+
+def per_token(batch, kv_heads, fbit):
+    return batch * kv_heads * 2 * sum(16 * f + 4 for f in fbit)
+
+
+class Pair:
+    """A GPU cache and the oracle's model of the same block, fed identically."""
+
+    def __init__(self, kvq, orc, batch, kv_heads, n_f, fbit, lam=None):
+        self.batch, self.kv_heads, self.n_f, self.fbit = batch, kv_heads, n_f, fbit
+        self.gpu = kvq.KVQCache(1, batch, kv_heads, n_f * per_token(batch, kv_heads, [fbit]), [fbit])
+        assert self.gpu.max_tokens == n_f
+        self.orc = orc.Layer(batch, kv_heads, n_f, fbit)
+        self.lam = lam
+        if lam is not None:
+            self.gpu.set_lambda(0, lam)
+
+    def append(self, k, v):
+        """k, v: CPU tensors [batch][n][kv_heads][128] (bf16 or fp32)."""
+        self.gpu.append(0, k.cuda(), v.cuda())
+        rc = self.orc.append(k.float().numpy(), v.float().numpy(), self.lam)
+        assert rc == 0
+
+    def check_codes(self, streams=None):
+        q = self.gpu.query(0)
+        assert q["tokens"] == self.orc.n and q["bits"] == self.orc.bits
+        assert q["n_shrinks"] == self.orc.n_shrinks
+        okc, ovc, okm, ovm = self.orc.k_codes(), self.orc.v_codes(), self.orc.k_meta(), self.orc.v_meta()
+        streams = streams or [(b, j) for b in range(self.batch) for j in range(self.kv_heads)]
+        for b, j in streams:
+            kc, vc, km, vm = self.gpu.export(0, b, j)
+            assert np.array_equal(km, okm[b, j]), (b, j, "k meta")
+            assert np.array_equal(vm, ovm[b, j]), (b, j, "v meta")
+            if not np.array_equal(kc, okc[b, j]):
+                bad = np.argwhere(kc != okc[b, j])
+                raise AssertionError(f"K codes differ at {len(bad)} places, first {bad[:5].tolist()}")
+            if not np.array_equal(vc, ovc[b, j]):
+                bad = np.argwhere(vc != ovc[b, j])
+                raise AssertionError(f"V codes differ at {len(bad)} places, first {bad[:5].tolist()}")
+
+    def check_attention(self, q, sm_scale=None):
+        """q: CPU bf16 [batch][q_heads][128]."""
+        sm_scale = sm_scale if sm_scale is not None else 1 / math.sqrt(128)
+        out = self.gpu.decode_attn(0, q.cuda(), sm_scale).cpu().numpy().astype(np.float64)
+        torch.cuda.synchronize()
+        self.gpu.device_status()
+        ref = self.orc.attention(q.float().numpy(), self.lam, sm_scale)
+        err = np.abs(out - ref).max(axis=-1) / np.abs(ref).max(axis=-1)
+        assert np.isfinite(out).all()
+        assert err.max() <= TOL, f"max rel err {err.max():.3e} at {np.unravel_index(err.argmax(), err.shape)}"
+        return float(err.max())
+
+
+def lam_for(k):
+    from oracle import oracle as orc
+    return orc.lambda_from_keys(k.float()[0].numpy(), 0.5)
+
+
+def test_tiny_config_progressive_one_by_one(kvq, orc):
+    """1 block, batch 1, 2 KV heads, 4 query heads, Fbit 4, 4096 fp32 tokens
+    appended one at a time: 16 bits to 1024, 8 bits to 2048, then 4 bits.
+    Codes/meta bit-exact and attention within tolerance after every shrink."""
+    T = 4096
+    k, v = S.keys_values(0, 0, 1, T, 2, 0, 4, dtype=torch.float32)
+    lam = lam_for(k)
+    P = Pair(kvq, orc, 1, 2, 4096, 4, lam)
+    checkpoints = {1000, 1024, 1025, 1500, 2048, 2049, 3000, 4096}
+    step = 0
+    for t in range(T):
+        P.append(k[:, t:t + 1], v[:, t:t + 1])
+        if t + 1 in checkpoints:
+            P.check_codes()
+            q = S.queries(0, 0, step, 1, 4, t + 1, dtype=torch.bfloat16)
+            P.check_attention(q)
+            step += 1
+    assert P.orc.shrink_at == [1024, 2048]
+    assert kvq.kvq_query(P.gpu.handle, 0) == {"tokens": 4096, "bits": 4, "capacity": 4096, "n_shrinks": 2}
+    for s in range(16):  # 16 decode queries at the end
+        P.check_attention(S.queries(0, 0, 100 + s, 1, 4, T, dtype=torch.bfloat16))
+    with pytest.raises(kvq.KVQError) as e:
+        P.gpu.append(0, k[:, :1].cuda(), v[:, :1].cuda())
+    assert e.value.status == 2
+
+
+@pytest.mark.parametrize("fbit,chunks", [
+    (2, [700, 300, 600, 1000, 1000, 400, 96]),   # crosses 16->8->4->2 inside chunks
+    (8, [1, 15, 16, 17, 2000]),
+    (16, [63, 65, 512, 1]),
+])
+def test_chunked_append_bit_exact(kvq, orc, fbit, chunks):
+    B, H = 2, 3
+    n_f = 4096
+    P = Pair(kvq, orc, B, H, n_f, fbit, None)
+    pos = 0
+    for i, n in enumerate(chunks):
+        if pos + n > n_f:
+            break
+        k, v = S.keys_values(1, i, B, n, H, pos, 3, dtype=torch.bfloat16)
+        P.append(k, v)
+        pos += n
+        P.check_codes(streams=[(0, 0), (1, 2)])
+    P.check_codes()
+
+
+@pytest.mark.parametrize("G", [2, 5, 7, 8])
+@pytest.mark.parametrize("T,fbit", [(1, 2), (17, 2), (300, 4), (1500, 4), (3000, 2), (4096, 2)])
+def test_decode_attention(kvq, orc, G, T, fbit):
+    B, H = 2, 2
+    k, v = S.keys_values(2, T, B, T, H, 0, 3, dtype=torch.bfloat16)
+    lam = lam_for(k)
+    P = Pair(kvq, orc, B, H, 4096, fbit, lam)
+    P.append(k, v)
+    q = S.queries(2, T, 0, B, H * G, T, dtype=torch.bfloat16)
+    P.check_attention(q)
+
+
+def test_forced_shrink_matches_oracle(kvq, orc):
+    B, H = 1, 2
+    P = Pair(kvq, orc, B, H, 4096, 2, None)
+    k, v = S.keys_values(3, 0, B, 512, H, 0, 2, dtype=torch.float32)
+    P.append(k, v)  # 512 = capacity at 16 bits for Fbit 2
+    assert P.gpu.query(0)["capacity"] == 512
+    P.gpu.shrink(0)
+    assert P.orc.shrink() == 0
+    P.check_codes()
+    with pytest.raises(kvq.KVQError) as e:
+        P.gpu.shrink(0)  # not full at 8 bits
+    assert e.value.status == 3
+    P.check_attention(S.queries(3, 0, 0, B, 4, 512))
+
+
+def test_decode_rejects_small_workspace(kvq, orc):
+    P = Pair(kvq, orc, 1, 2, 4096, 4, None)
+    k, v = S.keys_values(4, 0, 1, 10, 2, 0, 1, dtype=torch.float32)
+    P.append(k, v)
+    q = S.queries(4, 0, 0, 1, 4, 10).cuda()
+    out = torch.empty(1, 4, 128, device="cuda")
+    ws = torch.empty(16, device="cuda")
+    with pytest.raises(kvq.KVQError) as e:
+        kvq.kvq_decode_attn(P.gpu.handle, 0, q, 0.1, out, ws)
+    assert e.value.status == 6
