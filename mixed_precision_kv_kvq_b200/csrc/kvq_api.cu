@@ -54,8 +54,9 @@ struct LayerState {
   int nt;  // tiles per stream
   int pf;  // meta slots per tile
   bool counters_zeroed;
-  size_t off_lam, off_lam_inv, off_counters, off_codes, off_meta;
+  size_t off_lam, off_lam_inv, off_perm, off_counters, off_codes, off_meta;
   bool lambda_set;
+  std::vector<uint8_t> perm;  // host copy of the Key channel order [kv_heads][128]
 };
 
 struct Plan {
@@ -99,12 +100,14 @@ bool make_plan(int layers, int batch, int kv_heads, int head_dim, size_t budget,
     off += align_up((size_t)kv_heads * kHeadDim * 4);
     L.off_lam_inv = off;
     off += align_up((size_t)kv_heads * kHeadDim * 4);
+    L.off_perm = off;
+    off += align_up((size_t)kv_heads * kHeadDim);
     L.off_counters = off;
     off += align_up(n_streams * 4);
     L.off_codes = off;
-    off += align_up(n_streams * 2 * (size_t)L.nt * kTileBytes);
+    off += align_up(n_streams * (size_t)L.nt * kTileBytes);
     L.off_meta = off;
-    off += align_up(n_streams * 2 * (size_t)L.nt * L.pf * 4);
+    off += align_up(n_streams * (size_t)L.nt * L.pf * 8);
   }
   p.bytes = off;
   *why = KVQ_OK;
@@ -151,6 +154,7 @@ struct kvq_cache {
   uint32_t* meta(int l) { return reinterpret_cast<uint32_t*>(pool + L[l].off_meta); }
   float* lam(int l) { return reinterpret_cast<float*>(pool + L[l].off_lam); }
   float* lam_inv(int l) { return reinterpret_cast<float*>(pool + L[l].off_lam_inv); }
+  uint8_t* perm(int l) { return pool + L[l].off_perm; }
   int* counters(int l) { return reinterpret_cast<int*>(pool + L[l].off_counters); }
   int* err() { return reinterpret_cast<int*>(pool); }
 };
@@ -251,10 +255,22 @@ kvq_status kvq_set_lambda(kvq_cache* c, int layer, const float* lambda_host) {
     if (!(v > 0.0f) || !std::isfinite(v)) return fail(KVQ_ERR_INVALID, "lambda[%zu] = %g is not finite and > 0", i, (double)v);
     inv[i] = (float)(1.0 / (double)v);
   }
+  if (c->L[layer].n != 0) return fail(KVQ_ERR_STATE, "layer %d already holds tokens; set lambda before the first append", layer);
+  // Key channel order: largest lambda first (ties by channel index).
+  std::vector<uint8_t> perm(n);
+  for (int j = 0; j < c->kv_heads; j++) {
+    std::vector<int> idx(kHeadDim);
+    for (int ch = 0; ch < kHeadDim; ch++) idx[ch] = ch;
+    const float* lj = lambda_host + (size_t)j * kHeadDim;
+    std::stable_sort(idx.begin(), idx.end(), [lj](int x, int y) { return lj[x] > lj[y]; });
+    for (int pos = 0; pos < kHeadDim; pos++) perm[(size_t)j * kHeadDim + pos] = (uint8_t)idx[pos];
+  }
   cudaError_t e = cudaMemcpy(c->lam(layer), lambda_host, n * 4, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(c->lam_inv(layer), inv.data(), n * 4, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(c->perm(layer), perm.data(), n, cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return cuda_fail(e, "lambda upload");
   c->L[layer].lambda_set = true;
+  c->L[layer].perm = perm;
   return KVQ_OK;
 }
 
@@ -277,7 +293,7 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* k, const void* v, int
   while (off < n_tokens) {
     const long long cap = capacity(L, c->n_f, L.bits);
     if (L.n == cap) {  // full: shrink one level first (bits > fbit is implied by the budget check)
-      ShrinkArgs sa{c->codes(layer), (long long)c->batch * c->kv_heads * 2 * L.nt, L.bits / 2};
+      ShrinkArgs sa{c->codes(layer), (long long)c->batch * c->kv_heads * L.nt, L.bits / 2};
       cudaError_t e = launch_shrink(sa, s);
       if (e != cudaSuccess) return cuda_fail(e, "shrink launch");
       L.bits /= 2;
@@ -304,6 +320,7 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* k, const void* v, int
     a.codes = c->codes(layer);
     a.meta = c->meta(layer);
     a.lam_inv = L.lambda_set ? c->lam_inv(layer) : nullptr;
+    a.perm = L.lambda_set ? c->perm(layer) : nullptr;
     cudaError_t e = launch_append(a, s);
     if (e != cudaSuccess) return cuda_fail(e, "append launch");
     L.n += cnt;
@@ -320,7 +337,7 @@ kvq_status kvq_shrink(kvq_cache* c, int layer, kvq_stream_t stream) {
   if (L.n != cap)
     return fail(KVQ_ERR_STATE, "layer %d holds %lld tokens; a shrink needs the block full (%lld at %d bits)", layer, L.n, cap,
                 L.bits);
-  ShrinkArgs sa{c->codes(layer), (long long)c->batch * c->kv_heads * 2 * L.nt, L.bits / 2};
+  ShrinkArgs sa{c->codes(layer), (long long)c->batch * c->kv_heads * L.nt, L.bits / 2};
   cudaError_t e = launch_shrink(sa, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "shrink launch");
   L.bits /= 2;
@@ -332,8 +349,7 @@ size_t kvq_decode_workspace(const kvq_cache* c, int layer, int q_heads) {
   if (!c || layer < 0 || layer >= c->layers || q_heads <= 0 || q_heads % c->kv_heads) return 0;
   const int G = q_heads / c->kv_heads;
   if (G > 8) return 0;
-  kvq_cache* m = const_cast<kvq_cache*>(c);
-  return decode_parts_bytes(decode_grid(m->sms()), c->batch * c->kv_heads, G);
+  return decode_parts_bytes(c->batch * c->kv_heads, G);
 }
 
 kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, float sm_scale, float* out,
@@ -350,8 +366,7 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, 
   LayerState& L = c->L[layer];
   if (L.n <= 0) return fail(KVQ_ERR_STATE, "layer %d is empty", layer);
   const int n_streams = c->batch * c->kv_heads;
-  const int max_grid = decode_grid(c->sms());
-  const size_t need = decode_parts_bytes(max_grid, n_streams, G);
+  const size_t need = decode_parts_bytes(n_streams, G);
   if (!workspace || ws_bytes < need)
     return fail(KVQ_ERR_WORKSPACE, "workspace of %zu bytes; %zu needed", workspace ? ws_bytes : (size_t)0, need);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -366,6 +381,7 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, 
   a.meta = c->meta(layer);
   a.q = q;
   a.lam = L.lambda_set ? c->lam(layer) : nullptr;
+  a.perm = L.lambda_set ? c->perm(layer) : nullptr;
   a.out = out;
   a.parts = static_cast<float*>(workspace);
   a.counters = c->counters(layer);
@@ -376,8 +392,7 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, 
   a.q_heads = q_heads;
   a.group = G;
   a.qscale = sm_scale * 1.4426950408889634f;
-  const long long tot = (long long)n_streams * a.fill.gps;
-  a.grid = (int)std::min<long long>(max_grid, tot);
+  a.splits = decode_splits(c->sms(), n_streams, a.fill.gps);
   cudaError_t e = launch_decode(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return KVQ_OK;
@@ -402,15 +417,13 @@ kvq_status kvq_export(const kvq_cache* c, int layer, int b, int j, uint16_t* k_c
     return fail(KVQ_ERR_INVALID, "stream (%d, %d) out of range", b, j);
   const LayerState& L = c->L[layer];
   kvq_cache* m = const_cast<kvq_cache*>(c);
-  const size_t code_bytes = (size_t)L.nt * kTileBytes, meta_words = (size_t)L.nt * L.pf;
-  const size_t sk = ((size_t)b * c->kv_heads + j) * 2, sv = sk + 1;
-  std::vector<uint8_t> kc(code_bytes), vc(code_bytes);
-  std::vector<uint32_t> km(meta_words), vm(meta_words);
+  const size_t code_bytes = (size_t)L.nt * kTileBytes, meta_words = (size_t)L.nt * L.pf * 2;
+  const size_t st = (size_t)b * c->kv_heads + j;
+  std::vector<uint8_t> cb(code_bytes);
+  std::vector<uint32_t> mw(meta_words);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemcpyAsync(kc.data(), m->codes(layer) + sk * code_bytes, code_bytes, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(vc.data(), m->codes(layer) + sv * code_bytes, code_bytes, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(km.data(), m->meta(layer) + sk * meta_words, meta_words * 4, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(vm.data(), m->meta(layer) + sv * meta_words, meta_words * 4, cudaMemcpyDeviceToHost, s);
+  cudaError_t e = cudaMemcpyAsync(cb.data(), m->codes(layer) + st * code_bytes, code_bytes, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(mw.data(), m->meta(layer) + st * meta_words, meta_words * 4, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "export copy");
   const int bits = L.bits, ppw = 16 / bits;
@@ -422,11 +435,12 @@ kvq_status kvq_export(const kvq_cache* c, int layer, int b, int j, uint16_t* k_c
     const size_t gbase = (size_t)tile * kTileBytes + (size_t)grp * group_bytes(bits);
     if (k_codes) {
       const int g = tok & 7, x = tok >> 3;
-      for (int ch = 0; ch < kHeadDim; ch++) {
-        const int sb = ch >> 4, rem = ch & 15, r = rem >> 3, t = (rem & 7) >> 1, mb = rem & 1;
+      const uint8_t* pm = L.lambda_set ? &L.perm[(size_t)j * kHeadDim] : nullptr;
+      for (int kp = 0; kp < kHeadDim; kp++) {  // Key position -> channel pm[kp]
+        const int sb = kp >> 4, rem = kp & 15, r = rem >> 3, t = (rem & 7) >> 1, mb = rem & 1;
         const int p = 2 * sb + r, word = x * bits + p / ppw, pos = p % ppw;
-        const uint32_t w = rd32(&kc[gbase + (size_t)(4 * g + t) * unit_bytes(bits) + 4 * word]);
-        k_codes[i * kHeadDim + ch] = (uint16_t)((w >> (16 * mb + bits * pos)) & mask);
+        const uint32_t w = rd32(&cb[gbase + (size_t)(4 * g + t) * unit_bytes(bits) + 4 * word]);
+        k_codes[i * kHeadDim + (pm ? pm[kp] : kp)] = (uint16_t)((w >> (16 * mb + bits * pos)) & mask);
       }
     }
     if (v_codes) {
@@ -434,18 +448,18 @@ kvq_status kvq_export(const kvq_cache* c, int layer, int b, int j, uint16_t* k_c
       for (int ch = 0; ch < kHeadDim; ch++) {
         const int sb = ch >> 4, rem = ch & 15, r = rem >> 3, g = rem & 7;
         const int p = 2 * sb + r, word = u * bits + p / ppw, pos = p % ppw;
-        const uint32_t w = rd32(&vc[gbase + (size_t)(4 * g + t) * unit_bytes(bits) + 4 * word]);
+        const uint32_t w = rd32(&cb[gbase + part_bytes(bits) + (size_t)(4 * g + t) * unit_bytes(bits) + 4 * word]);
         v_codes[i * kHeadDim + ch] = (uint16_t)((w >> (16 * mb + bits * pos)) & mask);
       }
     }
-    const size_t mi = (size_t)tile * L.pf + slot;
+    const size_t mi = ((size_t)tile * L.pf + slot) * 2;
     if (k_meta) {
-      k_meta[2 * i] = (uint16_t)(km[mi] & 0xffffu);
-      k_meta[2 * i + 1] = (uint16_t)(km[mi] >> 16);
+      k_meta[2 * i] = (uint16_t)(mw[mi] & 0xffffu);
+      k_meta[2 * i + 1] = (uint16_t)(mw[mi] >> 16);
     }
     if (v_meta) {
-      v_meta[2 * i] = (uint16_t)(vm[mi] & 0xffffu);
-      v_meta[2 * i + 1] = (uint16_t)(vm[mi] >> 16);
+      v_meta[2 * i] = (uint16_t)(mw[mi + 1] & 0xffffu);
+      v_meta[2 * i + 1] = (uint16_t)(mw[mi + 1] >> 16);
     }
   }
   return KVQ_OK;

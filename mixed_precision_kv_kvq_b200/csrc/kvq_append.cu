@@ -9,8 +9,9 @@
 //   x_c = k_c * lambda_inv_c            (K only)
 //   Z   = binary16 round-down(min x)    R = binary16 round-up(max x - Z)
 //   q_c = clamp(floor((x_c - Z) * ((2^b - 1) / R) + 1/2), 0, 2^b - 1)
-// (R = 0: all codes 0), then scatters the codes into the group's lane units
-// (see kvq_internal.cuh) and writes (R, Z) to the slot's meta word.
+// (R = 0: all codes 0), then scatters the codes into the lane units of the
+// group's K or V part (see kvq_internal.cuh) and writes (R, Z) to the slot's
+// K or V meta word.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -102,22 +103,26 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs 
   const int slot = a.h + (int)(m - (long long)tile * a.e);
   const int grp = slot >> 4;
   const int tok = slot & 15;
-  const size_t stream_kv = ((size_t)b * a.kv_heads + j) * 2 + kv;
-  uint8_t* gbase = a.codes + (stream_kv * a.nt + tile) * (size_t)kTileBytes + (size_t)grp * group_bytes(bits);
+  const size_t stream = (size_t)b * a.kv_heads + j;
+  uint8_t* gbase = a.codes + (stream * a.nt + tile) * (size_t)kTileBytes + (size_t)grp * group_bytes(bits) +
+                   (size_t)kv * part_bytes(bits);
   const int ppw = 16 / bits;  // pairs per 32-bit word (per 16-bit half)
 
   if (kv == 0) {
     // Token tok: g = tok % 8, x = tok / 8.  Lane units 4g + t (t = 0..3) each
     // get `bits` words: unit word x*bits + jw holds pairs P = 16x + jw*ppw + kk.
+    // Positions map to channels through the block's Key channel order.
+    const uint8_t* pm = a.perm ? a.perm + (size_t)j * kHeadDim : nullptr;
     const int g = tok & 7, xs = tok >> 3;
     for (int wi = lane; wi < 4 * bits; wi += 32) {
       const int t = wi / bits, jw = wi - t * bits;
       uint32_t word = 0;
       for (int kk = 0; kk < ppw; kk++) {
         const int p = jw * ppw + kk;  // pair within the token's half: p = 2s + rr
-        const int ch0 = 16 * (p >> 1) + 2 * t + 8 * (p & 1);
-        word |= (uint32_t)sc[ch0] << (bits * kk);
-        word |= (uint32_t)sc[ch0 + 1] << (16 + bits * kk);
+        const int pos0 = 16 * (p >> 1) + 2 * t + 8 * (p & 1);
+        const int c0 = pm ? pm[pos0] : pos0, c1 = pm ? pm[pos0 + 1] : pos0 + 1;
+        word |= (uint32_t)sc[c0] << (bits * kk);
+        word |= (uint32_t)sc[c1] << (16 + bits * kk);
       }
       uint32_t* dst = reinterpret_cast<uint32_t*>(gbase + (4 * g + t) * unit_bytes(bits)) + xs * bits + jw;
       *dst = word;
@@ -142,7 +147,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs 
   }
   if (lane == 0) {
     const uint32_t mw = (uint32_t)__half_as_ushort(rh) | ((uint32_t)__half_as_ushort(zh) << 16);
-    a.meta[(stream_kv * a.nt + tile) * (size_t)a.pf + slot] = mw;
+    a.meta[((stream * a.nt + tile) * (size_t)a.pf + slot) * 2 + kv] = mw;
   }
 }
 

@@ -14,23 +14,23 @@
 // channels of codes and B = q' (N = 8 query heads; q' is carried as a hi + lo
 // pair of fp16 values, two MMAs on the same A registers, because one fp16
 // rounding of q' alone moves large outlier-channel scores by up to ~2^-12 of
-// their size, enough to break a 2e-3 output tolerance), PV with A = 16 channels x
-// 16 tokens of V codes and B = p R (transposed from the score fragment with
-// movmatrix).  Codes are widened to fp16 in registers with the 0x6400 exponent
-// trick (integer c in the low mantissa bits of 1024.0; one lop3 + one hfma2
-// per code pair).
+// their size, enough to break a 2e-3 output tolerance), PV with A = 16
+// channels x 16 tokens of V codes and B = p R (transposed from the score
+// fragment with movmatrix).  Codes are widened to fp16 in registers with the
+// 0x6400 exponent trick (integer c in the low mantissa bits of 1024.0; one
+// lop3 + one hfma2 per code pair).
 //
-// Work split: the groups (16 tokens) of all streams of the block form one
-// list; CTA c takes the contiguous slice [c*tot/grid, (c+1)*tot/grid).  One
-// producer warp streams the slice's codes and meta into a ring of shared-
-// memory stages with cp.async.bulk (TMA bulk copies) on mbarriers; eight
-// consumer warps take alternate groups of each stage and keep their own
-// online-softmax state, merged through shared memory when a stream segment
-// ends.  A stream split over several CTAs leaves one partial (max, sum,
-// unnormalised output) per CTA in the workspace; the last CTA to finish the
-// stream (atomic ticket, no waiting) merges them with log-sum-exp weights.
-// Every wait on an mbarrier is bounded in time; a kernel that gives up sets
-// the cache's error flag and carries on without hanging.
+// Work split: each stream is cut into `splits` equal slices of 16-token
+// groups, one CTA per slice (the host picks `splits` so the grid fills the
+// GPU in whole waves).  The CTA's four warps take contiguous quarters of the
+// slice; each warp streams its quarter through its own ring of shared-memory
+// stages filled by cp.async.bulk (TMA bulk copies) on mbarriers, a few KiB
+// ahead of its math, and keeps its own online-softmax state.  The warps merge
+// in shared memory; a stream cut into several slices leaves one partial
+// (max, sum, unnormalised output) per CTA in the workspace, and the last CTA
+// to finish the stream (atomic ticket, no waiting) merges them with
+// log-sum-exp weights.  Every mbarrier wait is bounded in time; a kernel that
+// gives up sets the cache's error flag and returns normally.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -39,17 +39,17 @@
 namespace kvq {
 namespace {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kStages = 4;
-constexpr int kChunkBytes = 8192;                 // K (and V) code bytes per stage
-constexpr int kMaxChunkGroups = kChunkBytes / 512; // 16 groups at 2 bits
-constexpr int kMetaBytes = kMaxChunkGroups * 64;  // 16 tokens * 4 B per group
-constexpr int kStageBytes = 2 * kChunkBytes + 2 * kMetaBytes;
-constexpr int kMaxGroup = 8;                      // query heads per KV head (MMA N)
-constexpr int kSmemBytes = kStages * kStageBytes + kMaxGroup * kHeadDim * 4 +
-                           3 * kConsumerWarps * kMaxGroup * 4 + 2 * kStages * 8 + 16;
-constexpr int kCtasPerSm = 2;
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr int kStages = 2;                 // per warp
+constexpr int kStageCode = 4096;           // code bytes per stage (K and V parts of whole groups)
+constexpr int kStageMeta = 512;            // meta bytes per stage (128 per group)
+constexpr int kWarpSmem = kStages * (kStageCode + kStageMeta);
+constexpr int kMaxGroup = 8;               // query heads per KV head (MMA N)
+constexpr int kCtasPerSm = 4;
+constexpr int kQfBytes = 8 * 32 * 16;      // q' B fragments: [s-block][lane] x (hi b0, hi b1, lo b0, lo b1)
+constexpr int kSmemBytes = kWarps * kWarpSmem + kQfBytes + kMaxGroup * 4 + 3 * kWarps * kMaxGroup * 4 +
+                           kWarps * kStages * 8 + kWarps * kStages * 8 + 16;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
 
 // ------------------------------------------------------------------ PTX
@@ -69,9 +69,6 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -84,12 +81,11 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 }
 // Bounded wait: true when the phase completed, false after kWaitNs (the
 // error flag is then set and *abort raised so later waits give up at once).
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err, volatile int* abort) {
-  if (mbar_try(bar, parity)) return true;
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, int* err, volatile int* abort) {
   const unsigned long long t0 = global_ns();
   for (unsigned it = 0;; it++) {
     if (mbar_try(bar, parity)) return true;
-    if ((it & 63) == 63) {
+    if ((it & 15) == 15) {
       if (*abort || global_ns() - t0 > kWaitNs) {
         *abort = 1;
         atomicExch(err, 1);
@@ -98,14 +94,15 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err, 
     }
   }
 }
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err, volatile int* abort) {
+  if (mbar_try(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, err, abort);
+}
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
-}
-__device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
 __device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
   uint32_t d;
@@ -141,22 +138,41 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 }
 
 // --------------------------------------------------------- code widening
-// Pair at field position POS of a word packed at BITS (BITS <= 8): the two
-// codes sit at bits [BITS*POS, +BITS) of each half-word.  Result: half2 of the
-// two codes as exact fp16 values.
+// Bit offset, within its byte, of the codes at field position POS of a word
+// packed at BITS (BITS <= 8); positions past the first byte are read from
+// the word shifted right by 8.
+template <int BITS, int POS>
+__host__ __device__ constexpr int field_shift() {
+  return BITS * ((POS % (16 / BITS)) % (8 / BITS));
+}
+// Pair at field position POS: the two codes sit at bits [BITS*POS, +BITS) of
+// each half-word.  Result: half2 (c0 * 2^e, c1 * 2^e), exact, with
+// e = field_shift: (0x6400 | c << e) is the fp16 number 1024 + c 2^e, and
+// subtracting 1024 is exact.  The 2^e is undone outside the inner loop (in
+// the q' operand for Keys, in the output rows for Values).
 template <int BITS, int POS>
 __device__ __forceinline__ uint32_t widen(uint32_t w, uint32_t w8) {
   constexpr int kPerByte = 8 / BITS;
-  constexpr int kp = POS % kPerByte;
+  constexpr int e = field_shift<BITS, POS>();
   constexpr uint32_t m = (1u << BITS) - 1u;
-  constexpr uint32_t mask = (m << (BITS * kp)) | (m << (16 + BITS * kp));
-  const uint32_t x = lop_and_or(POS >= kPerByte ? w8 : w, mask, 0x64006400u);  // 1024 + c*2^e
-  constexpr int e = BITS * kp;
-  constexpr uint32_t sc = (uint32_t)(15 - e) << 10;               // 2^-e
-  constexpr uint32_t bi = 0x8000u | ((uint32_t)(25 - e) << 10);   // -1024 * 2^-e
-  return hfma2_u(x, sc | (sc << 16), bi | (bi << 16));
+  constexpr uint32_t mask = (m << e) | (m << (16 + e));
+  const uint32_t x = lop_and_or((POS % (16 / BITS)) >= kPerByte ? w8 : w, mask, 0x64006400u);
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(x), "r"(0x64006400u));
+  return d;
 }
-// 16-bit codes: whole word is the pair; split each code into high and low byte.
+// Largest field shift at BITS: q' is scaled by 2^(kEmax - e) per channel so
+// every product c 2^e q' 2^(kEmax - e) carries the same factor 2^kEmax.
+template <int BITS>
+__host__ __device__ constexpr int emax() {
+  return BITS >= 8 ? 0 : 8 - BITS;
+}
+// field_shift of pair p (any p in 0..15) at BITS <= 8.
+template <int BITS>
+__host__ __device__ constexpr int pair_shift(int p) {
+  return BITS >= 16 ? 0 : BITS * ((p % (16 / BITS)) % (8 / BITS));
+}
+// 16-bit codes: the whole word is the pair; split each code into high and low byte.
 __device__ __forceinline__ uint32_t widen16_hi(uint32_t w) {
   return hfma2_u(lop_and_or(w >> 8, 0x00ff00ffu, 0x64006400u), 0x3c003c00u, 0xe400e400u);
 }
@@ -164,417 +180,559 @@ __device__ __forceinline__ uint32_t widen16_lo(uint32_t w) {
   return hfma2_u(lop_and_or(w, 0x00ff00ffu, 0x64006400u), 0x3c003c00u, 0xe400e400u);
 }
 
-// Word of a lane unit holding pair p (0..15) of half x at BITS, and its
-// position.
-template <int BITS>
-struct PairAddr {
-  static constexpr int ppw = 16 / BITS;
-  __device__ static constexpr int word(int x, int p) { return x * BITS + p / ppw; }
-  __device__ static constexpr int pos(int p) { return p % ppw; }
-};
-
-// A-fragment registers for MMA block s (channels or tokens 16s..16s+15).
-// K: a0a1 = (x=0, p=2s), a2a3 = (x=1, p=2s), a4a5 = (x=0, p=2s+1), a6a7 = (x=1, p=2s+1)
-// V: a0a1 = (x=0, p=2s), a2a3 = (x=0, p=2s+1), a4a5 = (x=1, p=2s), a6a7 = (x=1, p=2s+1)
-template <int BITS, int S>
-__device__ __forceinline__ uint32_t pair_at(const uint32_t* u, const uint32_t* u8, int x, int r) {
-  const int p = 2 * S + r;
-  const int wi = x * BITS + p / PairAddr<BITS>::ppw;
-  // POS must be a compile-time constant: expand over r.
-  if (r == 0) return widen<BITS, (2 * S) % (16 / BITS)>(u[wi], u8[wi]);
-  return widen<BITS, (2 * S + 1) % (16 / BITS)>(u[wi], u8[wi]);
+// Pair p = 2S + r of half x of a lane unit at BITS (<= 8), widened.
+template <int BITS, int S, int X, int R>
+__device__ __forceinline__ uint32_t pair_at(const uint32_t* u, const uint32_t* u8) {
+  constexpr int ppw = 16 / BITS;
+  constexpr int p = 2 * S + R;
+  constexpr int wi = X * BITS + p / ppw;
+  return widen<BITS, p % ppw>(u[wi], u8[wi]);
 }
 
-// ------------------------------------------------------------ work list
+// -------------------------------------------------------- group pieces
 
-struct Chunk {
-  int s;          // stream (b * kv_heads + j)
-  int tile, grp0, ng, tile_valid;
-};
-
-struct ChunkIter {
-  long long gidx, gend;
-  __device__ bool next(const Fill& f, int max_groups, Chunk& c) {
-    if (gidx >= gend) return false;
-    const long long s = gidx / f.gps;
-    const long long v = gidx - s * f.gps;
-    const GroupLoc loc = locate_group(f, v);
-    long long ng = loc.tile_groups - loc.grp;
-    if (ng > max_groups) ng = max_groups;
-    if (ng > gend - gidx) ng = gend - gidx;
-    c.s = (int)s;
-    c.tile = loc.tile;
-    c.grp0 = loc.grp;
-    c.ng = (int)ng;
-    c.tile_valid = loc.tile < f.k ? f.p : (loc.tile == f.k ? f.h + f.r : f.h);
-    gidx += ng;
-    return true;
+// Scores of NG 16-token groups: D[n][token][head] = sum over Key positions of
+// code * q' (all products carry 2^emax for BITS <= 8, 1/256 of the code for
+// BITS == 16).  The lo part of q' is added on the first LO k-blocks.  The
+// k-block loop is outermost so each q' fragment is loaded once for all
+// groups.
+template <int BITS, int LO, int NG>
+__device__ __forceinline__ void qk_groups(const uint32_t* const (&ku)[NG], const uint4* qfl, float (&d)[NG][4]) {
+  float dl[NG][4];
+#pragma unroll
+  for (int n = 0; n < NG; n++) d[n][0] = d[n][1] = d[n][2] = d[n][3] = dl[n][0] = dl[n][1] = dl[n][2] = dl[n][3] = 0.f;
+  if constexpr (BITS == 16) {
+#pragma unroll
+    for (int sb = 0; sb < 8; sb++) {
+      const uint4 q4 = qfl[32 * sb];
+      const uint32_t bl0 = hfma2_u(q4.x, 0x1c001c00u, 0u), bl1 = hfma2_u(q4.y, 0x1c001c00u, 0u);  // / 256
+#pragma unroll
+      for (int n = 0; n < NG; n++) {
+        const uint2 w0 = *reinterpret_cast<const uint2*>(ku[n] + 2 * sb);       // token g: pairs 2s, 2s+1
+        const uint2 w1 = *reinterpret_cast<const uint2*>(ku[n] + 16 + 2 * sb);  // token g+8
+        const uint32_t h0 = widen16_hi(w0.x), h1 = widen16_hi(w1.x), h2 = widen16_hi(w0.y), h3 = widen16_hi(w1.y);
+        mma(d[n], h0, h1, h2, h3, q4.x, q4.y);
+        if (sb < LO) mma(dl[n], h0, h1, h2, h3, q4.z, q4.w);
+        mma(dl[n], widen16_lo(w0.x), widen16_lo(w1.x), widen16_lo(w0.y), widen16_lo(w1.y), bl0, bl1);
+      }
+    }
+  } else {
+    uint32_t u[NG][2 * BITS], u8[NG][2 * BITS];
+#pragma unroll
+    for (int n = 0; n < NG; n++) {
+#pragma unroll
+      for (int i = 0; i < 2 * BITS; i += 4) {
+        const uint4 q4 = *reinterpret_cast<const uint4*>(ku[n] + i);
+        u[n][i] = q4.x; u[n][i + 1] = q4.y; u[n][i + 2] = q4.z; u[n][i + 3] = q4.w;
+      }
+#pragma unroll
+      for (int i = 0; i < 2 * BITS; i++) u8[n][i] = u[n][i] >> 8;
+    }
+#define KVQ_QK(S)                                                                                          \
+  {                                                                                                        \
+    const uint4 q4 = qfl[32 * S];                                                                          \
+    _Pragma("unroll") for (int n = 0; n < NG; n++) {                                                      \
+      const uint32_t a0 = pair_at<BITS, S, 0, 0>(u[n], u8[n]), a1 = pair_at<BITS, S, 1, 0>(u[n], u8[n]);   \
+      const uint32_t a2 = pair_at<BITS, S, 0, 1>(u[n], u8[n]), a3 = pair_at<BITS, S, 1, 1>(u[n], u8[n]);   \
+      mma(d[n], a0, a1, a2, a3, q4.x, q4.y);                                                               \
+      if constexpr (S < LO) mma(dl[n], a0, a1, a2, a3, q4.z, q4.w);                                        \
+    }                                                                                                      \
   }
+    KVQ_QK(0) KVQ_QK(1) KVQ_QK(2) KVQ_QK(3) KVQ_QK(4) KVQ_QK(5) KVQ_QK(6) KVQ_QK(7)
+#undef KVQ_QK
+  }
+#pragma unroll
+  for (int n = 0; n < NG; n++) {
+    d[n][0] += dl[n][0]; d[n][1] += dl[n][1]; d[n][2] += dl[n][2]; d[n][3] += dl[n][3];
+  }
+}
+
+// o[channel rows][heads] += V^T codes x P for NG groups (B fragments b0[n]:
+// tokens 2t, 2t+1, b1[n]: tokens 2t+8, 2t+9 of head g).
+template <int BITS, int NG>
+__device__ __forceinline__ void pv_groups(const uint32_t* const (&vu)[NG], const uint32_t (&b0)[NG],
+                                          const uint32_t (&b1)[NG], float (&o)[8][4]) {
+  if constexpr (BITS == 16) {
+    uint32_t b0l[NG], b1l[NG];
+#pragma unroll
+    for (int n = 0; n < NG; n++) {
+      b0l[n] = hfma2_u(b0[n], 0x1c001c00u, 0u);  // / 256
+      b1l[n] = hfma2_u(b1[n], 0x1c001c00u, 0u);
+    }
+#pragma unroll
+    for (int sb = 0; sb < 8; sb++) {
+#pragma unroll
+      for (int n = 0; n < NG; n++) {
+        const uint2 w0 = *reinterpret_cast<const uint2*>(vu[n] + 2 * sb);       // u = 0
+        const uint2 w1 = *reinterpret_cast<const uint2*>(vu[n] + 16 + 2 * sb);  // u = 1
+        mma(o[sb], widen16_hi(w0.x), widen16_hi(w0.y), widen16_hi(w1.x), widen16_hi(w1.y), b0[n], b1[n]);
+        mma(o[sb], widen16_lo(w0.x), widen16_lo(w0.y), widen16_lo(w1.x), widen16_lo(w1.y), b0l[n], b1l[n]);
+      }
+    }
+  } else {
+    uint32_t u[NG][2 * BITS], u8[NG][2 * BITS];
+#pragma unroll
+    for (int n = 0; n < NG; n++) {
+#pragma unroll
+      for (int i = 0; i < 2 * BITS; i += 4) {
+        const uint4 q4 = *reinterpret_cast<const uint4*>(vu[n] + i);
+        u[n][i] = q4.x; u[n][i + 1] = q4.y; u[n][i + 2] = q4.z; u[n][i + 3] = q4.w;
+      }
+#pragma unroll
+      for (int i = 0; i < 2 * BITS; i++) u8[n][i] = u[n][i] >> 8;
+    }
+#define KVQ_PV(S)                                                                                      \
+  _Pragma("unroll") for (int n = 0; n < NG; n++) {                                                    \
+    mma(o[S], pair_at<BITS, S, 0, 0>(u[n], u8[n]), pair_at<BITS, S, 0, 1>(u[n], u8[n]),               \
+        pair_at<BITS, S, 1, 0>(u[n], u8[n]), pair_at<BITS, S, 1, 1>(u[n], u8[n]), b0[n], b1[n]);         \
+  }
+    KVQ_PV(0) KVQ_PV(1) KVQ_PV(2) KVQ_PV(3) KVQ_PV(4) KVQ_PV(5) KVQ_PV(6) KVQ_PV(7)
+#undef KVQ_PV
+  }
+}
+
+// Online-softmax state of one warp for the heads 2t, 2t+1 of its lanes.
+struct Soft {
+  float m0, m1, l0, l1, pz0, pz1;
+  float o[8][4];
 };
 
-__device__ __forceinline__ long long cta_of(long long x, long long tot, int grid) {
-  return ((x + 1) * grid - 1) / tot;
+// NG consecutive groups of one stage: scores, one shared running-max update,
+// probabilities, then P V.  valid0: valid tokens from the first group on.
+template <int BITS, int LO, int NG>
+__device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* ms, int gi, int valid0, int lane,
+                                               const uint4* qfl, float sig0, float sig1, float kscale, Soft& st) {
+  constexpr int kGroupBytes = 512 * BITS, kPart = 256 * BITS;
+  const int g = lane >> 2;
+  const uint32_t* ku[NG];
+  const uint32_t* vu[NG];
+#pragma unroll
+  for (int n = 0; n < NG; n++) {
+    ku[n] = reinterpret_cast<const uint32_t*>(cs + (gi + n) * kGroupBytes + lane * unit_bytes(BITS));
+    vu[n] = reinterpret_cast<const uint32_t*>(cs + (gi + n) * kGroupBytes + kPart + lane * unit_bytes(BITS));
+  }
+  float d[NG][4];
+  qk_groups<BITS, LO, NG>(ku, qfl, d);
+  float s[NG][4], rv[NG][2], zv[NG][2];
+  bool partial = false;
+#pragma unroll
+  for (int n = 0; n < NG; n++) {
+    const uint2 mga = ms[(gi + n) * 16 + g], mgb = ms[(gi + n) * 16 + g + 8];
+    const float2 ka = __half22float2(*reinterpret_cast<const __half2*>(&mga.x));
+    const float2 kb = __half22float2(*reinterpret_cast<const __half2*>(&mgb.x));
+    const float2 va = __half22float2(*reinterpret_cast<const __half2*>(&mga.y));
+    const float2 vb = __half22float2(*reinterpret_cast<const __half2*>(&mgb.y));
+    const float rka = ka.x * kscale, rkb = kb.x * kscale;
+    s[n][0] = fmaf(rka, d[n][0], ka.y * sig0);  // token g,   head 2t
+    s[n][1] = fmaf(rka, d[n][1], ka.y * sig1);  // token g,   head 2t+1
+    s[n][2] = fmaf(rkb, d[n][2], kb.y * sig0);  // token g+8, head 2t
+    s[n][3] = fmaf(rkb, d[n][3], kb.y * sig1);  // token g+8, head 2t+1
+    rv[n][0] = va.x; zv[n][0] = va.y;
+    rv[n][1] = vb.x; zv[n][1] = vb.y;
+    partial |= valid0 - 16 * n < 16;
+  }
+  if (partial) {  // warp-uniform: only the last group of a stream's partial tile
+#pragma unroll
+    for (int n = 0; n < NG; n++) {
+      const int valid = valid0 - 16 * n;
+      if (g >= valid) {
+        s[n][0] = s[n][1] = -INFINITY;
+        rv[n][0] = zv[n][0] = 0.f;
+      }
+      if (g + 8 >= valid) {
+        s[n][2] = s[n][3] = -INFINITY;
+        rv[n][1] = zv[n][1] = 0.f;
+      }
+    }
+  }
+  float mx0 = fmaxf(s[0][0], s[0][2]), mx1 = fmaxf(s[0][1], s[0][3]);
+#pragma unroll
+  for (int n = 1; n < NG; n++) {
+    mx0 = fmaxf(mx0, fmaxf(s[n][0], s[n][2]));
+    mx1 = fmaxf(mx1, fmaxf(s[n][1], s[n][3]));
+  }
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+  }
+  const float n0 = fmaxf(st.m0, mx0), n1 = fmaxf(st.m1, mx1);
+  if (__any_sync(0xffffffffu, (n0 > st.m0) | (n1 > st.m1))) {
+    const float a0 = ex2(st.m0 - n0), a1 = ex2(st.m1 - n1);
+#pragma unroll
+    for (int sb = 0; sb < 8; sb++) {
+      st.o[sb][0] *= a0; st.o[sb][2] *= a0;
+      st.o[sb][1] *= a1; st.o[sb][3] *= a1;
+    }
+    st.l0 *= a0; st.pz0 *= a0;
+    st.l1 *= a1; st.pz1 *= a1;
+    st.m0 = n0;
+    st.m1 = n1;
+  }
+  uint32_t b0[NG], b1[NG];
+#pragma unroll
+  for (int n = 0; n < NG; n++) {
+    const float p00 = ex2(s[n][0] - st.m0), p01 = ex2(s[n][1] - st.m1);
+    const float p10 = ex2(s[n][2] - st.m0), p11 = ex2(s[n][3] - st.m1);
+    st.l0 += p00 + p10;
+    st.l1 += p01 + p11;
+    st.pz0 = fmaf(p00, zv[n][0], fmaf(p10, zv[n][1], st.pz0));
+    st.pz1 = fmaf(p01, zv[n][0], fmaf(p11, zv[n][1], st.pz1));
+    b0[n] = movmatrix_t(pack_h2(p00 * rv[n][0], p01 * rv[n][0]));  // tokens 2t, 2t+1 of head g
+    b1[n] = movmatrix_t(pack_h2(p10 * rv[n][1], p11 * rv[n][1]));  // tokens 2t+8, 2t+9
+  }
+  pv_groups<BITS, NG>(vu, b0, b1, st.o);
 }
 
 // ------------------------------------------------------------------ kernel
 
-template <int BITS>
-__global__ void __maxnreg__(112) decode_kernel(const DecodeArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  float* o_acc = reinterpret_cast<float*>(smem + kStages * kStageBytes);  // [8][128]
-  float* w_m = o_acc + kMaxGroup * kHeadDim;                               // [warps][8]
-  float* w_l = w_m + kConsumerWarps * kMaxGroup;
-  float* w_pz = w_l + kConsumerWarps * kMaxGroup;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(w_pz + kConsumerWarps * kMaxGroup);
-  volatile int* flags = reinterpret_cast<volatile int*>(bars + 2 * kStages);  // [0] abort, [1] last
-  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kStages);
+struct WarpSmem {
+  uint8_t code[kStages][kStageCode];
+  uint8_t meta[kStages][kStageMeta];
+};
 
-  constexpr int kGroupBytes = 256 * BITS;
-  constexpr int kChunkGroups = kChunkBytes / kGroupBytes;
+// LO: k-blocks that get the extra-precision q' term -- 1 when the Key
+// channels are ordered by lambda (outlier channels in k-block 0), else 8.
+template <int BITS, int LO>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  WarpSmem* ws = reinterpret_cast<WarpSmem*>(smem);
+  uint4* qf = reinterpret_cast<uint4*>(smem + kWarps * kWarpSmem);     // [8][32]
+  float* sig = reinterpret_cast<float*>(qf + 8 * 32);                 // [8] sum of q' per head
+  float* w_m = sig + kMaxGroup;                                        // [warps][8]
+  float* w_l = w_m + kWarps * kMaxGroup;
+  float* w_pz = w_l + kWarps * kMaxGroup;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(w_pz + kWarps * kMaxGroup);  // [warps][stages]
+  int2* desc = reinterpret_cast<int2*>(bars + kWarps * kStages);              // [warps][stages] (ng, valid0)
+  volatile int* flags = reinterpret_cast<volatile int*>(desc + kWarps * kStages);  // [0] abort, [1] last
+
+  constexpr int kGroupBytes = 512 * BITS;
+  constexpr int kPart = 256 * BITS;
+  constexpr bool kWide = BITS == 16;            // a 16-bit group (8 KiB) takes every code stage
+  constexpr int kS = kWide ? 1 : kStages;       // stages in use
+  constexpr int kChunkGroups = kWide ? 1 : kStageCode / kGroupBytes;
   constexpr float kCScale = (BITS == 16 ? 256.0f : 1.0f) / (float)((1u << BITS) - 1u);
+  constexpr float kKScale = kCScale / (float)(1 << emax<BITS>());  // QK products carry 2^emax
 
   const Fill f = a.fill;
-  const int n_streams = a.batch * a.kv_heads;
-  const long long tot = (long long)n_streams * f.gps;
-  const int cta = blockIdx.x;
-  const long long g_begin = tot * cta / a.grid, g_end = tot * (cta + 1) / a.grid;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; i++) {
-      mbar_init(full0 + 8 * i, 1);
-      mbar_init(empty0 + 8 * i, kConsumerWarps);
-    }
-    flags[0] = 0;
-    flags[1] = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  for (int i = threadIdx.x; i < kMaxGroup * kHeadDim; i += kThreads) o_acc[i] = 0.f;
-  __syncthreads();
-  if (g_begin >= g_end) return;
-
-  if (warp == kConsumerWarps) {
-    // ---------------- producer ----------------
-    if (lane == 0) {
-      ChunkIter it{g_begin, g_end};
-      Chunk c;
-      for (int ci = 0; it.next(f, kChunkGroups, c); ci++) {
-        const int st = ci % kStages;
-        if (ci >= kStages) {
-          if (!mbar_wait(empty0 + 8 * st, ((ci / kStages) - 1) & 1, a.err, flags)) break;
-        }
-        const uint32_t kb = (uint32_t)c.ng * kGroupBytes, mb = (uint32_t)c.ng * 64u;
-        mbar_expect_tx(full0 + 8 * st, 2 * kb + 2 * mb);
-        uint8_t* sb = smem + st * kStageBytes;
-        const size_t sk = (size_t)c.s * 2, sv = sk + 1;
-        const uint8_t* kc = a.codes + (sk * f.nt + c.tile) * (size_t)kTileBytes + (size_t)c.grp0 * kGroupBytes;
-        const uint8_t* vc = a.codes + (sv * f.nt + c.tile) * (size_t)kTileBytes + (size_t)c.grp0 * kGroupBytes;
-        const uint32_t* km = a.meta + (sk * f.nt + c.tile) * (size_t)f.pf + (size_t)c.grp0 * 16;
-        const uint32_t* vm = a.meta + (sv * f.nt + c.tile) * (size_t)f.pf + (size_t)c.grp0 * 16;
-        bulk_g2s(smem_u32(sb), kc, kb, full0 + 8 * st);
-        bulk_g2s(smem_u32(sb + kChunkBytes), vc, kb, full0 + 8 * st);
-        bulk_g2s(smem_u32(sb + 2 * kChunkBytes), km, mb, full0 + 8 * st);
-        bulk_g2s(smem_u32(sb + 2 * kChunkBytes + kMetaBytes), vm, mb, full0 + 8 * st);
-      }
-    }
-    return;
-  }
-
-  // ---------------- consumers ----------------
   const int g = lane >> 2, t = lane & 3;
   const int G = a.group;
-  uint32_t bq[8][2];      // q' B fragments (fp16x2), high part
-  uint32_t bqo[8][2];     // q' - high part, rounded to fp16 (low part)
-  uint32_t bql[8][2];     // high part / 256 (16-bit codes only)
-  float sig0 = 0.f, sig1 = 0.f;  // sum of q' for heads 2t, 2t+1
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f, pz0 = 0.f, pz1 = 0.f;
-  float o[8][4];
-  int cur = -1;
+  const int s = blockIdx.x / a.splits, split = blockIdx.x - s * a.splits;
+  const long long ca = f.gps * split / a.splits, cb = f.gps * (split + 1) / a.splits;
+  const long long wa = ca + (cb - ca) * warp / kWarps, wb = ca + (cb - ca) * (warp + 1) / kWarps;
+  WarpSmem& my = ws[warp];
+  const uint32_t bar0 = smem_u32(bars + warp * kStages);
+  int2* mydesc = desc + warp * kStages;
 
-  auto start_stream = [&](int s) {
-    const int b = s / a.kv_heads, j = s - b * a.kv_heads;
+  if (threadIdx.x == 0) {
+    flags[0] = 0;
+    flags[1] = 0;
+  }
+  if (threadIdx.x < kMaxGroup) sig[threadIdx.x] = 0.f;
+  if (lane == 0) {
+    for (int i = 0; i < kS; i++) mbar_init(bar0 + 8 * i, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  // ---- chunk iterator: lane 0 walks its groups tile by tile and issues the
+  // copies; everyone reads the per-stage descriptors (groups, valid tokens) ----
+  int left = (int)(wb - wa);  // groups this warp still has to issue
+  int it_tile = 0, it_grp = 0, it_tgroups = 0, it_tvalid = 0;
+  if (left > 0) {
+    const GroupLoc loc = locate_group(f, wa);
+    it_tile = loc.tile;
+    it_grp = loc.grp;
+    it_tgroups = loc.tile_groups;
+    it_tvalid = loc.tile < f.k ? f.p : (loc.tile == f.k ? f.h + f.r : f.h);
+  }
+  const uint8_t* sbase = a.codes + (size_t)s * f.nt * kTileBytes;
+  const uint32_t* mbase = a.meta + (size_t)s * f.nt * f.pf * 2;
+  auto issue = [&](int st) {  // lane 0 only: next chunk of this warp into stage st
+    if (left <= 0) {
+      mydesc[st] = make_int2(0, 0);
+      return;
+    }
+    int ng = it_tgroups - it_grp;
+    ng = ng < kChunkGroups ? ng : kChunkGroups;
+    ng = ng < left ? ng : left;
+    mydesc[st] = make_int2(ng, it_tvalid - 16 * it_grp);
+    const uint32_t cbytes = (uint32_t)ng * kGroupBytes, mbytes = (uint32_t)ng * 128u;
+    const uint32_t bar = bar0 + 8 * st;
+    mbar_expect_tx(bar, cbytes + mbytes);
+    bulk_g2s(smem_u32(my.code[st]), sbase + (size_t)it_tile * kTileBytes + (size_t)it_grp * kGroupBytes, cbytes, bar);
+    bulk_g2s(smem_u32(my.meta[st]), mbase + ((size_t)it_tile * f.pf + (size_t)it_grp * 16) * 2, mbytes, bar);
+    left -= ng;
+    it_grp += ng;
+    if (it_grp == it_tgroups) {  // next tile: full, the partial tile k, or a base tile
+      it_tile++;
+      it_grp = 0;
+      it_tgroups = it_tile < f.k ? f.gpt : (it_tile == f.k ? f.gk : f.gh);
+      it_tvalid = it_tile < f.k ? f.p : (it_tile == f.k ? f.h + f.r : f.h);
+    }
+  };
+
+  // start streaming before the q' set-up so DRAM latency overlaps it
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < kS - 1; i++) issue(i);
+  }
+  __syncwarp();
+
+  // ---- q' fragments for this stream (warp 0 builds them in shared memory) ----
+  // sum(q') must be taken over exactly the q' values the MMAs use, so that
+  // (R/(2^b-1)) q'.c + Z sum(q') stays the dot product of that q' with the
+  // dequantised key.
+  constexpr int lo_blocks = LO;
+  const int b = s / a.kv_heads, j = s - b * a.kv_heads;
+  {
+    // warp w builds the fragments of k-blocks 2w and 2w+1
     const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.q_heads + (size_t)j * G) * kHeadDim;
     const float* lam = a.lam ? a.lam + (size_t)j * kHeadDim : nullptr;
+    const uint8_t* pm = a.perm ? a.perm + (size_t)j * kHeadDim : nullptr;
     float part = 0.f;
 #pragma unroll
-    for (int sb = 0; sb < 8; sb++) {
+    for (int i = 0; i < 2; i++) {
+      const int sb = 2 * warp + i;
+      uint32_t hq[2], lq[2];
 #pragma unroll
       for (int hf = 0; hf < 2; hf++) {
         const int c0 = 16 * sb + 2 * t + 8 * hf;
         float v0 = 0.f, v1 = 0.f;
         if (g < G) {
-          const __nv_bfloat162 qq = *reinterpret_cast<const __nv_bfloat162*>(qb + (size_t)g * kHeadDim + c0);
-          v0 = __low2float(qq) * a.qscale;
-          v1 = __high2float(qq) * a.qscale;
+          // Key positions c0, c0+1 hold channels ch0, ch1 of the block's order
+          const int ch0 = pm ? pm[c0] : c0, ch1 = pm ? pm[c0 + 1] : c0 + 1;
+          const __nv_bfloat16* qr = qb + (size_t)g * kHeadDim;
+          v0 = __bfloat162float(qr[ch0]) * a.qscale;
+          v1 = __bfloat162float(qr[ch1]) * a.qscale;
           if (lam) {
-            v0 *= lam[c0];
-            v1 *= lam[c0 + 1];
+            v0 *= lam[ch0];
+            v1 *= lam[ch1];
           }
         }
-        const __half2 h = __floats2half2_rn(v0, v1);
-        const __half2 lo = __floats2half2_rn(v0 - __low2float(h), v1 - __high2float(h));
-        bq[sb][hf] = *reinterpret_cast<const uint32_t*>(&h);
-        bqo[sb][hf] = *reinterpret_cast<const uint32_t*>(&lo);
-        part += (__low2float(h) + __low2float(lo)) + (__high2float(h) + __high2float(lo));
-        if (BITS == 16) {
-          const __half2 hl = __hmul2(h, __float2half2_rn(1.0f / 256.0f));
-          bql[sb][hf] = *reinterpret_cast<const uint32_t*>(&hl);
-        }
+        // channel block sb, half hf = pair p = 2 sb + hf of the Key units
+        const float scl = kWide ? 1.0f : (float)(1 << (emax<BITS>() - pair_shift<BITS>(2 * sb + hf)));
+        const __half2 h = __floats2half2_rn(v0 * scl, v1 * scl);
+        const __half2 lo = __floats2half2_rn(v0 * scl - __low2float(h), v1 * scl - __high2float(h));
+        hq[hf] = *reinterpret_cast<const uint32_t*>(&h);
+        lq[hf] = *reinterpret_cast<const uint32_t*>(&lo);
+        const float lo0 = sb < lo_blocks ? __low2float(lo) : 0.f, lo1 = sb < lo_blocks ? __high2float(lo) : 0.f;
+        part += ((__low2float(h) + lo0) + (__high2float(h) + lo1)) / scl;
       }
+      qf[sb * 32 + lane] = make_uint4(hq[0], hq[1], lq[0], lq[1]);
     }
     part += __shfl_xor_sync(0xffffffffu, part, 1);
-    part += __shfl_xor_sync(0xffffffffu, part, 2);  // lanes 4g..4g+3: sum for head g
-    sig0 = __shfl_sync(0xffffffffu, part, 4 * (2 * t));
-    sig1 = __shfl_sync(0xffffffffu, part, 4 * (2 * t + 1));
-    m0 = m1 = -INFINITY;
-    l0 = l1 = pz0 = pz1 = 0.f;
-#pragma unroll
-    for (int sb = 0; sb < 8; sb++) o[sb][0] = o[sb][1] = o[sb][2] = o[sb][3] = 0.f;
-  };
+    part += __shfl_xor_sync(0xffffffffu, part, 2);  // lanes 4g..4g+3: this warp's sum for head g
+    if (t == 0) atomicAdd(&sig[g], part);
+  }
+  __syncthreads();
+  const float sig0 = sig[2 * t], sig1 = sig[2 * t + 1];  // sum of q' for heads 2t, 2t+1
+  const uint4* qfl = qf + lane;
 
-  auto finish_stream = [&](int s) {
-    // per-warp totals for heads 2t, 2t+1 (reduce the thread partials over g)
+  Soft sm;
+  sm.m0 = sm.m1 = -INFINITY;
+  sm.l0 = sm.l1 = sm.pz0 = sm.pz1 = 0.f;
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-      pz0 += __shfl_xor_sync(0xffffffffu, pz0, off);
-      pz1 += __shfl_xor_sync(0xffffffffu, pz1, off);
+  for (int sb = 0; sb < 8; sb++) sm.o[sb][0] = sm.o[sb][1] = sm.o[sb][2] = sm.o[sb][3] = 0.f;
+
+  for (int ci = 0;; ci++) {
+    const int st = kWide ? 0 : ci % kS;
+    if (!kWide && lane == 0) issue((ci + kS - 1) % kS);  // refills the stage used by chunk ci-1
+    if (kWide && lane == 0) issue(0);
+    __syncwarp();
+    const int2 dsc = mydesc[st];
+    if (dsc.x == 0) break;
+    const uint32_t parity = kWide ? (ci & 1) : ((ci / kS) & 1);
+    if (!mbar_wait(bar0 + 8 * st, parity, a.err, flags)) break;
+    const uint8_t* cs = my.code[st];
+    const uint2* ms = reinterpret_cast<const uint2*>(my.meta[st]);
+    int gi = 0;
+    if constexpr (kChunkGroups >= 2) {
+      for (; gi + 2 <= dsc.x; gi += 2)
+        process_groups<BITS, LO, 2>(cs, ms, gi, dsc.y - 16 * gi, lane, qfl, sig0, sig1, kKScale, sm);
     }
-    if (g == 0) {
-      w_m[warp * kMaxGroup + 2 * t] = m0;
-      w_m[warp * kMaxGroup + 2 * t + 1] = m1;
-      w_l[warp * kMaxGroup + 2 * t] = l0;
-      w_l[warp * kMaxGroup + 2 * t + 1] = l1;
-      w_pz[warp * kMaxGroup + 2 * t] = pz0;
-      w_pz[warp * kMaxGroup + 2 * t + 1] = pz1;
-    }
-    consumer_sync();
+    for (; gi < dsc.x; gi++)
+      process_groups<BITS, LO, 1>(cs, ms, gi, dsc.y - 16 * gi, lane, qfl, sig0, sig1, kKScale, sm);
+    __syncwarp();  // every lane is done with this stage before lane 0 refills it
+  }
+  float m0 = sm.m0, m1 = sm.m1, l0 = sm.l0, l1 = sm.l1, pz0 = sm.pz0, pz1 = sm.pz1;
+  float (&o)[8][4] = sm.o;
+
+  // ---- merge the four warps ----
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    pz0 += __shfl_xor_sync(0xffffffffu, pz0, off);
+    pz1 += __shfl_xor_sync(0xffffffffu, pz1, off);
+  }
+  if (g == 0) {
+    w_m[warp * kMaxGroup + 2 * t] = m0;
+    w_m[warp * kMaxGroup + 2 * t + 1] = m1;
+    w_l[warp * kMaxGroup + 2 * t] = l0;
+    w_l[warp * kMaxGroup + 2 * t + 1] = l1;
+    w_pz[warp * kMaxGroup + 2 * t] = pz0;
+    w_pz[warp * kMaxGroup + 2 * t + 1] = pz1;
+  }
+  __syncthreads();  // also: every stage of every warp is consumed (no copy in flight)
+  {
     float M0 = -INFINITY, M1 = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; w++) {
+    for (int w = 0; w < kWarps; w++) {
       M0 = fmaxf(M0, w_m[w * kMaxGroup + 2 * t]);
       M1 = fmaxf(M1, w_m[w * kMaxGroup + 2 * t + 1]);
     }
     const float sc0 = ex2(m0 - M0), sc1 = ex2(m1 - M1);
-    if (2 * t < G) {
+    float* ob = reinterpret_cast<float*>(my.code[0]);  // this warp's scaled o: [8][128]
 #pragma unroll
-      for (int sb = 0; sb < 8; sb++) {
-        atomicAdd(&o_acc[(2 * t) * kHeadDim + 16 * sb + g], sc0 * o[sb][0]);
-        atomicAdd(&o_acc[(2 * t) * kHeadDim + 16 * sb + g + 8], sc0 * o[sb][2]);
+    for (int sb = 0; sb < 8; sb++) {
+      // rows 16sb+g (pair 2sb) and 16sb+g+8 (pair 2sb+1) carry 2^field_shift
+      const float r0 = 1.0f / (float)(1 << pair_shift<BITS>(2 * sb));
+      const float r1 = 1.0f / (float)(1 << pair_shift<BITS>(2 * sb + 1));
+      ob[(2 * t) * kHeadDim + 16 * sb + g] = sc0 * r0 * o[sb][0];
+      ob[(2 * t + 1) * kHeadDim + 16 * sb + g] = sc1 * r0 * o[sb][1];
+      ob[(2 * t) * kHeadDim + 16 * sb + g + 8] = sc0 * r1 * o[sb][2];
+      ob[(2 * t + 1) * kHeadDim + 16 * sb + g + 8] = sc1 * r1 * o[sb][3];
+    }
+  }
+  __syncthreads();
+  float* outp = a.out + ((size_t)b * a.q_heads + (size_t)j * G) * kHeadDim;
+  const int nparts = a.splits;
+  float* mypart = a.parts + ((size_t)s * nparts + split) * G * (kHeadDim + 2);
+  for (int idx = threadIdx.x; idx < G * kHeadDim; idx += kThreads) {
+    const int h = idx / kHeadDim, c = idx - h * kHeadDim;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; w++) M = fmaxf(M, w_m[w * kMaxGroup + h]);
+    float L = 0.f, PZ = 0.f, O = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; w++) {
+      const float e = ex2(w_m[w * kMaxGroup + h] - M);
+      L += e * w_l[w * kMaxGroup + h];
+      PZ += e * w_pz[w * kMaxGroup + h];
+      O += reinterpret_cast<const float*>(ws[w].code[0])[idx];
+    }
+    O = O * kCScale + PZ;
+    if (nparts == 1) {
+      outp[idx] = O / L;
+    } else {
+      float* pr = mypart + (size_t)h * (kHeadDim + 2);
+      pr[2 + c] = O;
+      if (c == 0) {
+        pr[0] = M;
+        pr[1] = L;
       }
     }
-    if (2 * t + 1 < G) {
-#pragma unroll
-      for (int sb = 0; sb < 8; sb++) {
-        atomicAdd(&o_acc[(2 * t + 1) * kHeadDim + 16 * sb + g], sc1 * o[sb][1]);
-        atomicAdd(&o_acc[(2 * t + 1) * kHeadDim + 16 * sb + g + 8], sc1 * o[sb][3]);
-      }
+  }
+  if (nparts > 1) {
+    // Ticket: after the CTA barrier, one thread publishes the CTA's partial
+    // (fence, then the atomic); the CTA that takes the last ticket merges.
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      const int old = atomicAdd(a.counters + s, 1);
+      const int last = old == nparts - 1;
+      if (last) __threadfence();
+      flags[1] = last;
     }
-    consumer_sync();
-    const long long first = cta_of((long long)s * f.gps, tot, a.grid);
-    const long long last = cta_of((long long)(s + 1) * f.gps - 1, tot, a.grid);
-    const int nparts = (int)(last - first + 1);
-    const int b = s / a.kv_heads, j = s - b * a.kv_heads;
-    float* outp = a.out + ((size_t)b * a.q_heads + (size_t)j * G) * kHeadDim;
-    float* mypart = a.parts + (size_t)(cta + s) * G * (kHeadDim + 2);
-    for (int idx = threadIdx.x; idx < G * kHeadDim; idx += kConsumerWarps * 32) {
-      const int h = idx / kHeadDim, c = idx - h * kHeadDim;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; w++) M = fmaxf(M, w_m[w * kMaxGroup + h]);
-      float L = 0.f, PZ = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; w++) {
-        const float e = ex2(w_m[w * kMaxGroup + h] - M);
-        L += e * w_l[w * kMaxGroup + h];
-        PZ += e * w_pz[w * kMaxGroup + h];
+    __syncthreads();
+    if (flags[1]) {
+      const float* p0 = a.parts + (size_t)s * nparts * G * (kHeadDim + 2);
+      const size_t rec = (size_t)(kHeadDim + 2);
+      float* pmax = reinterpret_cast<float*>(ws[0].code[0]);  // [nparts][G]  (stage buffers are free now)
+      float* psum = pmax + kMaxSplits * kMaxGroup;
+      // every partial's (max, sum) at once
+      for (int i = threadIdx.x; i < nparts * G; i += kThreads) {
+        pmax[i] = __ldcg(p0 + (size_t)i * rec);
+        psum[i] = __ldcg(p0 + (size_t)i * rec + 1);
       }
-      const float O = o_acc[idx] * kCScale + PZ;
-      o_acc[idx] = 0.f;
-      if (nparts == 1) {
-        outp[idx] = O / L;
-      } else {
-        float* pr = mypart + (size_t)h * (kHeadDim + 2);
-        pr[2 + c] = O;
-        if (c == 0) {
-          pr[0] = M;
-          pr[1] = L;
+      __syncthreads();
+      if (threadIdx.x < G) {  // weight of partial k for head h: e^(M_k - M) / L
+        const int h = threadIdx.x;
+        float M = -INFINITY;
+        for (int k = 0; k < nparts; k++) M = fmaxf(M, pmax[k * G + h]);
+        float L = 0.f;
+        for (int k = 0; k < nparts; k++) {
+          const float e = ex2(pmax[k * G + h] - M);
+          pmax[k * G + h] = e;
+          L += e * psum[k * G + h];
         }
+        const float inv = 1.0f / L;
+        for (int k = 0; k < nparts; k++) pmax[k * G + h] *= inv;
       }
-    }
-    if (nparts > 1) {
-      __threadfence();  // this thread's partial is visible device-wide before the ticket
-      consumer_sync();
-      if (threadIdx.x == 0) {
-        __threadfence();
-        const int old = atomicAdd(a.counters + s, 1);
-        flags[1] = (old == nparts - 1);
-      }
-      consumer_sync();
-      if (flags[1]) {
-        __threadfence();
-        const float* p0 = a.parts + (size_t)(first + s) * G * (kHeadDim + 2);
-        for (int idx = threadIdx.x; idx < G * kHeadDim; idx += kConsumerWarps * 32) {
-          const int h = idx / kHeadDim, c = idx - h * kHeadDim;
-          float M = -INFINITY;
-          for (int k = 0; k < nparts; k++) M = fmaxf(M, __ldcg(p0 + ((size_t)k * G + h) * (kHeadDim + 2)));
-          float L = 0.f, O = 0.f;
-          for (int k = 0; k < nparts; k++) {
-            const float* pr = p0 + ((size_t)k * G + h) * (kHeadDim + 2);
-            const float e = ex2(__ldcg(pr) - M);
-            L += e * __ldcg(pr + 1);
-            O += e * __ldcg(pr + 2 + c);
-          }
-          outp[idx] = O / L;
+      __syncthreads();
+      static_assert(kThreads == kHeadDim, "one channel per thread");
+      const int c = threadIdx.x;  // one channel per thread
+      for (int h = 0; h < G; h++) {
+        const float* pr = p0 + (size_t)h * rec + 2 + c;
+        float acc[8];
+#pragma unroll
+        for (int u = 0; u < 8; u++) acc[u] = 0.f;
+        int k = 0;
+        for (; k + 8 <= nparts; k += 8) {
+#pragma unroll
+          for (int u = 0; u < 8; u++) acc[u] += pmax[(k + u) * G + h] * __ldcg(pr + (size_t)(k + u) * G * rec);
         }
-        if (threadIdx.x == 0) a.counters[s] = 0;
+        for (; k < nparts; k++) acc[0] += pmax[k * G + h] * __ldcg(pr + (size_t)k * G * rec);
+        outp[h * kHeadDim + c] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
       }
+      if (threadIdx.x == 0) a.counters[s] = 0;
     }
-    consumer_sync();
-  };
+  }
+}
 
-  ChunkIter it{g_begin, g_end};
-  Chunk c;
-  for (int ci = 0; it.next(f, kChunkGroups, c); ci++) {
-    if (c.s != cur) {
-      if (cur >= 0) finish_stream(cur);
-      start_stream(c.s);
-      cur = c.s;
-    }
-    const int st = ci % kStages;
-    const bool ok = mbar_wait(full0 + 8 * st, (ci / kStages) & 1, a.err, flags);
-    const uint8_t* sb = smem + st * kStageBytes;
-    for (int gi = warp; ok && gi < c.ng; gi += kConsumerWarps) {
-      const int valid = min(16, c.tile_valid - 16 * (c.grp0 + gi));
-      // ---- K unit -> scores ----
-      const uint32_t* ku = reinterpret_cast<const uint32_t*>(sb + (size_t)gi * kGroupBytes + lane * unit_bytes(BITS));
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
-      if constexpr (BITS == 16) {
-#pragma unroll
-        for (int sb2 = 0; sb2 < 8; sb2++) {
-          const uint2 w0 = *reinterpret_cast<const uint2*>(ku + 2 * sb2);        // token g: pairs 2s, 2s+1
-          const uint2 w1 = *reinterpret_cast<const uint2*>(ku + 16 + 2 * sb2);   // token g+8
-          const uint32_t h0 = widen16_hi(w0.x), h1 = widen16_hi(w1.x), h2 = widen16_hi(w0.y), h3 = widen16_hi(w1.y);
-          mma(d, h0, h1, h2, h3, bq[sb2][0], bq[sb2][1]);
-          mma(d, h0, h1, h2, h3, bqo[sb2][0], bqo[sb2][1]);
-          mma(d, widen16_lo(w0.x), widen16_lo(w1.x), widen16_lo(w0.y), widen16_lo(w1.y), bql[sb2][0], bql[sb2][1]);
-        }
-      } else {
-        uint32_t u[2 * BITS], u8[2 * BITS];
-#pragma unroll
-        for (int i = 0; i < 2 * BITS; i += 4) {
-          const uint4 q4 = *reinterpret_cast<const uint4*>(ku + i);
-          u[i] = q4.x; u[i + 1] = q4.y; u[i + 2] = q4.z; u[i + 3] = q4.w;
-        }
-#pragma unroll
-        for (int i = 0; i < 2 * BITS; i++) u8[i] = u[i] >> 8;
-#define KVQ_QK(S)                                                                                     \
-  {                                                                                                     \
-    const uint32_t a0 = pair_at<BITS, S>(u, u8, 0, 0), a1 = pair_at<BITS, S>(u, u8, 1, 0);             \
-    const uint32_t a2 = pair_at<BITS, S>(u, u8, 0, 1), a3 = pair_at<BITS, S>(u, u8, 1, 1);             \
-    mma(d, a0, a1, a2, a3, bq[S][0], bq[S][1]);                                                         \
-    mma(d, a0, a1, a2, a3, bqo[S][0], bqo[S][1]);                                                       \
+template <int BITS, int LO>
+cudaError_t launch_bits(const DecodeArgs& a, cudaStream_t s) {
+  static bool attr_set = false;  // per process; set before the first launch
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, LO>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_kernel<BITS, LO>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
   }
-        KVQ_QK(0) KVQ_QK(1) KVQ_QK(2) KVQ_QK(3) KVQ_QK(4) KVQ_QK(5) KVQ_QK(6) KVQ_QK(7)
-#undef KVQ_QK
-      }
-      // ---- meta for tokens g, g+8 ----
-      const uint32_t* kmeta = reinterpret_cast<const uint32_t*>(sb + 2 * kChunkBytes) + gi * 16;
-      const uint32_t* vmeta = reinterpret_cast<const uint32_t*>(sb + 2 * kChunkBytes + kMetaBytes) + gi * 16;
-      const bool va = g < valid, vb = g + 8 < valid;
-      const float2 ka = __half22float2(*reinterpret_cast<const __half2*>(kmeta + g));
-      const float2 kb = __half22float2(*reinterpret_cast<const __half2*>(kmeta + g + 8));
-      const float2 vma = __half22float2(*reinterpret_cast<const __half2*>(vmeta + g));
-      const float2 vmb = __half22float2(*reinterpret_cast<const __half2*>(vmeta + g + 8));
-      const float rka = ka.x * kCScale, rkb = kb.x * kCScale;
-      const float s00 = va ? fmaf(rka, d[0], ka.y * sig0) : -INFINITY;
-      const float s01 = va ? fmaf(rka, d[1], ka.y * sig1) : -INFINITY;
-      const float s10 = vb ? fmaf(rkb, d[2], kb.y * sig0) : -INFINITY;
-      const float s11 = vb ? fmaf(rkb, d[3], kb.y * sig1) : -INFINITY;
-      float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-      }
-      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-      if (__any_sync(0xffffffffu, (n0 > m0) | (n1 > m1))) {
-        const float a0 = ex2(m0 - n0), a1 = ex2(m1 - n1);
-#pragma unroll
-        for (int sb2 = 0; sb2 < 8; sb2++) {
-          o[sb2][0] *= a0; o[sb2][2] *= a0;
-          o[sb2][1] *= a1; o[sb2][3] *= a1;
-        }
-        l0 *= a0; pz0 *= a0;
-        l1 *= a1; pz1 *= a1;
-        m0 = n0;
-        m1 = n1;
-      }
-      const float p00 = ex2(s00 - m0), p01 = ex2(s01 - m1), p10 = ex2(s10 - m0), p11 = ex2(s11 - m1);
-      const float rva = va ? vma.x : 0.f, zva = va ? vma.y : 0.f;
-      const float rvb = vb ? vmb.x : 0.f, zvb = vb ? vmb.y : 0.f;
-      l0 += p00 + p10;
-      l1 += p01 + p11;
-      pz0 = fmaf(p00, zva, fmaf(p10, zvb, pz0));
-      pz1 = fmaf(p01, zva, fmaf(p11, zvb, pz1));
-      const uint32_t b0 = movmatrix_t(pack_h2(p00 * rva, p01 * rva));  // tokens 2t,2t+1 of head g
-      const uint32_t b1 = movmatrix_t(pack_h2(p10 * rvb, p11 * rvb));  // tokens 2t+8, 2t+9
-      // ---- V unit -> output ----
-      const uint32_t* vu = reinterpret_cast<const uint32_t*>(sb + kChunkBytes + (size_t)gi * kGroupBytes + lane * unit_bytes(BITS));
-      if constexpr (BITS == 16) {
-        const uint32_t b0l = hfma2_u(b0, 0x1c001c00u, 0u), b1l = hfma2_u(b1, 0x1c001c00u, 0u);  // /256
-#pragma unroll
-        for (int sb2 = 0; sb2 < 8; sb2++) {
-          const uint2 w0 = *reinterpret_cast<const uint2*>(vu + 2 * sb2);        // u = 0
-          const uint2 w1 = *reinterpret_cast<const uint2*>(vu + 16 + 2 * sb2);   // u = 1
-          mma(o[sb2], widen16_hi(w0.x), widen16_hi(w0.y), widen16_hi(w1.x), widen16_hi(w1.y), b0, b1);
-          mma(o[sb2], widen16_lo(w0.x), widen16_lo(w0.y), widen16_lo(w1.x), widen16_lo(w1.y), b0l, b1l);
-        }
-      } else {
-        uint32_t u[2 * BITS], u8[2 * BITS];
-#pragma unroll
-        for (int i = 0; i < 2 * BITS; i += 4) {
-          const uint4 q4 = *reinterpret_cast<const uint4*>(vu + i);
-          u[i] = q4.x; u[i + 1] = q4.y; u[i + 2] = q4.z; u[i + 3] = q4.w;
-        }
-#pragma unroll
-        for (int i = 0; i < 2 * BITS; i++) u8[i] = u[i] >> 8;
-#define KVQ_PV(S)                                                                                       \
-  mma(o[S], pair_at<BITS, S>(u, u8, 0, 0), pair_at<BITS, S>(u, u8, 0, 1), pair_at<BITS, S>(u, u8, 1, 0), \
-      pair_at<BITS, S>(u, u8, 1, 1), b0, b1);
-        KVQ_PV(0) KVQ_PV(1) KVQ_PV(2) KVQ_PV(3) KVQ_PV(4) KVQ_PV(5) KVQ_PV(6) KVQ_PV(7)
-#undef KVQ_PV
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty0 + 8 * st);
-  }
-  if (cur >= 0) finish_stream(cur);
+  const unsigned grid = (unsigned)(a.batch * a.kv_heads) * (unsigned)a.splits;
+  decode_kernel<BITS, LO><<<grid, kThreads, kSmemBytes, s>>>(a);
+  return cudaGetLastError();
 }
 
 template <int BITS>
 cudaError_t launch_bits(const DecodeArgs& a, cudaStream_t s) {
-  static bool attr_set = false;  // per process; set before the first launch
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  decode_kernel<BITS><<<a.grid, kThreads, kSmemBytes, s>>>(a);
-  return cudaGetLastError();
+  return a.perm ? launch_bits<BITS, 1>(a, s) : launch_bits<BITS, 8>(a, s);
 }
 
 }  // namespace
 
-int decode_grid(int num_sms) { return num_sms * kCtasPerSm; }
+int decode_splits(int num_sms, int n_streams, long long gps) {
+  // Smallest modelled makespan  waves(s) * (gps / s + c0)  over
+  // s = 1..min(kMaxSplits, gps), where a wave is num_sms * kCtasPerSm CTAs
+  // and c0 (in groups) stands for a CTA's fixed cost: pipeline fill, q'
+  // set-up, the warp merge and its share of the split merge.  Every CTA gets
+  // at least one group; ties go to fewer splits (fewer partials).
+  const long long slots = (long long)num_sms * kCtasPerSm;
+  const double c0 = 8.0;
+  const int smax = (int)(gps < kMaxSplits ? gps : kMaxSplits);
+  int best = 1;
+  double best_t = 1e300;
+  for (int sp = 1; sp <= smax; sp++) {
+    const long long waves = ((long long)n_streams * sp + slots - 1) / slots;
+    const double tm = (double)waves * ((double)gps / sp + c0 + (sp > 1 ? 0.25 * sp : 0.0));
+    if (tm < best_t * (1.0 - 1e-9)) {
+      best_t = tm;
+      best = sp;
+    }
+  }
+  return best;
+}
 
-size_t decode_parts_bytes(int grid, int n_streams, int group) {
-  return (size_t)(grid + n_streams) * group * (kHeadDim + 2) * sizeof(float);
+size_t decode_parts_bytes(int n_streams, int group) {
+  return (size_t)n_streams * kMaxSplits * group * (kHeadDim + 2) * sizeof(float);
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
-  if (a.group < 1 || a.group > kMaxGroup) return cudaErrorInvalidValue;
+  if (a.group < 1 || a.group > kMaxGroup || a.splits < 1 || a.splits > kMaxSplits) return cudaErrorInvalidValue;
   switch (a.fill.bits) {
     case 2: return launch_bits<2>(a, s);
     case 4: return launch_bits<4>(a, s);

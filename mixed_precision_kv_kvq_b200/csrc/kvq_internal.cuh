@@ -1,16 +1,17 @@
 // kvq_internal.cuh -- packed layout, block fill pattern and launch interfaces
 // shared by the libkvq kernels and the host scheduler.
 //
-// Packed layout (one "stream" = one (layer, sequence, KV head, K-or-V)):
-//   The stream is a region of NT tiles of 16 KiB.  At b bits a tile holds
-//   P_b = 1024 / b token slots (64 at 16 bits ... 512 at 2 bits), grouped in
-//   16-token groups of 256*b bytes.  A group is 32 "lane units" of 8*b bytes;
-//   unit L holds exactly the 64 codes that lane L of a warp needs as its
-//   mma.sync.m16n8k16 A-fragment registers:
-//     K (QK^T, A = K[token][channel]):  with L = 4g + t, tokens g and g+8 of
-//       the group, channels 16s + 2t + {0,1} + 8r  (s = 0..7, r = 0..1).
-//     V (P V,  A = V^T[channel][token]): channels 16s + g + 8r, tokens
-//       2t + {0,1} + 8u (u = 0..1).
+// Packed layout.  A "stream" is one (layer, sequence b, KV head j); it owns a
+// region of NT tiles of 16 KiB holding both its Keys and its Values.  At b
+// bits a tile holds P_b = 512 / b token slots (32 at 16 bits ... 256 at 2
+// bits) in 16-token groups of 512*b bytes: the group's K part (256*b bytes)
+// followed by its V part (256*b bytes).  Each part is 32 "lane units" of 8*b
+// bytes; unit L holds exactly the 64 codes that lane L of a warp needs as its
+// mma.sync.m16n8k16 A-fragment registers:
+//   K (QK^T, A = K[token][channel]):  with L = 4g + t, tokens g and g+8 of
+//     the group, channels 16s + 2t + {0,1} + 8r  (s = 0..7, r = 0..1).
+//   V (P V,  A = V^T[channel][token]): channels 16s + g + 8r, tokens
+//     2t + {0,1} + 8u (u = 0..1).
 //   Codes come in pairs that fill one half2 register: for K a pair is two
 //   adjacent channels of one token, for V the same channel of tokens 2t+8u and
 //   2t+8u+1.  A unit holds 32 pairs; pair index P = 16*x + 2*s + r, where x
@@ -19,9 +20,10 @@
 //   k = P % (16/b): the first member at bits [b*k, b*k+b), the second at
 //   bits [16 + b*k, 16 + b*k + b).  So each 16-bit half-word packs 16/b codes.
 //   Because this order is the same at every width, the shift 2b -> b maps
-//   input words (2J, 2J+1) of a tile to output word J of the same tile, with
-//   no data moving between tiles: a shrink compacts every tile into its first
-//   half in place and token slots keep their indices.
+//   input words (2J, 2J+1) of a tile to output word J of the same tile (the
+//   K/V interleave of the groups is preserved too), with no data moving
+//   between tiles: a shrink compacts every tile into its first half in place
+//   and token slots keep their indices.
 //
 // Fill pattern of a block (the slot map): before the first shrink tokens
 // fill tile 0, tile 1, ... (P_16 each).  A shrink happens only when every
@@ -30,9 +32,18 @@
 // therefore: tiles < k full, tile k holding h + r, tiles > k holding h.
 // Attention does not depend on token order, so nothing is ever reordered.
 //
-// Meta: one 32-bit word per (stream, tile, slot) = binary16 R (low half) and
-// binary16 Z (high half), sized for P_F slots per tile (F = the block's Fbit,
-// the widest a tile ever gets).  A shrink never touches it.
+// Key channel order: within every Key unit, "channel" above means a
+// position of the block's per-KV-head channel order perm[j][pos] (logical
+// channel at that position), which puts the 16 channels with the largest
+// migration factor lambda in positions 0..15, i.e. the first MMA k-block.
+// Outlier channels carry the largest q'.k products, and only that k-block
+// gets the extra-precision (hi + lo) q' term in the attention kernel.  Values
+// keep the natural channel order.
+//
+// Meta: two 32-bit words per (stream, tile, slot), the Key's then the
+// Value's, each binary16 R (low half) and binary16 Z (high half); P_F slots
+// per tile (F = the block's Fbit, the widest a tile ever gets).  A shrink
+// never touches meta.
 #pragma once
 #include <cstddef>
 #include <cstdint>
@@ -44,8 +55,9 @@ constexpr int kHeadDim = 128;
 constexpr int kTileBytes = 16384;
 constexpr int kGroupTokens = 16;
 
-__host__ __device__ constexpr int slots_per_tile(int bits) { return 1024 / bits; }
-__host__ __device__ constexpr int group_bytes(int bits) { return 256 * bits; }
+__host__ __device__ constexpr int slots_per_tile(int bits) { return 512 / bits; }
+__host__ __device__ constexpr int group_bytes(int bits) { return 512 * bits; }  // K part + V part
+__host__ __device__ constexpr int part_bytes(int bits) { return 256 * bits; }   // offset of the V part
 __host__ __device__ constexpr int unit_bytes(int bits) { return 8 * bits; }
 
 // Fill pattern of one block at its current width (identical for every stream
@@ -135,14 +147,15 @@ struct AppendArgs {
   long long n0;       // logical index of the first token of this launch
   int bits, h, e, nt, pf;
   int batch, kv_heads;
-  uint8_t* codes;     // layer base: [batch][kv_heads][2][nt][16 KiB]
-  uint32_t* meta;     // layer base: [batch][kv_heads][2][nt][pf]
+  uint8_t* codes;     // layer base: [batch][kv_heads][nt][16 KiB]
+  uint32_t* meta;     // layer base: [batch][kv_heads][nt][pf][2]
   const float* lam_inv;  // [kv_heads][128] or null
+  const uint8_t* perm;   // [kv_heads][128] Key position -> channel, or null (identity)
 };
 
 struct ShrinkArgs {
   uint8_t* codes;     // layer base
-  long long n_tiles;  // batch * kv_heads * 2 * nt
+  long long n_tiles;  // batch * kv_heads * nt
   int bits_to;        // 8, 4 or 2
 };
 
@@ -151,18 +164,21 @@ struct DecodeArgs {
   const uint32_t* meta;
   const void* q;        // bf16 [batch][q_heads][128]
   const float* lam;     // [kv_heads][128] or null
+  const uint8_t* perm;  // [kv_heads][128] Key position -> channel, or null (identity)
   float* out;           // fp32 [batch][q_heads][128]
-  float* parts;         // workspace partials
+  float* parts;         // workspace partials [batch*kv_heads][splits][group][2 + 128]
   int* counters;        // [batch*kv_heads] ticket counters (zero between calls)
   int* err;             // device error flag
   Fill fill;
   int batch, kv_heads, q_heads, group;
   float qscale;         // sm_scale * log2(e)
-  int grid;             // CTAs launched
+  int splits;           // CTAs per stream
 };
 
-int decode_grid(int num_sms);
-size_t decode_parts_bytes(int grid, int n_streams, int group);
+// CTAs per stream for a launch over n_streams streams on num_sms SMs.
+int decode_splits(int num_sms, int n_streams, long long groups_per_stream);
+constexpr int kMaxSplits = 64;
+size_t decode_parts_bytes(int n_streams, int group);
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t s);
