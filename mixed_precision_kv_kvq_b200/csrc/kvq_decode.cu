@@ -51,6 +51,10 @@ constexpr int kQfBytes = 8 * 32 * 16;      // q' B fragments: [s-block][lane] x 
 constexpr int kSmemBytes = kWarps * kWarpSmem + kQfBytes + kMaxGroup * 4 + 3 * kWarps * kMaxGroup * 4 +
                            kWarps * kStages * 8 + kWarps * kStages * 8 + 16;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
+constexpr int kPartFloats = 2 * kMaxGroup + kHeadDim * kMaxGroup;  // one CTA's partial record
+// Largest amount (log2 units) a score may exceed the running max before the
+// max is moved: p <= 2^8, and p * R stays well inside fp16 for R < 255.
+constexpr float kRebase = 8.0f;
 
 // ------------------------------------------------------------------ PTX
 
@@ -356,8 +360,10 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
   }
+  // Lazy rebase: the running max moves only when a score exceeds it by more
+  // than kRebase (log2 units), so p = 2^(s - m) <= 2^kRebase.
   const float n0 = fmaxf(st.m0, mx0), n1 = fmaxf(st.m1, mx1);
-  if (__any_sync(0xffffffffu, (n0 > st.m0) | (n1 > st.m1))) {
+  if (__any_sync(0xffffffffu, (mx0 > st.m0 + kRebase) | (mx1 > st.m1 + kRebase))) {
     const float a0 = ex2(st.m0 - n0), a1 = ex2(st.m1 - n1);
 #pragma unroll
     for (int sb = 0; sb < 8; sb++) {
@@ -597,11 +603,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     }
   }
   __syncthreads();
+  // Final state of this CTA for every head h < G and channel c = thread:
+  //   M = max over warps, L and PZ = e^(m_w - M)-weighted sums, O = sum of the
+  //   warps' scaled rows (times 2^-e and 1/(2^b-1)) + PZ  (unnormalised).
   float* outp = a.out + ((size_t)b * a.q_heads + (size_t)j * G) * kHeadDim;
   const int nparts = a.splits;
-  float* mypart = a.parts + ((size_t)s * nparts + split) * G * (kHeadDim + 2);
-  for (int idx = threadIdx.x; idx < G * kHeadDim; idx += kThreads) {
-    const int h = idx / kHeadDim, c = idx - h * kHeadDim;
+  const int c = threadIdx.x;  // one channel per thread
+  static_assert(kThreads == kHeadDim, "one channel per thread");
+  float Oc[kMaxGroup], Mh[kMaxGroup], Lh[kMaxGroup];
+#pragma unroll
+  for (int h = 0; h < kMaxGroup; h++) {
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kWarps; w++) M = fmaxf(M, w_m[w * kMaxGroup + h]);
@@ -611,75 +622,81 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
       const float e = ex2(w_m[w * kMaxGroup + h] - M);
       L += e * w_l[w * kMaxGroup + h];
       PZ += e * w_pz[w * kMaxGroup + h];
-      O += reinterpret_cast<const float*>(ws[w].code[0])[idx];
+      O += reinterpret_cast<const float*>(ws[w].code[0])[h * kHeadDim + c];
     }
-    O = O * kCScale + PZ;
-    if (nparts == 1) {
-      outp[idx] = O / L;
-    } else {
-      float* pr = mypart + (size_t)h * (kHeadDim + 2);
-      pr[2 + c] = O;
-      if (c == 0) {
-        pr[0] = M;
-        pr[1] = L;
-      }
+    Oc[h] = O * kCScale + PZ;
+    Mh[h] = M;
+    Lh[h] = L;
+  }
+  if (nparts == 1) {
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; h++)
+      if (h < G) outp[h * kHeadDim + c] = Oc[h] / Lh[h];
+    return;
+  }
+  // Partial record of this CTA: M[8], L[8], then O[128 channels][8 heads].
+  float* mypart = a.parts + ((size_t)s * nparts + split) * kPartFloats;
+  if (c == 0) {
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; h += 4) {
+      *reinterpret_cast<float4*>(mypart + h) = make_float4(Mh[h], Mh[h + 1], Mh[h + 2], Mh[h + 3]);
+      *reinterpret_cast<float4*>(mypart + kMaxGroup + h) = make_float4(Lh[h], Lh[h + 1], Lh[h + 2], Lh[h + 3]);
     }
   }
-  if (nparts > 1) {
-    // Ticket: after the CTA barrier, one thread publishes the CTA's partial
-    // (fence, then the atomic); the CTA that takes the last ticket merges.
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      __threadfence();
-      const int old = atomicAdd(a.counters + s, 1);
-      const int last = old == nparts - 1;
-      if (last) __threadfence();
-      flags[1] = last;
-    }
-    __syncthreads();
-    if (flags[1]) {
-      const float* p0 = a.parts + (size_t)s * nparts * G * (kHeadDim + 2);
-      const size_t rec = (size_t)(kHeadDim + 2);
-      float* pmax = reinterpret_cast<float*>(ws[0].code[0]);  // [nparts][G]  (stage buffers are free now)
-      float* psum = pmax + kMaxSplits * kMaxGroup;
-      // every partial's (max, sum) at once
-      for (int i = threadIdx.x; i < nparts * G; i += kThreads) {
-        pmax[i] = __ldcg(p0 + (size_t)i * rec);
-        psum[i] = __ldcg(p0 + (size_t)i * rec + 1);
-      }
-      __syncthreads();
-      if (threadIdx.x < G) {  // weight of partial k for head h: e^(M_k - M) / L
-        const int h = threadIdx.x;
-        float M = -INFINITY;
-        for (int k = 0; k < nparts; k++) M = fmaxf(M, pmax[k * G + h]);
-        float L = 0.f;
-        for (int k = 0; k < nparts; k++) {
-          const float e = ex2(pmax[k * G + h] - M);
-          pmax[k * G + h] = e;
-          L += e * psum[k * G + h];
-        }
-        const float inv = 1.0f / L;
-        for (int k = 0; k < nparts; k++) pmax[k * G + h] *= inv;
-      }
-      __syncthreads();
-      static_assert(kThreads == kHeadDim, "one channel per thread");
-      const int c = threadIdx.x;  // one channel per thread
-      for (int h = 0; h < G; h++) {
-        const float* pr = p0 + (size_t)h * rec + 2 + c;
-        float acc[8];
-#pragma unroll
-        for (int u = 0; u < 8; u++) acc[u] = 0.f;
-        int k = 0;
-        for (; k + 8 <= nparts; k += 8) {
-#pragma unroll
-          for (int u = 0; u < 8; u++) acc[u] += pmax[(k + u) * G + h] * __ldcg(pr + (size_t)(k + u) * G * rec);
-        }
-        for (; k < nparts; k++) acc[0] += pmax[k * G + h] * __ldcg(pr + (size_t)k * G * rec);
-        outp[h * kHeadDim + c] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-      }
-      if (threadIdx.x == 0) a.counters[s] = 0;
-    }
+  *reinterpret_cast<float4*>(mypart + 2 * kMaxGroup + c * kMaxGroup) = make_float4(Oc[0], Oc[1], Oc[2], Oc[3]);
+  *reinterpret_cast<float4*>(mypart + 2 * kMaxGroup + c * kMaxGroup + 4) = make_float4(Oc[4], Oc[5], Oc[6], Oc[7]);
+  // Ticket: after the CTA barrier one thread publishes the CTA's partial
+  // (fence, then the atomic); the CTA that takes the last ticket merges.
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const int old = atomicAdd(a.counters + s, 1);
+    const int last = old == nparts - 1;
+    if (last) __threadfence();
+    flags[1] = last;
   }
+  __syncthreads();
+  if (!flags[1]) return;
+  const float* p0 = a.parts + (size_t)s * nparts * kPartFloats;
+  float* wk = reinterpret_cast<float*>(ws[0].code[0]);  // [nparts][8] (the stage buffers are free now)
+  float* lk = wk + kMaxSplits * kMaxGroup;
+  for (int i = threadIdx.x; i < nparts * 2 * kMaxGroup / 4; i += kThreads) {  // every partial's M, L at once
+    const int k = i / (2 * kMaxGroup / 4), q4 = i - k * (2 * kMaxGroup / 4);
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(p0 + (size_t)k * kPartFloats) + q4);
+    float* dst = q4 < 2 ? wk + k * kMaxGroup + 4 * q4 : lk + k * kMaxGroup + 4 * (q4 - 2);
+    dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+  }
+  __syncthreads();
+  if (threadIdx.x < kMaxGroup) {  // weight of partial k for head h: e^(M_k - M) / L
+    const int h = threadIdx.x;
+    float M = -INFINITY;
+    for (int k = 0; k < nparts; k++) M = fmaxf(M, wk[k * kMaxGroup + h]);
+    float L = 0.f;
+    for (int k = 0; k < nparts; k++) {
+      const float e = ex2(wk[k * kMaxGroup + h] - M);
+      wk[k * kMaxGroup + h] = e;
+      L += e * lk[k * kMaxGroup + h];
+    }
+    const float inv = 1.0f / L;
+    for (int k = 0; k < nparts; k++) wk[k * kMaxGroup + h] *= inv;
+  }
+  __syncthreads();
+  float acc[kMaxGroup];
+#pragma unroll
+  for (int h = 0; h < kMaxGroup; h++) acc[h] = 0.f;
+  const float* oc = p0 + 2 * kMaxGroup + c * kMaxGroup;
+#pragma unroll 4
+  for (int k = 0; k < nparts; k++) {
+    const float4 v0 = __ldcg(reinterpret_cast<const float4*>(oc + (size_t)k * kPartFloats));
+    const float4 v1 = __ldcg(reinterpret_cast<const float4*>(oc + (size_t)k * kPartFloats + 4));
+    const float* w = wk + k * kMaxGroup;
+    acc[0] += w[0] * v0.x; acc[1] += w[1] * v0.y; acc[2] += w[2] * v0.z; acc[3] += w[3] * v0.w;
+    acc[4] += w[4] * v1.x; acc[5] += w[5] * v1.y; acc[6] += w[6] * v1.z; acc[7] += w[7] * v1.w;
+  }
+#pragma unroll
+  for (int h = 0; h < kMaxGroup; h++)
+    if (h < G) outp[h * kHeadDim + c] = acc[h];
+  if (threadIdx.x == 0) a.counters[s] = 0;
 }
 
 template <int BITS, int LO>
@@ -728,7 +745,8 @@ int decode_splits(int num_sms, int n_streams, long long gps) {
 }
 
 size_t decode_parts_bytes(int n_streams, int group) {
-  return (size_t)n_streams * kMaxSplits * group * (kHeadDim + 2) * sizeof(float);
+  (void)group;
+  return (size_t)n_streams * kMaxSplits * kPartFloats * sizeof(float);
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {

@@ -166,7 +166,7 @@ struct DecodeArgs {
   const float* lam;     // [kv_heads][128] or null
   const uint8_t* perm;  // [kv_heads][128] Key position -> channel, or null (identity)
   float* out;           // fp32 [batch][q_heads][128]
-  float* parts;         // workspace partials [batch*kv_heads][splits][group][2 + 128]
+  float* parts;         // workspace partials: [batch*kv_heads][splits] records of M[8], L[8], O[128][8]
   int* counters;        // [batch*kv_heads] ticket counters (zero between calls)
   int* err;             // device error flag
   Fill fill;
