@@ -118,6 +118,22 @@ size_t kvq_decode_workspace(const kvq_cache* c, int layer, int q_heads);
 kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, float sm_scale,
                            float* out, void* workspace, size_t ws_bytes, kvq_stream_t stream);
 
+/* Decode attention that allocates nothing and takes no workspace; same
+ * arguments, result and errors as kvq_decode_attn otherwise.  The paper has
+ * no counterpart to this call: it exists for callers that cannot allocate device
+ * memory where they run decode (an allocator owned by a host framework, a
+ * serving loop that must not allocate after start-up, a host that only hands
+ * out inputs and outputs).  The split partials go to a 24 MiB buffer that is
+ * part of the library: every GPU that loads the library holds it until the
+ * process exits.  A block whose batch * kv_heads streams need more than that
+ * is rejected with KVQ_ERR_WORKSPACE (use kvq_decode_attn).  The first call
+ * on a device looks up the buffer's device address (a CUDA runtime query,
+ * no allocation); make that first call before any stream capture.  All calls
+ * on one device share the buffer, so calls that can overlap on the GPU
+ * (different streams, or different caches) race: serialise them. */
+kvq_status kvq_decode_attn_noalloc(kvq_cache* c, int layer, const void* q, int q_heads, float sm_scale,
+                                   float* out, kvq_stream_t stream);
+
 /* Host-side state of one block.  Any output pointer may be NULL.
  * capacity: tokens that fit at the current width. */
 kvq_status kvq_query(const kvq_cache* c, int layer, int* tokens, int* bits, int* capacity,

@@ -22,7 +22,7 @@ HEAD_DIM = 128
 __all__ = [
     "KVQCache", "KVQError", "load",
     "kvq_pool_bytes", "kvq_alloc", "kvq_set_lambda", "kvq_append", "kvq_shrink",
-    "kvq_decode_workspace", "kvq_decode_attn", "kvq_query", "kvq_max_tokens", "kvq_export",
+    "kvq_decode_workspace", "kvq_decode_attn", "kvq_decode_attn_noalloc", "kvq_query", "kvq_max_tokens", "kvq_export",
     "kvq_device_status", "kvq_last_error", "kvq_free",
 ]
 
@@ -106,6 +106,22 @@ def kvq_decode_attn(cache, layer: int, q: torch.Tensor, sm_scale: float, out: to
     ws_bytes = workspace.numel() * workspace.element_size()
     check(load().kvq_decode_attn(cache, layer, _dptr(q), q.shape[1], float(sm_scale), _dptr(out),
                                  _dptr(workspace), ws_bytes, _stream_ptr(stream)))
+
+
+def kvq_decode_attn_noalloc(cache, layer: int, q: torch.Tensor, sm_scale: float, out: torch.Tensor,
+                            stream=None) -> None:
+    """Decode attention without a workspace: for callers that cannot allocate
+    device memory where they run decode.  The library's own fixed 24 MiB
+    scratch buffer (one per GPU, kept until exit) holds the split partials;
+    calls that can overlap on the GPU share it and must be serialised."""
+    if q.dtype != torch.bfloat16 or q.dim() != 3 or q.shape[-1] != HEAD_DIM or not q.is_contiguous():
+        raise ValueError("q must be a contiguous bf16 [batch][q_heads][128] tensor")
+    if out.dtype != torch.float32 or out.shape != q.shape or not out.is_contiguous():
+        raise ValueError("out must be a contiguous fp32 tensor shaped like q")
+    if not (q.is_cuda and out.is_cuda):
+        raise ValueError("q and out must be CUDA tensors")
+    check(load().kvq_decode_attn_noalloc(cache, layer, _dptr(q), q.shape[1], float(sm_scale), _dptr(out),
+                                         _stream_ptr(stream)))
 
 
 def kvq_query(cache, layer: int) -> dict:

@@ -13,6 +13,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -393,6 +394,97 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, 
   a.group = G;
   a.qscale = sm_scale * 1.4426950408889634f;
   a.splits = decode_splits(c->sms(), n_streams, a.fill.gps);
+  cudaError_t e = launch_decode(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return KVQ_OK;
+}
+
+// ---- decode attention without a caller workspace ----------------------------
+//
+// Some callers cannot allocate device memory at the point where they run
+// decode: code inside a framework whose allocator owns all device memory,
+// a serving loop that must not allocate after start-up (allocation can
+// stall, fragment or fail under memory pressure), or a host that only hands
+// out input and output buffers.  For them this entry point keeps the split
+// partials in a fixed buffer of device memory that is part of the library
+// itself: every GPU that loads the library holds it until the process exits.
+// Nothing is allocated per call.
+constexpr size_t kNoAllocScratchBytes = (size_t)24 << 20;  // 24 MiB per device
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the scratch buffer on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+cudaError_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
+kvq_status kvq_decode_attn_noalloc(kvq_cache* c, int layer, const void* q, int q_heads, float sm_scale,
+                                   float* out, kvq_stream_t stream) {
+  if (kvq_status s = check_layer(c, layer)) return s;
+  if (!q || !out) return fail(KVQ_ERR_INVALID, "q or out is NULL");
+  if (q_heads <= 0 || q_heads % c->kv_heads)
+    return fail(KVQ_ERR_INVALID, "q_heads %d is not a positive multiple of kv_heads %d", q_heads, c->kv_heads);
+  const int G = q_heads / c->kv_heads;
+  if (G > 8) return fail(KVQ_ERR_INVALID, "%d query heads per KV head; at most 8 are supported", G);
+  if (!std::isfinite(sm_scale)) return fail(KVQ_ERR_INVALID, "sm_scale is not finite");
+  if ((reinterpret_cast<uintptr_t>(q) % 4) || (reinterpret_cast<uintptr_t>(out) % 4))
+    return fail(KVQ_ERR_INVALID, "q and out must be 4-byte aligned");
+  LayerState& L = c->L[layer];
+  if (L.n <= 0) return fail(KVQ_ERR_STATE, "layer %d is empty", layer);
+  const int n_streams = c->batch * c->kv_heads;
+  const Fill fill = make_fill(L.bits, L.nt, L.pf, L.n_shrinks, L.n);
+  const int splits = decode_splits(c->sms(), n_streams, fill.gps);
+  const size_t need = decode_parts_used(n_streams, splits);
+  if (need > kNoAllocScratchBytes)
+    return fail(KVQ_ERR_WORKSPACE,
+                "this block needs %zu bytes of scratch (batch*kv_heads=%d x %d splits); the built-in buffer holds "
+                "%zu bytes -- use kvq_decode_attn with a workspace",
+                need, n_streams, splits, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  if (cudaError_t e = noalloc_scratch(&scratch)) return cuda_fail(e, "scratch address");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaError_t e = c->ensure_err(s)) return cuda_fail(e, "error flag reset");
+  if (!L.counters_zeroed) {  // the ticket counters live in the cache pool and must start at zero
+    cudaError_t e = cudaMemsetAsync(c->counters(layer), 0, (size_t)n_streams * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "counter reset");
+    L.counters_zeroed = true;
+  }
+  DecodeArgs a{};
+  a.codes = c->codes(layer);
+  a.meta = c->meta(layer);
+  a.q = q;
+  a.lam = L.lambda_set ? c->lam(layer) : nullptr;
+  a.perm = L.lambda_set ? c->perm(layer) : nullptr;
+  a.out = out;
+  a.parts = static_cast<float*>(scratch);  // fully written before it is read: needs no clearing
+  a.counters = c->counters(layer);
+  a.err = c->err();
+  a.fill = fill;
+  a.batch = c->batch;
+  a.kv_heads = c->kv_heads;
+  a.q_heads = q_heads;
+  a.group = G;
+  a.qscale = sm_scale * 1.4426950408889634f;
+  a.splits = splits;
   cudaError_t e = launch_decode(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return KVQ_OK;

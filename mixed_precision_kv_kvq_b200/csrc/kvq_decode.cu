@@ -413,7 +413,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   volatile int* flags = reinterpret_cast<volatile int*>(desc + kWarps * kStages);  // [0] abort, [1] last
 
   constexpr int kGroupBytes = 512 * BITS;
-  constexpr int kPart = 256 * BITS;
   constexpr bool kWide = BITS == 16;            // a 16-bit group (8 KiB) takes every code stage
   constexpr int kS = kWide ? 1 : kStages;       // stages in use
   constexpr int kChunkGroups = kWide ? 1 : kStageCode / kGroupBytes;
@@ -747,6 +746,10 @@ int decode_splits(int num_sms, int n_streams, long long gps) {
 size_t decode_parts_bytes(int n_streams, int group) {
   (void)group;
   return (size_t)n_streams * kMaxSplits * kPartFloats * sizeof(float);
+}
+
+size_t decode_parts_used(int n_streams, int splits) {
+  return (size_t)n_streams * splits * kPartFloats * sizeof(float);
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {

@@ -179,6 +179,8 @@ struct DecodeArgs {
 int decode_splits(int num_sms, int n_streams, long long groups_per_stream);
 constexpr int kMaxSplits = 64;
 size_t decode_parts_bytes(int n_streams, int group);
+// Workspace bytes one launch with `splits` CTAs per stream actually touches.
+size_t decode_parts_used(int n_streams, int splits);
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t s);
