@@ -35,6 +35,8 @@ __device__ __forceinline__ float warp_max(float x) {
 
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs a) {
   __shared__ uint16_t codes_sh[kWarpsPerBlock][kHeadDim];
+  pdl_wait();  // k/v and the cache may come from earlier kernels in the stream
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
   const long long w = (long long)blockIdx.x * kWarpsPerBlock + wib;
@@ -157,8 +159,7 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
   const long long warps = (long long)a.batch * a.cnt * a.kv_heads * 2;
   if (warps <= 0) return cudaSuccess;
   const long long blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  append_kernel<<<(unsigned)blocks, kWarpsPerBlock * 32, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(append_kernel, dim3((unsigned)blocks), dim3(kWarpsPerBlock * 32), 0, s, a);
 }
 
 }  // namespace kvq

@@ -439,6 +439,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     for (int i = 0; i < kS; i++) mbar_init(bar0 + 8 * i, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  pdl_wait();  // the cache, q and the counters may be written by earlier kernels
   __syncthreads();
 
   // ---- chunk iterator: lane 0 walks its groups tile by tile and issues the
@@ -564,6 +565,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   float m0 = sm.m0, m1 = sm.m1, l0 = sm.l0, l1 = sm.l1, pz0 = sm.pz0, pz1 = sm.pz1;
   float (&o)[8][4] = sm.o;
 
+  pdl_launch_dependents();  // the next kernel may start to launch while this one merges
   // ---- merge the four warps ----
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
@@ -710,8 +712,7 @@ cudaError_t launch_bits(const DecodeArgs& a, cudaStream_t s) {
     attr_set = true;
   }
   const unsigned grid = (unsigned)(a.batch * a.kv_heads) * (unsigned)a.splits;
-  decode_kernel<BITS, LO><<<grid, kThreads, kSmemBytes, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(decode_kernel<BITS, LO>, dim3(grid), dim3(kThreads), kSmemBytes, s, a);
 }
 
 template <int BITS>

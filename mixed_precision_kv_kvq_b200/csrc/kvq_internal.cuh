@@ -182,6 +182,29 @@ size_t decode_parts_bytes(int n_streams, int group);
 // Workspace bytes one launch with `splits` CTAs per stream actually touches.
 size_t decode_parts_used(int n_streams, int splits);
 
+// Programmatic dependent launch: kernels of libkvq are launched so that the
+// next kernel in the stream may be scheduled while the previous one drains;
+// each kernel waits (griddepcontrol.wait) before it touches memory an earlier
+// kernel may have written, so results are exactly as with plain launches.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+template <typename Kernel, typename Args>
+inline cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s, const Args& args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args);
+}
+
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
