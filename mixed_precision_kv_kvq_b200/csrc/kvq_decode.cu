@@ -118,6 +118,11 @@ __device__ __forceinline__ uint32_t hfma2_u(uint32_t x, uint32_t m, uint32_t a) 
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(x), "r"(m), "r"(a));
   return d;
 }
+__device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
 __device__ __forceinline__ void mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                     uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -301,10 +306,11 @@ struct Soft {
   float o[8][4];
 };
 
-// NG consecutive groups of one stage: scores, one shared running-max update,
-// probabilities, then P V.  valid0: valid tokens from the first group on.
-template <int BITS, int LO, int NG>
-__device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* ms, int gi, int valid0, int lane,
+// NG consecutive groups of one stage (cs, ms point at the first): scores,
+// one shared running-max update, probabilities, then P V.  valid0: valid
+// tokens from the first group on (FULL: all NG groups are full).
+template <int BITS, int LO, int NG, bool FULL>
+__device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* ms, int valid0, int lane,
                                                const uint4* qfl, float sig0, float sig1, float kscale, Soft& st) {
   constexpr int kGroupBytes = 512 * BITS, kPart = 256 * BITS;
   const int g = lane >> 2;
@@ -312,48 +318,54 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
   const uint32_t* vu[NG];
 #pragma unroll
   for (int n = 0; n < NG; n++) {
-    ku[n] = reinterpret_cast<const uint32_t*>(cs + (gi + n) * kGroupBytes + lane * unit_bytes(BITS));
-    vu[n] = reinterpret_cast<const uint32_t*>(cs + (gi + n) * kGroupBytes + kPart + lane * unit_bytes(BITS));
+    ku[n] = reinterpret_cast<const uint32_t*>(cs + n * kGroupBytes + lane * unit_bytes(BITS));
+    vu[n] = reinterpret_cast<const uint32_t*>(cs + n * kGroupBytes + kPart + lane * unit_bytes(BITS));
   }
   float d[NG][4];
   qk_groups<BITS, LO, NG>(ku, qfl, d);
-  float s[NG][4], rv[NG][2], zv[NG][2];
-  bool partial = false;
+  // Scores relative to the running max: x = R k-scale d + (Z sum(q') - m).
+  // Before the first group m is -inf; scores are then taken relative to 0.
+  const float me0 = st.m0 == -INFINITY ? 0.f : st.m0, me1 = st.m1 == -INFINITY ? 0.f : st.m1;
+  float x[NG][4], zv[NG][2];
+  uint32_t rv2[NG][2];  // (R^V, R^V) of tokens g and g+8 as half2
 #pragma unroll
   for (int n = 0; n < NG; n++) {
-    const uint2 mga = ms[(gi + n) * 16 + g], mgb = ms[(gi + n) * 16 + g + 8];
+    const uint2 mga = ms[n * 16 + g], mgb = ms[n * 16 + g + 8];
     const float2 ka = __half22float2(*reinterpret_cast<const __half2*>(&mga.x));
     const float2 kb = __half22float2(*reinterpret_cast<const __half2*>(&mgb.x));
-    const float2 va = __half22float2(*reinterpret_cast<const __half2*>(&mga.y));
-    const float2 vb = __half22float2(*reinterpret_cast<const __half2*>(&mgb.y));
     const float rka = ka.x * kscale, rkb = kb.x * kscale;
-    s[n][0] = fmaf(rka, d[n][0], ka.y * sig0);  // token g,   head 2t
-    s[n][1] = fmaf(rka, d[n][1], ka.y * sig1);  // token g,   head 2t+1
-    s[n][2] = fmaf(rkb, d[n][2], kb.y * sig0);  // token g+8, head 2t
-    s[n][3] = fmaf(rkb, d[n][3], kb.y * sig1);  // token g+8, head 2t+1
-    rv[n][0] = va.x; zv[n][0] = va.y;
-    rv[n][1] = vb.x; zv[n][1] = vb.y;
-    partial |= valid0 - 16 * n < 16;
+    x[n][0] = fmaf(rka, d[n][0], fmaf(ka.y, sig0, -me0));  // token g,   head 2t
+    x[n][1] = fmaf(rka, d[n][1], fmaf(ka.y, sig1, -me1));  // token g,   head 2t+1
+    x[n][2] = fmaf(rkb, d[n][2], fmaf(kb.y, sig0, -me0));  // token g+8, head 2t
+    x[n][3] = fmaf(rkb, d[n][3], fmaf(kb.y, sig1, -me1));  // token g+8, head 2t+1
+    zv[n][0] = __high2float(*reinterpret_cast<const __half2*>(&mga.y));
+    zv[n][1] = __high2float(*reinterpret_cast<const __half2*>(&mgb.y));
+    rv2[n][0] = __byte_perm(mga.y, 0, 0x1010);  // low half twice
+    rv2[n][1] = __byte_perm(mgb.y, 0, 0x1010);
   }
-  if (partial) {  // warp-uniform: only the last group of a stream's partial tile
+  if constexpr (!FULL) {
+    if (valid0 < 16 * NG) {  // warp-uniform: only the last group of a stream's partial tile
 #pragma unroll
-    for (int n = 0; n < NG; n++) {
-      const int valid = valid0 - 16 * n;
-      if (g >= valid) {
-        s[n][0] = s[n][1] = -INFINITY;
-        rv[n][0] = zv[n][0] = 0.f;
-      }
-      if (g + 8 >= valid) {
-        s[n][2] = s[n][3] = -INFINITY;
-        rv[n][1] = zv[n][1] = 0.f;
+      for (int n = 0; n < NG; n++) {
+        const int valid = valid0 - 16 * n;
+        if (g >= valid) {
+          x[n][0] = x[n][1] = -INFINITY;
+          rv2[n][0] = 0u;
+          zv[n][0] = 0.f;
+        }
+        if (g + 8 >= valid) {
+          x[n][2] = x[n][3] = -INFINITY;
+          rv2[n][1] = 0u;
+          zv[n][1] = 0.f;
+        }
       }
     }
   }
-  float mx0 = fmaxf(s[0][0], s[0][2]), mx1 = fmaxf(s[0][1], s[0][3]);
+  float mx0 = fmaxf(x[0][0], x[0][2]), mx1 = fmaxf(x[0][1], x[0][3]);
 #pragma unroll
   for (int n = 1; n < NG; n++) {
-    mx0 = fmaxf(mx0, fmaxf(s[n][0], s[n][2]));
-    mx1 = fmaxf(mx1, fmaxf(s[n][1], s[n][3]));
+    mx0 = fmaxf(mx0, fmaxf(x[n][0], x[n][2]));
+    mx1 = fmaxf(mx1, fmaxf(x[n][1], x[n][3]));
   }
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
@@ -362,9 +374,11 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
   }
   // Lazy rebase: the running max moves only when a score exceeds it by more
   // than kRebase (log2 units), so p = 2^(s - m) <= 2^kRebase.
-  const float n0 = fmaxf(st.m0, mx0), n1 = fmaxf(st.m1, mx1);
-  if (__any_sync(0xffffffffu, (mx0 > st.m0 + kRebase) | (mx1 > st.m1 + kRebase))) {
-    const float a0 = ex2(st.m0 - n0), a1 = ex2(st.m1 - n1);
+  if (__any_sync(0xffffffffu, (mx0 > kRebase) | (mx1 > kRebase) | (st.m0 == -INFINITY) | (st.m1 == -INFINITY))) {
+    // new max = old max + shift (exact for the first group: relative to 0)
+    const float d0 = st.m0 == -INFINITY ? mx0 : fmaxf(mx0, 0.f);
+    const float d1 = st.m1 == -INFINITY ? mx1 : fmaxf(mx1, 0.f);
+    const float a0 = ex2(-d0), a1 = ex2(-d1);  // 0 when the old max was -inf (o, l, pz are 0 then)
 #pragma unroll
     for (int sb = 0; sb < 8; sb++) {
       st.o[sb][0] *= a0; st.o[sb][2] *= a0;
@@ -372,20 +386,26 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
     }
     st.l0 *= a0; st.pz0 *= a0;
     st.l1 *= a1; st.pz1 *= a1;
-    st.m0 = n0;
-    st.m1 = n1;
+    st.m0 = me0 + d0;
+    st.m1 = me1 + d1;
+#pragma unroll
+    for (int n = 0; n < NG; n++) {
+      x[n][0] -= d0; x[n][2] -= d0;
+      x[n][1] -= d1; x[n][3] -= d1;
+    }
   }
   uint32_t b0[NG], b1[NG];
 #pragma unroll
   for (int n = 0; n < NG; n++) {
-    const float p00 = ex2(s[n][0] - st.m0), p01 = ex2(s[n][1] - st.m1);
-    const float p10 = ex2(s[n][2] - st.m0), p11 = ex2(s[n][3] - st.m1);
+    const float p00 = ex2(x[n][0]), p01 = ex2(x[n][1]);
+    const float p10 = ex2(x[n][2]), p11 = ex2(x[n][3]);
     st.l0 += p00 + p10;
     st.l1 += p01 + p11;
     st.pz0 = fmaf(p00, zv[n][0], fmaf(p10, zv[n][1], st.pz0));
     st.pz1 = fmaf(p01, zv[n][0], fmaf(p11, zv[n][1], st.pz1));
-    b0[n] = movmatrix_t(pack_h2(p00 * rv[n][0], p01 * rv[n][0]));  // tokens 2t, 2t+1 of head g
-    b1[n] = movmatrix_t(pack_h2(p10 * rv[n][1], p11 * rv[n][1]));  // tokens 2t+8, 2t+9
+    // P = p R^V in fp16, transposed to the B fragment (tokens 2t, 2t+1 / 2t+8, 2t+9 of head g)
+    b0[n] = movmatrix_t(hmul2_u(pack_h2(p00, p01), rv2[n][0]));
+    b1[n] = movmatrix_t(hmul2_u(pack_h2(p10, p11), rv2[n][1]));
   }
   pv_groups<BITS, NG>(vu, b0, b1, st.o);
 }
@@ -553,13 +573,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     if (!mbar_wait(bar0 + 8 * st, parity, a.err, flags)) break;
     const uint8_t* cs = my.code[st];
     const uint2* ms = reinterpret_cast<const uint2*>(my.meta[st]);
-    int gi = 0;
-    if constexpr (kChunkGroups >= 2) {
-      for (; gi + 2 <= dsc.x; gi += 2)
-        process_groups<BITS, LO, 2>(cs, ms, gi, dsc.y - 16 * gi, lane, qfl, sig0, sig1, kKScale, sm);
+    if (dsc.x == kChunkGroups && dsc.y >= 16 * kChunkGroups) {
+      // full chunk: fixed offsets, no masking
+      constexpr int kNG = kChunkGroups >= 2 ? 2 : 1;
+#pragma unroll 1
+      for (int gi = 0; gi < kChunkGroups; gi += kNG)
+        process_groups<BITS, LO, kNG, true>(cs + gi * kGroupBytes, ms + gi * 16, 16 * kNG, lane, qfl, sig0, sig1,
+                                            kKScale, sm);
+    } else {
+      for (int gi = 0; gi < dsc.x; gi++)
+        process_groups<BITS, LO, 1, false>(cs + gi * kGroupBytes, ms + gi * 16, dsc.y - 16 * gi, lane, qfl, sig0,
+                                           sig1, kKScale, sm);
     }
-    for (; gi < dsc.x; gi++)
-      process_groups<BITS, LO, 1>(cs, ms, gi, dsc.y - 16 * gi, lane, qfl, sig0, sig1, kKScale, sm);
     __syncwarp();  // every lane is done with this stage before lane 0 refills it
   }
   float m0 = sm.m0, m1 = sm.m1, l0 = sm.l0, l1 = sm.l1, pz0 = sm.pz0, pz1 = sm.pz1;
