@@ -77,6 +77,36 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def source_digest():
+    """sha256 of the decode kernel's sources: ncu counters stay valid only
+    while it matches the digest recorded with them."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("kvq_decode.cu", "kvq_internal.cuh"):
+        with open(os.path.join(ROOT, "mixed_precision_kv_kvq_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def decode_traffic(fbit):
+    """DRAM bytes per decode launch (ncu dram__bytes_read.sum +
+    dram__bytes_write.sum, averaged over the layers' bit widths) from the
+    committed profile summary, or None when the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", "decode_kernel_7b_b16_t32k.md")
+    try:
+        with open(path) as f:
+            line = next(l for l in f if l.startswith("traffic-json: "))
+        rec = json.loads(line[len("traffic-json: "):])
+    except (OSError, StopIteration, ValueError):
+        return None, "no ncu summary"
+    if rec.get("source_digest") != source_digest():
+        return None, "kernel changed since the ncu capture"
+    per = rec["bytes_per_launch"]
+    if not all(f"{b}bit" in per for b in fbit):
+        return None, "no capture for some bit width"
+    return int(sum(per[f"{b}bit"] for b in fbit) / len(fbit)), "profiles/decode_kernel_7b_b16_t32k.md"
+
+
 def calib_lambda(k):
     """Migration factor from the first chunk of a block's keys (the note's
     calibration rule lambda_i = (max_m |K_m,i|)^alpha, alpha = 1/2)."""
@@ -238,8 +268,8 @@ def run_gpu(args, rank, world):
     layers = args.layers
     fbit = FBIT7 if layers == L7 else [4 if l % 2 == 1 else 2 for l in range(layers)]
     K, W = args.steps, args.warmup
-    if K + W > ROOM:
-        raise SystemExit(f"--steps + --warmup must be <= {ROOM}")
+    if 3 * K + W > ROOM:
+        raise SystemExit(f"3 * --steps + --warmup must be <= {ROOM}")
     n_f = T7 + ROOM
     n_out = S.outliers_for(HKV7)
     seed = SEED + 1000 * rank
@@ -247,7 +277,7 @@ def run_gpu(args, rank, world):
     sm_scale = HEAD_DIM ** -0.5
 
     # per-step inputs, generated up front on the device
-    nsteps = K + W
+    nsteps = 2 * K + W  # warm-up, timed steps, per-launch-event steps
     g = torch.Generator(device=dev)
     g.manual_seed(seed + 7)
     kin = torch.randn((nsteps, layers, B7, 1, HKV7, HEAD_DIM), generator=g, device=dev).to(torch.bfloat16)
@@ -302,7 +332,8 @@ def run_gpu(args, rank, world):
     t0_tokens = cache.query(0)["tokens"]
 
     # ---- timed region (device-only inputs) ----
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(layers)] for _ in range(K)]
+    # No events between launches here: an event record between two kernels
+    # would break the programmatic dependent launch of append -> decode.
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
@@ -311,24 +342,42 @@ def run_gpu(args, rank, world):
         torch.cuda.nvtx.range_push("timed")
         e_start.record(stream)
         for i in range(K):
-            step(W + i, evs[i])
+            step(W + i)
         e_end.record(stream)
         torch.cuda.synchronize(dev)
         torch.cuda.nvtx.range_pop()
     cache.device_status()
     total_ms = e_start.elapsed_time(e_end)
-    dec_ms = sum(evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(K) for l in range(layers))
-    tot_bytes, dec_bytes = 0, 0
+    tot_bytes = 0
     for i in range(K):
-        tb, db = bytes_of_step(t0_tokens + i)
-        tot_bytes += tb
-        dec_bytes += db
+        tot_bytes += bytes_of_step(t0_tokens + i)[0]
     if world > 1:
         t = torch.tensor([total_ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         total_ms = float(t.item())
     value = world * tot_bytes / (total_ms / 1e3) / 1e9
     launches = K * layers * 2
+
+    # ---- per-launch decode durations: the same step again, K more times,
+    # with CUDA events on the launch stream around every decode launch ----
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(layers)] for _ in range(K)]
+    t1_tokens = cache.query(0)["tokens"]
+    torch.cuda.synchronize(dev)
+    r_start, r_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    r_start.record(stream)
+    for i in range(K):
+        step(W + K + i, evs[i])
+    r_end.record(stream)
+    torch.cuda.synchronize(dev)
+    cache.device_status()
+    dec_ms = sum(evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(K) for l in range(layers))
+    dec_ms_bits = {}
+    dec_bytes = 0
+    for i in range(K):
+        dec_bytes += bytes_of_step(t1_tokens + i)[1]
+        for l in range(layers):
+            dec_ms_bits.setdefault(fbit[l], []).append(evs[i][l][0].elapsed_time(evs[i][l][1]))
+    ev_step_ms = r_start.elapsed_time(r_end) / K
 
     # ---- e2e: the same step through the public API with host buffers ----
     e2e = None
@@ -337,7 +386,7 @@ def run_gpu(args, rank, world):
         vh = vin.cpu().pin_memory()
         qh = qin.cpu().pin_memory()
         oh = torch.empty((layers, B7, HQ7, HEAD_DIM), dtype=torch.float32).pin_memory()
-        E = min(K, ROOM - K - W)
+        E = min(K, ROOM - 2 * K - W)
         if E > 0:
             torch.cuda.synchronize(dev)
             if world > 1:
@@ -367,11 +416,17 @@ def run_gpu(args, rank, world):
     # ---- roofline of the decode kernel ----
     peak, peak_kind = peaks()
     achieved = dec_bytes / (dec_ms / 1e3) / 1e9
+    n_dec = K * layers
+    traffic, traffic_src = decode_traffic(fbit)
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs (copy)",
-            "traffic": None, "kernel": "decode_kernel (kvq_decode_attn)",
-            "avg_launch_us": round(dec_ms * 1e3 / (K * layers), 2),
-            "bytes_per_launch": int(dec_bytes / (K * layers))}
+            "traffic": traffic, "traffic_source": traffic_src,
+            "kernel": "decode_kernel (kvq_decode_attn)",
+            "avg_launch_us": round(dec_ms * 1e3 / n_dec, 2),
+            "bytes_per_launch": int(dec_bytes / n_dec),
+            "per_bits_us": {f"{b}bit": round(statistics.mean(v) * 1e3, 2) for b, v in sorted(dec_ms_bits.items())},
+            "timing": f"CUDA events around each of {n_dec} decode launches ({K} more steps after the timed "
+                      f"ones; {ev_step_ms:.4f} ms/step with the events)"}
 
     extra = {}
     if not args.no_shrink and rank == 0:
@@ -389,7 +444,7 @@ def run_gpu(args, rank, world):
         "config": {"workload": WORKLOAD, "layers": layers, "batch": B7, "q_heads": HQ7, "kv_heads": HKV7,
                    "head_dim": HEAD_DIM, "context": T7, "fbit": fbit, "parallelism": f"replicas x{world}",
                    "l2": "no flush: every block's cache read (151-285 MB) exceeds the 126 MB L2",
-                   "decode_ms_share": round(dec_ms / total_ms, 3)},
+                   "decode_ms_share": round(dec_ms / (ev_step_ms * K), 3)},
         "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
         **extra,
     }
