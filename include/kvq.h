@@ -109,8 +109,8 @@ size_t kvq_decode_workspace(const kvq_cache* c, int layer, int q_heads);
 /* GQA decode attention over the block's quantized cache:
  *   out[b][h] = sum_t softmax_t(sm_scale * (q[b][h] * lambda) . k^_t) v^_t
  * over every cached token, query head h reading KV head h / (q_heads /
- * kv_heads).  q: device bf16 [batch][q_heads][128]; out: device fp32
- * [batch][q_heads][128]; workspace: device buffer of at least
+ * kv_heads).  q: device bf16 [batch][q_heads][128], 16-byte aligned; out:
+ * device fp32 [batch][q_heads][128]; workspace: device buffer of at least
  * kvq_decode_workspace(c, layer, q_heads) bytes (contents need no
  * initialisation; the call owns it until it completes on the stream).
  * q_heads must be a multiple of kv_heads with at most 8 query heads per KV

@@ -362,8 +362,8 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, 
   const int G = q_heads / c->kv_heads;
   if (G > 8) return fail(KVQ_ERR_INVALID, "%d query heads per KV head; at most 8 are supported", G);
   if (!std::isfinite(sm_scale)) return fail(KVQ_ERR_INVALID, "sm_scale is not finite");
-  if ((reinterpret_cast<uintptr_t>(q) % 4) || (reinterpret_cast<uintptr_t>(out) % 4))
-    return fail(KVQ_ERR_INVALID, "q and out must be 4-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(q) % 16) || (reinterpret_cast<uintptr_t>(out) % 4))
+    return fail(KVQ_ERR_INVALID, "q must be 16-byte aligned and out 4-byte aligned");
   LayerState& L = c->L[layer];
   if (L.n <= 0) return fail(KVQ_ERR_STATE, "layer %d is empty", layer);
   const int n_streams = c->batch * c->kv_heads;
@@ -446,8 +446,8 @@ kvq_status kvq_decode_attn_noalloc(kvq_cache* c, int layer, const void* q, int q
   const int G = q_heads / c->kv_heads;
   if (G > 8) return fail(KVQ_ERR_INVALID, "%d query heads per KV head; at most 8 are supported", G);
   if (!std::isfinite(sm_scale)) return fail(KVQ_ERR_INVALID, "sm_scale is not finite");
-  if ((reinterpret_cast<uintptr_t>(q) % 4) || (reinterpret_cast<uintptr_t>(out) % 4))
-    return fail(KVQ_ERR_INVALID, "q and out must be 4-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(q) % 16) || (reinterpret_cast<uintptr_t>(out) % 4))
+    return fail(KVQ_ERR_INVALID, "q must be 16-byte aligned and out 4-byte aligned");
   LayerState& L = c->L[layer];
   if (L.n <= 0) return fail(KVQ_ERR_STATE, "layer %d is empty", layer);
   const int n_streams = c->batch * c->kv_heads;

@@ -367,14 +367,16 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
     mx0 = fmaxf(mx0, fmaxf(x[n][0], x[n][2]));
     mx1 = fmaxf(mx1, fmaxf(x[n][1], x[n][3]));
   }
-#pragma unroll
-  for (int off = 4; off < 32; off <<= 1) {
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-  }
   // Lazy rebase: the running max moves only when a score exceeds it by more
-  // than kRebase (log2 units), so p = 2^(s - m) <= 2^kRebase.
-  if (__any_sync(0xffffffffu, (mx0 > kRebase) | (mx1 > kRebase) | (st.m0 == -INFINITY) | (st.m1 == -INFINITY))) {
+  // than kRebase (log2 units), so p = 2^(s - m) <= 2^kRebase.  Whether any
+  // lane needs it is one vote; the maxima over the tokens are only formed
+  // when it does.
+  if (__any_sync(0xffffffffu, (fmaxf(mx0, mx1) > kRebase) | (st.m0 == -INFINITY))) {
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
     // new max = old max + shift (exact for the first group: relative to 0)
     const float d0 = st.m0 == -INFINITY ? mx0 : fmaxf(mx0, 0.f);
     const float d1 = st.m1 == -INFINITY ? mx1 : fmaxf(mx1, 0.f);
@@ -459,8 +461,33 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     for (int i = 0; i < kS; i++) mbar_init(bar0 + 8 * i, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  // q, lambda and the Key channel order are staged in shared memory (in warp
+  // 0's second code stage, unused until the main loop starts).  lambda and
+  // the channel order are fixed while kernels run on the block, so they are
+  // fetched before waiting for the previous kernel.
+  const int b = s / a.kv_heads, j = s - b * a.kv_heads;
+  __nv_bfloat16* s_q = reinterpret_cast<__nv_bfloat16*>(ws[0].code[kStages - 1]);  // [8][128]
+  float* s_lam = reinterpret_cast<float*>(s_q + kMaxGroup * kHeadDim);               // [128]
+  uint8_t* s_perm = reinterpret_cast<uint8_t*>(s_lam + kHeadDim);                    // [128]
+  if (warp == 1) {
+    const float4 lv = a.lam ? __ldg(reinterpret_cast<const float4*>(a.lam + (size_t)j * kHeadDim) + lane)
+                            : make_float4(1.f, 1.f, 1.f, 1.f);
+    reinterpret_cast<float4*>(s_lam)[lane] = lv;
+  } else if (warp == 2 && lane < kHeadDim / 16) {
+    uint4 pv;
+    if (a.perm) {
+      pv = __ldg(reinterpret_cast<const uint4*>(a.perm + (size_t)j * kHeadDim) + lane);
+    } else {
+      const uint32_t c0 = 16u * lane;
+      pv = make_uint4(c0 * 0x01010101u + 0x03020100u, c0 * 0x01010101u + 0x07060504u,
+                      c0 * 0x01010101u + 0x0b0a0908u, c0 * 0x01010101u + 0x0f0e0d0cu);
+    }
+    reinterpret_cast<uint4*>(s_perm)[lane] = pv;
+  }
   pdl_wait();  // the cache, q and the counters may be written by earlier kernels
-  __syncthreads();
+  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.q_heads + (size_t)j * G) * kHeadDim;
+  uint4 qv = make_uint4(0u, 0u, 0u, 0u);  // 8 bf16 of q: head threadIdx/16, channels 8 (threadIdx%16) ..
+  if ((int)threadIdx.x < G * (kHeadDim / 8)) qv = reinterpret_cast<const uint4*>(qb)[threadIdx.x];
 
   // ---- chunk iterator: lane 0 walks its groups tile by tile and issues the
   // copies; everyone reads the per-stage descriptors (groups, valid tokens) ----
@@ -506,17 +533,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   }
   __syncwarp();
 
-  // ---- q' fragments for this stream (warp 0 builds them in shared memory) ----
+  // ---- q' fragments for this stream, built in shared memory ----
   // sum(q') must be taken over exactly the q' values the MMAs use, so that
   // (R/(2^b-1)) q'.c + Z sum(q') stays the dot product of that q' with the
   // dequantised key.
   constexpr int lo_blocks = LO;
-  const int b = s / a.kv_heads, j = s - b * a.kv_heads;
+  reinterpret_cast<uint4*>(s_q)[threadIdx.x] = qv;  // heads >= G are zero
+  __syncthreads();
   {
     // warp w builds the fragments of k-blocks 2w and 2w+1
-    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.q_heads + (size_t)j * G) * kHeadDim;
-    const float* lam = a.lam ? a.lam + (size_t)j * kHeadDim : nullptr;
-    const uint8_t* pm = a.perm ? a.perm + (size_t)j * kHeadDim : nullptr;
     float part = 0.f;
 #pragma unroll
     for (int i = 0; i < 2; i++) {
@@ -524,19 +549,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
       uint32_t hq[2], lq[2];
 #pragma unroll
       for (int hf = 0; hf < 2; hf++) {
+        // Key positions c0, c0+1 hold channels ch0, ch1 of the block's order
         const int c0 = 16 * sb + 2 * t + 8 * hf;
-        float v0 = 0.f, v1 = 0.f;
-        if (g < G) {
-          // Key positions c0, c0+1 hold channels ch0, ch1 of the block's order
-          const int ch0 = pm ? pm[c0] : c0, ch1 = pm ? pm[c0 + 1] : c0 + 1;
-          const __nv_bfloat16* qr = qb + (size_t)g * kHeadDim;
-          v0 = __bfloat162float(qr[ch0]) * a.qscale;
-          v1 = __bfloat162float(qr[ch1]) * a.qscale;
-          if (lam) {
-            v0 *= lam[ch0];
-            v1 *= lam[ch1];
-          }
-        }
+        const int ch0 = s_perm[c0], ch1 = s_perm[c0 + 1];
+        const float v0 = __bfloat162float(s_q[g * kHeadDim + ch0]) * a.qscale * s_lam[ch0];
+        const float v1 = __bfloat162float(s_q[g * kHeadDim + ch1]) * a.qscale * s_lam[ch1];
         // channel block sb, half hf = pair p = 2 sb + hf of the Key units
         const float scl = kWide ? 1.0f : (float)(1 << (emax<BITS>() - pair_shift<BITS>(2 * sb + hf)));
         const __half2 h = __floats2half2_rn(v0 * scl, v1 * scl);
