@@ -529,10 +529,19 @@ kvq_status kvq_export(const kvq_cache* c, int layer, int b, int j, uint16_t* k_c
       const int g = tok & 7, x = tok >> 3;
       const uint8_t* pm = L.lambda_set ? &L.perm[(size_t)j * kHeadDim] : nullptr;
       for (int kp = 0; kp < kHeadDim; kp++) {  // Key position -> channel pm[kp]
-        const int sb = kp >> 4, rem = kp & 15, r = rem >> 3, t = (rem & 7) >> 1, mb = rem & 1;
-        const int p = 2 * sb + r, word = x * bits + p / ppw, pos = p % ppw;
+        // position 32s + 16r + 4t + i: member i of quad p = 2s + r in unit 4g + t
+        const int p = 2 * (kp >> 5) + ((kp >> 4) & 1), t = (kp >> 2) & 3, mi = kp & 3;
+        int word, shift;
+        if (bits == 16) {
+          word = x * bits + 2 * p + (mi >> 1);
+          shift = 16 * (mi & 1);
+        } else {
+          const int qpw = 8 / bits;
+          word = x * bits + p / qpw;
+          shift = 8 * mi + bits * (p % qpw);
+        }
         const uint32_t w = rd32(&cb[gbase + (size_t)(4 * g + t) * unit_bytes(bits) + 4 * word]);
-        k_codes[i * kHeadDim + (pm ? pm[kp] : kp)] = (uint16_t)((w >> (16 * mb + bits * pos)) & mask);
+        k_codes[i * kHeadDim + (pm ? pm[kp] : kp)] = (uint16_t)((w >> shift) & mask);
       }
     }
     if (v_codes) {

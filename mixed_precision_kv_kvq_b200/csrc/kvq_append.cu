@@ -108,23 +108,33 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs 
   const size_t stream = (size_t)b * a.kv_heads + j;
   uint8_t* gbase = a.codes + (stream * a.nt + tile) * (size_t)kTileBytes + (size_t)grp * group_bytes(bits) +
                    (size_t)kv * part_bytes(bits);
-  const int ppw = 16 / bits;  // pairs per 32-bit word (per 16-bit half)
 
   if (kv == 0) {
     // Token tok: g = tok % 8, x = tok / 8.  Lane units 4g + t (t = 0..3) each
-    // get `bits` words: unit word x*bits + jw holds pairs P = 16x + jw*ppw + kk.
-    // Positions map to channels through the block's Key channel order.
+    // get `bits` words of this token, unit words x*bits + jw, holding its
+    // quads Q = 8x + p, p = 2s + r: positions 32s + 16r + 4t + i (member i
+    // in byte i).  Positions map to channels through the block's Key
+    // channel order.
     const uint8_t* pm = a.perm ? a.perm + (size_t)j * kHeadDim : nullptr;
     const int g = tok & 7, xs = tok >> 3;
     for (int wi = lane; wi < 4 * bits; wi += 32) {
       const int t = wi / bits, jw = wi - t * bits;
       uint32_t word = 0;
-      for (int kk = 0; kk < ppw; kk++) {
-        const int p = jw * ppw + kk;  // pair within the token's half: p = 2s + rr
-        const int pos0 = 16 * (p >> 1) + 2 * t + 8 * (p & 1);
-        const int c0 = pm ? pm[pos0] : pos0, c1 = pm ? pm[pos0 + 1] : pos0 + 1;
-        word |= (uint32_t)sc[c0] << (bits * kk);
-        word |= (uint32_t)sc[c1] << (16 + bits * kk);
+      if (bits == 16) {  // half a quad: members 2(jw%2), 2(jw%2)+1 of quad p = jw/2
+        const int p = jw >> 1;
+        const int pos = 32 * (p >> 1) + 16 * (p & 1) + 4 * t + 2 * (jw & 1);
+        word = (uint32_t)sc[pm ? pm[pos] : pos] | ((uint32_t)sc[pm ? pm[pos + 1] : pos + 1] << 16);
+      } else {
+        const int qpw = 8 / bits;  // quads per word
+        for (int kk = 0; kk < qpw; kk++) {
+          const int p = jw * qpw + kk;
+          const int pos0 = 32 * (p >> 1) + 16 * (p & 1) + 4 * t;
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            const int c = pm ? pm[pos0 + i] : pos0 + i;
+            word |= (uint32_t)sc[c] << (8 * i + bits * kk);
+          }
+        }
       }
       uint32_t* dst = reinterpret_cast<uint32_t*>(gbase + (4 * g + t) * unit_bytes(bits)) + xs * bits + jw;
       *dst = word;
@@ -134,6 +144,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs 
     // Units 4g + t (g = 0..7): word u*bits + jw, half mb, pairs p = 2s + rr of
     // channel 16s + g + 8rr.
     const int t = (tok & 7) >> 1, mb = tok & 1, u = tok >> 3;
+    const int ppw = 16 / bits;  // pairs per 32-bit word (per 16-bit half)
     for (int hw = lane; hw < 8 * bits; hw += 32) {
       const int g = hw / bits, jw = hw - g * bits;
       uint32_t half = 0;

@@ -9,17 +9,18 @@
 // query).  Dequantisation is folded out of the inner loop:
 //   q'.k^_t = (R_t / (2^b-1)) (q'.c_t) + Z_t sum(q'),
 //   sum_t p_t v^_t = (sum_t p_t R_t c_t) / (2^b-1) + sum_t p_t Z_t,
-// so the raw codes go straight into mma.sync.m16n8k16 operands (fp16, exact
-// for codes < 2^11; 16-bit codes as two bytes): QK^T with A = 16 tokens x 16
-// channels of codes and B = q' (N = 8 query heads; q' is carried as a hi + lo
-// pair of fp16 values, two MMAs on the same A registers, because one fp16
-// rounding of q' alone moves large outlier-channel scores by up to ~2^-12 of
-// their size, enough to break a 2e-3 output tolerance), PV with A = 16
-// channels x 16 tokens of V codes and B = p R (transposed from the score
-// fragment with movmatrix).  Codes are widened to fp16 in registers with the
-// 0x6400 exponent trick (integer c in the low mantissa bits of 1024.0; one
-// lop3 + one hfma2 per code pair).
-//
+// so the raw codes go straight into tensor-core operands:
+//   QK^T: int8 mma.sync.m16n8k32, A = 16 tokens x 32 Key positions of codes
+//   (byte quads, each code moved to the top of its byte: c 2^(8-b), exact in
+//   u8), B = the query as an exact per-head int16, q' = s_h (256 hi + lo)
+//   with hi s8 and lo u8, two MMAs on the same A registers, int32
+//   accumulation (no rounding until one int -> float conversion per score);
+//   PV: fp16 mma.sync.m16n8k16, A = 16 channels x 16 tokens of V codes
+//   widened in registers with the 0x6400 exponent trick (integer c in the
+//   low mantissa bits of 1024.0; one lop3 + one sub.f16x2 per code pair),
+//   B = p R (transposed from the score fragment with movmatrix).
+// 16-bit codes go in as two bytes (Keys) or two fp16 halves (Values).
+
 // Work split: each stream is cut into `splits` equal slices of 16-token
 // groups, one CTA per slice (the host picks `splits` so the grid fills the
 // GPU in whole waves).  The CTA's four warps take contiguous quarters of the
@@ -47,8 +48,8 @@ constexpr int kStageMeta = 512;            // meta bytes per stage (128 per grou
 constexpr int kWarpSmem = kStages * (kStageCode + kStageMeta);
 constexpr int kMaxGroup = 8;               // query heads per KV head (MMA N)
 constexpr int kCtasPerSm = 4;
-constexpr int kQfBytes = 8 * 32 * 16;      // q' B fragments: [s-block][lane] x (hi b0, hi b1, lo b0, lo b1)
-constexpr int kSmemBytes = kWarps * kWarpSmem + kQfBytes + kMaxGroup * 4 + 3 * kWarps * kMaxGroup * 4 +
+constexpr int kQfBytes = 4 * 32 * 16;      // q' B fragments: [k-block][lane] x (hi b0, hi b1, lo b0, lo b1)
+constexpr int kSmemBytes = kWarps * kWarpSmem + kQfBytes + 3 * kWarps * kMaxGroup * 4 +
                            kWarps * kStages * 8 + kWarps * kStages * 8 + 16;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
 constexpr int kPartFloats = 2 * kMaxGroup + kHeadDim * kMaxGroup;  // one CTA's partial record
@@ -131,6 +132,34 @@ __device__ __forceinline__ void mma(float (&d)[4], uint32_t a0, uint32_t a1, uin
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+// int8 MMA, A = u8 codes, B = s8 (hi byte of q') or u8 (lo byte of q').
+__device__ __forceinline__ void imma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void imma_u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// w * 2^SH as an integer multiply (keeps the shift off the logic pipe)
+template <int SH>
+__device__ __forceinline__ uint32_t shl_mul(uint32_t w) {
+  if constexpr (SH == 0) {
+    return w;
+  } else {
+    uint32_t d;
+    asm("mul.lo.u32 %0, %1, %2;" : "=r"(d) : "r"(w), "n"(1 << SH));
+    return d;
+  }
+}
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
   uint32_t d;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(x));
@@ -157,8 +186,8 @@ __host__ __device__ constexpr int field_shift() {
 // Pair at field position POS: the two codes sit at bits [BITS*POS, +BITS) of
 // each half-word.  Result: half2 (c0 * 2^e, c1 * 2^e), exact, with
 // e = field_shift: (0x6400 | c << e) is the fp16 number 1024 + c 2^e, and
-// subtracting 1024 is exact.  The 2^e is undone outside the inner loop (in
-// the q' operand for Keys, in the output rows for Values).
+// subtracting 1024 is exact.  The 2^e is undone outside the inner loop, in
+// the output rows.
 template <int BITS, int POS>
 __device__ __forceinline__ uint32_t widen(uint32_t w, uint32_t w8) {
   constexpr int kPerByte = 8 / BITS;
@@ -169,12 +198,6 @@ __device__ __forceinline__ uint32_t widen(uint32_t w, uint32_t w8) {
   uint32_t d;
   asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(x), "r"(0x64006400u));
   return d;
-}
-// Largest field shift at BITS: q' is scaled by 2^(kEmax - e) per channel so
-// every product c 2^e q' 2^(kEmax - e) carries the same factor 2^kEmax.
-template <int BITS>
-__host__ __device__ constexpr int emax() {
-  return BITS >= 8 ? 0 : 8 - BITS;
 }
 // field_shift of pair p (any p in 0..15) at BITS <= 8.
 template <int BITS>
@@ -200,59 +223,92 @@ __device__ __forceinline__ uint32_t pair_at(const uint32_t* u, const uint32_t* u
 
 // -------------------------------------------------------- group pieces
 
+// Key quads.  A quad is the 4 codes of one token at 4 consecutive Key
+// positions, one int8 A-fragment register of mma.m16n8k32; member i sits in
+// byte i of its word at the quad's field (kvq_internal.cuh).  quad_reg gives
+// the register of quad (k-block S, token half X, column half R), its codes
+// moved to the top bits of each byte: c * 2^(8 - BITS), exact in u8.
+template <int BITS, int F>
+__device__ __forceinline__ uint32_t quad_field(uint32_t w) {
+  constexpr uint32_t top = (((1u << BITS) - 1u) << (8 - BITS)) * 0x01010101u;
+  return shl_mul<8 - BITS - BITS * F>(w) & top;
+}
+template <int BITS, int S, int X, int R>
+__device__ __forceinline__ uint32_t quad_reg(const uint32_t* u) {
+  constexpr int qpw = 8 / BITS;  // quads per word
+  constexpr int Q = 8 * X + 2 * S + R;
+  return quad_field<BITS, Q % qpw>(u[Q / qpw]);
+}
+
 // Scores of NG 16-token groups: D[n][token][head] = sum over Key positions of
-// code * q' (all products carry 2^emax for BITS <= 8, 1/256 of the code for
-// BITS == 16).  The lo part of q' is added on the first LO k-blocks.  The
-// k-block loop is outermost so each q' fragment is loaded once for all
-// groups.
-template <int BITS, int LO, int NG>
+// A * q'_int, with A = c 2^(8 - BITS) (BITS <= 8) or the 16-bit code itself,
+// and q'_int = 256 hi + lo the per-head int16 query (hi: s8, lo: u8); every
+// product and sum is exact in int32.  The k-block loop is outermost so each
+// q' fragment is loaded once for all groups.
+template <int BITS, int NG>
 __device__ __forceinline__ void qk_groups(const uint32_t* const (&ku)[NG], const uint4* qfl, float (&d)[NG][4]) {
-  float dl[NG][4];
-#pragma unroll
-  for (int n = 0; n < NG; n++) d[n][0] = d[n][1] = d[n][2] = d[n][3] = dl[n][0] = dl[n][1] = dl[n][2] = dl[n][3] = 0.f;
   if constexpr (BITS == 16) {
+    int hh[NG][4], hl[NG][4], lh[NG][4], ll[NG][4];
 #pragma unroll
-    for (int sb = 0; sb < 8; sb++) {
+    for (int n = 0; n < NG; n++)
+#pragma unroll
+      for (int e = 0; e < 4; e++) hh[n][e] = hl[n][e] = lh[n][e] = ll[n][e] = 0;
+#pragma unroll
+    for (int sb = 0; sb < 4; sb++) {
       const uint4 q4 = qfl[32 * sb];
-      const uint32_t bl0 = hfma2_u(q4.x, 0x1c001c00u, 0u), bl1 = hfma2_u(q4.y, 0x1c001c00u, 0u);  // / 256
 #pragma unroll
       for (int n = 0; n < NG; n++) {
-        const uint2 w0 = *reinterpret_cast<const uint2*>(ku[n] + 2 * sb);       // token g: pairs 2s, 2s+1
-        const uint2 w1 = *reinterpret_cast<const uint2*>(ku[n] + 16 + 2 * sb);  // token g+8
-        const uint32_t h0 = widen16_hi(w0.x), h1 = widen16_hi(w1.x), h2 = widen16_hi(w0.y), h3 = widen16_hi(w1.y);
-        mma(d[n], h0, h1, h2, h3, q4.x, q4.y);
-        if (sb < LO) mma(dl[n], h0, h1, h2, h3, q4.z, q4.w);
-        mma(dl[n], widen16_lo(w0.x), widen16_lo(w1.x), widen16_lo(w0.y), widen16_lo(w1.y), bl0, bl1);
+        // quad Q = 8x + 2s + r spans words 2Q (members 0, 1) and 2Q + 1 (members 2, 3)
+        const uint2 w00 = *reinterpret_cast<const uint2*>(ku[n] + 4 * sb);            // x 0, r 0
+        const uint2 w01 = *reinterpret_cast<const uint2*>(ku[n] + 4 * sb + 2);        // x 0, r 1
+        const uint2 w10 = *reinterpret_cast<const uint2*>(ku[n] + 16 + 4 * sb);       // x 1, r 0
+        const uint2 w11 = *reinterpret_cast<const uint2*>(ku[n] + 16 + 4 * sb + 2);   // x 1, r 1
+        const uint32_t l0 = __byte_perm(w00.x, w00.y, 0x6420), h0 = __byte_perm(w00.x, w00.y, 0x7531);
+        const uint32_t l1 = __byte_perm(w10.x, w10.y, 0x6420), h1 = __byte_perm(w10.x, w10.y, 0x7531);
+        const uint32_t l2 = __byte_perm(w01.x, w01.y, 0x6420), h2 = __byte_perm(w01.x, w01.y, 0x7531);
+        const uint32_t l3 = __byte_perm(w11.x, w11.y, 0x6420), h3 = __byte_perm(w11.x, w11.y, 0x7531);
+        imma_s8(hh[n], h0, h1, h2, h3, q4.x, q4.y);
+        imma_u8(hl[n], h0, h1, h2, h3, q4.z, q4.w);
+        imma_s8(lh[n], l0, l1, l2, l3, q4.x, q4.y);
+        imma_u8(ll[n], l0, l1, l2, l3, q4.z, q4.w);
       }
     }
+#pragma unroll
+    for (int n = 0; n < NG; n++)
+#pragma unroll
+      for (int e = 0; e < 4; e++)
+        d[n][e] = 256.0f * (float)(hh[n][e] * 256 + hl[n][e]) + (float)(lh[n][e] * 256 + ll[n][e]);
   } else {
-    uint32_t u[NG][2 * BITS], u8[NG][2 * BITS];
+    uint32_t u[NG][2 * BITS];
 #pragma unroll
     for (int n = 0; n < NG; n++) {
 #pragma unroll
       for (int i = 0; i < 2 * BITS; i += 4) {
-        const uint4 q4 = *reinterpret_cast<const uint4*>(ku[n] + i);
-        u[n][i] = q4.x; u[n][i + 1] = q4.y; u[n][i + 2] = q4.z; u[n][i + 3] = q4.w;
+        const uint4 w4 = *reinterpret_cast<const uint4*>(ku[n] + i);
+        u[n][i] = w4.x; u[n][i + 1] = w4.y; u[n][i + 2] = w4.z; u[n][i + 3] = w4.w;
       }
-#pragma unroll
-      for (int i = 0; i < 2 * BITS; i++) u8[n][i] = u[n][i] >> 8;
     }
-#define KVQ_QK(S)                                                                                          \
-  {                                                                                                        \
-    const uint4 q4 = qfl[32 * S];                                                                          \
-    _Pragma("unroll") for (int n = 0; n < NG; n++) {                                                      \
-      const uint32_t a0 = pair_at<BITS, S, 0, 0>(u[n], u8[n]), a1 = pair_at<BITS, S, 1, 0>(u[n], u8[n]);   \
-      const uint32_t a2 = pair_at<BITS, S, 0, 1>(u[n], u8[n]), a3 = pair_at<BITS, S, 1, 1>(u[n], u8[n]);   \
-      mma(d[n], a0, a1, a2, a3, q4.x, q4.y);                                                               \
-      if constexpr (S < LO) mma(dl[n], a0, a1, a2, a3, q4.z, q4.w);                                        \
-    }                                                                                                      \
-  }
-    KVQ_QK(0) KVQ_QK(1) KVQ_QK(2) KVQ_QK(3) KVQ_QK(4) KVQ_QK(5) KVQ_QK(6) KVQ_QK(7)
-#undef KVQ_QK
-  }
+    int ah[NG][4], al[NG][4];
 #pragma unroll
-  for (int n = 0; n < NG; n++) {
-    d[n][0] += dl[n][0]; d[n][1] += dl[n][1]; d[n][2] += dl[n][2]; d[n][3] += dl[n][3];
+    for (int n = 0; n < NG; n++)
+#pragma unroll
+      for (int e = 0; e < 4; e++) ah[n][e] = al[n][e] = 0;
+#define KVQ_QK(S)                                                                                    \
+  {                                                                                                  \
+    const uint4 q4 = qfl[32 * S];                                                                    \
+    _Pragma("unroll") for (int n = 0; n < NG; n++) {                                                \
+      const uint32_t a0 = quad_reg<BITS, S, 0, 0>(u[n]), a1 = quad_reg<BITS, S, 1, 0>(u[n]);         \
+      const uint32_t a2 = quad_reg<BITS, S, 0, 1>(u[n]), a3 = quad_reg<BITS, S, 1, 1>(u[n]);         \
+      imma_s8(ah[n], a0, a1, a2, a3, q4.x, q4.y);                                                    \
+      imma_u8(al[n], a0, a1, a2, a3, q4.z, q4.w);                                                    \
+    }                                                                                                \
+  }
+    KVQ_QK(0) KVQ_QK(1) KVQ_QK(2) KVQ_QK(3)
+#undef KVQ_QK
+#pragma unroll
+    for (int n = 0; n < NG; n++)
+#pragma unroll
+      for (int e = 0; e < 4; e++) d[n][e] = (float)(ah[n][e] * 256 + al[n][e]);
   }
 }
 
@@ -309,9 +365,10 @@ struct Soft {
 // NG consecutive groups of one stage (cs, ms point at the first): scores,
 // one shared running-max update, probabilities, then P V.  valid0: valid
 // tokens from the first group on (FULL: all NG groups are full).
-template <int BITS, int LO, int NG, bool FULL>
+template <int BITS, int NG, bool FULL>
 __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* ms, int valid0, int lane,
-                                               const uint4* qfl, float sig0, float sig1, float kscale, Soft& st) {
+                                               const uint4* qfl, float ks0, float ks1, float sig0, float sig1,
+                                               Soft& st) {
   constexpr int kGroupBytes = 512 * BITS, kPart = 256 * BITS;
   const int g = lane >> 2;
   const uint32_t* ku[NG];
@@ -322,8 +379,9 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
     vu[n] = reinterpret_cast<const uint32_t*>(cs + n * kGroupBytes + kPart + lane * unit_bytes(BITS));
   }
   float d[NG][4];
-  qk_groups<BITS, LO, NG>(ku, qfl, d);
-  // Scores relative to the running max: x = R k-scale d + (Z sum(q') - m).
+  qk_groups<BITS, NG>(ku, qfl, d);
+  // Scores relative to the running max: x = R ks_h d + (Z sum(q'_h) - m),
+  // ks_h = (q' scale of head h) / (code scale).
   // Before the first group m is -inf; scores are then taken relative to 0.
   const float me0 = st.m0 == -INFINITY ? 0.f : st.m0, me1 = st.m1 == -INFINITY ? 0.f : st.m1;
   float x[NG][4], zv[NG][2];
@@ -333,11 +391,10 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
     const uint2 mga = ms[n * 16 + g], mgb = ms[n * 16 + g + 8];
     const float2 ka = __half22float2(*reinterpret_cast<const __half2*>(&mga.x));
     const float2 kb = __half22float2(*reinterpret_cast<const __half2*>(&mgb.x));
-    const float rka = ka.x * kscale, rkb = kb.x * kscale;
-    x[n][0] = fmaf(rka, d[n][0], fmaf(ka.y, sig0, -me0));  // token g,   head 2t
-    x[n][1] = fmaf(rka, d[n][1], fmaf(ka.y, sig1, -me1));  // token g,   head 2t+1
-    x[n][2] = fmaf(rkb, d[n][2], fmaf(kb.y, sig0, -me0));  // token g+8, head 2t
-    x[n][3] = fmaf(rkb, d[n][3], fmaf(kb.y, sig1, -me1));  // token g+8, head 2t+1
+    x[n][0] = fmaf(ka.x * ks0, d[n][0], fmaf(ka.y, sig0, -me0));  // token g,   head 2t
+    x[n][1] = fmaf(ka.x * ks1, d[n][1], fmaf(ka.y, sig1, -me1));  // token g,   head 2t+1
+    x[n][2] = fmaf(kb.x * ks0, d[n][2], fmaf(kb.y, sig0, -me0));  // token g+8, head 2t
+    x[n][3] = fmaf(kb.x * ks1, d[n][3], fmaf(kb.y, sig1, -me1));  // token g+8, head 2t+1
     zv[n][0] = __high2float(*reinterpret_cast<const __half2*>(&mga.y));
     zv[n][1] = __high2float(*reinterpret_cast<const __half2*>(&mgb.y));
     rv2[n][0] = __byte_perm(mga.y, 0, 0x1010);  // low half twice
@@ -419,15 +476,12 @@ struct WarpSmem {
   uint8_t meta[kStages][kStageMeta];
 };
 
-// LO: k-blocks that get the extra-precision q' term -- 1 when the Key
-// channels are ordered by lambda (outlier channels in k-block 0), else 8.
-template <int BITS, int LO>
+template <int BITS>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   WarpSmem* ws = reinterpret_cast<WarpSmem*>(smem);
   uint4* qf = reinterpret_cast<uint4*>(smem + kWarps * kWarpSmem);     // [8][32]
-  float* sig = reinterpret_cast<float*>(qf + 8 * 32);                 // [8] sum of q' per head
-  float* w_m = sig + kMaxGroup;                                        // [warps][8]
+  float* w_m = reinterpret_cast<float*>(qf + 4 * 32);                 // [warps][8]
   float* w_l = w_m + kWarps * kMaxGroup;
   float* w_pz = w_l + kWarps * kMaxGroup;
   uint64_t* bars = reinterpret_cast<uint64_t*>(w_pz + kWarps * kMaxGroup);  // [warps][stages]
@@ -439,7 +493,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   constexpr int kS = kWide ? 1 : kStages;       // stages in use
   constexpr int kChunkGroups = kWide ? 1 : kStageCode / kGroupBytes;
   constexpr float kCScale = (BITS == 16 ? 256.0f : 1.0f) / (float)((1u << BITS) - 1u);
-  constexpr float kKScale = kCScale / (float)(1 << emax<BITS>());  // QK products carry 2^emax
+  // QK products carry the code as A = c 2^(8 - BITS) (BITS <= 8) or c (16)
+  constexpr float kKCode = 1.0f / ((float)((1u << BITS) - 1u) * (float)(BITS >= 8 ? 1 : 1 << (8 - BITS)));
 
   const Fill f = a.fill;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -456,7 +511,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     flags[0] = 0;
     flags[1] = 0;
   }
-  if (threadIdx.x < kMaxGroup) sig[threadIdx.x] = 0.f;
   if (lane == 0) {
     for (int i = 0; i < kS; i++) mbar_init(bar0 + 8 * i, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -533,45 +587,71 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   }
   __syncwarp();
 
-  // ---- q' fragments for this stream, built in shared memory ----
-  // sum(q') must be taken over exactly the q' values the MMAs use, so that
-  // (R/(2^b-1)) q'.c + Z sum(q') stays the dot product of that q' with the
+  // ---- q' for this stream: exact int16 per head, as int8 MMA B fragments ----
+  // q'_h = q_h * lambda * qscale at the Key positions, then per head h
+  //   s_h = max|q'_h| / 32767,  q_int = round(q'_h / s_h) = 256 hi + lo
+  // (hi: s8, lo: u8).  The MMAs compute sum A q_int exactly, and sum(q'_h)
+  // is taken as s_h sum(q_int), over exactly the values the MMAs use, so
+  // (R/(2^b-1)) q'.c + Z sum(q') is the dot product of s_h q_int with the
   // dequantised key.
-  constexpr int lo_blocks = LO;
+  float* s_qv = reinterpret_cast<float*>(ws[1].code[kStages - 1]);  // [8][128] q' (warp 1's free stage)
+  unsigned* s_amax = reinterpret_cast<unsigned*>(w_m);              // [8] bits of max|q'| (w_m is free here)
+  int* s_isum = reinterpret_cast<int*>(w_l);                         // [8] sum of q_int
   reinterpret_cast<uint4*>(s_q)[threadIdx.x] = qv;  // heads >= G are zero
-  __syncthreads();
-  {
-    // warp w builds the fragments of k-blocks 2w and 2w+1
-    float part = 0.f;
-#pragma unroll
-    for (int i = 0; i < 2; i++) {
-      const int sb = 2 * warp + i;
-      uint32_t hq[2], lq[2];
-#pragma unroll
-      for (int hf = 0; hf < 2; hf++) {
-        // Key positions c0, c0+1 hold channels ch0, ch1 of the block's order
-        const int c0 = 16 * sb + 2 * t + 8 * hf;
-        const int ch0 = s_perm[c0], ch1 = s_perm[c0 + 1];
-        const float v0 = __bfloat162float(s_q[g * kHeadDim + ch0]) * a.qscale * s_lam[ch0];
-        const float v1 = __bfloat162float(s_q[g * kHeadDim + ch1]) * a.qscale * s_lam[ch1];
-        // channel block sb, half hf = pair p = 2 sb + hf of the Key units
-        const float scl = kWide ? 1.0f : (float)(1 << (emax<BITS>() - pair_shift<BITS>(2 * sb + hf)));
-        const __half2 h = __floats2half2_rn(v0 * scl, v1 * scl);
-        const __half2 lo = __floats2half2_rn(v0 * scl - __low2float(h), v1 * scl - __high2float(h));
-        hq[hf] = *reinterpret_cast<const uint32_t*>(&h);
-        lq[hf] = *reinterpret_cast<const uint32_t*>(&lo);
-        const float lo0 = sb < lo_blocks ? __low2float(lo) : 0.f, lo1 = sb < lo_blocks ? __high2float(lo) : 0.f;
-        part += ((__low2float(h) + lo0) + (__high2float(h) + lo1)) / scl;
-      }
-      qf[sb * 32 + lane] = make_uint4(hq[0], hq[1], lq[0], lq[1]);
-    }
-    part += __shfl_xor_sync(0xffffffffu, part, 1);
-    part += __shfl_xor_sync(0xffffffffu, part, 2);  // lanes 4g..4g+3: this warp's sum for head g
-    if (t == 0) atomicAdd(&sig[g], part);
+  if (threadIdx.x < kMaxGroup) {
+    s_amax[threadIdx.x] = 0u;
+    s_isum[threadIdx.x] = 0;
   }
   __syncthreads();
-  const float sig0 = sig[2 * t], sig1 = sig[2 * t + 1];  // sum of q' for heads 2t, 2t+1
+  {
+    const int pos = threadIdx.x;  // Key position
+    const int ch = s_perm[pos];
+    const float f = a.qscale * s_lam[ch];
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; h++) {
+      const float v = __bfloat162float(s_q[h * kHeadDim + ch]) * f;
+      s_qv[h * kHeadDim + pos] = v;
+      float m = fabsf(v);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (lane == 0) atomicMax(s_amax + h, __float_as_uint(m));
+    }
+  }
+  __syncthreads();
+  {
+    // warp w builds k-block w: lane (g, t) holds positions 32w + 4t + i (b0)
+    // and 32w + 16 + 4t + i (b1), i = 0..3, of head g
+    const float am = __uint_as_float(s_amax[g]);
+    const float inv = am > 0.f ? 32767.0f / am : 0.f;
+    uint32_t hb[2] = {0u, 0u}, lb[2] = {0u, 0u};
+    int part = 0;
+#pragma unroll
+    for (int hf = 0; hf < 2; hf++) {
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const float v = s_qv[g * kHeadDim + 32 * warp + 16 * hf + 4 * t + i];
+        const int qi = max(-32767, min(32767, __float2int_rn(v * inv)));
+        part += qi;
+        hb[hf] |= (uint32_t)((qi >> 8) & 0xff) << (8 * i);
+        lb[hf] |= (uint32_t)(qi & 0xff) << (8 * i);
+      }
+    }
+    qf[warp * 32 + lane] = make_uint4(hb[0], hb[1], lb[0], lb[1]);
+    part += __shfl_xor_sync(0xffffffffu, part, 1);
+    part += __shfl_xor_sync(0xffffffffu, part, 2);  // lanes 4g..4g+3: this k-block's sum for head g
+    if (t == 0) atomicAdd(s_isum + g, part);
+  }
+  __syncthreads();
+  float ks0, ks1, sig0, sig1;  // heads 2t, 2t+1
+  {
+    const float s0 = __uint_as_float(s_amax[2 * t]) / 32767.0f, s1 = __uint_as_float(s_amax[2 * t + 1]) / 32767.0f;
+    ks0 = s0 * kKCode;
+    ks1 = s1 * kKCode;
+    sig0 = s0 * (float)s_isum[2 * t];
+    sig1 = s1 * (float)s_isum[2 * t + 1];
+  }
   const uint4* qfl = qf + lane;
+  __syncthreads();  // w_m / w_l are reused by the merge
 
   Soft sm;
   sm.m0 = sm.m1 = -INFINITY;
@@ -595,12 +675,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
       constexpr int kNG = kChunkGroups >= 2 ? 2 : 1;
 #pragma unroll 1
       for (int gi = 0; gi < kChunkGroups; gi += kNG)
-        process_groups<BITS, LO, kNG, true>(cs + gi * kGroupBytes, ms + gi * 16, 16 * kNG, lane, qfl, sig0, sig1,
-                                            kKScale, sm);
+        process_groups<BITS, kNG, true>(cs + gi * kGroupBytes, ms + gi * 16, 16 * kNG, lane, qfl, ks0, ks1, sig0,
+                                        sig1, sm);
     } else {
       for (int gi = 0; gi < dsc.x; gi++)
-        process_groups<BITS, LO, 1, false>(cs + gi * kGroupBytes, ms + gi * 16, dsc.y - 16 * gi, lane, qfl, sig0,
-                                           sig1, kKScale, sm);
+        process_groups<BITS, 1, false>(cs + gi * kGroupBytes, ms + gi * 16, dsc.y - 16 * gi, lane, qfl, ks0, ks1,
+                                       sig0, sig1, sm);
     }
     __syncwarp();  // every lane is done with this stage before lane 0 refills it
   }
@@ -742,24 +822,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   if (threadIdx.x == 0) a.counters[s] = 0;
 }
 
-template <int BITS, int LO>
+template <int BITS>
 cudaError_t launch_bits(const DecodeArgs& a, cudaStream_t s) {
   static bool attr_set = false;  // per process; set before the first launch
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, LO>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(decode_kernel<BITS, LO>, cudaFuncAttributePreferredSharedMemoryCarveout,
+      e = cudaFuncSetAttribute(decode_kernel<BITS>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const unsigned grid = (unsigned)(a.batch * a.kv_heads) * (unsigned)a.splits;
-  return launch_pdl(decode_kernel<BITS, LO>, dim3(grid), dim3(kThreads), kSmemBytes, s, a);
-}
-
-template <int BITS>
-cudaError_t launch_bits(const DecodeArgs& a, cudaStream_t s) {
-  return a.perm ? launch_bits<BITS, 1>(a, s) : launch_bits<BITS, 8>(a, s);
+  return launch_pdl(decode_kernel<BITS>, dim3(grid), dim3(kThreads), kSmemBytes, s, a);
 }
 
 }  // namespace

@@ -6,25 +6,34 @@
 // bits a tile holds P_b = 512 / b token slots (32 at 16 bits ... 256 at 2
 // bits) in 16-token groups of 512*b bytes: the group's K part (256*b bytes)
 // followed by its V part (256*b bytes).  Each part is 32 "lane units" of 8*b
-// bytes; unit L holds exactly the 64 codes that lane L of a warp needs as its
-// mma.sync.m16n8k16 A-fragment registers:
-//   K (QK^T, A = K[token][channel]):  with L = 4g + t, tokens g and g+8 of
-//     the group, channels 16s + 2t + {0,1} + 8r  (s = 0..7, r = 0..1).
-//   V (P V,  A = V^T[channel][token]): channels 16s + g + 8r, tokens
-//     2t + {0,1} + 8u (u = 0..1).
-//   Codes come in pairs that fill one half2 register: for K a pair is two
-//   adjacent channels of one token, for V the same channel of tokens 2t+8u and
-//   2t+8u+1.  A unit holds 32 pairs; pair index P = 16*x + 2*s + r, where x
-//   selects the token (K: g or g+8) or token pair (V: u).  At b bits pair P
-//   lives in 32-bit word P / (16/b) of the unit at field position
-//   k = P % (16/b): the first member at bits [b*k, b*k+b), the second at
-//   bits [16 + b*k, 16 + b*k + b).  So each 16-bit half-word packs 16/b codes.
-//   Because this order is the same at every width, the shift 2b -> b maps
-//   input words (2J, 2J+1) of a tile to output word J of the same tile (the
-//   K/V interleave of the groups is preserved too), with no data moving
-//   between tiles: a shrink compacts every tile into its first half in place
-//   and token slots keep their indices.
-//
+// bytes; unit L (lane L = 4g + t of a warp) holds exactly the 64 codes that
+// lane needs as its MMA A-fragment registers:
+//   K (QK^T, int8 mma.m16n8k32, A = K[token][position]): tokens g and g+8
+//     of the group, positions 32s + 16r + 4t + i (k-block s = 0..3, column
+//     half r = 0..1, member i = 0..3).  The 4 codes (i = 0..3) of one token,
+//     k-block and column half form a "quad" = one A register of 4 bytes.  A
+//     unit holds 16 quads, quad index Q = 8x + 2s + r with x = 0 for token
+//     g and 1 for token g+8.  At b <= 8 bits quad Q lives in 32-bit word
+//     Q / (8/b) of the unit at field k = Q % (8/b): member i at bits
+//     [8i + b*k, 8i + b*k + b), so each byte packs 8/b codes.  At 16 bits
+//     quad Q spans words 2Q (members 0, 1 as half-words) and 2Q + 1
+//     (members 2, 3).
+//   V (P V, fp16 mma.m16n8k16, A = V^T[channel][token]): channels
+//     16s + g + 8r, tokens 2t + {0,1} + 8u (s = 0..7, r, u = 0..1).  Codes
+//     come in pairs that fill one half2 register: the same channel of tokens
+//     2t+8u and 2t+8u+1.  A unit holds 32 pairs, pair index P = 16u + 2s + r.
+//     At b bits pair P lives in 32-bit word P / (16/b) of the unit at field
+//     k = P % (16/b): the first member at bits [b*k, b*k+b), the second at
+//     bits [16 + b*k, 16 + b*k + b), so each 16-bit half-word packs 16/b
+//     codes.
+//   In both parts the order of quads (pairs) is the same at every width, so
+//   the shift 2b -> b maps input words (2J, 2J+1) of a tile to output word J
+//   of the same tile (the K/V interleave of the groups is preserved too),
+//   with no data moving between tiles: a shrink compacts every tile into its
+//   first half in place and token slots keep their indices.  Every word of
+//   a Key part belongs to one token (x is the outermost quad index), so a
+//   single-token append writes whole words there.
+
 // Fill pattern of a block (the slot map): before the first shrink tokens
 // fill tile 0, tile 1, ... (P_16 each).  A shrink happens only when every
 // tile is full, so afterwards every tile is exactly half full (h = P_b / 2)
@@ -32,13 +41,11 @@
 // therefore: tiles < k full, tile k holding h + r, tiles > k holding h.
 // Attention does not depend on token order, so nothing is ever reordered.
 //
-// Key channel order: within every Key unit, "channel" above means a
-// position of the block's per-KV-head channel order perm[j][pos] (logical
-// channel at that position), which puts the 16 channels with the largest
-// migration factor lambda in positions 0..15, i.e. the first MMA k-block.
-// Outlier channels carry the largest q'.k products, and only that k-block
-// gets the extra-precision (hi + lo) q' term in the attention kernel.  Values
-// keep the natural channel order.
+// Key channel order: "position" above is a position of the block's
+// per-KV-head channel order perm[j][pos] (the logical channel at that
+// position; channels sorted by decreasing migration factor lambda).
+// Attention and export apply the same order, so any permutation is valid.
+// Values keep the natural channel order.
 //
 // Meta: two 32-bit words per (stream, tile, slot), the Key's then the
 // Value's, each binary16 R (low half) and binary16 Z (high half); P_F slots

@@ -23,9 +23,10 @@ namespace {
 
 constexpr int kShrinkThreads = 256;
 
-// in0, in1: two consecutive input words (each half-word packs 16/(2b) codes
-// of width 2b).  Returns the output word: half-word h of the output is the
-// shifted codes of half h of in0 (low byte) and of in1 (high byte).
+// Value parts: in0, in1 are two consecutive input words (each half-word
+// packs 16/(2b) codes of width 2b).  Returns the output word: half-word h of
+// the output is the shifted codes of half h of in0 (low byte) and of in1
+// (high byte).
 template <int BTO>
 __device__ __forceinline__ uint32_t ers_pair(uint32_t in0, uint32_t in1);
 
@@ -65,6 +66,63 @@ __device__ __forceinline__ uint32_t ers_pair<2>(uint32_t in0, uint32_t in1) {
   return ers_half_words_2(in0) | (ers_half_words_2(in1) << 8);
 }
 
+// Key parts hold byte quads (member i of a quad in byte i of its word, see
+// kvq_internal.cuh): output byte i gets the shifted member i of the input
+// quads, in field order.
+template <int BTO>
+__device__ __forceinline__ uint32_t ers_quads(uint32_t in0, uint32_t in1);
+
+template <>
+__device__ __forceinline__ uint32_t ers_quads<8>(uint32_t in0, uint32_t in1) {
+  // one quad spans two input words (members 0, 1 in in0; 2, 3 in in1)
+  const uint32_t mul = 65281u;
+  uint32_t a = ((in0 & 0xffffu) + 128u) * mul >> 24;
+  uint32_t b = ((in0 >> 16) + 128u) * mul >> 24;
+  uint32_t c = ((in1 & 0xffffu) + 128u) * mul >> 24;
+  uint32_t d = ((in1 >> 16) + 128u) * mul >> 24;
+  return a | (b << 8) | (c << 16) | (d << 24);
+}
+
+__device__ __forceinline__ uint32_t ers_lanes16_4(uint32_t x) {  // 8-bit codes in 16-bit lanes -> 4 bits
+  return ((x + 0x00080008u) * 241u >> 12) & 0x000f000fu;
+}
+
+template <>
+__device__ __forceinline__ uint32_t ers_quads<4>(uint32_t in0, uint32_t in1) {
+  // in0 holds quad 2J (-> low nibbles), in1 quad 2J+1 (-> high nibbles)
+  const uint32_t ev = ers_lanes16_4(in0 & 0x00ff00ffu) | (ers_lanes16_4(in1 & 0x00ff00ffu) << 4);
+  const uint32_t od = ers_lanes16_4((in0 >> 8) & 0x00ff00ffu) | (ers_lanes16_4((in1 >> 8) & 0x00ff00ffu) << 4);
+  return ev | (od << 8);
+}
+
+__device__ __forceinline__ uint32_t ers_lanes8_2(uint32_t x) {  // 4-bit codes in 8-bit lanes -> 2 bits
+  return ((x + 0x02020202u) * 13u >> 6) & 0x03030303u;
+}
+
+template <>
+__device__ __forceinline__ uint32_t ers_quads<2>(uint32_t in0, uint32_t in1) {
+  // in0 holds quads 4J, 4J+1 (nibbles), in1 quads 4J+2, 4J+3 -> fields 0..3
+  return ers_lanes8_2(in0 & 0x0f0f0f0fu) | (ers_lanes8_2((in0 >> 4) & 0x0f0f0f0fu) << 2) |
+         (ers_lanes8_2(in1 & 0x0f0f0f0fu) << 4) | (ers_lanes8_2((in1 >> 4) & 0x0f0f0f0fu) << 6);
+}
+
+template <int BTO>
+__device__ __forceinline__ uint4 ers_uint4(uint4 a, uint4 b, bool key) {
+  uint4 o;
+  if (key) {
+    o.x = ers_quads<BTO>(a.x, a.y);
+    o.y = ers_quads<BTO>(a.z, a.w);
+    o.z = ers_quads<BTO>(b.x, b.y);
+    o.w = ers_quads<BTO>(b.z, b.w);
+  } else {
+    o.x = ers_pair<BTO>(a.x, a.y);
+    o.y = ers_pair<BTO>(a.z, a.w);
+    o.z = ers_pair<BTO>(b.x, b.y);
+    o.w = ers_pair<BTO>(b.z, b.w);
+  }
+  return o;
+}
+
 template <int BTO>
 __global__ void __launch_bounds__(kShrinkThreads) shrink_kernel(uint8_t* codes) {
   // Tile = 1024 uint4 in, 512 uint4 out.  Thread i produces output uint4
@@ -77,15 +135,11 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_kernel(uint8_t* codes) 
   in[2] = __ldcs(tile + 2 * (i + 256));
   in[3] = __ldcs(tile + 2 * (i + 256) + 1);
   __syncthreads();  // every read of the tile is done before any write
-  uint4 o0, o1;
-  o0.x = ers_pair<BTO>(in[0].x, in[0].y);
-  o0.y = ers_pair<BTO>(in[0].z, in[0].w);
-  o0.z = ers_pair<BTO>(in[1].x, in[1].y);
-  o0.w = ers_pair<BTO>(in[1].z, in[1].w);
-  o1.x = ers_pair<BTO>(in[2].x, in[2].y);
-  o1.y = ers_pair<BTO>(in[2].z, in[2].w);
-  o1.z = ers_pair<BTO>(in[3].x, in[3].y);
-  o1.w = ers_pair<BTO>(in[3].z, in[3].w);
+  // Output uint4 u lies in a Key part when (u mod 32*BTO) < 16*BTO (a group
+  // at BTO bits is 32*BTO uint4: Key part, then Value part); warp-uniform.
+  constexpr int kGroupU4 = 32 * BTO, kPartU4 = 16 * BTO;
+  const uint4 o0 = ers_uint4<BTO>(in[0], in[1], (i % kGroupU4) < kPartU4);
+  const uint4 o1 = ers_uint4<BTO>(in[2], in[3], ((i + 256) % kGroupU4) < kPartU4);
   tile[i] = o0;
   tile[i + 256] = o1;
 }
