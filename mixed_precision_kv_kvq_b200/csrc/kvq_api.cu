@@ -52,6 +52,12 @@ struct LayerState {
   int bits;
   long long n;
   int n_shrinks;
+  // Tokens whose slots no library kernel still in flight can be writing when
+  // a later kernel on the same stream starts early (programmatic dependent
+  // launch): the append kernel triggers its dependents only after its own
+  // predecessors completed, and the shrink kernel never triggers early, so
+  // only the most recent append kernel of the block can still be running.
+  long long n_stable;
   int nt;  // tiles per stream
   int pf;  // meta slots per tile
   bool counters_zeroed;
@@ -93,6 +99,7 @@ bool make_plan(int layers, int batch, int kv_heads, int head_dim, size_t budget,
     L.bits = 16;
     L.n = 0;
     L.n_shrinks = 0;
+    L.n_stable = 0;
     L.pf = slots_per_tile(L.fbit);
     L.nt = (int)(n_f / L.pf);
     L.counters_zeroed = false;
@@ -184,6 +191,15 @@ void slot_of(const LayerState& L, long long i, int* tile, int* slot) {
   const long long m = i - (long long)L.nt * h;
   *tile = (int)(m / ee);
   *slot = h + (int)(m % ee);
+}
+
+// Groups (in the kernels' group order, see locate_group) of every stream
+// that hold only slots of tokens before n_stable.
+long long stable_groups(const LayerState& L, const Fill& f) {
+  if (L.n_stable >= L.n) return f.gps;
+  int tile, slot;
+  slot_of(L, L.n_stable, &tile, &slot);
+  return (long long)tile * f.gpt + slot / kGroupTokens;
 }
 
 uint32_t rd32(const uint8_t* p) {
@@ -324,6 +340,7 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* k, const void* v, int
     a.perm = L.lambda_set ? c->perm(layer) : nullptr;
     cudaError_t e = launch_append(a, s);
     if (e != cudaSuccess) return cuda_fail(e, "append launch");
+    L.n_stable = L.n;
     L.n += cnt;
     off += cnt;
   }
@@ -343,6 +360,7 @@ kvq_status kvq_shrink(kvq_cache* c, int layer, kvq_stream_t stream) {
   if (e != cudaSuccess) return cuda_fail(e, "shrink launch");
   L.bits /= 2;
   L.n_shrinks++;
+  L.n_stable = L.n;
   return KVQ_OK;
 }
 
@@ -394,6 +412,7 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, 
   a.group = G;
   a.qscale = sm_scale * 1.4426950408889634f;
   a.splits = decode_splits(c->sms(), n_streams, a.fill.gps);
+  a.safe = stable_groups(L, a.fill);
   cudaError_t e = launch_decode(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return KVQ_OK;
@@ -485,6 +504,7 @@ kvq_status kvq_decode_attn_noalloc(kvq_cache* c, int layer, const void* q, int q
   a.group = G;
   a.qscale = sm_scale * 1.4426950408889634f;
   a.splits = splits;
+  a.safe = stable_groups(L, fill);
   cudaError_t e = launch_decode(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return KVQ_OK;

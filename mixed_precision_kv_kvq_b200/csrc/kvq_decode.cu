@@ -538,11 +538,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     }
     reinterpret_cast<uint4*>(s_perm)[lane] = pv;
   }
-  pdl_wait();  // the cache, q and the counters may be written by earlier kernels
-  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.q_heads + (size_t)j * G) * kHeadDim;
-  uint4 qv = make_uint4(0u, 0u, 0u, 0u);  // 8 bf16 of q: head threadIdx/16, channels 8 (threadIdx%16) ..
-  if ((int)threadIdx.x < G * (kHeadDim / 8)) qv = reinterpret_cast<const uint4*>(qb)[threadIdx.x];
-
   // ---- chunk iterator: lane 0 walks its groups tile by tile and issues the
   // copies; everyone reads the per-stage descriptors (groups, valid tokens) ----
   int left = (int)(wb - wa);  // groups this warp still has to issue
@@ -580,8 +575,26 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     }
   };
 
+  // A first chunk that lies wholly in groups no kernel still in flight can
+  // be writing (a.safe: before the slots of the most recent append) is
+  // fetched before waiting for the previous kernel.
+  bool pre = false;
+  if constexpr (!kWide) {
+    if (lane == 0 && left > 0) {
+      const int ng0 = min(min(it_tgroups - it_grp, kChunkGroups), left);
+      if (wa + ng0 <= a.safe) {
+        issue(0);
+        pre = true;
+      }
+    }
+  }
+  pdl_wait();  // the rest of the cache, q and the counters may be written by earlier kernels
+  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.q_heads + (size_t)j * G) * kHeadDim;
+  uint4 qv = make_uint4(0u, 0u, 0u, 0u);  // 8 bf16 of q: head threadIdx/16, channels 8 (threadIdx%16) ..
+  if ((int)threadIdx.x < G * (kHeadDim / 8)) qv = reinterpret_cast<const uint4*>(qb)[threadIdx.x];
+
   // start streaming before the q' set-up so DRAM latency overlaps it
-  if (lane == 0) {
+  if (lane == 0 && !pre) {
 #pragma unroll
     for (int i = 0; i < kS - 1; i++) issue(i);
   }
@@ -594,52 +607,49 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   // is taken as s_h sum(q_int), over exactly the values the MMAs use, so
   // (R/(2^b-1)) q'.c + Z sum(q') is the dot product of s_h q_int with the
   // dequantised key.
-  float* s_qv = reinterpret_cast<float*>(ws[1].code[kStages - 1]);  // [8][128] q' (warp 1's free stage)
-  unsigned* s_amax = reinterpret_cast<unsigned*>(w_m);              // [8] bits of max|q'| (w_m is free here)
-  int* s_isum = reinterpret_cast<int*>(w_l);                         // [8] sum of q_int
+  unsigned* s_amax = reinterpret_cast<unsigned*>(w_m);  // [8] bits of max|q'| (w_m is free here)
+  int* s_isum = reinterpret_cast<int*>(w_l);             // [8] sum of q_int
   reinterpret_cast<uint4*>(s_q)[threadIdx.x] = qv;  // heads >= G are zero
-  if (threadIdx.x < kMaxGroup) {
-    s_amax[threadIdx.x] = 0u;
-    s_isum[threadIdx.x] = 0;
-  }
   __syncthreads();
   {
-    const int pos = threadIdx.x;  // Key position
-    const int ch = s_perm[pos];
-    const float f = a.qscale * s_lam[ch];
+    // Warp w quantizes heads 2w and 2w+1: lane L takes head gq = 2w + L/16
+    // and writes the B fragment of k-block sq = L%4 for MMA lane 4 gq + tq,
+    // tq = (L/4)%4: positions 32 sq + 16 hf + 4 tq + i (hf = 0..1, i = 0..3).
+    // The 16 lanes of a head cover its 128 positions.
+    const int gq = 2 * warp + (lane >> 4), tq = (lane >> 2) & 3, sq = lane & 3;
+    float v[2][4];
+    float m = 0.f;
 #pragma unroll
-    for (int h = 0; h < kMaxGroup; h++) {
-      const float v = __bfloat162float(s_q[h * kHeadDim + ch]) * f;
-      s_qv[h * kHeadDim + pos] = v;
-      float m = fabsf(v);
+    for (int hf = 0; hf < 2; hf++) {
 #pragma unroll
-      for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if (lane == 0) atomicMax(s_amax + h, __float_as_uint(m));
+      for (int i = 0; i < 4; i++) {
+        const int ch = s_perm[32 * sq + 16 * hf + 4 * tq + i];
+        v[hf][i] = __bfloat162float(s_q[gq * kHeadDim + ch]) * a.qscale * s_lam[ch];
+        m = fmaxf(m, fabsf(v[hf][i]));
+      }
     }
-  }
-  __syncthreads();
-  {
-    // warp w builds k-block w: lane (g, t) holds positions 32w + 4t + i (b0)
-    // and 32w + 16 + 4t + i (b1), i = 0..3, of head g
-    const float am = __uint_as_float(s_amax[g]);
-    const float inv = am > 0.f ? 32767.0f / am : 0.f;
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float inv = m > 0.f ? 32767.0f / m : 0.f;
     uint32_t hb[2] = {0u, 0u}, lb[2] = {0u, 0u};
     int part = 0;
 #pragma unroll
     for (int hf = 0; hf < 2; hf++) {
 #pragma unroll
       for (int i = 0; i < 4; i++) {
-        const float v = s_qv[g * kHeadDim + 32 * warp + 16 * hf + 4 * t + i];
-        const int qi = max(-32767, min(32767, __float2int_rn(v * inv)));
+        const int qi = max(-32767, min(32767, __float2int_rn(v[hf][i] * inv)));
         part += qi;
         hb[hf] |= (uint32_t)((qi >> 8) & 0xff) << (8 * i);
         lb[hf] |= (uint32_t)(qi & 0xff) << (8 * i);
       }
     }
-    qf[warp * 32 + lane] = make_uint4(hb[0], hb[1], lb[0], lb[1]);
-    part += __shfl_xor_sync(0xffffffffu, part, 1);
-    part += __shfl_xor_sync(0xffffffffu, part, 2);  // lanes 4g..4g+3: this k-block's sum for head g
-    if (t == 0) atomicAdd(s_isum + g, part);
+    qf[sq * 32 + 4 * gq + tq] = make_uint4(hb[0], hb[1], lb[0], lb[1]);
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if ((lane & 15) == 0) {
+      s_amax[gq] = __float_as_uint(m);
+      s_isum[gq] = part;
+    }
   }
   __syncthreads();
   float ks0, ks1, sig0, sig1;  // heads 2t, 2t+1
@@ -781,6 +791,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   __syncthreads();
   if (!flags[1]) return;
   const float* p0 = a.parts + (size_t)s * nparts * kPartFloats;
+  // The first kPre partials' outputs for this thread's channel are loaded
+  // now, in flight while the weights are formed from every partial's M, L.
+  constexpr int kPre = 8;
+  const float* oc = p0 + 2 * kMaxGroup + c * kMaxGroup;
+  float4 ov[kPre][2];
+#pragma unroll
+  for (int k = 0; k < kPre; k++) {
+    if (k < nparts) {
+      ov[k][0] = __ldcg(reinterpret_cast<const float4*>(oc + (size_t)k * kPartFloats));
+      ov[k][1] = __ldcg(reinterpret_cast<const float4*>(oc + (size_t)k * kPartFloats + 4));
+    }
+  }
   float* wk = reinterpret_cast<float*>(ws[0].code[0]);  // [nparts][8] (the stage buffers are free now)
   float* lk = wk + kMaxSplits * kMaxGroup;
   for (int i = threadIdx.x; i < nparts * 2 * kMaxGroup / 4; i += kThreads) {  // every partial's M, L at once
@@ -790,32 +812,43 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
   }
   __syncthreads();
-  if (threadIdx.x < kMaxGroup) {  // weight of partial k for head h: e^(M_k - M) / L
-    const int h = threadIdx.x;
-    float M = -INFINITY;
-    for (int k = 0; k < nparts; k++) M = fmaxf(M, wk[k * kMaxGroup + h]);
-    float L = 0.f;
-    for (int k = 0; k < nparts; k++) {
-      const float e = ex2(wk[k * kMaxGroup + h] - M);
-      wk[k * kMaxGroup + h] = e;
-      L += e * lk[k * kMaxGroup + h];
-    }
-    const float inv = 1.0f / L;
-    for (int k = 0; k < nparts; k++) wk[k * kMaxGroup + h] *= inv;
-  }
-  __syncthreads();
-  float acc[kMaxGroup];
+  // Every thread forms the log-sum-exp weights itself (broadcast reads):
+  // w_k = e^(M_k - M) for head h, out = sum_k w_k O_k / sum_k w_k L_k.
+  float Mx[kMaxGroup], Ls[kMaxGroup], acc[kMaxGroup];
 #pragma unroll
-  for (int h = 0; h < kMaxGroup; h++) acc[h] = 0.f;
-  const float* oc = p0 + 2 * kMaxGroup + c * kMaxGroup;
-#pragma unroll 4
+  for (int h = 0; h < kMaxGroup; h++) {
+    Mx[h] = -INFINITY;
+    Ls[h] = 0.f;
+    acc[h] = 0.f;
+  }
   for (int k = 0; k < nparts; k++) {
+    const float4 m0 = *reinterpret_cast<const float4*>(wk + k * kMaxGroup);
+    const float4 m1 = *reinterpret_cast<const float4*>(wk + k * kMaxGroup + 4);
+    Mx[0] = fmaxf(Mx[0], m0.x); Mx[1] = fmaxf(Mx[1], m0.y); Mx[2] = fmaxf(Mx[2], m0.z); Mx[3] = fmaxf(Mx[3], m0.w);
+    Mx[4] = fmaxf(Mx[4], m1.x); Mx[5] = fmaxf(Mx[5], m1.y); Mx[6] = fmaxf(Mx[6], m1.z); Mx[7] = fmaxf(Mx[7], m1.w);
+  }
+  auto add = [&](int k, const float4& o0, const float4& o1) {
+    const float* mk = wk + k * kMaxGroup;
+    const float* lkk = lk + k * kMaxGroup;
+    const float ov8[kMaxGroup] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; h++) {
+      const float e = ex2(mk[h] - Mx[h]);
+      Ls[h] = fmaf(e, lkk[h], Ls[h]);
+      acc[h] = fmaf(e, ov8[h], acc[h]);
+    }
+  };
+#pragma unroll
+  for (int k = 0; k < kPre; k++)
+    if (k < nparts) add(k, ov[k][0], ov[k][1]);
+#pragma unroll 4
+  for (int k = kPre; k < nparts; k++) {
     const float4 v0 = __ldcg(reinterpret_cast<const float4*>(oc + (size_t)k * kPartFloats));
     const float4 v1 = __ldcg(reinterpret_cast<const float4*>(oc + (size_t)k * kPartFloats + 4));
-    const float* w = wk + k * kMaxGroup;
-    acc[0] += w[0] * v0.x; acc[1] += w[1] * v0.y; acc[2] += w[2] * v0.z; acc[3] += w[3] * v0.w;
-    acc[4] += w[4] * v1.x; acc[5] += w[5] * v1.y; acc[6] += w[6] * v1.z; acc[7] += w[7] * v1.w;
+    add(k, v0, v1);
   }
+#pragma unroll
+  for (int h = 0; h < kMaxGroup; h++) acc[h] /= Ls[h];
 #pragma unroll
   for (int h = 0; h < kMaxGroup; h++)
     if (h < G) outp[h * kHeadDim + c] = acc[h];

@@ -180,6 +180,7 @@ struct DecodeArgs {
   int batch, kv_heads, q_heads, group;
   float qscale;         // sm_scale * log2(e)
   int splits;           // CTAs per stream
+  long long safe;       // groups [0, safe) of every stream are not written by kernels still in flight
 };
 
 // CTAs per stream for a launch over n_streams streams on num_sms SMs.
