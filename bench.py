@@ -257,6 +257,83 @@ def measure_append_chunk(kvq, dev, flush_buf, reps=3):
     return {"gbs": nb / t / 1e9, "us": t * 1e6, "bytes": nb, "bits": bits, "tokens": 4096, "batch": batch}
 
 
+def _decode_args(kvq, cache, q, out, ws, stream):
+    import ctypes as C
+    return (cache.handle, 0, C.c_void_p(q.data_ptr()), q.shape[1], C.c_float(HEAD_DIM ** -0.5),
+            C.c_void_p(out.data_ptr()), C.c_void_p(ws.data_ptr()), ws.numel() * 4, C.c_void_p(stream.cuda_stream))
+
+
+def measure_decode_configs(kvq, dev, reps=20):
+    """Decode attention of one block of each model-shaped workload at both of
+    its widths: `reps` back-to-back launches on one block (CUDA events around
+    the batch; the block's read exceeds L2), mean per launch."""
+    lib = kvq.load()
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    cfgs = (("qwen7b", 16, 4, 28, 32768, 32768 + ROOM),
+            ("qwen32b", 16, 8, 40, 32768, 55296),
+            ("llama70b", 8, 8, 64, 131072, 131072))
+    for name, batch, kv_heads, q_heads, tokens, n_f in cfgs:
+        for fbit in (2, 4):
+            cache = build_cache(kvq, dev, 1, batch, kv_heads, [fbit], tokens, n_f, SEED + 31, S.outliers_for(kv_heads),
+                                chunk=8192)
+            assert cache.query(0)["bits"] == fbit
+            q = S.queries(SEED, 0, 0, batch, q_heads, tokens, dtype=torch.bfloat16, device=dev)
+            out = torch.empty((batch, q_heads, HEAD_DIM), dtype=torch.float32, device=dev)
+            ws = cache.workspace(0, q_heads)
+            a = _decode_args(kvq, cache, q, out, ws, stream)
+            for _ in range(3):
+                kvq.check(lib.kvq_decode_attn(*a))
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                lib.kvq_decode_attn(*a)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            cache.device_status()
+            us = e0.elapsed_time(e1) / reps * 1e3
+            nb = decode_bytes(batch, kv_heads, q_heads, tokens, fbit)
+            res[f"{name}_{fbit}bit"] = {"us": round(us, 2), "gbs": round(nb / us / 1e3, 1), "bytes": nb,
+                                        "batch": batch, "kv_heads": kv_heads, "q_heads": q_heads, "tokens": tokens}
+            cache.free()
+            del cache
+    res["timing"] = f"{reps} back-to-back launches on one block, CUDA events around the batch, mean per launch"
+    return res
+
+
+def measure_append_token(kvq, dev, reps=200):
+    """Single-token append on a 7B-shaped block (batch 16, 4 KV heads, 2-bit,
+    32768 tokens cached): `reps` back-to-back calls through the C ABI, mean."""
+    import ctypes as C
+    lib = kvq.load()
+    stream = torch.cuda.current_stream(dev)
+    cache = build_cache(kvq, dev, 1, B7, HKV7, [2], T7, T7 + ROOM, SEED + 41, S.outliers_for(HKV7), chunk=8192)
+    g = torch.Generator(device=dev)
+    g.manual_seed(SEED + 43)
+    kin = torch.randn((reps + 3, B7, 1, HKV7, HEAD_DIM), generator=g, device=dev).to(torch.bfloat16)
+    vin = torch.randn((reps + 3, B7, 1, HKV7, HEAD_DIM), generator=g, device=dev).to(torch.bfloat16)
+    sp = C.c_void_p(stream.cuda_stream)
+    for i in range(3):
+        kvq.check(lib.kvq_append(cache.handle, 0, C.c_void_p(kin[i].data_ptr()), C.c_void_p(vin[i].data_ptr()),
+                                 kvq.KVQ_DTYPE_BF16, 1, sp))
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(3, reps + 3):
+        lib.kvq_append(cache.handle, 0, C.c_void_p(kin[i].data_ptr()), C.c_void_p(vin[i].data_ptr()),
+                       kvq.KVQ_DTYPE_BF16, 1, sp)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) / reps * 1e3
+    assert cache.query(0)["tokens"] == T7 + reps + 3
+    cache.free()
+    nb = append_bytes(B7, HKV7, 1, 2)
+    return {"us": round(us, 2), "gbs": round(nb / us / 1e3, 2), "bytes": nb, "batch": B7, "kv_heads": HKV7,
+            "bits": 2, "timing": f"{reps} back-to-back single-token appends, CUDA events around the batch; "
+                                 "launch-latency bound"}
+
+
 def run_gpu(args, rank, world):
     from mixed_precision_kv_kvq_b200 import build as kbuild
 
@@ -379,6 +456,54 @@ def run_gpu(args, rank, world):
             dec_ms_bits.setdefault(fbit[l], []).append(evs[i][l][0].elapsed_time(evs[i][l][1]))
     ev_step_ms = r_start.elapsed_time(r_end) / K
 
+    # ---- the decode half of the step captured in one CUDA graph ----
+    graph = None
+    if not args.no_shrink:
+        gs = torch.cuda.Stream(dev)
+        gsp = C.c_void_p(gs.cuda_stream)
+        qg = qin[W + 2 * K - 1]
+        gargs = [(h, l, C.c_void_p(qg[l].data_ptr()), HQ7, scale_c, op[l], wp[l][0], wp[l][1], gsp)
+                 for l in range(layers)]
+        gs.wait_stream(stream)
+        with torch.cuda.stream(gs):
+            for l in range(layers):  # warm the side stream
+                kvq.check(lib.kvq_decode_attn(*gargs[l]))
+        gs.synchronize()
+        cg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cg, stream=gs):
+            for l in range(layers):
+                lib.kvq_decode_attn(*gargs[l])
+        torch.cuda.synchronize(dev)
+        nrep = max(K, 20)
+        for _ in range(3):
+            cg.replay()
+        torch.cuda.synchronize(dev)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(nrep):
+            cg.replay()
+        g1.record(stream)
+        torch.cuda.synchronize(dev)
+        graph_ms = g0.elapsed_time(g1) / nrep
+        # the same launches without the graph
+        n0, n1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        plain = [(h, l, C.c_void_p(qg[l].data_ptr()), HQ7, scale_c, op[l], wp[l][0], wp[l][1], sp)
+                 for l in range(layers)]
+        n0.record(stream)
+        for _ in range(nrep):
+            for l in range(layers):
+                lib.kvq_decode_attn(*plain[l])
+        n1.record(stream)
+        torch.cuda.synchronize(dev)
+        plain_ms = n0.elapsed_time(n1) / nrep
+        cache.device_status()
+        dbytes = sum(decode_bytes(B7, HKV7, HQ7, cache.query(l)["tokens"], fbit[l]) for l in range(layers))
+        graph = {"ms_per_step": round(graph_ms, 4), "gbs": round(dbytes / graph_ms / 1e6, 1),
+                 "ms_per_step_no_graph": round(plain_ms, 4), "gbs_no_graph": round(dbytes / plain_ms / 1e6, 1),
+                 "what": f"the {layers} decode launches of one step in one CUDA graph, {nrep} replays "
+                         "(appends cannot be replayed: the host scheduler state moves with every token)"}
+        del cg
+
     # ---- e2e: the same step through the public API with host buffers ----
     e2e = None
     if not args.no_e2e:
@@ -437,6 +562,9 @@ def run_gpu(args, rank, world):
         extra["shrink"] = measure_shrink(kvq, dev, flush)
         extra["shrink"]["unit"] = "GB/s"
         extra["append_chunk"] = measure_append_chunk(kvq, dev, flush)
+        extra["append_token"] = measure_append_token(kvq, dev)
+        extra["decode_configs"] = measure_decode_configs(kvq, dev)
+        extra["decode_graph"] = graph
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(total_ms / K, 4), "higher_is_better": True, "scaling": "weak",
