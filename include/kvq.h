@@ -155,6 +155,23 @@ kvq_status kvq_export(const kvq_cache* c, int layer, int b, int j, uint16_t* k_c
  * bounded wait (KVQ_ERR_TIMEOUT) since the last check; clears the flag. */
 kvq_status kvq_device_status(kvq_cache* c, kvq_stream_t stream);
 
+/* Block-wise bit allocation (key design 2): choose one width per block from
+ * the candidate widths bits[0..n_opts) (each 2, 4, 8 or 16, distinct;
+ * n_opts <= 4) minimising  sum_i sens[i][o_i]  subject to the cache's budget
+ * rule for max_tokens tokens in every block:
+ *   batch * kv_heads * 2 * max_tokens * sum_i (16 * bits[o_i] + 4) <= budget_bytes.
+ * sens: host double [layers][n_opts], the sensitivity s_{i,b} of block i at
+ * width bits[o] (computed offline from gradients; an input here).  The
+ * solution is exact (dynamic programming over the budget in units of
+ * batch * kv_heads * 2 * max_tokens * 4 bytes); among assignments of equal
+ * objective the first found (blocks in order, options in the given order)
+ * is returned.  fbit_out: host int [layers], ready for kvq_pool_bytes /
+ * kvq_alloc; objective_out (may be NULL): the minimal sum.  Pure host
+ * computation.  Errors: INVALID (arguments), BUDGET (no assignment fits). */
+kvq_status kvq_allocate_bits(int layers, int n_opts, const int* bits, const double* sens, int batch,
+                             int kv_heads, int head_dim, long long max_tokens, size_t budget_bytes,
+                             int* fbit_out, double* objective_out);
+
 /* Message of the last failed call on this thread ("" if none). */
 const char* kvq_last_error(void);
 

@@ -23,7 +23,7 @@ __all__ = [
     "KVQCache", "KVQError", "load",
     "kvq_pool_bytes", "kvq_alloc", "kvq_set_lambda", "kvq_append", "kvq_shrink",
     "kvq_decode_workspace", "kvq_decode_attn", "kvq_decode_attn_noalloc", "kvq_query", "kvq_max_tokens", "kvq_export",
-    "kvq_device_status", "kvq_last_error", "kvq_free",
+    "kvq_device_status", "kvq_last_error", "kvq_free", "kvq_allocate_bits",
 ]
 
 
@@ -148,6 +148,21 @@ def kvq_export(cache, layer: int, b: int, j: int, stream=None):
 
 def kvq_device_status(cache, stream=None) -> None:
     check(load().kvq_device_status(cache, _stream_ptr(stream)))
+
+
+def kvq_allocate_bits(sens, bits: Sequence[int], batch: int, kv_heads: int, max_tokens: int,
+                      budget_bytes: int, head_dim: int = HEAD_DIM):
+    """sens: [layers][n_opts] sensitivities (host).  -> (fbit list, objective)."""
+    sens = np.ascontiguousarray(sens, dtype=np.float64)
+    if sens.ndim != 2 or sens.shape[1] != len(bits):
+        raise ValueError("sens must be [layers][len(bits)]")
+    layers = sens.shape[0]
+    b = (C.c_int * len(bits))(*[int(x) for x in bits])
+    out = (C.c_int * layers)()
+    obj = C.c_double()
+    check(load().kvq_allocate_bits(layers, len(bits), b, sens.ctypes.data_as(C.c_void_p), batch, kv_heads,
+                                   head_dim, max_tokens, budget_bytes, out, C.byref(obj)))
+    return list(out), obj.value
 
 
 def kvq_last_error() -> str:

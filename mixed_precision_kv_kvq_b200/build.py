@@ -10,7 +10,7 @@ PKG = Path(__file__).resolve().parent
 ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIB = PKG / "libkvq.so"
-SOURCES = ["kvq_api.cu", "kvq_append.cu", "kvq_shrink.cu", "kvq_decode.cu"]
+SOURCES = ["kvq_api.cu", "kvq_append.cu", "kvq_shrink.cu", "kvq_decode.cu", "kvq_bitalloc.cu"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

@@ -41,6 +41,16 @@ kvq_status cuda_fail(cudaError_t e, const char* what) {
   return fail(KVQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+}  // namespace
+
+namespace kvq {
+// Records the message of a failed call (for the host-only entry points in
+// other files).
+kvq_status api_fail(kvq_status s, const char* msg) { return fail(s, "%s", msg); }
+}  // namespace kvq
+
+namespace {
+
 constexpr size_t kAlign = 256;
 constexpr int kTokenRound = 512;  // tokens per tile at 2 bits: a multiple for every width
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }

@@ -263,3 +263,34 @@ def attention_dense(q: np.ndarray, k: np.ndarray, v: np.ndarray, sm_scale: float
     lib().orc_attention_dense(_ptr(q), _ptr(k), _ptr(v), T, q.shape[0], hkv, d, float(sm_scale),
                               _ptr(out))
     return out
+
+
+def block_bytes(bits: int, batch: int, kv_heads: int, max_tokens: int) -> int:
+    """KV-cache bytes of one block at `bits` for max_tokens tokens: codes
+    (16 bits bytes per token-head, K and V) plus binary16 (R, Z) per group."""
+    return batch * kv_heads * 2 * max_tokens * (16 * bits + 4)
+
+
+def allocate_bits_brute(sens, bits, batch: int, kv_heads: int, max_tokens: int, budget: int):
+    """Block-wise bit allocation of the PM-KVQ note (key design 2), by
+    enumeration: every assignment of one width per block whose total KV
+    memory fits the budget M, and the least  sum_i s_{i,b_i}.  Returns
+    (objective, [every optimal assignment as a tuple of widths]) or
+    (None, []) if nothing fits.  Small cases only (n_opts ** layers)."""
+    import itertools
+
+    sens = np.asarray(sens, dtype=np.float64)
+    layers, n_opts = sens.shape
+    cost = [block_bytes(b, batch, kv_heads, max_tokens) for b in bits]
+    best, arg = None, []
+    for choice in itertools.product(range(n_opts), repeat=layers):
+        if sum(cost[o] for o in choice) > budget:
+            continue
+        obj = 0.0
+        for i, o in enumerate(choice):
+            obj += float(sens[i, o])
+        if best is None or obj < best - 1e-12 * max(1.0, abs(best)):
+            best, arg = obj, [tuple(bits[o] for o in choice)]
+        elif abs(obj - best) <= 1e-12 * max(1.0, abs(best)):
+            arg.append(tuple(bits[o] for o in choice))
+    return best, arg
