@@ -230,6 +230,21 @@ uint32_t orc_ers(uint32_t x2b, int b) {
 /* Scale after a shrink, as a function of the scale before it (S_b = (2^b+1) S_2b). */
 double orc_scale_after_shrink(double s2b, int b) { return (double)((1u << b) + 1u) * s2b; }
 
+/* Direct Right Shift (the first row of the note's ablation): keep only the
+ * high b bits of the 2b-bit code, X_b = X_2b >> b, with Z_b = Z_2b and the
+ * scale of the kept bits S_b = 2^b S_2b (reading: the plain scale of a
+ * truncation; the note gives no formula).  In the range form R = (2^b - 1) S
+ * that is R_b = 2^b R_2b / (2^b + 1), computed as fp32(fp32(R 2^b) / (2^b + 1))
+ * and rounded to binary16 to nearest (reading: the meta format is binary16). */
+uint32_t orc_drs(uint32_t x2b, int b) { return x2b >> b; }
+
+uint16_t orc_drs_range(uint16_t r_bits, int b) {
+  const float r = (float)orc_f16_to_f64(r_bits);
+  const float num = r * (float)(1u << b); /* exact: a power of two */
+  const float q = num / (float)((1u << b) + 1u);
+  return orc_f16_from_f64((double)q, 0);
+}
+
 /* ------------------------------------------------------------------------ */
 /* Progressive cache model of one transformer block (Key design 1).          */
 /* Codes and meta are kept in logical token order.                          */
@@ -243,6 +258,7 @@ typedef struct {
   uint16_t* vc;
   uint16_t* km; /* [batch][kv_heads][n_f][2]  (R bits, Z bits) */
   uint16_t* vm;
+  int shift_mode; /* 0: Equivalent Right Shift, 1: Direct Right Shift */
 } orc_layer;
 
 size_t orc_layer_sizeof(void) { return sizeof(orc_layer); }
@@ -281,18 +297,29 @@ static size_t orc_slot(const orc_layer* L, int b, int h, int t) {
   return ((size_t)b * L->kv_heads + h) * L->n_f + t;
 }
 
-/* Shrink every stored code one level (2b -> b).  Meta is untouched: with the
- * range form R = (2^b - 1) S, S_b = (2^b + 1) S_2b keeps R fixed. */
+/* Shrink every stored code one level (2b -> b).  Equivalent Right Shift:
+ * meta is untouched (with the range form R = (2^b - 1) S, S_b = (2^b + 1) S_2b
+ * keeps R fixed).  Direct Right Shift: every stored R is rescaled. */
 int orc_layer_shrink(orc_layer* L) {
   if (L->bits <= L->fbit) return -1;
   int b = L->bits / 2;
   for (int bb = 0; bb < L->batch; bb++)
     for (int h = 0; h < L->kv_heads; h++)
       for (int t = 0; t < L->n; t++) {
-        size_t base = orc_slot(L, bb, h, t) * ORC_D;
+        size_t slot = orc_slot(L, bb, h, t);
+        size_t base = slot * ORC_D;
         for (int c = 0; c < ORC_D; c++) {
-          L->kc[base + c] = (uint16_t)orc_ers(L->kc[base + c], b);
-          L->vc[base + c] = (uint16_t)orc_ers(L->vc[base + c], b);
+          if (L->shift_mode == 1) {
+            L->kc[base + c] = (uint16_t)orc_drs(L->kc[base + c], b);
+            L->vc[base + c] = (uint16_t)orc_drs(L->vc[base + c], b);
+          } else {
+            L->kc[base + c] = (uint16_t)orc_ers(L->kc[base + c], b);
+            L->vc[base + c] = (uint16_t)orc_ers(L->vc[base + c], b);
+          }
+        }
+        if (L->shift_mode == 1) {
+          L->km[slot * 2] = orc_drs_range(L->km[slot * 2], b);
+          L->vm[slot * 2] = orc_drs_range(L->vm[slot * 2], b);
         }
       }
   if (L->n_shrinks < 8) L->shrink_at[L->n_shrinks] = L->n;
@@ -326,6 +353,14 @@ int orc_layer_append(orc_layer* L, const float* k, const float* v, int n, const 
       }
     L->n++;
   }
+  return 0;
+}
+
+/* Choose the shift of a block before its first shrink (0 ERS, 1 DRS). */
+int orc_layer_set_shift_mode(orc_layer* L, int mode) {
+  if (mode != 0 && mode != 1) return -1;
+  if (L->n_shrinks > 0) return -2;
+  L->shift_mode = mode;
   return 0;
 }
 

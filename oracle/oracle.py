@@ -47,6 +47,7 @@ class _Layer(C.Structure):
         ("shrink_at", C.c_int * 8),
         ("kc", C.POINTER(C.c_uint16)), ("vc", C.POINTER(C.c_uint16)),
         ("km", C.POINTER(C.c_uint16)), ("vm", C.POINTER(C.c_uint16)),
+        ("shift_mode", C.c_int),
     ]
 
 
@@ -74,6 +75,11 @@ def lib():
         L.orc_ers.restype = C.c_uint32
         L.orc_scale_after_shrink.argtypes = [C.c_double, C.c_int]
         L.orc_scale_after_shrink.restype = C.c_double
+        L.orc_drs.argtypes = [C.c_uint32, C.c_int]
+        L.orc_drs.restype = C.c_uint32
+        L.orc_drs_range.argtypes = [C.c_uint16, C.c_int]
+        L.orc_drs_range.restype = C.c_uint16
+        L.orc_layer_set_shift_mode.argtypes = [P, C.c_int]
         L.orc_layer_sizeof.restype = C.c_size_t
         L.orc_layer_capacity.argtypes = [P, C.c_int]
         L.orc_layer_init.argtypes = [P, C.c_int, C.c_int, C.c_int, C.c_int]
@@ -168,6 +174,16 @@ def scale_after_shrink(s2b: float, b: int) -> float:
     return lib().orc_scale_after_shrink(float(s2b), int(b))
 
 
+def drs(x2b: int, b: int) -> int:
+    """Direct Right Shift (the note's ablation): keep the high b bits."""
+    return lib().orc_drs(int(x2b), int(b))
+
+
+def drs_range(r_bits: int, b: int) -> int:
+    """Range after a Direct Right Shift: binary16 RN of fp32(R 2^b / (2^b + 1))."""
+    return lib().orc_drs_range(int(r_bits), int(b))
+
+
 # --- progressive cache model of one block -------------------------------------
 
 class Layer:
@@ -218,6 +234,10 @@ class Layer:
 
     def shrink(self) -> int:
         return lib().orc_layer_force_shrink(C.byref(self._s))
+
+    def set_shift_mode(self, mode: int) -> int:
+        """0: Equivalent Right Shift (default), 1: Direct Right Shift; before the first shrink."""
+        return lib().orc_layer_set_shift_mode(C.byref(self._s), int(mode))
 
     def _arr(self, p, last):
         shape = (self.batch, self.kv_heads, self.n_f, last)
