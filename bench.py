@@ -172,10 +172,13 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- GPU arm
 
-def build_cache(kvq, dev, layers, batch, kv_heads, fbit, tokens, n_f, seed, n_out, chunk=4096):
+def build_cache(kvq, dev, layers, batch, kv_heads, fbit, tokens, n_f, seed, n_out, chunk=4096, shift_mode=None):
     budget = n_f * per_token_bytes(batch, kv_heads, fbit)
     cache = kvq.KVQCache(layers, batch, kv_heads, budget, fbit, device=dev)
     assert cache.max_tokens == n_f, (cache.max_tokens, n_f)
+    if shift_mode is not None:
+        for l in range(layers):
+            cache.set_shift_mode(l, shift_mode)
     for l in range(layers):
         pos = 0
         while pos < tokens:
@@ -194,23 +197,26 @@ def flush_l2(buf):
 
 
 def measure_shrink(kvq, dev, flush_buf, reps=3):
-    """Equivalent Right Shift kernel GB/s (algorithmic: whole region read,
-    half written).  (a) Llama-70B-shape layer (batch 8, 8 KV heads), Fbit 2,
-    a block full with 131072 tokens at 4 bits shrinking to 2 bits.  (b) the
+    """Shrink kernel GB/s (algorithmic: whole region read, half written; the
+    Direct Right Shift also reads and rewrites the meta of every token).
+    (a) Llama-70B-shape layer (batch 8, 8 KV heads), Fbit 2, a block full with
+    131072 tokens at 4 bits shrinking to 2 bits, with either shift.  (b) the
     7B progressive stream (batch 8, 4 KV heads, 32768 tokens at Fbit 2):
     events 16->8 at 4096, 8->4 at 8192, 4->2 at 16384 tokens."""
     res = {}
 
-    def one(batch, kv_heads, n_f, fbit, fill_tokens, tag):
+    def one(batch, kv_heads, n_f, fbit, fill_tokens, tag, direct=False):
         times = []
         nbytes = None
         for r in range(reps):
             cache = build_cache(kvq, dev, 1, batch, kv_heads, [fbit], fill_tokens, n_f, SEED + 17 + r, 10,
-                                chunk=8192)
+                                chunk=8192, shift_mode=kvq.KVQ_SHIFT_DIRECT if direct else None)
             st = cache.query(0)
             assert st["tokens"] == st["capacity"], st
             region = batch * kv_heads * 2 * n_f * 16 * fbit  # code bytes of the block
             nbytes = region + region // 2
+            if direct:  # the meta of every stored token is read and rewritten too
+                nbytes += 2 * batch * kv_heads * st["tokens"] * 2 * 4
             flush_l2(flush_buf)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
@@ -228,6 +234,7 @@ def measure_shrink(kvq, dev, flush_buf, reps=3):
                     "reps": reps}
 
     one(8, 8, 262144, 2, 131072, "llama70b_128k_4to2")
+    one(8, 8, 262144, 2, 131072, "llama70b_128k_4to2_direct_shift", direct=True)
     for tokens, tag in ((4096, "qwen7b_16to8"), (8192, "qwen7b_8to4"), (16384, "qwen7b_4to2")):
         one(8, 4, 32768, 2, tokens, tag)
     return res

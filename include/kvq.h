@@ -102,6 +102,21 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* k, const void* v, int
  * is already at its Fbit. */
 kvq_status kvq_shrink(kvq_cache* c, int layer, kvq_stream_t stream);
 
+/* Shift a block uses when it shrinks (before its first shrink; the default
+ * is the Equivalent Right Shift):
+ *   KVQ_SHIFT_EQUIVALENT  key design 1: X_b = ((2^2b - 2^b + 1)(X_2b + 2^(b-1)))
+ *                         >> 3b, Z_b = Z_2b, S_b = (2^b + 1) S_2b (meta untouched);
+ *   KVQ_SHIFT_DIRECT      the "Direct Right Shift" row of the note's ablation:
+ *                         keep the high b bits, X_b = X_2b >> b, Z_b = Z_2b and
+ *                         the truncation's scale S_b = 2^b S_2b, i.e. every
+ *                         stored range becomes binary16_RN(fp32(R 2^b) / (2^b + 1))
+ *                         (the shrink also rewrites the block's meta).
+ * The ablation's "Modified Right Shift" has no definition on the pages and is
+ * not offered.  Errors: INVALID (mode), STATE (the block has already shrunk
+ * with the other shift). */
+enum { KVQ_SHIFT_EQUIVALENT = 0, KVQ_SHIFT_DIRECT = 1 };
+kvq_status kvq_set_shift_mode(kvq_cache* c, int layer, int mode);
+
 /* Bytes of device workspace kvq_decode_attn needs for this block and number
  * of query heads (any token count).  0 on invalid arguments. */
 size_t kvq_decode_workspace(const kvq_cache* c, int layer, int q_heads);

@@ -15,13 +15,14 @@ from typing import Optional, Sequence
 import numpy as np
 import torch
 
-from ._lib import (KVQ_DTYPE_BF16, KVQ_DTYPE_F32, KVQError, check, load)  # noqa: F401
+from ._lib import (KVQ_DTYPE_BF16, KVQ_DTYPE_F32, KVQ_SHIFT_DIRECT, KVQ_SHIFT_EQUIVALENT,  # noqa: F401
+                   KVQError, check, load)
 
 HEAD_DIM = 128
 
 __all__ = [
     "KVQCache", "KVQError", "load",
-    "kvq_pool_bytes", "kvq_alloc", "kvq_set_lambda", "kvq_append", "kvq_shrink",
+    "kvq_pool_bytes", "kvq_alloc", "kvq_set_lambda", "kvq_append", "kvq_shrink", "kvq_set_shift_mode",
     "kvq_decode_workspace", "kvq_decode_attn", "kvq_decode_attn_noalloc", "kvq_query", "kvq_max_tokens", "kvq_export",
     "kvq_device_status", "kvq_last_error", "kvq_free", "kvq_allocate_bits",
 ]
@@ -88,6 +89,11 @@ def kvq_append(cache, layer: int, k: torch.Tensor, v: torch.Tensor, stream=None)
 
 def kvq_shrink(cache, layer: int, stream=None) -> None:
     check(load().kvq_shrink(cache, layer, _stream_ptr(stream)))
+
+
+def kvq_set_shift_mode(cache, layer: int, mode: int) -> None:
+    """KVQ_SHIFT_EQUIVALENT (default) or KVQ_SHIFT_DIRECT, before the block's first shrink."""
+    check(load().kvq_set_shift_mode(cache, layer, int(mode)))
 
 
 def kvq_decode_workspace(cache, layer: int, q_heads: int) -> int:
@@ -224,6 +230,9 @@ class KVQCache:
 
     def shrink(self, layer: int, stream=None) -> None:
         kvq_shrink(self.handle, layer, stream)
+
+    def set_shift_mode(self, layer: int, mode: int) -> None:
+        kvq_set_shift_mode(self.handle, layer, mode)
 
     def decode_attn(self, layer: int, q: torch.Tensor, sm_scale: Optional[float] = None,
                     out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

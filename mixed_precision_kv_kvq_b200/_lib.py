@@ -24,6 +24,8 @@ STATUS_NAMES = {
 }
 KVQ_DTYPE_BF16 = 0
 KVQ_DTYPE_F32 = 1
+KVQ_SHIFT_EQUIVALENT = 0
+KVQ_SHIFT_DIRECT = 1
 
 # name -> (restype, argtypes); the exported symbols of include/kvq.h
 P = C.c_void_p
@@ -35,6 +37,7 @@ SIGNATURES = {
     "kvq_set_lambda": (I, [P, I, P]),
     "kvq_append": (I, [P, I, P, P, I, I, P]),
     "kvq_shrink": (I, [P, I, P]),
+    "kvq_set_shift_mode": (I, [P, I, I]),
     "kvq_decode_workspace": (SZ, [P, I, I]),
     "kvq_decode_attn": (I, [P, I, P, I, C.c_float, P, P, SZ, P]),
     "kvq_decode_attn_noalloc": (I, [P, I, P, I, C.c_float, P, P]),

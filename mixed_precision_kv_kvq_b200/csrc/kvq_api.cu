@@ -68,6 +68,7 @@ struct LayerState {
   // predecessors completed, and the shrink kernel never triggers early, so
   // only the most recent append kernel of the block can still be running.
   long long n_stable;
+  int shift_mode;  // KVQ_SHIFT_EQUIVALENT or KVQ_SHIFT_DIRECT
   int nt;  // tiles per stream
   int pf;  // meta slots per tile
   bool counters_zeroed;
@@ -110,6 +111,7 @@ bool make_plan(int layers, int batch, int kv_heads, int head_dim, size_t budget,
     L.n = 0;
     L.n_shrinks = 0;
     L.n_stable = 0;
+    L.shift_mode = KVQ_SHIFT_EQUIVALENT;
     L.pf = slots_per_tile(L.fbit);
     L.nt = (int)(n_f / L.pf);
     L.counters_zeroed = false;
@@ -201,6 +203,20 @@ void slot_of(const LayerState& L, long long i, int* tile, int* slot) {
   const long long m = i - (long long)L.nt * h;
   *tile = (int)(m / ee);
   *slot = h + (int)(m % ee);
+}
+
+// Shrink of block `layer` from its current width to half of it.
+ShrinkArgs shrink_args(kvq_cache* c, int layer) {
+  const LayerState& L = c->L[layer];
+  ShrinkArgs sa{};
+  sa.codes = c->codes(layer);
+  sa.n_tiles = (long long)c->batch * c->kv_heads * L.nt;
+  sa.bits_to = L.bits / 2;
+  sa.direct = L.shift_mode == KVQ_SHIFT_DIRECT;
+  sa.meta = c->meta(layer);
+  sa.pf = L.pf;
+  sa.p_from = slots_per_tile(L.bits);
+  return sa;
 }
 
 // Groups (in the kernels' group order, see locate_group) of every stream
@@ -320,7 +336,7 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* k, const void* v, int
   while (off < n_tokens) {
     const long long cap = capacity(L, c->n_f, L.bits);
     if (L.n == cap) {  // full: shrink one level first (bits > fbit is implied by the budget check)
-      ShrinkArgs sa{c->codes(layer), (long long)c->batch * c->kv_heads * L.nt, L.bits / 2};
+      const ShrinkArgs sa = shrink_args(c, layer);
       cudaError_t e = launch_shrink(sa, s);
       if (e != cudaSuccess) return cuda_fail(e, "shrink launch");
       L.bits /= 2;
@@ -365,12 +381,22 @@ kvq_status kvq_shrink(kvq_cache* c, int layer, kvq_stream_t stream) {
   if (L.n != cap)
     return fail(KVQ_ERR_STATE, "layer %d holds %lld tokens; a shrink needs the block full (%lld at %d bits)", layer, L.n, cap,
                 L.bits);
-  ShrinkArgs sa{c->codes(layer), (long long)c->batch * c->kv_heads * L.nt, L.bits / 2};
+  const ShrinkArgs sa = shrink_args(c, layer);
   cudaError_t e = launch_shrink(sa, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "shrink launch");
   L.bits /= 2;
   L.n_shrinks++;
   L.n_stable = L.n;
+  return KVQ_OK;
+}
+
+kvq_status kvq_set_shift_mode(kvq_cache* c, int layer, int mode) {
+  if (kvq_status s = check_layer(c, layer)) return s;
+  if (mode != KVQ_SHIFT_EQUIVALENT && mode != KVQ_SHIFT_DIRECT) return fail(KVQ_ERR_INVALID, "shift mode %d unknown", mode);
+  LayerState& L = c->L[layer];
+  if (L.n_shrinks > 0 && mode != L.shift_mode)
+    return fail(KVQ_ERR_STATE, "layer %d has already shrunk; its shift is fixed", layer);
+  L.shift_mode = mode;
   return KVQ_OK;
 }
 

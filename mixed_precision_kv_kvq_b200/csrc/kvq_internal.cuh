@@ -164,6 +164,10 @@ struct ShrinkArgs {
   uint8_t* codes;     // layer base
   long long n_tiles;  // batch * kv_heads * nt
   int bits_to;        // 8, 4 or 2
+  bool direct;        // Direct Right Shift (also rescales the ranges in meta)
+  uint32_t* meta;     // layer base of the meta (used when direct)
+  int pf;             // meta slots per tile
+  int p_from;         // valid slots per tile before the shrink (the tile is full)
 };
 
 struct DecodeArgs {

@@ -130,6 +130,11 @@ def test_alloc_initial_state_and_validation(kvq):
         assert lib.kvq_set_lambda(h, 0, bad.ctypes.data_as(C.c_void_p)) == 1
         # export of an out-of-range stream
         assert lib.kvq_export(h, 0, 1, 0, None, None, None, None, None) == 1
+        # shift mode: two known modes, per block, before the first shrink
+        assert lib.kvq_set_shift_mode(h, 0, 2) == 1
+        assert lib.kvq_set_shift_mode(h, 1, 1) == 1
+        assert lib.kvq_set_shift_mode(h, 0, kvq.KVQ_SHIFT_DIRECT) == 0
+        assert lib.kvq_set_shift_mode(h, 0, kvq.KVQ_SHIFT_EQUIVALENT) == 0
     finally:
         kvq.kvq_free(h)
 

@@ -55,7 +55,7 @@ def per_token(batch, kv_heads, fbit):
 class Sampled:
     """A full-size GPU block plus oracle replays of a few of its streams."""
 
-    def __init__(self, kvq, orc, batch, kv_heads, n_f, fbit, streams, layer, seed=SEED):
+    def __init__(self, kvq, orc, batch, kv_heads, n_f, fbit, streams, layer, seed=SEED, shift_mode=0):
         self.kvq, self.orc_mod = kvq, orc
         self.batch, self.kv_heads, self.n_f, self.fbit = batch, kv_heads, n_f, fbit
         self.streams, self.layer, self.seed = streams, layer, seed
@@ -65,6 +65,10 @@ class Sampled:
         self.lam = None
         self.pos = 0
         self.n_out = S.outliers_for(kv_heads)
+        if shift_mode:
+            self.gpu.set_shift_mode(0, shift_mode)
+            for o in self.orc.values():
+                assert o.set_shift_mode(shift_mode) == 0
 
     def _set_lambda(self, k):
         self.lam = self.orc_mod.lambda_from_keys(k[0].float().cpu().numpy(), 0.5)
@@ -208,6 +212,22 @@ def test_70b_final_4to2_shrink_then_decode(kvq, orc):
         assert o.shrink() == 0
     st = x.check_state()
     assert st["bits"] == 2
+    x.check_codes()
+    x.check_attention(HQ)
+    x.free()
+
+
+def test_70b_final_4to2_direct_shift_then_decode(kvq, orc):
+    """The same 128K-token 4 -> 2 event with the ablation's Direct Right Shift
+    (codes X >> 2, every stored range rescaled by 4/5)."""
+    B, H, HQ, T = 8, 8, 64, 131072
+    x = Sampled(kvq, orc, B, H, 2 * T, 2, corners(B, H), 2, shift_mode=kvq.KVQ_SHIFT_DIRECT)
+    x.fill(T, chunk=8192)
+    assert x.check_state()["bits"] == 4
+    x.gpu.shrink(0)
+    for o in x.orc.values():
+        assert o.shrink() == 0
+    assert x.check_state()["bits"] == 2
     x.check_codes()
     x.check_attention(HQ)
     x.free()

@@ -36,7 +36,7 @@ def per_token(batch, kv_heads, fbit):
 class Pair:
     """A GPU cache and the oracle's model of the same block, fed identically."""
 
-    def __init__(self, kvq, orc, batch, kv_heads, n_f, fbit, lam=None):
+    def __init__(self, kvq, orc, batch, kv_heads, n_f, fbit, lam=None, shift_mode=0):
         self.batch, self.kv_heads, self.n_f, self.fbit = batch, kv_heads, n_f, fbit
         self.gpu = kvq.KVQCache(1, batch, kv_heads, n_f * per_token(batch, kv_heads, [fbit]), [fbit])
         assert self.gpu.max_tokens == n_f
@@ -44,6 +44,9 @@ class Pair:
         self.lam = lam
         if lam is not None:
             self.gpu.set_lambda(0, lam)
+        if shift_mode:
+            self.gpu.set_shift_mode(0, shift_mode)
+            assert self.orc.set_shift_mode(shift_mode) == 0
 
     def append(self, k, v):
         """k, v: CPU tensors [batch][n][kv_heads][128] (bf16 or fp32)."""
@@ -169,3 +172,46 @@ def test_decode_rejects_small_workspace(kvq, orc):
     with pytest.raises(kvq.KVQError) as e:
         kvq.kvq_decode_attn(P.gpu.handle, 0, q, 0.1, out, ws)
     assert e.value.status == 6
+
+
+# ---------------------------------------------------- Direct Right Shift (ablation)
+
+def test_direct_shift_tiny_config_one_by_one(kvq, orc):
+    """The tiny configuration with the ablation's Direct Right Shift: the same
+    schedule (16 -> 8 at 1024, 8 -> 4 at 2048); codes = X >> b and rescaled
+    ranges bit-exact after every shrink; attention within tolerance."""
+    T = 2100
+    k, v = S.keys_values(5, 0, 1, T, 2, 0, 4, dtype=torch.float32)
+    lam = lam_for(k)
+    P = Pair(kvq, orc, 1, 2, 4096, 4, lam, shift_mode=kvq.KVQ_SHIFT_DIRECT)
+    checkpoints = {1024, 1025, 2048, 2049, 2100}
+    for t in range(T):
+        P.append(k[:, t:t + 1], v[:, t:t + 1])
+        if t + 1 in checkpoints:
+            P.check_codes()
+            P.check_attention(S.queries(5, 0, t, 1, 4, t + 1, dtype=torch.bfloat16))
+    assert P.orc.shrink_at == [1024, 2048]
+    with pytest.raises(kvq.KVQError) as e:
+        P.gpu.set_shift_mode(0, kvq.KVQ_SHIFT_EQUIVALENT)  # fixed once the block has shrunk
+    assert e.value.status == 3
+
+
+@pytest.mark.parametrize("fbit", [2, 8])
+def test_direct_shift_chunked_bf16(kvq, orc, fbit):
+    """Chunks crossing every shrink of a 2-bit block (16 -> 8 -> 4 -> 2) and an
+    8-bit one, batch 3, 4 KV heads, bf16 inputs, Direct Right Shift."""
+    B, H, n_f = 3, 4, 4096
+    cap16 = n_f * fbit // 16
+    k, v = S.keys_values(6, fbit, B, n_f, H, 0, 5, dtype=torch.bfloat16)
+    lam = lam_for(k)
+    P = Pair(kvq, orc, B, H, n_f, fbit, lam, shift_mode=kvq.KVQ_SHIFT_DIRECT)
+    pos = 0
+    for n in (cap16 - 7, 300, 900, 1600, n_f):
+        n = min(n, n_f - pos)
+        if n <= 0:
+            break
+        P.append(k[:, pos:pos + n], v[:, pos:pos + n])
+        pos += n
+    assert P.gpu.query(0)["bits"] == fbit and pos == n_f
+    P.check_codes()
+    P.check_attention(S.queries(6, fbit, 0, B, 4 * H, n_f, dtype=torch.bfloat16))
