@@ -372,6 +372,126 @@ int orc_layer_force_shrink(orc_layer* L) {
 }
 
 /* ------------------------------------------------------------------------ */
+/* Sink token + recent window (training strategy: the KIVI trick the note    */
+/* keeps -- the first token and the most recent 128 tokens are stored as     */
+/* INT16).  Readings: a token is quantized at 16 bits when it arrives; when  */
+/* it leaves the window (token t arrives, t - 128 >= 1 leaves) it moves into */
+/* the block's progressive cache at that cache's current width by the        */
+/* block's own shift applied 16 -> 8 -> ... -> b, R and Z kept (rescaled R   */
+/* under the Direct Right Shift) -- the same codes it would have if it had   */
+/* been stored at 16 bits and shrunk with the block; the sink never leaves.  */
+/* The progressive cache (tokens 1 .. n - 129) follows the budget schedule   */
+/* on its own token count.                                                   */
+/* ------------------------------------------------------------------------ */
+
+#define ORC_WINDOW 128
+
+typedef struct {
+  orc_layer main; /* the progressive cache: token 1 + m at index m */
+  int n;          /* tokens appended */
+  int n_max;      /* main.n_f + 1 + ORC_WINDOW */
+  uint16_t* kc;   /* [batch][kv_heads][n_max][128]: INT16 codes of every token */
+  uint16_t* vc;
+  uint16_t* km; /* [batch][kv_heads][n_max][2] */
+  uint16_t* vm;
+} orc_wlayer;
+
+size_t orc_wlayer_sizeof(void) { return sizeof(orc_wlayer); }
+
+int orc_wlayer_init(orc_wlayer* W, int batch, int kv_heads, int n_f, int fbit) {
+  memset(W, 0, sizeof(*W));
+  int rc = orc_layer_init(&W->main, batch, kv_heads, n_f, fbit);
+  if (rc) return rc;
+  W->n_max = n_f + 1 + ORC_WINDOW;
+  size_t ncode = (size_t)batch * kv_heads * W->n_max * ORC_D;
+  size_t nmeta = (size_t)batch * kv_heads * W->n_max * 2;
+  W->kc = (uint16_t*)calloc(ncode, 2);
+  W->vc = (uint16_t*)calloc(ncode, 2);
+  W->km = (uint16_t*)calloc(nmeta, 2);
+  W->vm = (uint16_t*)calloc(nmeta, 2);
+  if (!W->kc || !W->vc || !W->km || !W->vm) return -2;
+  return 0;
+}
+
+void orc_wlayer_free(orc_wlayer* W) {
+  orc_layer_free(&W->main);
+  free(W->kc);
+  free(W->vc);
+  free(W->km);
+  free(W->vm);
+  memset(W, 0, sizeof(*W));
+}
+
+static size_t orc_wslot(const orc_wlayer* W, int b, int h, int t) {
+  return ((size_t)b * W->main.kv_heads + h) * W->n_max + t;
+}
+
+/* One INT16 code (and its group's range) brought down to `bits` by the
+ * block's shift, one level at a time. */
+static uint32_t orc_chain_code(uint32_t x, int bits, int mode) {
+  for (int b = 8; b >= bits; b /= 2) x = mode == 1 ? orc_drs(x, b) : orc_ers(x, b);
+  return x;
+}
+static uint16_t orc_chain_range(uint16_t r, int bits, int mode) {
+  if (mode == 1)
+    for (int b = 8; b >= bits; b /= 2) r = orc_drs_range(r, b);
+  return r;
+}
+
+/* Move token e (>= 1) from the INT16 store into the progressive cache. */
+static void orc_wlayer_evict(orc_wlayer* W, int e) {
+  orc_layer* L = &W->main;
+  if (L->n == orc_layer_capacity(L, L->bits)) orc_layer_shrink(L); /* budget checked by the caller */
+  for (int bb = 0; bb < L->batch; bb++)
+    for (int h = 0; h < L->kv_heads; h++) {
+      size_t src = orc_wslot(W, bb, h, e), dst = orc_slot(L, bb, h, L->n);
+      for (int c = 0; c < ORC_D; c++) {
+        L->kc[dst * ORC_D + c] = (uint16_t)orc_chain_code(W->kc[src * ORC_D + c], L->bits, L->shift_mode);
+        L->vc[dst * ORC_D + c] = (uint16_t)orc_chain_code(W->vc[src * ORC_D + c], L->bits, L->shift_mode);
+      }
+      L->km[dst * 2] = orc_chain_range(W->km[src * 2], L->bits, L->shift_mode);
+      L->km[dst * 2 + 1] = W->km[src * 2 + 1];
+      L->vm[dst * 2] = orc_chain_range(W->vm[src * 2], L->bits, L->shift_mode);
+      L->vm[dst * 2 + 1] = W->vm[src * 2 + 1];
+    }
+  L->n++;
+}
+
+/* Append n tokens (same arguments as orc_layer_append).  Returns 1 when the
+ * progressive cache could not hold its share at Fbit (nothing written). */
+int orc_wlayer_append(orc_wlayer* W, const float* k, const float* v, int n, const float* lambda) {
+  orc_layer* L = &W->main;
+  if (n < 0) return -1;
+  int64_t main_after = (int64_t)W->n + n - 1 - ORC_WINDOW;
+  if (main_after > (int64_t)L->n_f) return 1;
+  float x[ORC_D];
+  for (int i = 0; i < n; i++) {
+    int t = W->n;
+    for (int bb = 0; bb < L->batch; bb++)
+      for (int h = 0; h < L->kv_heads; h++) {
+        size_t in = (((size_t)bb * n + i) * L->kv_heads + h) * ORC_D;
+        size_t slot = orc_wslot(W, bb, h, t);
+        for (int c = 0; c < ORC_D; c++)
+          x[c] = lambda ? orc_migrate(k[in + c], lambda[h * ORC_D + c]) : k[in + c];
+        orc_quantize_group(x, ORC_D, 16, W->kc + slot * ORC_D, W->km + slot * 2, W->km + slot * 2 + 1);
+        orc_quantize_group(v + in, ORC_D, 16, W->vc + slot * ORC_D, W->vm + slot * 2, W->vm + slot * 2 + 1);
+      }
+    W->n++;
+    if (t - ORC_WINDOW >= 1) orc_wlayer_evict(W, t - ORC_WINDOW);
+  }
+  return 0;
+}
+
+/* Tokens held at INT16: the sink and the window, oldest first. */
+int orc_wlayer_window_tokens(const orc_wlayer* W, int* tokens) {
+  int c = 0;
+  if (W->n > 0) tokens[c++] = 0;
+  int lo = W->n - ORC_WINDOW > 1 ? W->n - ORC_WINDOW : 1;
+  for (int t = lo; t < W->n; t++) tokens[c++] = t;
+  return c;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Decode attention over the quantized cache, fp64.                          */
 /* q: [batch][q_heads][128] (fp32 values of the bf16 queries).               */
 /* lambda: [kv_heads][128] or NULL.  out: [batch][q_heads][128].             */
@@ -417,6 +537,68 @@ int orc_attention(const orc_layer* L, const float* q, int q_heads, const float* 
       }
     }
   free(s);
+  return 0;
+}
+
+/* Decode attention over a block with the sink + window: every token the
+ * block holds -- the sink and the window at 16 bits, the progressive cache
+ * at its width -- dequantized and attended in fp64. */
+int orc_wattention(const orc_wlayer* W, const float* q, int q_heads, const float* lambda, double sm_scale,
+                   double* out) {
+  const orc_layer* L = &W->main;
+  if (W->n <= 0 || q_heads % L->kv_heads) return -1;
+  int g = q_heads / L->kv_heads;
+  int* wt = (int*)malloc(sizeof(int) * (ORC_WINDOW + 1));
+  int nw = orc_wlayer_window_tokens(W, wt);
+  int T = L->n + nw;
+  double* s = (double*)malloc(sizeof(double) * (size_t)T);
+  double qp[ORC_D];
+  if (!s || !wt) return -2;
+  for (int bb = 0; bb < L->batch; bb++)
+    for (int hq = 0; hq < q_heads; hq++) {
+      int h = hq / g;
+      const float* qq = q + ((size_t)bb * q_heads + hq) * ORC_D;
+      for (int c = 0; c < ORC_D; c++)
+        qp[c] = (double)qq[c] * (lambda ? (double)lambda[h * ORC_D + c] : 1.0);
+      double mx = -INFINITY;
+      for (int t = 0; t < T; t++) {
+        const uint16_t *kc, *km;
+        int bits;
+        if (t < L->n) {
+          size_t slot = orc_slot(L, bb, h, t);
+          kc = L->kc + slot * ORC_D, km = L->km + slot * 2, bits = L->bits;
+        } else {
+          size_t slot = orc_wslot(W, bb, h, wt[t - L->n]);
+          kc = W->kc + slot * ORC_D, km = W->km + slot * 2, bits = 16;
+        }
+        double acc = 0.0;
+        for (int c = 0; c < ORC_D; c++) acc += qp[c] * orc_dequant(kc[c], km[0], km[1], bits);
+        s[t] = sm_scale * acc;
+        if (s[t] > mx) mx = s[t];
+      }
+      double den = 0.0;
+      for (int t = 0; t < T; t++) {
+        s[t] = exp(s[t] - mx);
+        den += s[t];
+      }
+      double* o = out + ((size_t)bb * q_heads + hq) * ORC_D;
+      for (int c = 0; c < ORC_D; c++) o[c] = 0.0;
+      for (int t = 0; t < T; t++) {
+        const uint16_t *vc, *vm;
+        int bits;
+        if (t < L->n) {
+          size_t slot = orc_slot(L, bb, h, t);
+          vc = L->vc + slot * ORC_D, vm = L->vm + slot * 2, bits = L->bits;
+        } else {
+          size_t slot = orc_wslot(W, bb, h, wt[t - L->n]);
+          vc = W->vc + slot * ORC_D, vm = W->vm + slot * 2, bits = 16;
+        }
+        double p = s[t] / den;
+        for (int c = 0; c < ORC_D; c++) o[c] += p * orc_dequant(vc[c], vm[0], vm[1], bits);
+      }
+    }
+  free(s);
+  free(wt);
   return 0;
 }
 

@@ -51,6 +51,17 @@ class _Layer(C.Structure):
     ]
 
 
+class _WLayer(C.Structure):
+    _fields_ = [
+        ("main", _Layer), ("n", C.c_int), ("n_max", C.c_int),
+        ("kc", C.POINTER(C.c_uint16)), ("vc", C.POINTER(C.c_uint16)),
+        ("km", C.POINTER(C.c_uint16)), ("vm", C.POINTER(C.c_uint16)),
+    ]
+
+
+WINDOW = 128
+
+
 def lib():
     global _lib
     if _lib is None:
@@ -80,6 +91,12 @@ def lib():
         L.orc_drs_range.argtypes = [C.c_uint16, C.c_int]
         L.orc_drs_range.restype = C.c_uint16
         L.orc_layer_set_shift_mode.argtypes = [P, C.c_int]
+        L.orc_wlayer_sizeof.restype = C.c_size_t
+        L.orc_wlayer_init.argtypes = [P, C.c_int, C.c_int, C.c_int, C.c_int]
+        L.orc_wlayer_free.argtypes = [P]
+        L.orc_wlayer_append.argtypes = [P, P, P, C.c_int, P]
+        L.orc_wlayer_window_tokens.argtypes = [P, P]
+        L.orc_wattention.argtypes = [P, P, C.c_int, P, C.c_double, P]
         L.orc_layer_sizeof.restype = C.c_size_t
         L.orc_layer_capacity.argtypes = [P, C.c_int]
         L.orc_layer_init.argtypes = [P, C.c_int, C.c_int, C.c_int, C.c_int]
@@ -91,6 +108,7 @@ def lib():
         L.orc_attention_dense.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, C.c_int,
                                           C.c_double, P]
         assert L.orc_layer_sizeof() == C.sizeof(_Layer)
+        assert L.orc_wlayer_sizeof() == C.sizeof(_WLayer)
     return _lib
 
 
@@ -197,6 +215,8 @@ class Layer:
         self.batch, self.kv_heads, self.n_f, self.fbit = batch, kv_heads, n_f, fbit
 
     def __del__(self):
+        if getattr(self, "_view", False):  # owned by a WLayer
+            return
         try:
             lib().orc_layer_free(C.byref(self._s))
         except Exception:
@@ -314,3 +334,77 @@ def allocate_bits_brute(sens, bits, batch: int, kv_heads: int, max_tokens: int, 
         elif abs(obj - best) <= 1e-12 * max(1.0, abs(best)):
             arg.append(tuple(bits[o] for o in choice))
     return best, arg
+
+
+class WLayer:
+    """A block with the sink token and the recent-128 window held at INT16
+    (training strategy of the PM-KVQ note: the KIVI trick it keeps); older
+    tokens live in the block's progressive cache (`main`, a Layer view)."""
+
+    def __init__(self, batch: int, kv_heads: int, n_f: int, fbit: int):
+        self._s = _WLayer()
+        rc = lib().orc_wlayer_init(C.byref(self._s), batch, kv_heads, n_f, fbit)
+        if rc != 0:
+            raise ValueError(f"orc_wlayer_init failed ({rc})")
+        self.batch, self.kv_heads, self.n_f, self.fbit = batch, kv_heads, n_f, fbit
+        self.main = Layer.__new__(Layer)  # a view of the embedded progressive cache
+        self.main._s = self._s.main
+        self.main.batch, self.main.kv_heads, self.main.n_f, self.main.fbit = batch, kv_heads, n_f, fbit
+        self.main._view = True
+
+    def __del__(self):
+        try:
+            lib().orc_wlayer_free(C.byref(self._s))
+        except Exception:
+            pass
+
+    @property
+    def n(self) -> int:
+        return self._s.n
+
+    def set_shift_mode(self, mode: int) -> int:
+        return lib().orc_layer_set_shift_mode(C.byref(self._s.main), int(mode))
+
+    def append(self, k: np.ndarray, v: np.ndarray, lam: np.ndarray | None) -> int:
+        k = np.ascontiguousarray(k, dtype=np.float32)
+        v = np.ascontiguousarray(v, dtype=np.float32)
+        assert k.shape == v.shape and k.shape[0] == self.batch and k.shape[2] == self.kv_heads
+        lp = None
+        if lam is not None:
+            lam = np.ascontiguousarray(lam, dtype=np.float32)
+            lp = _ptr(lam)
+        return lib().orc_wlayer_append(C.byref(self._s), _ptr(k), _ptr(v), k.shape[1], lp)
+
+    def window_tokens(self) -> list:
+        """Token indices held at INT16: the sink, then the window oldest first."""
+        out = (C.c_int * (WINDOW + 1))()
+        n = lib().orc_wlayer_window_tokens(C.byref(self._s), out)
+        return list(out[:n])
+
+    def _all(self, p, last):
+        shape = (self.batch, self.kv_heads, self._s.n_max, last)
+        return np.ctypeslib.as_array(p, shape=(int(np.prod(shape)),)).reshape(shape)
+
+    def int16_codes(self):
+        """(k codes, v codes, k meta, v meta) of every appended token at INT16,
+        [batch][kv_heads][n][...] (tokens since moved keep their INT16 record)."""
+        n = self.n
+        return tuple(self._all(p, d)[:, :, :n].copy() for p, d in
+                     ((self._s.kc, HEAD_DIM), (self._s.vc, HEAD_DIM), (self._s.km, 2), (self._s.vm, 2)))
+
+    def window_codes(self):
+        """The sink and window tokens' INT16 codes and meta, oldest first."""
+        idx = self.window_tokens()
+        return tuple(a[:, :, idx] for a in self.int16_codes())
+
+    def attention(self, q: np.ndarray, lam: np.ndarray | None, sm_scale: float) -> np.ndarray:
+        q = np.ascontiguousarray(q, dtype=np.float32)
+        out = np.empty(q.shape, np.float64)
+        lp = None
+        if lam is not None:
+            lam = np.ascontiguousarray(lam, dtype=np.float32)
+            lp = _ptr(lam)
+        rc = lib().orc_wattention(C.byref(self._s), _ptr(q), q.shape[1], lp, float(sm_scale), _ptr(out))
+        if rc != 0:
+            raise ValueError(f"orc_wattention failed ({rc})")
+        return out

@@ -363,6 +363,118 @@ def test_progressive_model_with_drs(orc):
     assert L.set_shift_mode(0) == -2  # fixed once the block has shrunk
 
 
+# ------------------------------------------ sink token + recent window at INT16
+
+def _chain(orc, codes, bits, mode=0):
+    """Shift INT16 codes down to `bits` one level at a time (Python, from the
+    operators pinned above)."""
+    out = codes.astype(np.int64)
+    b = 8
+    while b >= bits:
+        f = (lambda x, b=b: orc.drs(int(x), b)) if mode else (lambda x, b=b: orc.ers(int(x), b))
+        out = np.vectorize(f)(out)
+        b //= 2
+    return out
+
+
+def test_window_short_block_is_all_int16(orc):
+    """Up to 129 tokens everything is held at INT16: the progressive cache is
+    empty and attention equals that of a 16-bit block of the same tokens."""
+    k, v = _cfg0_inputs(129, seed=7)
+    W = orc.WLayer(1, 2, 4096, 4)
+    P = orc.Layer(1, 2, 4096, 16)
+    assert W.append(k, v, None) == 0 and P.append(k, v, None) == 0
+    assert W.main.n == 0 and W.window_tokens() == list(range(129))
+    q = torch.randn(1, 4, 128, generator=torch.Generator().manual_seed(1)).numpy()
+    np.testing.assert_allclose(W.attention(q, None, 0.1), P.attention(q, None, 0.1), rtol=1e-13, atol=1e-13)
+    kc, vc, km, vm = W.window_codes()
+    assert np.array_equal(kc, P.k_codes()) and np.array_equal(km, P.k_meta())
+
+
+def test_window_fbit16_block_equals_plain_block(orc):
+    """A 16-bit block never shrinks, so moving a token out of the window
+    changes nothing: codes and attention equal the plain block's."""
+    k, v = _cfg0_inputs(700, seed=8)
+    W = orc.WLayer(1, 2, 1024, 16)
+    P = orc.Layer(1, 2, 1024, 16)
+    W.append(k, v, None)
+    P.append(k, v, None)
+    assert W.main.n == 700 - 129
+    assert np.array_equal(W.main.k_codes(), P.k_codes()[:, :, 1:1 + W.main.n])
+    assert np.array_equal(W.main.v_meta(), P.v_meta()[:, :, 1:1 + W.main.n])
+    q = torch.randn(1, 4, 128, generator=torch.Generator().manual_seed(2)).numpy()
+    np.testing.assert_allclose(W.attention(q, None, 0.1), P.attention(q, None, 0.1), rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_window_moved_tokens_are_the_shift_chain(orc, mode):
+    """Tokens that left the window hold the block's shift chain of their INT16
+    codes (ERS; or the direct shift with its range chain), whatever the
+    shrinks in between; Z is kept."""
+    k, v = _cfg0_inputs(900, seed=9)
+    W = orc.WLayer(1, 2, 1024, 2)  # shrinks at progressive counts 128, 256, 512
+    assert W.set_shift_mode(mode) == 0
+    for t0 in range(0, 900, 150):
+        assert W.append(k[:, t0:t0 + 150], v[:, t0:t0 + 150], None) == 0
+    m = W.main
+    assert m.n == 900 - 129 and m.bits == 2 and m.shrink_at == [128, 256, 512]
+    kc16, vc16, km16, vm16 = W.int16_codes()
+    sel = slice(1, 1 + m.n)
+    assert np.array_equal(m.k_codes(), _chain(orc, kc16[:, :, sel], m.bits, mode))
+    assert np.array_equal(m.v_codes(), _chain(orc, vc16[:, :, sel], m.bits, mode))
+    assert np.array_equal(m.k_meta()[..., 1], km16[:, :, sel, 1])
+    if mode:
+        rr = km16[:, :, sel, 0].astype(np.int64)
+        for b in (8, 4, 2):
+            rr = np.vectorize(lambda r, b=b: orc.drs_range(int(r), b))(rr)
+        assert np.array_equal(m.k_meta()[..., 0], rr)
+    else:
+        assert np.array_equal(m.k_meta(), km16[:, :, sel])
+    assert W.window_tokens() == [0] + list(range(900 - 128, 900))
+
+
+def test_window_chunked_equals_token_by_token(orc):
+    k, v = _cfg0_inputs(700, seed=10)
+    lam = np.exp(np.random.default_rng(3).uniform(0, 1.5, (2, 128))).astype(np.float32)
+    A = orc.WLayer(1, 2, 1024, 4)
+    B = orc.WLayer(1, 2, 1024, 4)
+    for t in range(700):
+        assert A.append(k[:, t:t + 1], v[:, t:t + 1], lam) == 0
+    for t0 in range(0, 700, 97):
+        assert B.append(k[:, t0:t0 + 97], v[:, t0:t0 + 97], lam) == 0
+    assert A.main.n_shrinks == B.main.n_shrinks == 2
+    for x, y in zip(A.int16_codes() + (A.main.k_codes(), A.main.v_codes(), A.main.k_meta()),
+                    B.int16_codes() + (B.main.k_codes(), B.main.v_codes(), B.main.k_meta())):
+        assert np.array_equal(x, y)
+
+
+def test_window_attention_over_three_segments(orc):
+    """Attention of a windowed block = dense fp64 attention over the
+    dequantized sink, progressive cache and window, assembled here."""
+    k, v = _cfg0_inputs(400, seed=11)
+    lam = np.exp(np.random.default_rng(4).uniform(0, 1.0, (2, 128))).astype(np.float32)
+    W = orc.WLayer(1, 2, 512, 4)
+    W.append(k, v, lam)
+    m = W.main
+    wk, wv, wkm, wvm = W.window_codes()
+    K = np.concatenate([orc.dequant_array(m.k_codes(), m.k_meta(), m.bits), orc.dequant_array(wk, wkm, 16)], axis=2)
+    V = np.concatenate([orc.dequant_array(m.v_codes(), m.v_meta(), m.bits), orc.dequant_array(wv, wvm, 16)], axis=2)
+    q = torch.randn(1, 4, 128, generator=torch.Generator().manual_seed(5)).numpy()
+    qp = q[0].astype(np.float64) * np.repeat(lam.astype(np.float64), 2, axis=0)
+    want = orc.attention_dense(qp, K[0].transpose(1, 0, 2), V[0].transpose(1, 0, 2), 0.1)
+    np.testing.assert_allclose(W.attention(q, lam, 0.1)[0], want, rtol=1e-11, atol=1e-12)
+
+
+def test_window_budget(orc):
+    """The progressive cache holds N_F tokens at Fbit; with the sink and the
+    window the block refuses the (N_F + 130)-th token."""
+    k, v = _cfg0_inputs(512 + 130, seed=12)
+    W = orc.WLayer(1, 2, 512, 4)
+    assert W.append(k[:, :512 + 129], v[:, :512 + 129], None) == 0
+    assert W.main.n == 512 and W.main.bits == 4
+    assert W.append(k[:, -1:], v[:, -1:], None) == 1 and W.n == 512 + 129
+
+
 # ---------------------------------------------------------------- attention
 
 def _small_layer(orc, T, bits_target=4, seed=0, lam=None):
