@@ -172,10 +172,11 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- GPU arm
 
-def build_cache(kvq, dev, layers, batch, kv_heads, fbit, tokens, n_f, seed, n_out, chunk=4096, shift_mode=None):
+def build_cache(kvq, dev, layers, batch, kv_heads, fbit, tokens, n_f, seed, n_out, chunk=4096, shift_mode=None,
+                sink_window=False):
     budget = n_f * per_token_bytes(batch, kv_heads, fbit)
-    cache = kvq.KVQCache(layers, batch, kv_heads, budget, fbit, device=dev)
-    assert cache.max_tokens == n_f, (cache.max_tokens, n_f)
+    cache = kvq.KVQCache(layers, batch, kv_heads, budget, fbit, device=dev, sink_window=sink_window)
+    assert cache.max_tokens == n_f + (129 if sink_window else 0), (cache.max_tokens, n_f)
     if shift_mode is not None:
         for l in range(layers):
             cache.set_shift_mode(l, shift_mode)
@@ -280,42 +281,49 @@ def measure_decode_configs(kvq, dev, reps=20):
     cfgs = (("qwen7b", 16, 4, 28, 32768, 32768 + ROOM),
             ("qwen32b", 16, 8, 40, 32768, 55296),
             ("llama70b", 8, 8, 64, 131072, 131072))
-    for name, batch, kv_heads, q_heads, tokens, n_f in cfgs:
-        for fbit in (2, 4):
-            cache = build_cache(kvq, dev, 1, batch, kv_heads, [fbit], tokens, n_f, SEED + 31, S.outliers_for(kv_heads),
-                                chunk=8192)
-            assert cache.query(0)["bits"] == fbit
-            q = S.queries(SEED, 0, 0, batch, q_heads, tokens, dtype=torch.bfloat16, device=dev)
-            out = torch.empty((batch, q_heads, HEAD_DIM), dtype=torch.float32, device=dev)
-            ws = cache.workspace(0, q_heads)
-            a = _decode_args(kvq, cache, q, out, ws, stream)
-            for _ in range(3):
-                kvq.check(lib.kvq_decode_attn(*a))
-            torch.cuda.synchronize(dev)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(reps):
-                lib.kvq_decode_attn(*a)
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-            cache.device_status()
-            us = e0.elapsed_time(e1) / reps * 1e3
-            nb = decode_bytes(batch, kv_heads, q_heads, tokens, fbit)
-            res[f"{name}_{fbit}bit"] = {"us": round(us, 2), "gbs": round(nb / us / 1e3, 1), "bytes": nb,
-                                        "batch": batch, "kv_heads": kv_heads, "q_heads": q_heads, "tokens": tokens}
-            cache.free()
-            del cache
-    res["timing"] = f"{reps} back-to-back launches on one block, CUDA events around the batch, mean per launch"
+    runs = [(c, fbit, False) for c in cfgs for fbit in (2, 4)]
+    runs.append((("qwen7b_sink_window", 16, 4, 28, 32768 + 129, 32768), 2, True))
+    for (name, batch, kv_heads, q_heads, tokens, n_f), fbit, window in runs:
+        cache = build_cache(kvq, dev, 1, batch, kv_heads, [fbit], tokens, n_f, SEED + 31, S.outliers_for(kv_heads),
+                            chunk=8192, sink_window=window)
+        assert cache.query(0)["bits"] == fbit
+        q = S.queries(SEED, 0, 0, batch, q_heads, tokens, dtype=torch.bfloat16, device=dev)
+        out = torch.empty((batch, q_heads, HEAD_DIM), dtype=torch.float32, device=dev)
+        ws = cache.workspace(0, q_heads)
+        a = _decode_args(kvq, cache, q, out, ws, stream)
+        for _ in range(3):
+            kvq.check(lib.kvq_decode_attn(*a))
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            lib.kvq_decode_attn(*a)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        cache.device_status()
+        us = e0.elapsed_time(e1) / reps * 1e3
+        nb = decode_bytes(batch, kv_heads, q_heads, tokens, fbit)
+        if window:  # the sink and the window are read at 16 bits
+            nb = decode_bytes(batch, kv_heads, q_heads, tokens - 129, fbit) + \
+                decode_bytes(batch, kv_heads, q_heads, 129, 16) - batch * q_heads * HEAD_DIM * (2 + 4)
+        res[f"{name}_{fbit}bit"] = {"us": round(us, 2), "gbs": round(nb / us / 1e3, 1), "bytes": nb,
+                                    "batch": batch, "kv_heads": kv_heads, "q_heads": q_heads, "tokens": tokens}
+        cache.free()
+        del cache
+    res["timing"] = (f"{reps} back-to-back calls on one block, CUDA events around the batch, mean per call "
+                     "(with the sink + window: two launches a call, the window at 16 bits and the rest)")
     return res
 
 
-def measure_append_token(kvq, dev, reps=200):
+def measure_append_token(kvq, dev, reps=200, sink_window=False):
     """Single-token append on a 7B-shaped block (batch 16, 4 KV heads, 2-bit,
-    32768 tokens cached): `reps` back-to-back calls through the C ABI, mean."""
+    32768 tokens cached): `reps` back-to-back calls through the C ABI, mean.
+    With the sink + window every call also moves the token leaving the window."""
     import ctypes as C
     lib = kvq.load()
     stream = torch.cuda.current_stream(dev)
-    cache = build_cache(kvq, dev, 1, B7, HKV7, [2], T7, T7 + ROOM, SEED + 41, S.outliers_for(HKV7), chunk=8192)
+    cache = build_cache(kvq, dev, 1, B7, HKV7, [2], T7, T7 + ROOM, SEED + 41, S.outliers_for(HKV7), chunk=8192,
+                        sink_window=sink_window)
     g = torch.Generator(device=dev)
     g.manual_seed(SEED + 43)
     kin = torch.randn((reps + 3, B7, 1, HKV7, HEAD_DIM), generator=g, device=dev).to(torch.bfloat16)
@@ -570,6 +578,7 @@ def run_gpu(args, rank, world):
         extra["shrink"]["unit"] = "GB/s"
         extra["append_chunk"] = measure_append_chunk(kvq, dev, flush)
         extra["append_token"] = measure_append_token(kvq, dev)
+        extra["append_token_sink_window"] = measure_append_token(kvq, dev, sink_window=True)
         extra["decode_configs"] = measure_decode_configs(kvq, dev)
         extra["decode_graph"] = graph
     res = {

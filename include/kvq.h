@@ -68,6 +68,26 @@ enum { KVQ_DTYPE_BF16 = 0, KVQ_DTYPE_F32 = 1 };
 size_t kvq_pool_bytes(int layers, int batch, int kv_heads, int head_dim, size_t budget_bytes,
                       const int* fbit /* host [layers], each 2, 4, 8 or 16 */);
 
+/* Options of kvq_pool_bytes_ex / kvq_alloc_ex.
+ *   KVQ_OPT_SINK_WINDOW  the deployed configuration of the pages (training
+ *     strategy, the KIVI trick the note keeps): every block holds token 0
+ *     (the sink) and its latest 128 tokens at 16 bits; a token that leaves
+ *     the window moves into the block's progressive cache at that cache's
+ *     current width by the block's shift applied 16 -> 8 -> ... -> b (R and Z
+ *     kept; R rescaled under KVQ_SHIFT_DIRECT) -- the codes it would have had
+ *     had it been stored at 16 bits and shrunk with the block.  The budget
+ *     rule (N tokens per block) applies to the progressive cache; the window
+ *     adds 5 tiles of 16 KiB plus 1,280 bytes of meta per (sequence, KV head)
+ *     and block to the pool, outside the budget.  With the option: kvq_query
+ *     reports every token (tokens), the progressive cache's width (bits) and
+ *     capacity + 129; kvq_max_tokens is N + 129; kvq_export returns the
+ *     progressive cache (tokens 1 .. n-129) and kvq_export_window the sink
+ *     and the window; kvq_shrink needs the progressive cache full;
+ *     attention covers all three. */
+enum { KVQ_OPT_SINK_WINDOW = 1 };
+size_t kvq_pool_bytes_ex(int layers, int batch, int kv_heads, int head_dim, size_t budget_bytes,
+                         const int* fbit, int options);
+
 /* Create a cache.  fbit: host [layers].  dev_pool: a device buffer of at least
  * kvq_pool_bytes(...) bytes, owned by the caller and kept alive until
  * kvq_free; or NULL, and the library cudaMallocs the pool itself.  With a
@@ -76,6 +96,12 @@ size_t kvq_pool_bytes(int layers, int batch, int kv_heads, int head_dim, size_t 
  * smaller than 512 tokens), OOM. */
 kvq_status kvq_alloc(kvq_cache** out, int layers, int batch, int kv_heads, int head_dim,
                      size_t budget_bytes, const int* fbit, void* dev_pool, size_t pool_bytes);
+
+/* kvq_alloc with options (KVQ_OPT_*; 0 = kvq_alloc).  dev_pool, when given,
+ * must hold kvq_pool_bytes_ex(..., options) bytes.  Errors as kvq_alloc;
+ * INVALID for unknown option bits. */
+kvq_status kvq_alloc_ex(kvq_cache** out, int layers, int batch, int kv_heads, int head_dim,
+                        size_t budget_bytes, const int* fbit, void* dev_pool, size_t pool_bytes, int options);
 
 /* Per-channel migration factor of one block (key design 3).  lambda_host:
  * host float [kv_heads][128], every value finite and > 0.  Stored Keys become
@@ -165,6 +191,16 @@ int kvq_max_tokens(const kvq_cache* c);
 kvq_status kvq_export(const kvq_cache* c, int layer, int b, int j, uint16_t* k_codes,
                       uint16_t* v_codes, uint16_t* k_meta, uint16_t* v_meta,
                       kvq_stream_t stream);
+
+/* The sink and window tokens of one stream (caches made with
+ * KVQ_OPT_SINK_WINDOW), oldest first: token 0, then the latest min(n - 1,
+ * 128) tokens, at 16 bits:
+ *   k_codes, v_codes: host uint16 [129][128]; k_meta, v_meta: host uint16 [129][2]
+ * (buffers for 129 tokens; the first *n_tokens rows are written).  Any of
+ * the four may be NULL.  Synchronous.  Errors: INVALID (no window, stream). */
+kvq_status kvq_export_window(const kvq_cache* c, int layer, int b, int j, uint16_t* k_codes,
+                             uint16_t* v_codes, uint16_t* k_meta, uint16_t* v_meta, int* n_tokens,
+                             kvq_stream_t stream);
 
 /* Wait for the stream and report whether a kernel of this cache gave up on a
  * bounded wait (KVQ_ERR_TIMEOUT) since the last check; clears the flag. */

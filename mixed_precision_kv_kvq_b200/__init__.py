@@ -15,14 +15,14 @@ from typing import Optional, Sequence
 import numpy as np
 import torch
 
-from ._lib import (KVQ_DTYPE_BF16, KVQ_DTYPE_F32, KVQ_SHIFT_DIRECT, KVQ_SHIFT_EQUIVALENT,  # noqa: F401
-                   KVQError, check, load)
+from ._lib import (KVQ_DTYPE_BF16, KVQ_DTYPE_F32, KVQ_OPT_SINK_WINDOW, KVQ_SHIFT_DIRECT,  # noqa: F401
+                   KVQ_SHIFT_EQUIVALENT, WINDOW_TOKENS, KVQError, check, load)
 
 HEAD_DIM = 128
 
 __all__ = [
     "KVQCache", "KVQError", "load",
-    "kvq_pool_bytes", "kvq_alloc", "kvq_set_lambda", "kvq_append", "kvq_shrink", "kvq_set_shift_mode",
+    "kvq_pool_bytes", "kvq_pool_bytes_ex", "kvq_alloc", "kvq_alloc_ex", "kvq_export_window", "kvq_set_lambda", "kvq_append", "kvq_shrink", "kvq_set_shift_mode",
     "kvq_decode_workspace", "kvq_decode_attn", "kvq_decode_attn_noalloc", "kvq_query", "kvq_max_tokens", "kvq_export",
     "kvq_device_status", "kvq_last_error", "kvq_free", "kvq_allocate_bits",
 ]
@@ -54,13 +54,23 @@ def kvq_pool_bytes(layers: int, batch: int, kv_heads: int, head_dim: int, budget
     return load().kvq_pool_bytes(layers, batch, kv_heads, head_dim, budget_bytes, _fbit_array(fbit))
 
 
+def kvq_pool_bytes_ex(layers: int, batch: int, kv_heads: int, head_dim: int, budget_bytes: int,
+                      fbit: Sequence[int], options: int) -> int:
+    return load().kvq_pool_bytes_ex(layers, batch, kv_heads, head_dim, budget_bytes, _fbit_array(fbit), options)
+
+
 def kvq_alloc(layers: int, batch: int, kv_heads: int, head_dim: int, budget_bytes: int,
               fbit: Sequence[int], dev_pool: Optional[torch.Tensor] = None) -> C.c_void_p:
+    return kvq_alloc_ex(layers, batch, kv_heads, head_dim, budget_bytes, fbit, dev_pool, 0)
+
+
+def kvq_alloc_ex(layers: int, batch: int, kv_heads: int, head_dim: int, budget_bytes: int,
+                 fbit: Sequence[int], dev_pool: Optional[torch.Tensor] = None, options: int = 0) -> C.c_void_p:
     h = C.c_void_p()
     pool_ptr = _dptr(dev_pool) if dev_pool is not None else C.c_void_p(None)
     pool_bytes = dev_pool.numel() * dev_pool.element_size() if dev_pool is not None else 0
-    check(load().kvq_alloc(C.byref(h), layers, batch, kv_heads, head_dim, budget_bytes,
-                           _fbit_array(fbit), pool_ptr, pool_bytes))
+    check(load().kvq_alloc_ex(C.byref(h), layers, batch, kv_heads, head_dim, budget_bytes,
+                              _fbit_array(fbit), pool_ptr, pool_bytes, options))
     return h
 
 
@@ -140,9 +150,13 @@ def kvq_max_tokens(cache) -> int:
     return load().kvq_max_tokens(cache)
 
 
-def kvq_export(cache, layer: int, b: int, j: int, stream=None):
-    """-> (k_codes [T][128], v_codes [T][128], k_meta [T][2], v_meta [T][2]) uint16 numpy."""
+def kvq_export(cache, layer: int, b: int, j: int, stream=None, sink_window: bool = False):
+    """-> (k_codes [T][128], v_codes [T][128], k_meta [T][2], v_meta [T][2]) uint16 numpy.
+    With the sink + window option (sink_window=True) T counts the
+    progressive cache only: tokens 1 .. n - 129."""
     T = kvq_query(cache, layer)["tokens"]
+    if sink_window:
+        T = max(0, T - WINDOW_TOKENS - 1)
     kc = np.zeros((T, HEAD_DIM), np.uint16)
     vc = np.zeros((T, HEAD_DIM), np.uint16)
     km = np.zeros((T, 2), np.uint16)
@@ -150,6 +164,20 @@ def kvq_export(cache, layer: int, b: int, j: int, stream=None):
     p = lambda a: a.ctypes.data_as(C.c_void_p)  # noqa: E731
     check(load().kvq_export(cache, layer, b, j, p(kc), p(vc), p(km), p(vm), _stream_ptr(stream)))
     return kc, vc, km, vm
+
+
+def kvq_export_window(cache, layer: int, b: int, j: int, stream=None):
+    """-> (k_codes [n][128], v_codes, k_meta [n][2], v_meta) uint16 numpy: the
+    sink and window tokens at 16 bits, oldest first."""
+    n1 = WINDOW_TOKENS + 1
+    kc = np.zeros((n1, HEAD_DIM), np.uint16)
+    vc = np.zeros((n1, HEAD_DIM), np.uint16)
+    km = np.zeros((n1, 2), np.uint16)
+    vm = np.zeros((n1, 2), np.uint16)
+    n = C.c_int()
+    p = lambda a: a.ctypes.data_as(C.c_void_p)  # noqa: E731
+    check(load().kvq_export_window(cache, layer, b, j, p(kc), p(vc), p(km), p(vm), C.byref(n), _stream_ptr(stream)))
+    return kc[:n.value], vc[:n.value], km[:n.value], vm[:n.value]
 
 
 def kvq_device_status(cache, stream=None) -> None:
@@ -191,15 +219,17 @@ class KVQCache:
     the call (pinned memory makes the copy asynchronous)."""
 
     def __init__(self, layers: int, batch: int, kv_heads: int, budget_bytes: int,
-                 fbit: Sequence[int], head_dim: int = HEAD_DIM, device=None):
+                 fbit: Sequence[int], head_dim: int = HEAD_DIM, device=None, sink_window: bool = False):
         self.layers, self.batch, self.kv_heads = layers, batch, kv_heads
         self.fbit = list(fbit)
         self.device = torch.device(device if device is not None else "cuda")
-        nbytes = kvq_pool_bytes(layers, batch, kv_heads, head_dim, budget_bytes, fbit)
+        self.sink_window = sink_window
+        options = KVQ_OPT_SINK_WINDOW if sink_window else 0
+        nbytes = kvq_pool_bytes_ex(layers, batch, kv_heads, head_dim, budget_bytes, fbit, options)
         if nbytes == 0:
             raise KVQError(1, "invalid cache parameters or budget too small")
         self.pool = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
-        self.handle = kvq_alloc(layers, batch, kv_heads, head_dim, budget_bytes, fbit, self.pool)
+        self.handle = kvq_alloc_ex(layers, batch, kv_heads, head_dim, budget_bytes, fbit, self.pool, options)
         self._ws = {}
         self._stage = {}
 
@@ -252,7 +282,10 @@ class KVQCache:
         return kvq_max_tokens(self.handle)
 
     def export(self, layer: int, b: int, j: int, stream=None):
-        return kvq_export(self.handle, layer, b, j, stream)
+        return kvq_export(self.handle, layer, b, j, stream, self.sink_window)
+
+    def export_window(self, layer: int, b: int, j: int, stream=None):
+        return kvq_export_window(self.handle, layer, b, j, stream)
 
     def device_status(self, stream=None) -> None:
         kvq_device_status(self.handle, stream)

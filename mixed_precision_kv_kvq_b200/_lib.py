@@ -26,6 +26,8 @@ KVQ_DTYPE_BF16 = 0
 KVQ_DTYPE_F32 = 1
 KVQ_SHIFT_EQUIVALENT = 0
 KVQ_SHIFT_DIRECT = 1
+KVQ_OPT_SINK_WINDOW = 1
+WINDOW_TOKENS = 128
 
 # name -> (restype, argtypes); the exported symbols of include/kvq.h
 P = C.c_void_p
@@ -33,7 +35,9 @@ I = C.c_int
 SZ = C.c_size_t
 SIGNATURES = {
     "kvq_pool_bytes": (SZ, [I, I, I, I, SZ, P]),
+    "kvq_pool_bytes_ex": (SZ, [I, I, I, I, SZ, P, I]),
     "kvq_alloc": (I, [C.POINTER(P), I, I, I, I, SZ, P, P, SZ]),
+    "kvq_alloc_ex": (I, [C.POINTER(P), I, I, I, I, SZ, P, P, SZ, I]),
     "kvq_set_lambda": (I, [P, I, P]),
     "kvq_append": (I, [P, I, P, P, I, I, P]),
     "kvq_shrink": (I, [P, I, P]),
@@ -44,6 +48,7 @@ SIGNATURES = {
     "kvq_query": (I, [P, I, P, P, P, P]),
     "kvq_max_tokens": (I, [P]),
     "kvq_export": (I, [P, I, I, I, P, P, P, P, P]),
+    "kvq_export_window": (I, [P, I, I, I, P, P, P, P, P, P]),
     "kvq_device_status": (I, [P, P]),
     "kvq_allocate_bits": (I, [I, I, P, P, I, I, I, C.c_longlong, SZ, P, P]),
     "kvq_last_error": (C.c_char_p, []),

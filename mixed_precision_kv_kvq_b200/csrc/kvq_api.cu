@@ -73,6 +73,10 @@ struct LayerState {
   int pf;  // meta slots per tile
   bool counters_zeroed;
   size_t off_lam, off_lam_inv, off_perm, off_counters, off_codes, off_meta;
+  // sink + window option: n counts the progressive cache; n_all every token
+  bool window;
+  long long n_all;
+  size_t off_wcodes, off_wmeta;
   bool lambda_set;
   std::vector<uint8_t> perm;  // host copy of the Key channel order [kv_heads][128]
 };
@@ -84,10 +88,12 @@ struct Plan {
 };
 
 // Budget split: every block holds the same N tokens at its own Fbit.
-bool make_plan(int layers, int batch, int kv_heads, int head_dim, size_t budget, const int* fbit, Plan& p,
-               kvq_status* why) {
+bool make_plan(int layers, int batch, int kv_heads, int head_dim, size_t budget, const int* fbit, int options,
+               Plan& p, kvq_status* why) {
   *why = KVQ_ERR_INVALID;
   if (layers < 1 || batch < 1 || kv_heads < 1 || head_dim != kHeadDim || !fbit) return false;
+  if (options & ~KVQ_OPT_SINK_WINDOW) return false;
+  const bool window = (options & KVQ_OPT_SINK_WINDOW) != 0;
   unsigned long long per_token = 0;  // bytes per token over all blocks
   const unsigned long long streams = (unsigned long long)batch * kv_heads * 2;
   for (int l = 0; l < layers; l++) {
@@ -128,6 +134,15 @@ bool make_plan(int layers, int batch, int kv_heads, int head_dim, size_t budget,
     off += align_up(n_streams * (size_t)L.nt * kTileBytes);
     L.off_meta = off;
     off += align_up(n_streams * (size_t)L.nt * L.pf * 8);
+    L.window = window;
+    L.n_all = 0;
+    L.off_wcodes = L.off_wmeta = 0;
+    if (window) {  // token 0 and the latest 128 tokens at 16 bits, outside the budget rule
+      L.off_wcodes = off;
+      off += align_up(n_streams * (size_t)kWindowTiles * kTileBytes);
+      L.off_wmeta = off;
+      off += align_up(n_streams * (size_t)kWindowTiles * slots_per_tile(16) * 8);
+    }
   }
   p.bytes = off;
   *why = KVQ_OK;
@@ -172,6 +187,8 @@ struct kvq_cache {
   }
   uint8_t* codes(int l) { return pool + L[l].off_codes; }
   uint32_t* meta(int l) { return reinterpret_cast<uint32_t*>(pool + L[l].off_meta); }
+  uint8_t* wcodes(int l) { return pool + L[l].off_wcodes; }
+  uint32_t* wmeta(int l) { return reinterpret_cast<uint32_t*>(pool + L[l].off_wmeta); }
   float* lam(int l) { return reinterpret_cast<float*>(pool + L[l].off_lam); }
   float* lam_inv(int l) { return reinterpret_cast<float*>(pool + L[l].off_lam_inv); }
   uint8_t* perm(int l) { return pool + L[l].off_perm; }
@@ -228,6 +245,70 @@ long long stable_groups(const LayerState& L, const Fill& f) {
   return (long long)tile * f.gpt + slot / kGroupTokens;
 }
 
+// The decode launches of one call: the progressive cache (if it holds
+// tokens) and, with the sink + window option, the window (one CTA per
+// stream, 16 bits); every CTA leaves one partial and the last to finish a
+// stream merges them all.
+struct DecodePlan {
+  Fill fill, wfill;
+  int splits = 0, wsplits = 0, nparts = 0;
+};
+
+DecodePlan plan_decode(kvq_cache* c, const LayerState& L) {
+  DecodePlan d;
+  const int n_streams = c->batch * c->kv_heads;
+  if (L.n > 0) {
+    d.fill = make_fill(L.bits, L.nt, L.pf, L.n_shrinks, L.n);
+    d.splits = decode_splits(c->sms(), n_streams, d.fill.gps);
+  }
+  if (L.window) {
+    d.wfill = make_fill(16, kWindowTiles, slots_per_tile(16), 0, std::min<long long>(L.n_all, kWindowTokens + 1));
+    d.wsplits = 1;
+    if (d.splits > kMaxSplits - 1) d.splits = kMaxSplits - 1;
+  }
+  d.nparts = d.splits + d.wsplits;
+  return d;
+}
+
+cudaError_t enqueue_decode(kvq_cache* c, int layer, const DecodePlan& d, const void* q, int q_heads, float sm_scale,
+                           float* out, float* parts, cudaStream_t s) {
+  const LayerState& L = c->L[layer];
+  DecodeArgs a{};
+  a.q = q;
+  a.lam = L.lambda_set ? c->lam(layer) : nullptr;
+  a.perm = L.lambda_set ? c->perm(layer) : nullptr;
+  a.out = out;
+  a.parts = parts;
+  a.counters = c->counters(layer);
+  a.err = c->err();
+  a.batch = c->batch;
+  a.kv_heads = c->kv_heads;
+  a.q_heads = q_heads;
+  a.group = q_heads / c->kv_heads;
+  a.qscale = sm_scale * 1.4426950408889634f;
+  a.nparts = d.nparts;
+  if (d.wsplits) {  // the window first: its partials are in place when the other launch's CTAs merge
+    DecodeArgs w = a;
+    w.codes = c->wcodes(layer);
+    w.meta = c->wmeta(layer);
+    w.fill = d.wfill;
+    w.splits = d.wsplits;
+    w.part_base = 0;
+    w.safe = 0;  // every window slot may be rewritten by an append in flight
+    if (cudaError_t e = launch_decode(w, s)) return e;
+  }
+  if (d.splits) {
+    a.codes = c->codes(layer);
+    a.meta = c->meta(layer);
+    a.fill = d.fill;
+    a.splits = d.splits;
+    a.part_base = d.wsplits;
+    a.safe = stable_groups(L, d.fill);
+    if (cudaError_t e = launch_decode(a, s)) return e;
+  }
+  return cudaSuccess;
+}
+
 uint32_t rd32(const uint8_t* p) {
   uint32_t w;
   memcpy(&w, p, 4);
@@ -238,23 +319,28 @@ uint32_t rd32(const uint8_t* p) {
 
 extern "C" {
 
-size_t kvq_pool_bytes(int layers, int batch, int kv_heads, int head_dim, size_t budget_bytes, const int* fbit) {
+size_t kvq_pool_bytes_ex(int layers, int batch, int kv_heads, int head_dim, size_t budget_bytes, const int* fbit,
+                         int options) {
   Plan p;
   kvq_status why;
-  if (!make_plan(layers, batch, kv_heads, head_dim, budget_bytes, fbit, p, &why)) return 0;
+  if (!make_plan(layers, batch, kv_heads, head_dim, budget_bytes, fbit, options, p, &why)) return 0;
   return p.bytes;
 }
 
-kvq_status kvq_alloc(kvq_cache** out, int layers, int batch, int kv_heads, int head_dim, size_t budget_bytes,
-                     const int* fbit, void* dev_pool, size_t pool_bytes) {
+size_t kvq_pool_bytes(int layers, int batch, int kv_heads, int head_dim, size_t budget_bytes, const int* fbit) {
+  return kvq_pool_bytes_ex(layers, batch, kv_heads, head_dim, budget_bytes, fbit, 0);
+}
+
+kvq_status kvq_alloc_ex(kvq_cache** out, int layers, int batch, int kv_heads, int head_dim, size_t budget_bytes,
+                        const int* fbit, void* dev_pool, size_t pool_bytes, int options) {
   if (!out) return fail(KVQ_ERR_INVALID, "out is NULL");
   *out = nullptr;
   Plan p;
   kvq_status why;
-  if (!make_plan(layers, batch, kv_heads, head_dim, budget_bytes, fbit, p, &why)) {
+  if (!make_plan(layers, batch, kv_heads, head_dim, budget_bytes, fbit, options, p, &why)) {
     if (why == KVQ_ERR_BUDGET) return fail(why, "budget of %zu bytes holds fewer than %d tokens per block", budget_bytes, kTokenRound);
-    return fail(why, "invalid shape or fbit (layers=%d batch=%d kv_heads=%d head_dim=%d; fbit must be 2/4/8/16, head_dim 128)",
-                layers, batch, kv_heads, head_dim);
+    return fail(why, "invalid shape, fbit or options (layers=%d batch=%d kv_heads=%d head_dim=%d options=%d; fbit must be "
+                "2/4/8/16, head_dim 128)", layers, batch, kv_heads, head_dim, options);
   }
   if (dev_pool && pool_bytes < p.bytes)
     return fail(KVQ_ERR_INVALID, "pool of %zu bytes is smaller than the %zu bytes needed", pool_bytes, p.bytes);
@@ -286,6 +372,11 @@ kvq_status kvq_alloc(kvq_cache** out, int layers, int batch, int kv_heads, int h
   c->pool_bytes = p.bytes;
   *out = c;
   return KVQ_OK;
+}
+
+kvq_status kvq_alloc(kvq_cache** out, int layers, int batch, int kv_heads, int head_dim, size_t budget_bytes,
+                     const int* fbit, void* dev_pool, size_t pool_bytes) {
+  return kvq_alloc_ex(out, layers, batch, kv_heads, head_dim, budget_bytes, fbit, dev_pool, pool_bytes, 0);
 }
 
 kvq_status kvq_set_lambda(kvq_cache* c, int layer, const float* lambda_host) {
@@ -327,15 +418,23 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* k, const void* v, int
   if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) % 16)
     return fail(KVQ_ERR_INVALID, "k and v must be 16-byte aligned");
   LayerState& L = c->L[layer];
-  if (L.n + n_tokens > c->n_f)
+  const long long W1 = kWindowTokens + 1;  // sink + window
+  if (!L.window && L.n + n_tokens > c->n_f)
     return fail(KVQ_ERR_BUDGET, "layer %d holds %lld of %lld tokens at Fbit %d; %d more do not fit", layer, L.n, c->n_f,
                 L.fbit, n_tokens);
+  if (L.window && std::max(0LL, L.n_all + n_tokens - W1) > c->n_f)
+    return fail(KVQ_ERR_BUDGET, "layer %d holds %lld tokens (%lld in the window); %d more do not fit at Fbit %d", layer,
+                L.n_all, std::min(L.n_all, W1), n_tokens, L.fbit);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaError_t e = c->ensure_err(s)) return cuda_fail(e, "error flag reset");
   int off = 0;
   while (off < n_tokens) {
     const long long cap = capacity(L, c->n_f, L.bits);
-    if (L.n == cap) {  // full: shrink one level first (bits > fbit is implied by the budget check)
+    // tokens this launch moves into the progressive cache: with the window,
+    // token t >= 129 moves token t - 128 (to index t - 129)
+    const long long t0 = L.window ? L.n_all : 0;
+    const bool moves_next = L.window ? t0 >= W1 : true;
+    if (L.n == cap && moves_next) {  // full: shrink one level first (bits > fbit is implied by the budget check)
       const ShrinkArgs sa = shrink_args(c, layer);
       cudaError_t e = launch_shrink(sa, s);
       if (e != cudaSuccess) return cuda_fail(e, "shrink launch");
@@ -343,7 +442,16 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* k, const void* v, int
       L.n_shrinks++;
       continue;
     }
-    const int cnt = (int)std::min<long long>(n_tokens - off, cap - L.n);
+    int cnt;
+    if (L.window) {
+      // at most 128 tokens a launch (their window slots are distinct), and no
+      // more moves than the progressive cache holds at this width
+      long long lim = std::min<long long>(n_tokens - off, kWindowTokens);
+      lim = std::min(lim, cap + W1 - t0);  // keeps t0 + cnt - 129 <= cap
+      cnt = (int)lim;
+    } else {
+      cnt = (int)std::min<long long>(n_tokens - off, cap - L.n);
+    }
     AppendArgs a{};
     a.k = k;
     a.v = v;
@@ -364,10 +472,20 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* k, const void* v, int
     a.meta = c->meta(layer);
     a.lam_inv = L.lambda_set ? c->lam_inv(layer) : nullptr;
     a.perm = L.lambda_set ? c->perm(layer) : nullptr;
+    a.window = L.window;
+    a.direct = L.shift_mode == KVQ_SHIFT_DIRECT;
+    a.t0 = t0;
+    a.wcodes = L.window ? c->wcodes(layer) : nullptr;
+    a.wmeta = L.window ? c->wmeta(layer) : nullptr;
     cudaError_t e = launch_append(a, s);
     if (e != cudaSuccess) return cuda_fail(e, "append launch");
     L.n_stable = L.n;
-    L.n += cnt;
+    if (L.window) {
+      L.n_all += cnt;
+      L.n = std::max(0LL, L.n_all - W1);
+    } else {
+      L.n += cnt;
+    }
     off += cnt;
   }
   return KVQ_OK;
@@ -419,7 +537,7 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, 
   if ((reinterpret_cast<uintptr_t>(q) % 16) || (reinterpret_cast<uintptr_t>(out) % 4))
     return fail(KVQ_ERR_INVALID, "q must be 16-byte aligned and out 4-byte aligned");
   LayerState& L = c->L[layer];
-  if (L.n <= 0) return fail(KVQ_ERR_STATE, "layer %d is empty", layer);
+  if ((L.window ? L.n_all : L.n) <= 0) return fail(KVQ_ERR_STATE, "layer %d is empty", layer);
   const int n_streams = c->batch * c->kv_heads;
   const size_t need = decode_parts_bytes(n_streams, G);
   if (!workspace || ws_bytes < need)
@@ -431,25 +549,8 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, 
     if (e != cudaSuccess) return cuda_fail(e, "counter reset");
     L.counters_zeroed = true;
   }
-  DecodeArgs a{};
-  a.codes = c->codes(layer);
-  a.meta = c->meta(layer);
-  a.q = q;
-  a.lam = L.lambda_set ? c->lam(layer) : nullptr;
-  a.perm = L.lambda_set ? c->perm(layer) : nullptr;
-  a.out = out;
-  a.parts = static_cast<float*>(workspace);
-  a.counters = c->counters(layer);
-  a.err = c->err();
-  a.fill = make_fill(L.bits, L.nt, L.pf, L.n_shrinks, L.n);
-  a.batch = c->batch;
-  a.kv_heads = c->kv_heads;
-  a.q_heads = q_heads;
-  a.group = G;
-  a.qscale = sm_scale * 1.4426950408889634f;
-  a.splits = decode_splits(c->sms(), n_streams, a.fill.gps);
-  a.safe = stable_groups(L, a.fill);
-  cudaError_t e = launch_decode(a, s);
+  const DecodePlan d = plan_decode(c, L);
+  cudaError_t e = enqueue_decode(c, layer, d, q, q_heads, sm_scale, out, static_cast<float*>(workspace), s);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return KVQ_OK;
 }
@@ -504,16 +605,15 @@ kvq_status kvq_decode_attn_noalloc(kvq_cache* c, int layer, const void* q, int q
   if ((reinterpret_cast<uintptr_t>(q) % 16) || (reinterpret_cast<uintptr_t>(out) % 4))
     return fail(KVQ_ERR_INVALID, "q must be 16-byte aligned and out 4-byte aligned");
   LayerState& L = c->L[layer];
-  if (L.n <= 0) return fail(KVQ_ERR_STATE, "layer %d is empty", layer);
+  if ((L.window ? L.n_all : L.n) <= 0) return fail(KVQ_ERR_STATE, "layer %d is empty", layer);
   const int n_streams = c->batch * c->kv_heads;
-  const Fill fill = make_fill(L.bits, L.nt, L.pf, L.n_shrinks, L.n);
-  const int splits = decode_splits(c->sms(), n_streams, fill.gps);
-  const size_t need = decode_parts_used(n_streams, splits);
+  const DecodePlan d = plan_decode(c, L);
+  const size_t need = decode_parts_used(n_streams, d.nparts);
   if (need > kNoAllocScratchBytes)
     return fail(KVQ_ERR_WORKSPACE,
                 "this block needs %zu bytes of scratch (batch*kv_heads=%d x %d splits); the built-in buffer holds "
                 "%zu bytes -- use kvq_decode_attn with a workspace",
-                need, n_streams, splits, kNoAllocScratchBytes);
+                need, n_streams, d.nparts, kNoAllocScratchBytes);
   void* scratch = nullptr;
   if (cudaError_t e = noalloc_scratch(&scratch)) return cuda_fail(e, "scratch address");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -523,25 +623,8 @@ kvq_status kvq_decode_attn_noalloc(kvq_cache* c, int layer, const void* q, int q
     if (e != cudaSuccess) return cuda_fail(e, "counter reset");
     L.counters_zeroed = true;
   }
-  DecodeArgs a{};
-  a.codes = c->codes(layer);
-  a.meta = c->meta(layer);
-  a.q = q;
-  a.lam = L.lambda_set ? c->lam(layer) : nullptr;
-  a.perm = L.lambda_set ? c->perm(layer) : nullptr;
-  a.out = out;
-  a.parts = static_cast<float*>(scratch);  // fully written before it is read: needs no clearing
-  a.counters = c->counters(layer);
-  a.err = c->err();
-  a.fill = fill;
-  a.batch = c->batch;
-  a.kv_heads = c->kv_heads;
-  a.q_heads = q_heads;
-  a.group = G;
-  a.qscale = sm_scale * 1.4426950408889634f;
-  a.splits = splits;
-  a.safe = stable_groups(L, fill);
-  cudaError_t e = launch_decode(a, s);
+  // the scratch is fully written before it is read: it needs no clearing
+  cudaError_t e = enqueue_decode(c, layer, d, q, q_heads, sm_scale, out, static_cast<float*>(scratch), s);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return KVQ_OK;
 }
@@ -549,14 +632,18 @@ kvq_status kvq_decode_attn_noalloc(kvq_cache* c, int layer, const void* q, int q
 kvq_status kvq_query(const kvq_cache* c, int layer, int* tokens, int* bits, int* cap, int* n_shrinks) {
   if (kvq_status s = check_layer(c, layer)) return s;
   const LayerState& L = c->L[layer];
-  if (tokens) *tokens = (int)L.n;
+  const int w = L.window ? kWindowTokens + 1 : 0;
+  if (tokens) *tokens = (int)(L.window ? L.n_all : L.n);
   if (bits) *bits = L.bits;
-  if (cap) *cap = (int)capacity(L, c->n_f, L.bits);
+  if (cap) *cap = (int)capacity(L, c->n_f, L.bits) + w;
   if (n_shrinks) *n_shrinks = L.n_shrinks;
   return KVQ_OK;
 }
 
-int kvq_max_tokens(const kvq_cache* c) { return c ? (int)c->n_f : 0; }
+int kvq_max_tokens(const kvq_cache* c) {
+  if (!c) return 0;
+  return (int)c->n_f + (c->layers > 0 && c->L[0].window ? kWindowTokens + 1 : 0);
+}
 
 kvq_status kvq_export(const kvq_cache* c, int layer, int b, int j, uint16_t* k_codes, uint16_t* v_codes,
                       uint16_t* k_meta, uint16_t* v_meta, kvq_stream_t stream) {
@@ -619,6 +706,67 @@ kvq_status kvq_export(const kvq_cache* c, int layer, int b, int j, uint16_t* k_c
       v_meta[2 * i + 1] = (uint16_t)(mw[mi + 1] >> 16);
     }
   }
+  return KVQ_OK;
+}
+
+kvq_status kvq_export_window(const kvq_cache* c, int layer, int b, int j, uint16_t* k_codes, uint16_t* v_codes,
+                             uint16_t* k_meta, uint16_t* v_meta, int* n_tokens, kvq_stream_t stream) {
+  if (kvq_status s = check_layer(c, layer)) return s;
+  if (b < 0 || b >= c->batch || j < 0 || j >= c->kv_heads)
+    return fail(KVQ_ERR_INVALID, "stream (%d, %d) out of range", b, j);
+  const LayerState& L = c->L[layer];
+  if (!L.window) return fail(KVQ_ERR_INVALID, "the cache was made without KVQ_OPT_SINK_WINDOW");
+  kvq_cache* m = const_cast<kvq_cache*>(c);
+  constexpr int P16 = slots_per_tile(16);
+  const size_t code_bytes = (size_t)kWindowTiles * kTileBytes, meta_words = (size_t)kWindowTiles * P16 * 2;
+  const size_t st = (size_t)b * c->kv_heads + j;
+  std::vector<uint8_t> cb(code_bytes);
+  std::vector<uint32_t> mw(meta_words);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(cb.data(), m->wcodes(layer) + st * code_bytes, code_bytes, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(mw.data(), m->wmeta(layer) + st * meta_words, meta_words * 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "export copy");
+  // tokens held: 0, then max(1, n - 128) .. n - 1; token t >= 1 sits in slot 1 + (t - 1) mod 128
+  std::vector<long long> toks;
+  if (L.n_all > 0) toks.push_back(0);
+  for (long long t = std::max(1LL, L.n_all - kWindowTokens); t < L.n_all; t++) toks.push_back(t);
+  const uint8_t* pm = L.lambda_set ? &L.perm[(size_t)j * kHeadDim] : nullptr;
+  constexpr int kUnit = 8 * 16;  // unit bytes at 16 bits
+  for (size_t i = 0; i < toks.size(); i++) {
+    const long long t = toks[i];
+    const int rs = t == 0 ? 0 : 1 + (int)((t - 1) % kWindowTokens);
+    const int tile = rs / P16, slot = rs % P16, grp = slot >> 4, tok = slot & 15;
+    const size_t gbase = (size_t)tile * kTileBytes + (size_t)grp * group_bytes(16);
+    if (k_codes) {
+      const int g = tok & 7, x = tok >> 3;
+      for (int kp = 0; kp < kHeadDim; kp++) {
+        const int p = 2 * (kp >> 5) + ((kp >> 4) & 1), tt = (kp >> 2) & 3, mi = kp & 3;
+        const int word = x * 16 + 2 * p + (mi >> 1);
+        const uint32_t w = rd32(&cb[gbase + (size_t)(4 * g + tt) * kUnit + 4 * word]);
+        k_codes[i * kHeadDim + (pm ? pm[kp] : kp)] = (uint16_t)(w >> (16 * (mi & 1)));
+      }
+    }
+    if (v_codes) {
+      const int tt = (tok & 7) >> 1, mb = tok & 1, u = tok >> 3;
+      for (int ch = 0; ch < kHeadDim; ch++) {
+        const int sb = ch >> 4, r = (ch >> 3) & 1, g = ch & 7;
+        const int word = u * 16 + 2 * sb + r;
+        const uint32_t w = rd32(&cb[gbase + part_bytes(16) + (size_t)(4 * g + tt) * kUnit + 4 * word]);
+        v_codes[i * kHeadDim + ch] = (uint16_t)(w >> (16 * mb));
+      }
+    }
+    const size_t mi = ((size_t)tile * P16 + slot) * 2;
+    if (k_meta) {
+      k_meta[2 * i] = (uint16_t)(mw[mi] & 0xffffu);
+      k_meta[2 * i + 1] = (uint16_t)(mw[mi] >> 16);
+    }
+    if (v_meta) {
+      v_meta[2 * i] = (uint16_t)(mw[mi + 1] & 0xffffu);
+      v_meta[2 * i + 1] = (uint16_t)(mw[mi + 1] >> 16);
+    }
+  }
+  if (n_tokens) *n_tokens = (int)toks.size();
   return KVQ_OK;
 }
 

@@ -740,7 +740,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   //   M = max over warps, L and PZ = e^(m_w - M)-weighted sums, O = sum of the
   //   warps' scaled rows (times 2^-e and 1/(2^b-1)) + PZ  (unnormalised).
   float* outp = a.out + ((size_t)b * a.q_heads + (size_t)j * G) * kHeadDim;
-  const int nparts = a.splits;
+  const int nparts = a.nparts;  // partials of this stream over every launch of the call
   const int c = threadIdx.x;  // one channel per thread
   static_assert(kThreads == kHeadDim, "one channel per thread");
   float Oc[kMaxGroup], Mh[kMaxGroup], Lh[kMaxGroup];
@@ -768,7 +768,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     return;
   }
   // Partial record of this CTA: M[8], L[8], then O[128 channels][8 heads].
-  float* mypart = a.parts + ((size_t)s * nparts + split) * kPartFloats;
+  float* mypart = a.parts + ((size_t)s * nparts + a.part_base + split) * kPartFloats;
   if (c == 0) {
 #pragma unroll
     for (int h = 0; h < kMaxGroup; h += 4) {
@@ -904,7 +904,9 @@ size_t decode_parts_used(int n_streams, int splits) {
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
-  if (a.group < 1 || a.group > kMaxGroup || a.splits < 1 || a.splits > kMaxSplits) return cudaErrorInvalidValue;
+  if (a.group < 1 || a.group > kMaxGroup || a.splits < 1 || a.nparts > kMaxSplits || a.part_base < 0 ||
+      a.part_base + a.splits > a.nparts)
+    return cudaErrorInvalidValue;
   switch (a.fill.bits) {
     case 2: return launch_bits<2>(a, s);
     case 4: return launch_bits<4>(a, s);

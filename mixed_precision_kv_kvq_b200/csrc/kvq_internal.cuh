@@ -61,6 +61,11 @@ namespace kvq {
 constexpr int kHeadDim = 128;
 constexpr int kTileBytes = 16384;
 constexpr int kGroupTokens = 16;
+// Sink + window option: token 0 and the latest kWindowTokens tokens held at
+// 16 bits in kWindowTiles tiles per stream: slot 0 the sink, slot
+// 1 + (t - 1) mod kWindowTokens token t >= 1 (the slot its leaving token frees).
+constexpr int kWindowTokens = 128;
+constexpr int kWindowTiles = 5;  // 129 slots at 32 per 16-bit tile
 
 __host__ __device__ constexpr int slots_per_tile(int bits) { return 512 / bits; }
 __host__ __device__ constexpr int group_bytes(int bits) { return 512 * bits; }  // K part + V part
@@ -158,6 +163,12 @@ struct AppendArgs {
   uint32_t* meta;     // layer base: [batch][kv_heads][nt][pf][2]
   const float* lam_inv;  // [kv_heads][128] or null
   const uint8_t* perm;   // [kv_heads][128] Key position -> channel, or null (identity)
+  // sink + window (the block keeps token 0 and the latest kWindowTokens at 16 bits)
+  bool window;           // tokens enter the window; n0/bits/h/e/nt describe the progressive cache
+  bool direct;           // the block shrinks with the Direct Right Shift
+  long long t0;          // token index (all tokens) of the first token of this launch
+  uint8_t* wcodes;       // window codes: [batch][kv_heads][kWindowTiles][16 KiB]
+  uint32_t* wmeta;       // window meta:  [batch][kv_heads][kWindowTiles][32][2]
 };
 
 struct ShrinkArgs {
@@ -183,7 +194,9 @@ struct DecodeArgs {
   Fill fill;
   int batch, kv_heads, q_heads, group;
   float qscale;         // sm_scale * log2(e)
-  int splits;           // CTAs per stream
+  int splits;           // CTAs per stream in this launch
+  int nparts;           // partials per stream over every launch of the call (the ticket counts them all)
+  int part_base;        // index of this launch's first partial
   long long safe;       // groups [0, safe) of every stream are not written by kernels still in flight
 };
 

@@ -160,3 +160,36 @@ def test_per_layer_capacities(kvq):
         assert [kvq.kvq_query(h, l)["capacity"] for l in range(4)] == [512, 1024, 2048, 4096]
     finally:
         kvq.kvq_free(h)
+
+
+def test_window_option_host_side(kvq):
+    """The sink + window option adds 5 tiles of 16 KiB and 1,280 bytes of meta
+    per (sequence, KV head) and block to the pool, keeps the budget rule for
+    the progressive cache, and rejects unknown option bits."""
+    lib = kvq.load()
+    budget = 4096 * _per_token(2, 3, [2, 4])
+    plain = kvq.kvq_pool_bytes(2, 2, 3, 128, budget, [2, 4])
+    win = kvq.kvq_pool_bytes_ex(2, 2, 3, 128, budget, [2, 4], kvq.KVQ_OPT_SINK_WINDOW)
+    per_block = 2 * 3 * (5 * 16384 + 5 * 32 * 8)
+    assert plain < win <= plain + 2 * (per_block + 2 * 256)
+    assert kvq.kvq_pool_bytes_ex(2, 2, 3, 128, budget, [2, 4], 0) == plain
+    assert kvq.kvq_pool_bytes_ex(2, 2, 3, 128, budget, [2, 4], 2) == 0
+    pool = HostPool(win)
+    h = C.c_void_p()
+    fb = (C.c_int * 2)(2, 4)
+    assert lib.kvq_alloc_ex(C.byref(h), 2, 2, 3, 128, budget, fb, pool.ptr, win, 2) == 1
+    assert lib.kvq_alloc_ex(C.byref(h), 2, 2, 3, 128, budget, fb, pool.ptr, plain, 1) == 1  # pool too small
+    assert lib.kvq_alloc_ex(C.byref(h), 2, 2, 3, 128, budget, fb, pool.ptr, win, 1) == 0
+    try:
+        assert kvq.kvq_max_tokens(h) == 4096 + 129
+        assert kvq.kvq_query(h, 1) == {"tokens": 0, "bits": 16, "capacity": 1024 + 129, "n_shrinks": 0}
+        n = C.c_int()
+        assert lib.kvq_export_window(h, 0, 2, 0, None, None, None, None, C.byref(n), None) == 1  # stream
+    finally:
+        kvq.kvq_free(h)
+    h2, pool2 = _host_cache(kvq)
+    try:
+        n = C.c_int()
+        assert lib.kvq_export_window(h2, 0, 0, 0, None, None, None, None, C.byref(n), None) == 1  # no window
+    finally:
+        kvq.kvq_free(h2)

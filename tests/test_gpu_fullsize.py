@@ -55,13 +55,16 @@ def per_token(batch, kv_heads, fbit):
 class Sampled:
     """A full-size GPU block plus oracle replays of a few of its streams."""
 
-    def __init__(self, kvq, orc, batch, kv_heads, n_f, fbit, streams, layer, seed=SEED, shift_mode=0):
+    def __init__(self, kvq, orc, batch, kv_heads, n_f, fbit, streams, layer, seed=SEED, shift_mode=0,
+                 window=False):
         self.kvq, self.orc_mod = kvq, orc
         self.batch, self.kv_heads, self.n_f, self.fbit = batch, kv_heads, n_f, fbit
         self.streams, self.layer, self.seed = streams, layer, seed
-        self.gpu = kvq.KVQCache(1, batch, kv_heads, n_f * per_token(batch, kv_heads, fbit), [fbit])
-        assert self.gpu.max_tokens == n_f
-        self.orc = {s: orc.Layer(1, 1, n_f, fbit) for s in streams}
+        self.window = window
+        self.gpu = kvq.KVQCache(1, batch, kv_heads, n_f * per_token(batch, kv_heads, fbit), [fbit],
+                                sink_window=window)
+        assert self.gpu.max_tokens == n_f + (129 if window else 0)
+        self.orc = {s: (orc.WLayer if window else orc.Layer)(1, 1, n_f, fbit) for s in streams}
         self.lam = None
         self.pos = 0
         self.n_out = S.outliers_for(kv_heads)
@@ -110,11 +113,17 @@ class Sampled:
     def check_state(self):
         st = self.gpu.query(0)
         for o in self.orc.values():
-            assert (st["tokens"], st["bits"], st["n_shrinks"]) == (o.n, o.bits, o.n_shrinks), (st, o.shrink_at)
+            m = o.main if self.window else o
+            assert (st["tokens"], st["bits"], st["n_shrinks"]) == (o.n, m.bits, m.n_shrinks), (st, m.shrink_at)
         return st
 
     def check_codes(self):
-        for (b, j), o in self.orc.items():
+        for (b, j), w in self.orc.items():
+            o = w.main if self.window else w
+            if self.window:
+                got = self.gpu.export_window(0, b, j)
+                for name, x, y in zip(("wK", "wV", "wKm", "wVm"), got, w.window_codes()):
+                    assert np.array_equal(x, y[0, 0]), (b, j, name)
             kc, vc, km, vm = self.gpu.export(0, b, j)
             assert np.array_equal(km, o.k_meta()[0, 0]), (b, j, "K meta")
             assert np.array_equal(vm, o.v_meta()[0, 0]), (b, j, "V meta")
@@ -228,6 +237,19 @@ def test_70b_final_4to2_direct_shift_then_decode(kvq, orc):
     for o in x.orc.values():
         assert o.shrink() == 0
     assert x.check_state()["bits"] == 2
+    x.check_codes()
+    x.check_attention(HQ)
+    x.free()
+
+
+def test_7b_decode_sink_window_fullsize(kvq, orc):
+    """The 7B block with the pages' deployed configuration: the sink and the
+    latest 128 tokens at INT16, 32768 + 129 tokens, Fbit 2."""
+    B, H, HQ, T = 16, 4, 28, 32768 + 129
+    x = Sampled(kvq, orc, B, H, 32768, 2, corners(B, H), 9, window=True)
+    x.fill(T, chunk=4096)
+    st = x.check_state()
+    assert st["bits"] == 2 and st["tokens"] == T
     x.check_codes()
     x.check_attention(HQ)
     x.free()

@@ -215,3 +215,99 @@ def test_direct_shift_chunked_bf16(kvq, orc, fbit):
     assert P.gpu.query(0)["bits"] == fbit and pos == n_f
     P.check_codes()
     P.check_attention(S.queries(6, fbit, 0, B, 4 * H, n_f, dtype=torch.bfloat16))
+
+
+# ------------------------------------------ sink token + recent window at INT16
+
+class WPair:
+    """A GPU cache made with the sink + window option and the oracle's
+    windowed block, fed identically."""
+
+    def __init__(self, kvq, orc, batch, kv_heads, n_f, fbit, lam=None, shift_mode=0):
+        self.kvq = kvq
+        self.batch, self.kv_heads = batch, kv_heads
+        self.gpu = kvq.KVQCache(1, batch, kv_heads, n_f * per_token(batch, kv_heads, [fbit]), [fbit],
+                                sink_window=True)
+        assert self.gpu.max_tokens == n_f + 129
+        self.orc = orc.WLayer(batch, kv_heads, n_f, fbit)
+        self.lam = lam
+        if lam is not None:
+            self.gpu.set_lambda(0, lam)
+        if shift_mode:
+            self.gpu.set_shift_mode(0, shift_mode)
+            assert self.orc.set_shift_mode(shift_mode) == 0
+
+    def append(self, k, v):
+        self.gpu.append(0, k.cuda(), v.cuda())
+        assert self.orc.append(k.float().numpy(), v.float().numpy(), self.lam) == 0
+
+    def check_codes(self):
+        q = self.gpu.query(0)
+        m = self.orc.main
+        assert (q["tokens"], q["bits"], q["n_shrinks"]) == (self.orc.n, m.bits, m.n_shrinks), (q, m.shrink_at)
+        okc, ovc, okm, ovm = m.k_codes(), m.v_codes(), m.k_meta(), m.v_meta()
+        wkc, wvc, wkm, wvm = self.orc.window_codes()
+        for b in range(self.batch):
+            for j in range(self.kv_heads):
+                kc, vc, km, vm = self.gpu.export(0, b, j)
+                assert kc.shape[0] == m.n
+                for name, got, want in (("K", kc, okc[b, j]), ("V", vc, ovc[b, j]), ("K meta", km, okm[b, j]),
+                                        ("V meta", vm, ovm[b, j])):
+                    assert np.array_equal(got, want), (b, j, name, np.argwhere(got != want)[:4].tolist())
+                kc, vc, km, vm = self.gpu.export_window(0, b, j)
+                for name, got, want in (("window K", kc, wkc[b, j]), ("window V", vc, wvc[b, j]),
+                                        ("window K meta", km, wkm[b, j]), ("window V meta", vm, wvm[b, j])):
+                    assert np.array_equal(got, want), (b, j, name, np.argwhere(got != want)[:4].tolist())
+
+    def check_attention(self, q, sm_scale=1 / math.sqrt(128)):
+        out = self.gpu.decode_attn(0, q.cuda(), sm_scale).cpu().numpy().astype(np.float64)
+        torch.cuda.synchronize()
+        self.gpu.device_status()
+        ref = self.orc.attention(q.float().numpy(), self.lam, sm_scale)
+        err = np.abs(out - ref).max(axis=-1) / np.abs(ref).max(axis=-1)
+        assert np.isfinite(out).all()
+        assert err.max() <= TOL, f"max rel err {err.max():.3e} at {np.unravel_index(err.argmax(), err.shape)}"
+
+
+def test_window_tiny_one_by_one(kvq, orc):
+    """Token by token through: window filling (progressive cache empty),
+    the first move (token 129), and two shrinks of the progressive cache
+    (at 128 and 256 of its tokens); codes bit-exact, attention within 2e-3."""
+    T = 600
+    k, v = S.keys_values(7, 0, 1, T, 2, 0, 4, dtype=torch.float32)
+    lam = lam_for(k)
+    P = WPair(kvq, orc, 1, 2, 512, 4, lam)
+    checkpoints = {1, 2, 128, 129, 130, 131, 257, 258, 385, 386, 600}
+    for t in range(T):
+        P.append(k[:, t:t + 1], v[:, t:t + 1])
+        if t + 1 in checkpoints:
+            P.check_codes()
+            P.check_attention(S.queries(7, 0, t, 1, 4, t + 1, dtype=torch.bfloat16))
+    assert P.orc.main.shrink_at == [128, 256]
+
+
+@pytest.mark.parametrize("fbit,mode", [(2, 0), (2, 1), (8, 0)])
+def test_window_chunked_bf16(kvq, orc, fbit, mode):
+    """Chunks of every size around the window (1 .. 700 tokens: launches are
+    cut at 128 tokens and at the progressive cache's capacity), batch 3,
+    4 KV heads, through every shrink of the block, either shift."""
+    B, H, n_f = 3, 4, 1024
+    total = n_f + 129
+    k, v = S.keys_values(8, fbit, B, total, H, 0, 5, dtype=torch.bfloat16)
+    lam = lam_for(k)
+    P = WPair(kvq, orc, B, H, n_f, fbit, lam, shift_mode=mode)
+    pos = 0
+    for n in (1, 127, 1, 129, 300, 5, 700, total):
+        n = min(n, total - pos)
+        if n <= 0:
+            break
+        P.append(k[:, pos:pos + n], v[:, pos:pos + n])
+        pos += n
+        if pos in (1, 128, 258, 563):
+            P.check_codes()
+    assert pos == total and P.gpu.query(0)["bits"] == fbit
+    P.check_codes()
+    P.check_attention(S.queries(8, fbit, 0, B, 4 * H, total, dtype=torch.bfloat16))
+    with pytest.raises(kvq.KVQError) as e:  # the progressive cache is full at Fbit
+        P.gpu.append(0, k[:, :1].cuda(), v[:, :1].cuda())
+    assert e.value.status == 2
