@@ -263,7 +263,8 @@ DecodePlan plan_decode(kvq_cache* c, const LayerState& L) {
   }
   if (L.window) {
     d.wfill = make_fill(16, kWindowTiles, slots_per_tile(16), 0, std::min<long long>(L.n_all, kWindowTokens + 1));
-    d.wsplits = 1;
+    // up to 9 16-bit groups: 3 CTAs so the window's copies overlap; every CTA gets a group
+    d.wsplits = (int)std::min<long long>(3, d.wfill.gps);
     if (d.splits > kMaxSplits - 1) d.splits = kMaxSplits - 1;
   }
   d.nparts = d.splits + d.wsplits;
@@ -287,24 +288,31 @@ cudaError_t enqueue_decode(kvq_cache* c, int layer, const DecodePlan& d, const v
   a.group = q_heads / c->kv_heads;
   a.qscale = sm_scale * 1.4426950408889634f;
   a.nparts = d.nparts;
-  if (d.wsplits) {  // the window first: its partials are in place when the other launch's CTAs merge
-    DecodeArgs w = a;
-    w.codes = c->wcodes(layer);
-    w.meta = c->wmeta(layer);
-    w.fill = d.wfill;
-    w.splits = d.wsplits;
-    w.part_base = 0;
-    w.safe = 0;  // every window slot may be rewritten by an append in flight
-    if (cudaError_t e = launch_decode(w, s)) return e;
-  }
+  // The progressive cache first; the window launch follows it.  The first
+  // launch triggers its dependents only after its own dependency wait, so
+  // the window launch needs none: it runs in the shadow of the first one's
+  // merge.  The last CTA of a stream, in either launch, merges all partials.
   if (d.splits) {
     a.codes = c->codes(layer);
     a.meta = c->meta(layer);
     a.fill = d.fill;
     a.splits = d.splits;
-    a.part_base = d.wsplits;
+    a.part_base = 0;
     a.safe = stable_groups(L, d.fill);
+    a.trigger_early = d.wsplits > 0;
     if (cudaError_t e = launch_decode(a, s)) return e;
+    a.trigger_early = false;
+  }
+  if (d.wsplits) {
+    DecodeArgs w = a;
+    w.codes = c->wcodes(layer);
+    w.meta = c->wmeta(layer);
+    w.fill = d.wfill;
+    w.splits = d.wsplits;
+    w.part_base = d.splits;
+    w.after_decode = d.splits > 0;
+    w.safe = w.after_decode ? d.wfill.gps : 0;  // alone, every window slot may be rewritten by an append in flight
+    if (cudaError_t e = launch_decode(w, s)) return e;
   }
   return cudaSuccess;
 }

@@ -588,7 +588,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
       }
     }
   }
-  pdl_wait();  // the rest of the cache, q and the counters may be written by earlier kernels
+  // the rest of the cache, q and the counters may be written by earlier
+  // kernels -- unless this launch directly follows another decode launch of
+  // the same call, which triggers this one only after its own wait (then
+  // everything before that launch is complete).
+  if (!a.after_decode) pdl_wait();
+  if (a.trigger_early) pdl_launch_dependents();  // a window launch follows: let it fill free SMs now
   const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.q_heads + (size_t)j * G) * kHeadDim;
   uint4 qv = make_uint4(0u, 0u, 0u, 0u);  // 8 bf16 of q: head threadIdx/16, channels 8 (threadIdx%16) ..
   if ((int)threadIdx.x < G * (kHeadDim / 8)) qv = reinterpret_cast<const uint4*>(qb)[threadIdx.x];
@@ -697,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   float m0 = sm.m0, m1 = sm.m1, l0 = sm.l0, l1 = sm.l1, pz0 = sm.pz0, pz1 = sm.pz1;
   float (&o)[8][4] = sm.o;
 
-  pdl_launch_dependents();  // the next kernel may start to launch while this one merges
+  if (!a.trigger_early) pdl_launch_dependents();  // the next kernel may start to launch while this one merges
   // ---- merge the four warps ----
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
@@ -789,6 +794,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     flags[1] = last;
   }
   __syncthreads();
+  // A launch that skipped its dependency wait still completes only after the
+  // launch before it (so kernels after this one are ordered behind both).
+  // No deadlock: this grid started only once every CTA of that launch had
+  // triggered, i.e. was resident.
+  if (a.after_decode) pdl_wait();
   if (!flags[1]) return;
   const float* p0 = a.parts + (size_t)s * nparts * kPartFloats;
   // The first kPre partials' outputs for this thread's channel are loaded

@@ -198,6 +198,8 @@ struct DecodeArgs {
   int nparts;           // partials per stream over every launch of the call (the ticket counts them all)
   int part_base;        // index of this launch's first partial
   long long safe;       // groups [0, safe) of every stream are not written by kernels still in flight
+  bool after_decode;    // launched right after another decode launch of the same call: no dependency wait
+  bool trigger_early;   // another decode launch of the call follows: trigger it right after the wait
 };
 
 // CTAs per stream for a launch over n_streams streams on num_sms SMs.
