@@ -92,8 +92,8 @@ size_t kvq_pool_bytes_ex(int layers, int batch, int kv_heads, int head_dim, size
  * kvq_pool_bytes(...) bytes, owned by the caller and kept alive until
  * kvq_free; or NULL, and the library cudaMallocs the pool itself.  With a
  * caller pool this call makes no CUDA call.  Every block starts empty at 16
- * bits.  Errors: INVALID (shape, fbit, head_dim != 128), BUDGET (budget
- * smaller than 512 tokens), OOM. */
+ * bits.  Errors: INVALID (shape -- batch <= 65535 and kv_heads <= 4096 --,
+ * fbit, head_dim != 128), BUDGET (budget smaller than 512 tokens), OOM. */
 kvq_status kvq_alloc(kvq_cache** out, int layers, int batch, int kv_heads, int head_dim,
                      size_t budget_bytes, const int* fbit, void* dev_pool, size_t pool_bytes);
 

@@ -92,6 +92,7 @@ bool make_plan(int layers, int batch, int kv_heads, int head_dim, size_t budget,
                Plan& p, kvq_status* why) {
   *why = KVQ_ERR_INVALID;
   if (layers < 1 || batch < 1 || kv_heads < 1 || head_dim != kHeadDim || !fbit) return false;
+  if (batch > 65535 || kv_heads > 4096) return false;  // kernel grid limits
   if (options & ~KVQ_OPT_SINK_WINDOW) return false;
   const bool window = (options & KVQ_OPT_SINK_WINDOW) != 0;
   unsigned long long per_token = 0;  // bytes per token over all blocks

@@ -66,6 +66,7 @@ constexpr int kGroupTokens = 16;
 // 1 + (t - 1) mod kWindowTokens token t >= 1 (the slot its leaving token frees).
 constexpr int kWindowTokens = 128;
 constexpr int kWindowTiles = 5;  // 129 slots at 32 per 16-bit tile
+static_assert((kWindowTokens & (kWindowTokens - 1)) == 0, "window slots are taken modulo a power of two");
 
 __host__ __device__ constexpr int slots_per_tile(int bits) { return 512 / bits; }
 __host__ __device__ constexpr int group_bytes(int bits) { return 512 * bits; }  // K part + V part
