@@ -135,7 +135,7 @@ def test_chunked_append_bit_exact(kvq, orc, fbit, chunks):
     P.check_codes()
 
 
-@pytest.mark.parametrize("G", [2, 5, 7, 8])
+@pytest.mark.parametrize("G", [1, 2, 3, 5, 7, 8])
 @pytest.mark.parametrize("T,fbit", [(1, 2), (17, 2), (300, 4), (1500, 4), (3000, 2), (4096, 2)])
 def test_decode_attention(kvq, orc, G, T, fbit):
     B, H = 2, 2
@@ -311,3 +311,20 @@ def test_window_chunked_bf16(kvq, orc, fbit, mode):
     with pytest.raises(kvq.KVQError) as e:  # the progressive cache is full at Fbit
         P.gpu.append(0, k[:, :1].cuda(), v[:, :1].cuda())
     assert e.value.status == 2
+
+
+def test_window_noalloc_matches_workspace_entry(kvq, orc):
+    """The no-workspace entry point on a cache with the sink + window: the same
+    two launches, the same result as kvq_decode_attn."""
+    B, H, G = 2, 2, 4
+    T = 700
+    k, v = S.keys_values(9, 0, B, T, H, 0, 3, dtype=torch.bfloat16)
+    P = WPair(kvq, orc, B, H, 1024, 2, lam_for(k))
+    P.append(k, v)
+    q = S.queries(9, 0, 0, B, H * G, T, dtype=torch.bfloat16).cuda()
+    ref = P.gpu.decode_attn(0, q)
+    out = torch.empty_like(ref)
+    kvq.kvq_decode_attn_noalloc(P.gpu.handle, 0, q, 128 ** -0.5, out)
+    torch.cuda.synchronize()
+    assert torch.allclose(out, ref, rtol=0, atol=0)
+    P.check_attention(q.cpu())
