@@ -265,6 +265,21 @@ def measure_append_chunk(kvq, dev, flush_buf, reps=3):
     return {"gbs": nb / t / 1e9, "us": t * 1e6, "bytes": nb, "bits": bits, "tokens": 4096, "batch": batch}
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's device time (every rank passes its own)."""
+    if world <= 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(bytes_per_rank: int, ms: float, world: int) -> float:
+    """Replicas: every rank moves the same bytes; the job's rate is all
+    ranks' bytes over the slowest rank's time."""
+    return world * bytes_per_rank / (ms / 1e3) / 1e9
+
+
 def _decode_args(kvq, cache, q, out, ws, stream):
     import ctypes as C
     return (cache.handle, 0, C.c_void_p(q.data_ptr()), q.shape[1], C.c_float(HEAD_DIM ** -0.5),
@@ -443,11 +458,8 @@ def run_gpu(args, rank, world):
     tot_bytes = 0
     for i in range(K):
         tot_bytes += bytes_of_step(t0_tokens + i)[0]
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * tot_bytes / (total_ms / 1e3) / 1e9
+    total_ms = max_over_ranks(total_ms, world, dev)
+    value = whole_job_gbs(tot_bytes, total_ms, world)
     launches = K * layers * 2
 
     # ---- per-launch decode durations: the same step again, K more times,
@@ -541,15 +553,12 @@ def run_gpu(args, rank, world):
             f1.record(stream)
             torch.cuda.synchronize(dev)
             e2e_ms = f0.elapsed_time(f1)
-            if world > 1:
-                t = torch.tensor([e2e_ms], device=dev)
-                torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-                e2e_ms = float(t.item())
+            e2e_ms = max_over_ranks(e2e_ms, world, dev)
             eb = 0
             t1 = cache.query(0)["tokens"] - E
             for i in range(E):
                 eb += bytes_of_step(t1 + i)[0]
-            e2e = {"value": world * eb / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+            e2e = {"value": whole_job_gbs(eb, e2e_ms, world), "unit": "GB/s",
                    "h2d_bytes_per_step": layers * (kin[0, 0].numel() * 2 * 2 + qin[0, 0].numel() * 2),
                    "d2h_bytes_per_step": layers * out[0].numel() * 4, "steps": E}
 
@@ -636,7 +645,7 @@ def cpu_baseline(budget_s=15.0):
                       f"{HQ7 // HKV7} query heads, fp64 attention; {dt:.1f} s"}
 
 
-def run_reference(args):
+def run_reference(args, world=1):
     K, W = args.steps, args.warmup
     tokens = T7 if K + W <= 20 else max(1024, (T7 * 20 // (K + W)) // 512 * 512)
     L, q, lam = oracle_sample(tokens)
@@ -650,11 +659,12 @@ def run_reference(args):
     v = K * nb / dt / 1e9
     sample = (f"each step: one (sequence, KV head) stream of a 2-bit 7B-shape block, {tokens} tokens, "
               f"{HQ7 // HKV7} query heads, fp64 attention in the CPU oracle")
-    return {"impl": "reference", "metric": METRIC, "value": round(v, 5), "unit": "GB/s", "n_gpus": 1,
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 5), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": round(dt * 1e3 / K, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "layers": L7, "batch": B7, "q_heads": HQ7, "kv_heads": HKV7,
-                       "head_dim": HEAD_DIM, "context": T7, "fbit": FBIT7},
+                       "head_dim": HEAD_DIM, "context": T7, "fbit": FBIT7, "parallelism": f"replicas x{world}",
+                       "reference": "the CPU oracle on rank 0 only (the other ranks exit without work)"},
             "cpu_baseline": {"value": round(v, 5), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": round(v, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -678,7 +688,7 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(run_reference(args)), flush=True)
+            print(json.dumps(run_reference(args, world)), flush=True)
         return
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
