@@ -375,8 +375,8 @@ def run_gpu(args, rank, world):
     layers = args.layers
     fbit = FBIT7 if layers == L7 else [4 if l % 2 == 1 else 2 for l in range(layers)]
     K, W = args.steps, args.warmup
-    if 3 * K + W > ROOM:
-        raise SystemExit(f"3 * --steps + --warmup must be <= {ROOM}")
+    if 4 * K + W > ROOM:
+        raise SystemExit(f"4 * --steps + --warmup must be <= {ROOM}")
     n_f = T7 + ROOM
     n_out = S.outliers_for(HKV7)
     seed = SEED + 1000 * rank
@@ -384,7 +384,7 @@ def run_gpu(args, rank, world):
     sm_scale = HEAD_DIM ** -0.5
 
     # per-step inputs, generated up front on the device
-    nsteps = 2 * K + W  # warm-up, timed steps, per-launch-event steps
+    nsteps = 3 * K + W  # warm-up, timed steps, per-launch-event steps, two-call steps
     g = torch.Generator(device=dev)
     g.manual_seed(seed + 7)
     kin = torch.randn((nsteps, layers, B7, 1, HKV7, HEAD_DIM), generator=g, device=dev).to(torch.bfloat16)
@@ -407,17 +407,27 @@ def run_gpu(args, rank, world):
     scale_c = C.c_float(sm_scale)
 
     def step(i, ev=None):
+        # one decode step per block: the new token's append and the attention
+        # in one launch (kvq_append_decode)
         for l in range(layers):
-            st = lib.kvq_append(h, l, kp[i][l], vp[i][l], kvq.KVQ_DTYPE_BF16, 1, sp)
-            if st:
-                kvq.check(st)
             if ev is not None:
                 ev[l][0].record(stream)
-            st = lib.kvq_decode_attn(h, l, qp[i][l], HQ7, scale_c, op[l], wp[l][0], wp[l][1], sp)
+            st = lib.kvq_append_decode(h, l, kp[i][l], vp[i][l], kvq.KVQ_DTYPE_BF16, qp[i][l], HQ7, scale_c, op[l],
+                                       wp[l][0], wp[l][1], sp)
             if st:
                 kvq.check(st)
             if ev is not None:
                 ev[l][1].record(stream)
+
+    def step_two_calls(i):
+        # the same step as kvq_append then kvq_decode_attn (two launches per block)
+        for l in range(layers):
+            st = lib.kvq_append(h, l, kp[i][l], vp[i][l], kvq.KVQ_DTYPE_BF16, 1, sp)
+            if st:
+                kvq.check(st)
+            st = lib.kvq_decode_attn(h, l, qp[i][l], HQ7, scale_c, op[l], wp[l][0], wp[l][1], sp)
+            if st:
+                kvq.check(st)
 
     def bytes_of_step(t_before):
         """Algorithmic bytes of one step given the token count before it."""
@@ -460,7 +470,7 @@ def run_gpu(args, rank, world):
         tot_bytes += bytes_of_step(t0_tokens + i)[0]
     total_ms = max_over_ranks(total_ms, world, dev)
     value = whole_job_gbs(tot_bytes, total_ms, world)
-    launches = K * layers * 2
+    launches = K * layers  # one kvq_append_decode launch per block (no shrink in the timed steps)
 
     # ---- per-launch decode durations: the same step again, K more times,
     # with CUDA events on the launch stream around every decode launch ----
@@ -478,10 +488,25 @@ def run_gpu(args, rank, world):
     dec_ms_bits = {}
     dec_bytes = 0
     for i in range(K):
-        dec_bytes += bytes_of_step(t1_tokens + i)[1]
+        dec_bytes += bytes_of_step(t1_tokens + i)[0]  # the fused launch: attention + the new token
         for l in range(layers):
             dec_ms_bits.setdefault(fbit[l], []).append(evs[i][l][0].elapsed_time(evs[i][l][1]))
     ev_step_ms = r_start.elapsed_time(r_end) / K
+
+    # ---- the same steps as two calls per block (append, then attention) ----
+    t2_tokens = cache.query(0)["tokens"]
+    torch.cuda.synchronize(dev)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    for i in range(K):
+        step_two_calls(W + 2 * K + i)
+    c1.record(stream)
+    torch.cuda.synchronize(dev)
+    cache.device_status()
+    two_ms = c0.elapsed_time(c1) / K
+    two_bytes = sum(bytes_of_step(t2_tokens + i)[0] for i in range(K)) / K
+    two_calls = {"ms_per_step": round(two_ms, 4), "gbs": round(two_bytes / two_ms / 1e6, 1),
+                 "what": "the step as kvq_append + kvq_decode_attn per block (two launches)"}
 
     # ---- the decode half of the step captured in one CUDA graph ----
     graph = None
@@ -538,7 +563,7 @@ def run_gpu(args, rank, world):
         vh = vin.cpu().pin_memory()
         qh = qin.cpu().pin_memory()
         oh = torch.empty((layers, B7, HQ7, HEAD_DIM), dtype=torch.float32).pin_memory()
-        E = min(K, ROOM - 2 * K - W)
+        E = min(K, ROOM - 3 * K - W)
         if E > 0:
             torch.cuda.synchronize(dev)
             if world > 1:
@@ -554,8 +579,7 @@ def run_gpu(args, rank, world):
                 vd.copy_(vh[i], non_blocking=True)
                 qd.copy_(qh[i], non_blocking=True)
                 for l in range(layers):
-                    cache.append(l, kd[l], vd[l])
-                    cache.decode_attn(l, qd[l], sm_scale, out=out[l])
+                    cache.append_decode(l, kd[l], vd[l], qd[l], sm_scale, out=out[l])
                 oh.copy_(out, non_blocking=True)
             f1.record(stream)
             torch.cuda.synchronize(dev)
@@ -577,7 +601,7 @@ def run_gpu(args, rank, world):
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs (copy)",
             "traffic": traffic, "traffic_source": traffic_src,
-            "kernel": "decode_kernel (kvq_decode_attn)",
+            "kernel": "decode_kernel (kvq_append_decode: the step's new token and the attention)",
             "avg_launch_us": round(dec_ms * 1e3 / n_dec, 2),
             "bytes_per_launch": int(dec_bytes / n_dec),
             "per_bits_us": {f"{b}bit": round(statistics.mean(v) * 1e3, 2) for b, v in sorted(dec_ms_bits.items())},
@@ -606,6 +630,7 @@ def run_gpu(args, rank, world):
                    "l2": "no flush: every block's cache read (151-285 MB) exceeds the 126 MB L2",
                    "decode_ms_share": round(dec_ms / (ev_step_ms * K), 3)},
         "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
+        "two_call_step": two_calls,
         **extra,
     }
     return res

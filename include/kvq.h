@@ -159,6 +159,22 @@ size_t kvq_decode_workspace(const kvq_cache* c, int layer, int q_heads);
 kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, float sm_scale,
                            float* out, void* workspace, size_t ws_bytes, kvq_stream_t stream);
 
+/* One decode step of a block in one launch: kvq_append of one token per
+ * sequence (k, v: device [batch][1][kv_heads][128], dtype as kvq_append,
+ * 16-byte aligned) followed by kvq_decode_attn over every token including it
+ * (q, q_heads, sm_scale, out, workspace as kvq_decode_attn) -- the same codes,
+ * meta and output as the two calls.  The token is quantized and written by
+ * the attention kernel itself (by the warp whose share of the block holds the
+ * token's group, before it reads that group), which saves the append launch
+ * on the decode path.  A full block is first shrunk one level as kvq_append
+ * would (a separate launch).  With KVQ_OPT_SINK_WINDOW the call runs the two
+ * calls.  Errors: those of kvq_append (BUDGET, INVALID) and of
+ * kvq_decode_attn (WORKSPACE, INVALID, CUDA); on an error before a launch
+ * nothing has changed. */
+kvq_status kvq_append_decode(kvq_cache* c, int layer, const void* k, const void* v, int dtype, const void* q,
+                             int q_heads, float sm_scale, float* out, void* workspace, size_t ws_bytes,
+                             kvq_stream_t stream);
+
 /* Decode attention that allocates nothing and takes no workspace; same
  * arguments, result and errors as kvq_decode_attn otherwise.  The paper has
  * no counterpart to this call: it exists for callers that cannot allocate device

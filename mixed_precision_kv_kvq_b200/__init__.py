@@ -23,7 +23,7 @@ HEAD_DIM = 128
 __all__ = [
     "KVQCache", "KVQError", "load",
     "kvq_pool_bytes", "kvq_pool_bytes_ex", "kvq_alloc", "kvq_alloc_ex", "kvq_export_window", "kvq_set_lambda", "kvq_append", "kvq_shrink", "kvq_set_shift_mode",
-    "kvq_decode_workspace", "kvq_decode_attn", "kvq_decode_attn_noalloc", "kvq_query", "kvq_max_tokens", "kvq_export",
+    "kvq_decode_workspace", "kvq_decode_attn", "kvq_decode_attn_noalloc", "kvq_append_decode", "kvq_query", "kvq_max_tokens", "kvq_export",
     "kvq_device_status", "kvq_last_error", "kvq_free", "kvq_allocate_bits",
 ]
 
@@ -122,6 +122,23 @@ def kvq_decode_attn(cache, layer: int, q: torch.Tensor, sm_scale: float, out: to
     ws_bytes = workspace.numel() * workspace.element_size()
     check(load().kvq_decode_attn(cache, layer, _dptr(q), q.shape[1], float(sm_scale), _dptr(out),
                                  _dptr(workspace), ws_bytes, _stream_ptr(stream)))
+
+
+def kvq_append_decode(cache, layer: int, k: torch.Tensor, v: torch.Tensor, q: torch.Tensor, sm_scale: float,
+                      out: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:
+    """One decode step in one launch: append k, v (device [batch][1][kv_heads][128])
+    then attend with q (device bf16 [batch][q_heads][128]) into out (fp32)."""
+    if k.shape != v.shape or k.dtype != v.dtype or k.dim() != 4 or k.shape[1] != 1 or k.shape[-1] != HEAD_DIM:
+        raise ValueError("k and v must both be [batch][1][kv_heads][128] of one dtype")
+    if not (k.is_cuda and v.is_cuda and k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("k and v must be contiguous CUDA tensors")
+    if q.dtype != torch.bfloat16 or q.dim() != 3 or q.shape[-1] != HEAD_DIM or not q.is_contiguous():
+        raise ValueError("q must be a contiguous bf16 [batch][q_heads][128] tensor")
+    if out.dtype != torch.float32 or out.shape != q.shape or not out.is_contiguous():
+        raise ValueError("out must be a contiguous fp32 tensor shaped like q")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    check(load().kvq_append_decode(cache, layer, _dptr(k), _dptr(v), _dtype_code(k), _dptr(q), q.shape[1],
+                                   float(sm_scale), _dptr(out), _dptr(workspace), ws_bytes, _stream_ptr(stream)))
 
 
 def kvq_decode_attn_noalloc(cache, layer: int, q: torch.Tensor, sm_scale: float, out: torch.Tensor,
@@ -272,6 +289,17 @@ class KVQCache:
         if out is None:
             out = torch.empty(q.shape, dtype=torch.float32, device=self.device)
         kvq_decode_attn(self.handle, layer, q, sm_scale, out, self.workspace(layer, q.shape[1]), stream)
+        return out
+
+    def append_decode(self, layer: int, k: torch.Tensor, v: torch.Tensor, q: torch.Tensor,
+                      sm_scale: Optional[float] = None, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """append(layer, k, v) of one token per sequence, then decode_attn(layer, q), in one launch."""
+        k, v, q = self._dev(k), self._dev(v), self._dev(q)
+        if sm_scale is None:
+            sm_scale = HEAD_DIM ** -0.5
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=self.device)
+        kvq_append_decode(self.handle, layer, k, v, q, sm_scale, out, self.workspace(layer, q.shape[1]), stream)
         return out
 
     def query(self, layer: int) -> dict:

@@ -45,6 +45,7 @@ SIGNATURES = {
     "kvq_decode_workspace": (SZ, [P, I, I]),
     "kvq_decode_attn": (I, [P, I, P, I, C.c_float, P, P, SZ, P]),
     "kvq_decode_attn_noalloc": (I, [P, I, P, I, C.c_float, P, P]),
+    "kvq_append_decode": (I, [P, I, P, P, I, P, I, C.c_float, P, P, SZ, P]),
     "kvq_query": (I, [P, I, P, P, P, P]),
     "kvq_max_tokens": (I, [P]),
     "kvq_export": (I, [P, I, I, I, P, P, P, P, P]),

@@ -272,10 +272,20 @@ DecodePlan plan_decode(kvq_cache* c, const LayerState& L) {
   return d;
 }
 
+// The new token of a fused single-token append (kvq_append_decode).
+struct AppendOne {
+  long long group = -1;  // its group in the kernels' group order; < 0: no append
+  int tile = 0, slot = 0;
+  const void* k = nullptr;
+  const void* v = nullptr;
+  int dtype = 0;
+};
+
 cudaError_t enqueue_decode(kvq_cache* c, int layer, const DecodePlan& d, const void* q, int q_heads, float sm_scale,
-                           float* out, float* parts, cudaStream_t s) {
+                           float* out, float* parts, cudaStream_t s, const AppendOne& app = AppendOne()) {
   const LayerState& L = c->L[layer];
   DecodeArgs a{};
+  a.app_group = -1;
   a.q = q;
   a.lam = L.lambda_set ? c->lam(layer) : nullptr;
   a.perm = L.lambda_set ? c->perm(layer) : nullptr;
@@ -301,8 +311,19 @@ cudaError_t enqueue_decode(kvq_cache* c, int layer, const DecodePlan& d, const v
     a.part_base = 0;
     a.safe = stable_groups(L, d.fill);
     a.trigger_early = d.wsplits > 0;
+    if (app.group >= 0) {  // this launch writes the new token itself: keep the pre-wait copies clear of it
+      a.app_group = app.group;
+      a.app_tile = app.tile;
+      a.app_slot = app.slot;
+      a.ak = app.k;
+      a.av = app.v;
+      a.adtype = app.dtype;
+      a.lam_inv = L.lambda_set ? c->lam_inv(layer) : nullptr;
+      a.safe = std::min(a.safe, app.group);
+    }
     if (cudaError_t e = launch_decode(a, s)) return e;
     a.trigger_early = false;
+    a.app_group = -1;
   }
   if (d.wsplits) {
     DecodeArgs w = a;
@@ -561,6 +582,67 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, 
   const DecodePlan d = plan_decode(c, L);
   cudaError_t e = enqueue_decode(c, layer, d, q, q_heads, sm_scale, out, static_cast<float*>(workspace), s);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return KVQ_OK;
+}
+
+kvq_status kvq_append_decode(kvq_cache* c, int layer, const void* k, const void* v, int dtype, const void* q,
+                             int q_heads, float sm_scale, float* out, void* workspace, size_t ws_bytes,
+                             kvq_stream_t stream) {
+  if (kvq_status s = check_layer(c, layer)) return s;
+  LayerState& L = c->L[layer];
+  if (L.window) {  // the window's moves need the append kernel: the two calls
+    if (kvq_status st = kvq_append(c, layer, k, v, dtype, 1, stream)) return st;
+    return kvq_decode_attn(c, layer, q, q_heads, sm_scale, out, workspace, ws_bytes, stream);
+  }
+  if (!k || !v || !q || !out) return fail(KVQ_ERR_INVALID, "k, v, q or out is NULL");
+  if (dtype != KVQ_DTYPE_BF16 && dtype != KVQ_DTYPE_F32) return fail(KVQ_ERR_INVALID, "dtype %d unknown", dtype);
+  if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) % 16)
+    return fail(KVQ_ERR_INVALID, "k and v must be 16-byte aligned");
+  if (q_heads <= 0 || q_heads % c->kv_heads)
+    return fail(KVQ_ERR_INVALID, "q_heads %d is not a positive multiple of kv_heads %d", q_heads, c->kv_heads);
+  const int G = q_heads / c->kv_heads;
+  if (G > 8) return fail(KVQ_ERR_INVALID, "%d query heads per KV head; at most 8 are supported", G);
+  if (!std::isfinite(sm_scale)) return fail(KVQ_ERR_INVALID, "sm_scale is not finite");
+  if ((reinterpret_cast<uintptr_t>(q) % 16) || (reinterpret_cast<uintptr_t>(out) % 4))
+    return fail(KVQ_ERR_INVALID, "q must be 16-byte aligned and out 4-byte aligned");
+  if (L.n + 1 > c->n_f)
+    return fail(KVQ_ERR_BUDGET, "layer %d holds %lld of %lld tokens at Fbit %d; 1 more does not fit", layer, L.n, c->n_f,
+                L.fbit);
+  const int n_streams = c->batch * c->kv_heads;
+  const size_t need = decode_parts_bytes(n_streams, G);
+  if (!workspace || ws_bytes < need)
+    return fail(KVQ_ERR_WORKSPACE, "workspace of %zu bytes; %zu needed", workspace ? ws_bytes : (size_t)0, need);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaError_t e = c->ensure_err(s)) return cuda_fail(e, "error flag reset");
+  if (!L.counters_zeroed) {
+    cudaError_t e = cudaMemsetAsync(c->counters(layer), 0, (size_t)n_streams * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "counter reset");
+    L.counters_zeroed = true;
+  }
+  if (L.n == capacity(L, c->n_f, L.bits)) {  // full: shrink one level first, as kvq_append would
+    const ShrinkArgs sa = shrink_args(c, layer);
+    if (cudaError_t e = launch_shrink(sa, s)) return cuda_fail(e, "shrink launch");
+    L.bits /= 2;
+    L.n_shrinks++;
+  }
+  // the new token's slot (the append kernel's formula) and its group
+  const int p = slots_per_tile(L.bits);
+  const int h = L.n_shrinks > 0 ? p / 2 : 0;
+  const long long m = L.n - (long long)L.nt * h;
+  AppendOne app;
+  app.tile = (int)(m / (p - h));
+  app.slot = h + (int)(m % (p - h));
+  app.group = (long long)app.tile * (p / kGroupTokens) + app.slot / kGroupTokens;
+  app.k = k;
+  app.v = v;
+  app.dtype = dtype;
+  L.n += 1;  // the plan covers the new token
+  const DecodePlan d = plan_decode(c, L);
+  L.n -= 1;
+  cudaError_t e = enqueue_decode(c, layer, d, q, q_heads, sm_scale, out, static_cast<float*>(workspace), s, app);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  L.n_stable = L.n;
+  L.n += 1;
   return KVQ_OK;
 }
 

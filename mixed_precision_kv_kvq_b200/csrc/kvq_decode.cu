@@ -35,7 +35,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
-#include "kvq_internal.cuh"
+#include "kvq_quant.cuh"
 
 namespace kvq {
 namespace {
@@ -53,6 +53,11 @@ constexpr int kSmemBytes = kWarps * kWarpSmem + kQfBytes + 3 * kWarps * kMaxGrou
                            kWarps * kStages * 8 + kWarps * kStages * 8 + 16;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
 constexpr int kPartFloats = 2 * kMaxGroup + kHeadDim * kMaxGroup;  // one CTA's partial record
+// Scratch of the fused append in a warp's second code stage (unused until the
+// main loop; warp 0's holds q, lambda and the channel order below this).
+constexpr int kAppScratch = 3072;
+static_assert(kAppScratch >= 2 * kMaxGroup * kHeadDim + 4 * kHeadDim + kHeadDim, "clear of q, lambda, order");
+static_assert(kAppScratch + 2 * kHeadDim <= kStageCode, "the scratch fits the stage");
 // Largest amount (log2 units) a score may exceed the running max before the
 // max is moved: p <= 2^8, and p * R stays well inside fp16 for R < 255.
 constexpr float kRebase = 8.0f;
@@ -597,6 +602,44 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.q_heads + (size_t)j * G) * kHeadDim;
   uint4 qv = make_uint4(0u, 0u, 0u, 0u);  // 8 bf16 of q: head threadIdx/16, channels 8 (threadIdx%16) ..
   if ((int)threadIdx.x < G * (kHeadDim / 8)) qv = reinterpret_cast<const uint4*>(qb)[threadIdx.x];
+
+  // ---- fused single-token append: the warp whose range holds the new
+  // token's group quantizes and writes the token (K, then V) before it
+  // copies any group (a.safe kept the pre-wait copy away from that group) ----
+  if (a.app_group >= 0 && wa <= a.app_group && a.app_group < wb) {  // warp-uniform
+    uint16_t* sc = reinterpret_cast<uint16_t*>(ws[warp].code[kStages - 1] + kAppScratch);
+    const size_t tile = (size_t)s * f.nt + a.app_tile;
+#pragma unroll 1
+    for (int kv = 0; kv < 2; kv++) {
+      const size_t in_off = (((size_t)b * a.kv_heads + j) * kHeadDim) + 4 * lane;  // token 0 of a 1-token call
+      const void* src = kv ? a.av : a.ak;
+      float x[4];
+      if (a.adtype == 1) {
+        const float4 f4 = *reinterpret_cast<const float4*>(static_cast<const float*>(src) + in_off);
+        x[0] = f4.x; x[1] = f4.y; x[2] = f4.z; x[3] = f4.w;
+      } else {
+        const uint2 raw = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(src) + in_off);
+        x[0] = __uint_as_float(raw.x << 16); x[1] = __uint_as_float(raw.x & 0xffff0000u);
+        x[2] = __uint_as_float(raw.y << 16); x[3] = __uint_as_float(raw.y & 0xffff0000u);
+      }
+      if (kv == 0 && a.lam_inv) {
+        const float4 li = *reinterpret_cast<const float4*>(a.lam_inv + (size_t)j * kHeadDim + 4 * lane);
+        x[0] = __fmul_rn(x[0], li.x); x[1] = __fmul_rn(x[1], li.y);
+        x[2] = __fmul_rn(x[2], li.z); x[3] = __fmul_rn(x[3], li.w);
+      }
+      const uint32_t mw = quantize_group(x, BITS == 16 ? 65535u : (1u << BITS) - 1u, sc, lane);
+      __syncwarp();
+      uint8_t* gbase = const_cast<uint8_t*>(a.codes) + tile * kTileBytes + (size_t)(a.app_slot >> 4) * kGroupBytes +
+                       (size_t)kv * (kGroupBytes / 2);
+      const uint8_t* pm = (kv == 0 && a.perm) ? a.perm + (size_t)j * kHeadDim : nullptr;
+      pack_codes<BITS>(gbase, a.app_slot & 15, kv, sc, pm, lane);
+      if (lane == 0) const_cast<uint32_t*>(a.meta)[(tile * f.pf + a.app_slot) * 2 + kv] = mw;
+      __syncwarp();  // sc is rewritten for V
+    }
+    // this warp's own bulk copies (async proxy) must see these writes
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __syncwarp();
+  }
 
   // start streaming before the q' set-up so DRAM latency overlaps it
   if (lane == 0 && !pre) {

@@ -201,6 +201,15 @@ struct DecodeArgs {
   long long safe;       // groups [0, safe) of every stream are not written by kernels still in flight
   bool after_decode;    // launched right after another decode launch of the same call: no dependency wait
   bool trigger_early;   // another decode launch of the call follows: trigger it right after the wait
+  // fused single-token append (kvq_append_decode): the warp whose groups
+  // include group app_group writes the new token (slot app_slot of tile
+  // app_tile of every stream) before copying its groups; app_group < 0: none
+  long long app_group;
+  int app_tile, app_slot;
+  const void* ak;        // [batch][1][kv_heads][128] new Keys (bf16 or f32)
+  const void* av;        // new Values
+  int adtype;            // 0 bf16, 1 f32
+  const float* lam_inv;  // [kv_heads][128] or null
 };
 
 // CTAs per stream for a launch over n_streams streams on num_sms SMs.

@@ -253,3 +253,28 @@ def test_7b_decode_sink_window_fullsize(kvq, orc):
     x.check_codes()
     x.check_attention(HQ)
     x.free()
+
+
+def test_7b_fused_decode_steps_fullsize(kvq, orc):
+    """The benchmark's step on a full 7B block: three single-token
+    kvq_append_decode calls on top of 32768 tokens (2 bits), sampled streams
+    against the oracle after each."""
+    B, H, HQ, T = 16, 4, 28, 32768
+    x = Sampled(kvq, orc, B, H, T + 4096, 2, corners(B, H), 11)
+    x.fill(T)
+    for step in range(3):
+        k, v = S.keys_values(x.seed, x.layer, B, 1, H, x.pos, x.n_out, dtype=torch.bfloat16, device="cuda")
+        q = S.queries(x.seed, x.layer, 50 + step, B, HQ, x.pos + 1, dtype=torch.bfloat16, device="cuda")
+        out = x.gpu.append_decode(0, k, v, q).cpu().numpy().astype(np.float64)
+        torch.cuda.synchronize()
+        x._replay(k, v)
+        x.pos += 1
+        x.check_state()
+        qc = q.float().cpu().numpy()
+        for (b, j), o in x.orc.items():
+            G = HQ // H
+            ref = o.attention(qc[b:b + 1, j * G:(j + 1) * G], x.lam[j:j + 1], 1 / math.sqrt(128))[0]
+            err = np.abs(out[b, j * G:(j + 1) * G] - ref).max(axis=-1) / np.abs(ref).max(axis=-1)
+            assert err.max() <= TOL, (step, b, j, err.max())
+    x.check_codes()
+    x.free()

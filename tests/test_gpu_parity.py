@@ -328,3 +328,38 @@ def test_window_noalloc_matches_workspace_entry(kvq, orc):
     torch.cuda.synchronize()
     assert torch.allclose(out, ref, rtol=0, atol=0)
     P.check_attention(q.cpu())
+
+
+# ------------------------------------------------ fused single-token append + decode
+
+@pytest.mark.parametrize("fbit,t0,steps", [(2, 509, 6), (2, 1021, 5), (4, 3000, 4), (16, 250, 4)])
+def test_append_decode_equals_two_calls(kvq, orc, fbit, t0, steps):
+    """kvq_append_decode (one launch: the decode kernel writes the new token)
+    gives the same codes, meta and output, bit for bit, as kvq_append then
+    kvq_decode_attn -- including across a shrink -- and matches the oracle."""
+    B, H, G, n_f = 2, 3, 4, 4096
+    k, v = S.keys_values(10, fbit, B, t0 + steps, H, 0, 3, dtype=torch.bfloat16)
+    lam = lam_for(k)
+    P = Pair(kvq, orc, B, H, n_f, fbit, lam)  # separate calls, and the oracle
+    F = kvq.KVQCache(1, B, H, n_f * per_token(B, H, [fbit]), [fbit])
+    F.set_lambda(0, lam)
+    P.append(k[:, :t0], v[:, :t0])
+    F.append(0, k[:, :t0].cuda(), v[:, :t0].cuda())
+    for i in range(steps):
+        t = t0 + i
+        kt, vt = k[:, t:t + 1].contiguous(), v[:, t:t + 1].contiguous()
+        q = S.queries(10, fbit, i, B, H * G, t + 1, dtype=torch.bfloat16).cuda()
+        P.append(kt, vt)
+        o_sep = P.gpu.decode_attn(0, q)
+        o_fus = F.append_decode(0, kt.cuda(), vt.cuda(), q)
+        torch.cuda.synchronize()
+        assert torch.equal(o_sep, o_fus), (i, (o_sep - o_fus).abs().max().item())
+        assert F.query(0) == P.gpu.query(0)
+    F.device_status()
+    for b in range(B):
+        for j in range(H):
+            for x, y in zip(P.gpu.export(0, b, j), F.export(0, b, j)):
+                assert np.array_equal(x, y), (b, j)
+    P.check_codes()
+    P.check_attention(S.queries(10, fbit, 99, B, H * G, t0 + steps, dtype=torch.bfloat16))
+    F.free()
