@@ -629,11 +629,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
       }
       const uint32_t mw = quantize_group(x, BITS == 16 ? 65535u : (1u << BITS) - 1u, sc, lane);
       __syncwarp();
-      uint8_t* gbase = const_cast<uint8_t*>(a.codes) + tile * kTileBytes + (size_t)(a.app_slot >> 4) * kGroupBytes +
-                       (size_t)kv * (kGroupBytes / 2);
+      uint8_t* gbase = a.codes + tile * kTileBytes + (size_t)(a.app_slot >> 4) * kGroupBytes + (size_t)kv * (kGroupBytes / 2);
       const uint8_t* pm = (kv == 0 && a.perm) ? a.perm + (size_t)j * kHeadDim : nullptr;
       pack_codes<BITS>(gbase, a.app_slot & 15, kv, sc, pm, lane);
-      if (lane == 0) const_cast<uint32_t*>(a.meta)[(tile * f.pf + a.app_slot) * 2 + kv] = mw;
+      if (lane == 0) a.meta[(tile * f.pf + a.app_slot) * 2 + kv] = mw;
       __syncwarp();  // sc is rewritten for V
     }
     // this warp's own bulk copies (async proxy) must see these writes

@@ -183,8 +183,8 @@ struct ShrinkArgs {
 };
 
 struct DecodeArgs {
-  const uint8_t* codes;
-  const uint32_t* meta;
+  uint8_t* codes;       // the block's (or window's) codes; written only by a fused append
+  uint32_t* meta;
   const void* q;        // bf16 [batch][q_heads][128]
   const float* lam;     // [kv_heads][128] or null
   const uint8_t* perm;  // [kv_heads][128] Key position -> channel, or null (identity)
