@@ -568,19 +568,48 @@ def run_gpu(args, rank, world):
             torch.cuda.synchronize(dev)
             if world > 1:
                 torch.distributed.barrier()
-            # device staging of one step's inputs (the step's H2D lands here)
-            kd, vd, qd = torch.empty_like(kin[0]), torch.empty_like(vin[0]), torch.empty_like(qin[0])
+            # A serving loop's steps, double-buffered: a copy stream brings step
+            # i+1's K, V, Q in and takes step i-1's outputs out while step i runs
+            # (the public API per block, on device views).  Every copy of every
+            # step is inside the timed region.
+            cs = torch.cuda.Stream(dev)
+            bufs = [(torch.empty_like(kin[0]), torch.empty_like(vin[0]), torch.empty_like(qin[0]), torch.empty_like(out))
+                    for _ in range(2)]
+            in_ready = [torch.cuda.Event() for _ in range(2)]
+            done = [torch.cuda.Event() for _ in range(2)]      # step's compute finished (inputs read, output written)
+            drained = [torch.cuda.Event() for _ in range(2)]   # step's output copied out
+
+            def fetch(i):
+                b = i % 2
+                with torch.cuda.stream(cs):
+                    if i >= 2:
+                        cs.wait_event(done[b])  # the step that last read these buffers
+                    kd, vd, qd, _ = bufs[b]
+                    kd.copy_(kh[i], non_blocking=True)
+                    vd.copy_(vh[i], non_blocking=True)
+                    qd.copy_(qh[i], non_blocking=True)
+                    in_ready[b].record(cs)
+
             f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             f0.record(stream)
+            cs.wait_event(f0)
+            fetch(0)
             for i in range(E):
-                # a serving loop's step: this step's K, V, Q in (one copy each), the
-                # public API per block on device views, every block's output out
-                kd.copy_(kh[i], non_blocking=True)
-                vd.copy_(vh[i], non_blocking=True)
-                qd.copy_(qh[i], non_blocking=True)
+                b = i % 2
+                if i + 1 < E:
+                    fetch(i + 1)
+                kd, vd, qd, od = bufs[b]
+                stream.wait_event(in_ready[b])
+                if i >= 2:
+                    stream.wait_event(drained[b])  # output buffer b copied out by then
                 for l in range(layers):
-                    cache.append_decode(l, kd[l], vd[l], qd[l], sm_scale, out=out[l])
-                oh.copy_(out, non_blocking=True)
+                    cache.append_decode(l, kd[l], vd[l], qd[l], sm_scale, out=od[l])
+                done[b].record(stream)
+                with torch.cuda.stream(cs):
+                    cs.wait_event(done[b])
+                    oh.copy_(od, non_blocking=True)
+                    drained[b].record(cs)
+            stream.wait_stream(cs)
             f1.record(stream)
             torch.cuda.synchronize(dev)
             e2e_ms = f0.elapsed_time(f1)
