@@ -709,6 +709,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   }
   const uint4* qfl = qf + lane;
   __syncthreads();  // w_m / w_l are reused by the merge
+  // The staging areas (second code stages) are refilled by bulk copies from
+  // the first loop iteration on: order the generic accesses before them.
+  if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 
   Soft sm;
   sm.m0 = sm.m1 = -INFINITY;
