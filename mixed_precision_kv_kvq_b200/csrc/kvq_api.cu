@@ -72,13 +72,12 @@ struct LayerState {
   int nt;  // tiles per stream
   int pf;  // meta slots per tile
   bool counters_zeroed;
-  size_t off_lam, off_lam_inv, off_perm, off_counters, off_codes, off_meta;
+  size_t off_lam, off_lam_inv, off_counters, off_codes, off_meta;
   // sink + window option: n counts the progressive cache; n_all every token
   bool window;
   long long n_all;
   size_t off_wcodes, off_wmeta;
   bool lambda_set;
-  std::vector<uint8_t> perm;  // host copy of the Key channel order [kv_heads][128]
 };
 
 struct Plan {
@@ -127,8 +126,6 @@ bool make_plan(int layers, int batch, int kv_heads, int head_dim, size_t budget,
     off += align_up((size_t)kv_heads * kHeadDim * 4);
     L.off_lam_inv = off;
     off += align_up((size_t)kv_heads * kHeadDim * 4);
-    L.off_perm = off;
-    off += align_up((size_t)kv_heads * kHeadDim);
     L.off_counters = off;
     off += align_up(n_streams * 4);
     L.off_codes = off;
@@ -192,7 +189,6 @@ struct kvq_cache {
   uint32_t* wmeta(int l) { return reinterpret_cast<uint32_t*>(pool + L[l].off_wmeta); }
   float* lam(int l) { return reinterpret_cast<float*>(pool + L[l].off_lam); }
   float* lam_inv(int l) { return reinterpret_cast<float*>(pool + L[l].off_lam_inv); }
-  uint8_t* perm(int l) { return pool + L[l].off_perm; }
   int* counters(int l) { return reinterpret_cast<int*>(pool + L[l].off_counters); }
   int* err() { return reinterpret_cast<int*>(pool); }
 };
@@ -288,7 +284,6 @@ cudaError_t enqueue_decode(kvq_cache* c, int layer, const DecodePlan& d, const v
   a.app_group = -1;
   a.q = q;
   a.lam = L.lambda_set ? c->lam(layer) : nullptr;
-  a.perm = L.lambda_set ? c->perm(layer) : nullptr;
   a.out = out;
   a.parts = parts;
   a.counters = c->counters(layer);
@@ -420,21 +415,10 @@ kvq_status kvq_set_lambda(kvq_cache* c, int layer, const float* lambda_host) {
     inv[i] = (float)(1.0 / (double)v);
   }
   if (c->L[layer].n != 0) return fail(KVQ_ERR_STATE, "layer %d already holds tokens; set lambda before the first append", layer);
-  // Key channel order: largest lambda first (ties by channel index).
-  std::vector<uint8_t> perm(n);
-  for (int j = 0; j < c->kv_heads; j++) {
-    std::vector<int> idx(kHeadDim);
-    for (int ch = 0; ch < kHeadDim; ch++) idx[ch] = ch;
-    const float* lj = lambda_host + (size_t)j * kHeadDim;
-    std::stable_sort(idx.begin(), idx.end(), [lj](int x, int y) { return lj[x] > lj[y]; });
-    for (int pos = 0; pos < kHeadDim; pos++) perm[(size_t)j * kHeadDim + pos] = (uint8_t)idx[pos];
-  }
   cudaError_t e = cudaMemcpy(c->lam(layer), lambda_host, n * 4, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(c->lam_inv(layer), inv.data(), n * 4, cudaMemcpyHostToDevice);
-  if (e == cudaSuccess) e = cudaMemcpy(c->perm(layer), perm.data(), n, cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return cuda_fail(e, "lambda upload");
   c->L[layer].lambda_set = true;
-  c->L[layer].perm = perm;
   return KVQ_OK;
 }
 
@@ -501,8 +485,7 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* k, const void* v, int
     a.codes = c->codes(layer);
     a.meta = c->meta(layer);
     a.lam_inv = L.lambda_set ? c->lam_inv(layer) : nullptr;
-    a.perm = L.lambda_set ? c->perm(layer) : nullptr;
-    a.window = L.window;
+      a.window = L.window;
     a.direct = L.shift_mode == KVQ_SHIFT_DIRECT;
     a.t0 = t0;
     a.wcodes = L.window ? c->wcodes(layer) : nullptr;
@@ -761,9 +744,8 @@ kvq_status kvq_export(const kvq_cache* c, int layer, int b, int j, uint16_t* k_c
     const size_t gbase = (size_t)tile * kTileBytes + (size_t)grp * group_bytes(bits);
     if (k_codes) {
       const int g = tok & 7, x = tok >> 3;
-      const uint8_t* pm = L.lambda_set ? &L.perm[(size_t)j * kHeadDim] : nullptr;
-      for (int kp = 0; kp < kHeadDim; kp++) {  // Key position -> channel pm[kp]
-        // position 32s + 16r + 4t + i: member i of quad p = 2s + r in unit 4g + t
+      for (int kp = 0; kp < kHeadDim; kp++) {
+        // channel 32s + 16r + 4t + i: member i of quad p = 2s + r in unit 4g + t
         const int p = 2 * (kp >> 5) + ((kp >> 4) & 1), t = (kp >> 2) & 3, mi = kp & 3;
         int word, shift;
         if (bits == 16) {
@@ -775,7 +757,7 @@ kvq_status kvq_export(const kvq_cache* c, int layer, int b, int j, uint16_t* k_c
           shift = 8 * mi + bits * (p % qpw);
         }
         const uint32_t w = rd32(&cb[gbase + (size_t)(4 * g + t) * unit_bytes(bits) + 4 * word]);
-        k_codes[i * kHeadDim + (pm ? pm[kp] : kp)] = (uint16_t)((w >> shift) & mask);
+        k_codes[i * kHeadDim + kp] = (uint16_t)((w >> shift) & mask);
       }
     }
     if (v_codes) {
@@ -822,7 +804,6 @@ kvq_status kvq_export_window(const kvq_cache* c, int layer, int b, int j, uint16
   std::vector<long long> toks;
   if (L.n_all > 0) toks.push_back(0);
   for (long long t = std::max(1LL, L.n_all - kWindowTokens); t < L.n_all; t++) toks.push_back(t);
-  const uint8_t* pm = L.lambda_set ? &L.perm[(size_t)j * kHeadDim] : nullptr;
   constexpr int kUnit = 8 * 16;  // unit bytes at 16 bits
   for (size_t i = 0; i < toks.size(); i++) {
     const long long t = toks[i];
@@ -835,7 +816,7 @@ kvq_status kvq_export_window(const kvq_cache* c, int layer, int b, int j, uint16
         const int p = 2 * (kp >> 5) + ((kp >> 4) & 1), tt = (kp >> 2) & 3, mi = kp & 3;
         const int word = x * 16 + 2 * p + (mi >> 1);
         const uint32_t w = rd32(&cb[gbase + (size_t)(4 * g + tt) * kUnit + 4 * word]);
-        k_codes[i * kHeadDim + (pm ? pm[kp] : kp)] = (uint16_t)(w >> (16 * (mi & 1)));
+        k_codes[i * kHeadDim + kp] = (uint16_t)(w >> (16 * (mi & 1)));
       }
     }
     if (v_codes) {

@@ -42,7 +42,6 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs 
   const int tk0 = tb * kTokensPerWarp;
   const int ntk = min(kTokensPerWarp, a.cnt - tk0);
   const size_t stream = (size_t)b * a.kv_heads + j;
-  const uint8_t* pm = (kv == 0 && a.perm) ? a.perm + (size_t)j * kHeadDim : nullptr;
   uint16_t* sc = codes_sh[wib];
 
   // ---- load 4 channels per lane of every token of this warp, migrate Keys ----
@@ -110,7 +109,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs 
       if (t >= kWindowTokens + 1) {
         // token t - 128 leaves the window: its INT16 codes go to the progressive
         // cache at the current width (index t - 129) by the block's shift chain
-        unpack_codes16(wg, wtok, kv, sc, pm, lane);
+        unpack_codes16(wg, wtok, kv, sc, lane);
         __syncwarp();
 #pragma unroll
         for (int i = 0; i < 4; i++) sc[4 * lane + i] = (uint16_t)shift_chain<BITS>(sc[4 * lane + i], a.direct);
@@ -119,7 +118,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs 
         int slot;
         size_t tile;
         uint8_t* gbase = main_group(t - (kWindowTokens + 1), &slot, &tile);
-        pack_codes<BITS>(gbase, slot & 15, kv, sc, pm, lane);
+        pack_codes<BITS>(gbase, slot & 15, kv, sc, lane);
         if (lane == 0) {
           const uint32_t mw = (uint32_t)range_chain<BITS>((uint16_t)(old & 0xffffu), a.direct) | (old & 0xffff0000u);
           a.meta[(tile * (size_t)a.pf + slot) * 2 + kv] = mw;
@@ -133,13 +132,13 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs 
     __syncwarp();
 
     if (a.window) {
-      pack_codes<16>(wg, wtok, kv, sc, pm, lane);
+      pack_codes<16>(wg, wtok, kv, sc, lane);
       if (lane == 0) a.wmeta[wmi] = mw;
     } else {
       int slot;
       size_t tile;
       uint8_t* gbase = main_group(a.n0 + tkn, &slot, &tile);
-      pack_codes<BITS>(gbase, slot & 15, kv, sc, pm, lane);
+      pack_codes<BITS>(gbase, slot & 15, kv, sc, lane);
       if (lane == 0) a.meta[(tile * (size_t)a.pf + slot) * 2 + kv] = mw;
     }
     __syncwarp();  // sc is rewritten by the next token

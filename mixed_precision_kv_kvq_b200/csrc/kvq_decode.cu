@@ -10,7 +10,7 @@
 //   q'.k^_t = (R_t / (2^b-1)) (q'.c_t) + Z_t sum(q'),
 //   sum_t p_t v^_t = (sum_t p_t R_t c_t) / (2^b-1) + sum_t p_t Z_t,
 // so the raw codes go straight into tensor-core operands:
-//   QK^T: int8 mma.sync.m16n8k32, A = 16 tokens x 32 Key positions of codes
+//   QK^T: int8 mma.sync.m16n8k32, A = 16 tokens x 32 Key channels of codes
 //   (byte quads, each code moved to the top of its byte: c 2^(8-b), exact in
 //   u8), B = the query as an exact per-head int16, q' = s_h (256 hi + lo)
 //   with hi s8 and lo u8, two MMAs on the same A registers, int32
@@ -245,7 +245,7 @@ __device__ __forceinline__ uint32_t quad_reg(const uint32_t* u) {
   return quad_field<BITS, Q % qpw>(u[Q / qpw]);
 }
 
-// Scores of NG 16-token groups: D[n][token][head] = sum over Key positions of
+// Scores of NG 16-token groups: D[n][token][head] = sum over Key channels of
 // A * q'_int, with A = c 2^(8 - BITS) (BITS <= 8) or the 16-bit code itself,
 // and q'_int = 256 hi + lo the per-head int16 query (hi: s8, lo: u8); every
 // product and sum is exact in int32.  The k-block loop is outermost so each
@@ -520,28 +520,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     for (int i = 0; i < kS; i++) mbar_init(bar0 + 8 * i, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // q, lambda and the Key channel order are staged in shared memory (in warp
-  // 0's second code stage, unused until the main loop starts).  lambda and
-  // the channel order are fixed while kernels run on the block, so they are
-  // fetched before waiting for the previous kernel.
+  // q and lambda are staged in shared memory (in warp 0's second code stage,
+  // unused until the main loop starts).  lambda is fixed while kernels run on
+  // the block, so it is fetched before waiting for the previous kernel.
   const int b = s / a.kv_heads, j = s - b * a.kv_heads;
   __nv_bfloat16* s_q = reinterpret_cast<__nv_bfloat16*>(ws[0].code[kStages - 1]);  // [8][128]
   float* s_lam = reinterpret_cast<float*>(s_q + kMaxGroup * kHeadDim);               // [128]
-  uint8_t* s_perm = reinterpret_cast<uint8_t*>(s_lam + kHeadDim);                    // [128]
   if (warp == 1) {
     const float4 lv = a.lam ? __ldg(reinterpret_cast<const float4*>(a.lam + (size_t)j * kHeadDim) + lane)
                             : make_float4(1.f, 1.f, 1.f, 1.f);
     reinterpret_cast<float4*>(s_lam)[lane] = lv;
-  } else if (warp == 2 && lane < kHeadDim / 16) {
-    uint4 pv;
-    if (a.perm) {
-      pv = __ldg(reinterpret_cast<const uint4*>(a.perm + (size_t)j * kHeadDim) + lane);
-    } else {
-      const uint32_t c0 = 16u * lane;
-      pv = make_uint4(c0 * 0x01010101u + 0x03020100u, c0 * 0x01010101u + 0x07060504u,
-                      c0 * 0x01010101u + 0x0b0a0908u, c0 * 0x01010101u + 0x0f0e0d0cu);
-    }
-    reinterpret_cast<uint4*>(s_perm)[lane] = pv;
   }
   // ---- chunk iterator: lane 0 walks its groups tile by tile and issues the
   // copies; everyone reads the per-stage descriptors (groups, valid tokens) ----
@@ -630,8 +618,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
       const uint32_t mw = quantize_group(x, BITS == 16 ? 65535u : (1u << BITS) - 1u, sc, lane);
       __syncwarp();
       uint8_t* gbase = a.codes + tile * kTileBytes + (size_t)(a.app_slot >> 4) * kGroupBytes + (size_t)kv * (kGroupBytes / 2);
-      const uint8_t* pm = (kv == 0 && a.perm) ? a.perm + (size_t)j * kHeadDim : nullptr;
-      pack_codes<BITS>(gbase, a.app_slot & 15, kv, sc, pm, lane);
+      pack_codes<BITS>(gbase, a.app_slot & 15, kv, sc, lane);
       if (lane == 0) a.meta[(tile * f.pf + a.app_slot) * 2 + kv] = mw;
       __syncwarp();  // sc is rewritten for V
     }
@@ -648,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   __syncwarp();
 
   // ---- q' for this stream: exact int16 per head, as int8 MMA B fragments ----
-  // q'_h = q_h * lambda * qscale at the Key positions, then per head h
+  // q'_h = q_h * lambda * qscale at the Key channels, then per head h
   //   s_h = max|q'_h| / 32767,  q_int = round(q'_h / s_h) = 256 hi + lo
   // (hi: s8, lo: u8).  The MMAs compute sum A q_int exactly, and sum(q'_h)
   // is taken as s_h sum(q_int), over exactly the values the MMAs use, so
@@ -661,8 +648,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   {
     // Warp w quantizes heads 2w and 2w+1: lane L takes head gq = 2w + L/16
     // and writes the B fragment of k-block sq = L%4 for MMA lane 4 gq + tq,
-    // tq = (L/4)%4: positions 32 sq + 16 hf + 4 tq + i (hf = 0..1, i = 0..3).
-    // The 16 lanes of a head cover its 128 positions.
+    // tq = (L/4)%4: channels 32 sq + 16 hf + 4 tq + i (hf = 0..1, i = 0..3).
+    // The 16 lanes of a head cover its 128 channels.
     const int gq = 2 * warp + (lane >> 4), tq = (lane >> 2) & 3, sq = lane & 3;
     float v[2][4];
     float m = 0.f;
@@ -670,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     for (int hf = 0; hf < 2; hf++) {
 #pragma unroll
       for (int i = 0; i < 4; i++) {
-        const int ch = s_perm[32 * sq + 16 * hf + 4 * tq + i];
+        const int ch = 32 * sq + 16 * hf + 4 * tq + i;
         v[hf][i] = __bfloat162float(s_q[gq * kHeadDim + ch]) * a.qscale * s_lam[ch];
         m = fmaxf(m, fabsf(v[hf][i]));
       }

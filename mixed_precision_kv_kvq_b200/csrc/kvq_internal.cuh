@@ -8,8 +8,8 @@
 // followed by its V part (256*b bytes).  Each part is 32 "lane units" of 8*b
 // bytes; unit L (lane L = 4g + t of a warp) holds exactly the 64 codes that
 // lane needs as its MMA A-fragment registers:
-//   K (QK^T, int8 mma.m16n8k32, A = K[token][position]): tokens g and g+8
-//     of the group, positions 32s + 16r + 4t + i (k-block s = 0..3, column
+//   K (QK^T, int8 mma.m16n8k32, A = K[token][channel]): tokens g and g+8
+//     of the group, channels 32s + 16r + 4t + i (k-block s = 0..3, column
 //     half r = 0..1, member i = 0..3).  The 4 codes (i = 0..3) of one token,
 //     k-block and column half form a "quad" = one A register of 4 bytes.  A
 //     unit holds 16 quads, quad index Q = 8x + 2s + r with x = 0 for token
@@ -40,12 +40,6 @@
 // and new tokens fill the free halves tile by tile.  At any time the block is
 // therefore: tiles < k full, tile k holding h + r, tiles > k holding h.
 // Attention does not depend on token order, so nothing is ever reordered.
-//
-// Key channel order: "position" above is a position of the block's
-// per-KV-head channel order perm[j][pos] (the logical channel at that
-// position; channels sorted by decreasing migration factor lambda).
-// Attention and export apply the same order, so any permutation is valid.
-// Values keep the natural channel order.
 //
 // Meta: two 32-bit words per (stream, tile, slot), the Key's then the
 // Value's, each binary16 R (low half) and binary16 Z (high half); P_F slots
@@ -163,7 +157,6 @@ struct AppendArgs {
   uint8_t* codes;     // layer base: [batch][kv_heads][nt][16 KiB]
   uint32_t* meta;     // layer base: [batch][kv_heads][nt][pf][2]
   const float* lam_inv;  // [kv_heads][128] or null
-  const uint8_t* perm;   // [kv_heads][128] Key position -> channel, or null (identity)
   // sink + window (the block keeps token 0 and the latest kWindowTokens at 16 bits)
   bool window;           // tokens enter the window; n0/bits/h/e/nt describe the progressive cache
   bool direct;           // the block shrinks with the Direct Right Shift
@@ -187,7 +180,6 @@ struct DecodeArgs {
   uint32_t* meta;
   const void* q;        // bf16 [batch][q_heads][128]
   const float* lam;     // [kv_heads][128] or null
-  const uint8_t* perm;  // [kv_heads][128] Key position -> channel, or null (identity)
   float* out;           // fp32 [batch][q_heads][128]
   float* parts;         // workspace partials: [batch*kv_heads][splits] records of M[8], L[8], O[128][8]
   int* counters;        // [batch*kv_heads] ticket counters (zero between calls)

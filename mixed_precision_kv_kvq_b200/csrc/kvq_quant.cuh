@@ -37,15 +37,13 @@ __device__ __forceinline__ float warp_max(float x) {
 //   K: token tok -> g = tok % 8, x = tok / 8.  Byte B -> unit 4g + t, word
 //      x*b + jw, member i (t = B / 4b, jw = (B / 4) % b, i = B % 4); it holds
 //      member i of quads p = jw*(8/b) + k (k = 0 .. 8/b-1) at bits b*k, quad
-//      p = 2s + r being positions 32s + 16r + 4t + i, mapped to channels by
-//      the block's Key channel order.
+//      p = 2s + r being channels 32s + 16r + 4t + i.
 //   V: token tok -> t = (tok % 8) / 2, member mb = tok % 2, u = tok / 8.  Byte
 //      B -> unit 4g + t, word u*b + jw, half mb, byte hb of the half
 //      (g = B / 2b, jw = (B / 2) % b, hb = B % 2); it holds pairs p = jw*(16/b)
 //      + hb*(8/b) + k of channel 16(p/2) + g + 8(p%2) at bits b*k.
 template <int bits>
-__device__ __forceinline__ void pack_codes(uint8_t* gbase, int tok, int kv, const uint16_t* sc, const uint8_t* pm,
-                                           int lane) {
+__device__ __forceinline__ void pack_codes(uint8_t* gbase, int tok, int kv, const uint16_t* sc, int lane) {
   if constexpr (bits == 16) {  // two codes per 32-bit word
     if (kv == 0) {
       const int g = tok & 7, xs = tok >> 3;
@@ -53,7 +51,7 @@ __device__ __forceinline__ void pack_codes(uint8_t* gbase, int tok, int kv, cons
         const int t = wi >> 4, jw = wi & 15;
         const int p = jw >> 1;
         const int pos = 32 * (p >> 1) + 16 * (p & 1) + 4 * t + 2 * (jw & 1);
-        const uint32_t word = (uint32_t)sc[pm ? pm[pos] : pos] | ((uint32_t)sc[pm ? pm[pos + 1] : pos + 1] << 16);
+        const uint32_t word = (uint32_t)sc[pos] | ((uint32_t)sc[pos + 1] << 16);
         reinterpret_cast<uint32_t*>(gbase + (4 * g + t) * unit_bytes(16))[xs * 16 + jw] = word;
       }
     } else {
@@ -75,7 +73,7 @@ __device__ __forceinline__ void pack_codes(uint8_t* gbase, int tok, int kv, cons
       for (int k = 0; k < per_byte; k++) {
         const int p = jw * per_byte + k;
         const int pos = 32 * (p >> 1) + 16 * (p & 1) + 4 * t + i;
-        byte |= (uint32_t)sc[pm ? pm[pos] : pos] << (bits * k);
+        byte |= (uint32_t)sc[pos] << (bits * k);
       }
       // join the 4 bytes of the word (lanes 4w .. 4w+3)
       uint32_t word = byte << (8 * i);
@@ -106,8 +104,7 @@ __device__ __forceinline__ void pack_codes(uint8_t* gbase, int tok, int kv, cons
 
 // Read one token's 16-bit codes back from its group part (the inverse of
 // pack_codes at 16 bits) into sc, channel order.
-__device__ __forceinline__ void unpack_codes16(const uint8_t* gbase, int tok, int kv, uint16_t* sc,
-                                               const uint8_t* pm, int lane) {
+__device__ __forceinline__ void unpack_codes16(const uint8_t* gbase, int tok, int kv, uint16_t* sc, int lane) {
   const uint16_t* u16 = reinterpret_cast<const uint16_t*>(gbase);
   constexpr int kUnitHalves = 8 * 16 / 2;  // 128-byte units
   if (kv == 0) {
@@ -115,7 +112,7 @@ __device__ __forceinline__ void unpack_codes16(const uint8_t* gbase, int tok, in
     for (int pos = lane; pos < kHeadDim; pos += 32) {
       const int p = 2 * (pos >> 5) + ((pos >> 4) & 1), t = (pos >> 2) & 3, i = pos & 3;
       const int word = xs * 16 + 2 * p + (i >> 1);
-      sc[pm ? pm[pos] : pos] = u16[(4 * g + t) * kUnitHalves + 2 * word + (i & 1)];
+      sc[pos] = u16[(4 * g + t) * kUnitHalves + 2 * word + (i & 1)];
     }
   } else {
     const int t = (tok & 7) >> 1, mb = tok & 1, u = tok >> 3;
