@@ -8,7 +8,8 @@
 // the block's width; key design 3 folds the migration factor into the
 // query).  Dequantisation is folded out of the inner loop:
 //   q'.k^_t = (R_t / (2^b-1)) (q'.c_t) + Z_t sum(q'),
-//   sum_t p_t v^_t = (sum_t p_t R_t c_t) / (2^b-1) + sum_t p_t Z_t,
+//   sum_t p_t v^_t = (sum_t p_t R_t (c_t - h)) / (2^b-1) + sum_t p_t Z'_t,
+//   h = 2^(b-1), Z'_t = Z_t + R_t h / (2^b-1)  (codes centred),
 // so the raw codes go straight into tensor-core operands:
 //   QK^T: int8 mma.sync.m16n8k32, A = 16 tokens x 32 Key channels of codes
 //   (byte quads, each code moved to the top of its byte: c 2^(8-b), exact in
@@ -17,7 +18,8 @@
 //   accumulation (no rounding until one int -> float conversion per score);
 //   PV: fp16 mma.sync.m16n8k16, A = 16 channels x 16 tokens of V codes
 //   widened in registers with the 0x6400 exponent trick (integer c in the
-//   low mantissa bits of 1024.0; one lop3 + one sub.f16x2 per code pair),
+//   low mantissa bits of 1024.0; one lop3 + one sub.f16x2 per code pair,
+//   which also subtracts h),
 //   B = p R (transposed from the score fragment with movmatrix).
 // 16-bit codes go in as two bytes (Keys) or two fp16 halves (Values).
 
@@ -189,19 +191,25 @@ __host__ __device__ constexpr int field_shift() {
   return BITS * ((POS % (16 / BITS)) % (8 / BITS));
 }
 // Pair at field position POS: the two codes sit at bits [BITS*POS, +BITS) of
-// each half-word.  Result: half2 (c0 * 2^e, c1 * 2^e), exact, with
-// e = field_shift: (0x6400 | c << e) is the fp16 number 1024 + c 2^e, and
-// subtracting 1024 is exact.  The 2^e is undone outside the inner loop, in
-// the output rows.
+// each half-word.  Result: half2 ((c0 - 2^(BITS-1)) 2^e, (c1 - 2^(BITS-1)) 2^e),
+// exact, with e = field_shift: (0x6400 | c << e) is the fp16 number
+// 1024 + c 2^e, and subtracting the integer 1024 + 2^(BITS-1+e) is exact.
+// Centring the codes keeps the P V sum and the Z sum small (both near the
+// output instead of two large terms that cancel), so the fp32 accumulation
+// of the MMAs loses nothing to cancellation; the 2^(BITS-1) R / (2^BITS - 1)
+// taken out here is added to each token's zero.  The 2^e is undone outside
+// the inner loop, in the output rows.
 template <int BITS, int POS>
 __device__ __forceinline__ uint32_t widen(uint32_t w, uint32_t w8) {
   constexpr int kPerByte = 8 / BITS;
   constexpr int e = field_shift<BITS, POS>();
   constexpr uint32_t m = (1u << BITS) - 1u;
   constexpr uint32_t mask = (m << e) | (m << (16 + e));
+  constexpr uint32_t off = (0x6400u + (1u << (BITS - 1 + e))) * 0x00010001u;
+  static_assert((1u << (BITS - 1 + e)) < 1024u, "the offset is an integer below 2048");
   const uint32_t x = lop_and_or((POS % (16 / BITS)) >= kPerByte ? w8 : w, mask, 0x64006400u);
   uint32_t d;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(x), "r"(0x64006400u));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(x), "r"(off));
   return d;
 }
 // field_shift of pair p (any p in 0..15) at BITS <= 8.
@@ -209,9 +217,10 @@ template <int BITS>
 __host__ __device__ constexpr int pair_shift(int p) {
   return BITS >= 16 ? 0 : BITS * ((p % (16 / BITS)) % (8 / BITS));
 }
-// 16-bit codes: the whole word is the pair; split each code into high and low byte.
+// 16-bit codes: the whole word is the pair; split each code into high and low
+// byte, c - 2^15 = 256 (hi - 128) + lo (centred as above).
 __device__ __forceinline__ uint32_t widen16_hi(uint32_t w) {
-  return hfma2_u(lop_and_or(w >> 8, 0x00ff00ffu, 0x64006400u), 0x3c003c00u, 0xe400e400u);
+  return hfma2_u(lop_and_or(w >> 8, 0x00ff00ffu, 0x64006400u), 0x3c003c00u, 0xe480e480u);  // - 1152
 }
 __device__ __forceinline__ uint32_t widen16_lo(uint32_t w) {
   return hfma2_u(lop_and_or(w, 0x00ff00ffu, 0x64006400u), 0x3c003c00u, 0xe400e400u);
@@ -375,6 +384,7 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
                                                const uint4* qfl, float ks0, float ks1, float sig0, float sig1,
                                                Soft& st) {
   constexpr int kGroupBytes = 512 * BITS, kPart = 256 * BITS;
+  constexpr float kVMid = (float)(1u << (BITS - 1)) / (float)((1u << BITS) - 1u);
   const int g = lane >> 2;
   const uint32_t* ku[NG];
   const uint32_t* vu[NG];
@@ -400,8 +410,11 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
     x[n][1] = fmaf(ka.x * ks1, d[n][1], fmaf(ka.y, sig1, -me1));  // token g,   head 2t+1
     x[n][2] = fmaf(kb.x * ks0, d[n][2], fmaf(kb.y, sig0, -me0));  // token g+8, head 2t
     x[n][3] = fmaf(kb.x * ks1, d[n][3], fmaf(kb.y, sig1, -me1));  // token g+8, head 2t+1
-    zv[n][0] = __high2float(*reinterpret_cast<const __half2*>(&mga.y));
-    zv[n][1] = __high2float(*reinterpret_cast<const __half2*>(&mgb.y));
+    // Value zero moved by the centring of the codes: Z + R 2^(b-1) / (2^b - 1)
+    const float2 va = __half22float2(*reinterpret_cast<const __half2*>(&mga.y));
+    const float2 vb = __half22float2(*reinterpret_cast<const __half2*>(&mgb.y));
+    zv[n][0] = fmaf(va.x, kVMid, va.y);
+    zv[n][1] = fmaf(vb.x, kVMid, vb.y);
     rv2[n][0] = __byte_perm(mga.y, 0, 0x1010);  // low half twice
     rv2[n][1] = __byte_perm(mgb.y, 0, 0x1010);
   }
@@ -719,8 +732,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     const uint2* ms = reinterpret_cast<const uint2*>(my.meta[st]);
     if (dsc.x == kChunkGroups && dsc.y >= 16 * kChunkGroups) {
       // full chunk: fixed offsets, no masking
+      // unrolled: one pair's P V and the next pair's QK share a basic block
       constexpr int kNG = kChunkGroups >= 2 ? 2 : 1;
-#pragma unroll 1
+#pragma unroll
       for (int gi = 0; gi < kChunkGroups; gi += kNG)
         process_groups<BITS, kNG, true>(cs + gi * kGroupBytes, ms + gi * 16, 16 * kNG, lane, qfl, ks0, ks1, sig0,
                                         sig1, sm);
