@@ -492,6 +492,221 @@ int orc_wlayer_window_tokens(const orc_wlayer* W, int* tokens) {
 }
 
 /* ------------------------------------------------------------------------ */
+/* Per-channel Key groups (KIVI's axis; the PM-KVQ note's training strategy  */
+/* names group size 128 without an axis, and its comparison with KIVI names  */
+/* KIVI's per-channel Key / per-token Value split).  Readings:               */
+/*   - A Key group is one channel of one KV head over a block of 128         */
+/*     consecutive tokens; Value groups stay one token's 128 channels.       */
+/*   - The tokens of the block being filled (the last n mod 128) are held at */
+/*     INT16, each quantized per token (Keys after the migration), as the    */
+/*     note stores recent tokens at INT16.                                   */
+/*   - When a block's 128th token arrives the block enters the progressive   */
+/*     cache.  Keys: every staged INT16 Key is dequantized in fp32 as         */
+/*     x = Z + code * (R / 65535) (one division, one multiply, one add, each */
+/*     round-to-nearest, no fused multiply-add) and each channel's 128       */
+/*     values are quantized by the affine quantizer directly at the cache's  */
+/*     current width (tokens reach the cache directly at its width, as new   */
+/*     tokens do after a shrink).  Values move by the block's shift chain    */
+/*     from their INT16 codes, R and Z kept (R rescaled by the direct        */
+/*     shift), as tokens leaving the sink + window store do.                 */
+/*   - The progressive cache takes whole blocks: a block that does not fit   */
+/*     at the current width shrinks the cache first.  Its capacity at every  */
+/*     width is a multiple of 128 tokens (N * Fbit / 16 divisible by 128),   */
+/*     so a shrink always finds the cache full.  A shrink treats the         */
+/*     per-channel Key ranges as the per-token ones (kept by the Equivalent  */
+/*     Right Shift, rescaled by the Direct Right Shift).                     */
+/* ------------------------------------------------------------------------ */
+
+#define ORC_KBLOCK 128
+
+typedef struct {
+  orc_layer main; /* codes and Value meta per token; its Key meta is unused */
+  uint16_t* kmc;  /* [batch][kv_heads][n_f / 128][128][2]: per-channel Key (R, Z) per block */
+  int n;          /* tokens appended */
+  uint16_t* skc;  /* staging: [batch][kv_heads][128][128] INT16 codes, token t in slot t mod 128 */
+  uint16_t* svc;
+  uint16_t* skm; /* [batch][kv_heads][128][2] */
+  uint16_t* svm;
+} orc_clayer;
+
+size_t orc_clayer_sizeof(void) { return sizeof(orc_clayer); }
+
+int orc_clayer_init(orc_clayer* C, int batch, int kv_heads, int n_f, int fbit) {
+  memset(C, 0, sizeof(*C));
+  if (n_f <= 0 || ((int64_t)n_f * fbit / 16) % ORC_KBLOCK != 0 || ((int64_t)n_f * fbit) % 16 != 0) return -1;
+  int rc = orc_layer_init(&C->main, batch, kv_heads, n_f, fbit);
+  if (rc) return rc;
+  size_t streams = (size_t)batch * kv_heads;
+  C->kmc = (uint16_t*)calloc(streams * (size_t)n_f * 2, 2);
+  C->skc = (uint16_t*)calloc(streams * ORC_KBLOCK * ORC_D, 2);
+  C->svc = (uint16_t*)calloc(streams * ORC_KBLOCK * ORC_D, 2);
+  C->skm = (uint16_t*)calloc(streams * ORC_KBLOCK * 2, 2);
+  C->svm = (uint16_t*)calloc(streams * ORC_KBLOCK * 2, 2);
+  if (!C->kmc || !C->skc || !C->svc || !C->skm || !C->svm) return -2;
+  return 0;
+}
+
+void orc_clayer_free(orc_clayer* C) {
+  orc_layer_free(&C->main);
+  free(C->kmc);
+  free(C->skc);
+  free(C->svc);
+  free(C->skm);
+  free(C->svm);
+  memset(C, 0, sizeof(*C));
+}
+
+static size_t orc_cstage(const orc_clayer* C, int b, int h, int s) {
+  return ((size_t)b * C->main.kv_heads + h) * ORC_KBLOCK + s;
+}
+/* (R, Z) of channel c of block blk: index of its pair */
+static size_t orc_ckm(const orc_clayer* C, int b, int h, int blk, int c) {
+  return ((((size_t)b * C->main.kv_heads + h) * (C->main.n_f / ORC_KBLOCK) + blk) * ORC_D + c) * 2;
+}
+
+/* fp32 value of an INT16 code: Z + code * (R / 65535), three RN steps. */
+float orc_int16_value(uint16_t code, uint16_t r_bits, uint16_t z_bits) {
+  volatile float r = (float)orc_f16_to_f64(r_bits);
+  volatile float z = (float)orc_f16_to_f64(z_bits);
+  volatile float step = r / 65535.0f;
+  volatile float p = (float)code * step;
+  volatile float x = z + p;
+  return x;
+}
+
+static int orc_clayer_shrink(orc_clayer* C) {
+  orc_layer* L = &C->main;
+  int rc = orc_layer_shrink(L);
+  if (rc) return rc;
+  if (L->shift_mode == 1) {
+    int blocks = L->n / ORC_KBLOCK;
+    for (int bb = 0; bb < L->batch; bb++)
+      for (int h = 0; h < L->kv_heads; h++)
+        for (int k = 0; k < blocks; k++)
+          for (int c = 0; c < ORC_D; c++) {
+            size_t i = orc_ckm(C, bb, h, k, c);
+            C->kmc[i] = orc_drs_range(C->kmc[i], L->bits);
+          }
+  }
+  return 0;
+}
+
+/* The full staged block enters the progressive cache. */
+static void orc_clayer_move_block(orc_clayer* C) {
+  orc_layer* L = &C->main;
+  while (L->n + ORC_KBLOCK > orc_layer_capacity(L, L->bits))
+    if (orc_clayer_shrink(C) != 0) return; /* unreachable: the caller checked the budget */
+  const int blk = L->n / ORC_KBLOCK;
+  float col[ORC_KBLOCK];
+  uint16_t codes[ORC_KBLOCK];
+  for (int bb = 0; bb < L->batch; bb++)
+    for (int h = 0; h < L->kv_heads; h++) {
+      for (int c = 0; c < ORC_D; c++) {
+        for (int t = 0; t < ORC_KBLOCK; t++) {
+          size_t s = orc_cstage(C, bb, h, t);
+          col[t] = orc_int16_value(C->skc[s * ORC_D + c], C->skm[s * 2], C->skm[s * 2 + 1]);
+        }
+        size_t mi = orc_ckm(C, bb, h, blk, c);
+        orc_quantize_group(col, ORC_KBLOCK, L->bits, codes, &C->kmc[mi], &C->kmc[mi + 1]);
+        for (int t = 0; t < ORC_KBLOCK; t++) L->kc[orc_slot(L, bb, h, L->n + t) * ORC_D + c] = codes[t];
+      }
+      for (int t = 0; t < ORC_KBLOCK; t++) {
+        size_t s = orc_cstage(C, bb, h, t), dst = orc_slot(L, bb, h, L->n + t);
+        for (int c = 0; c < ORC_D; c++)
+          L->vc[dst * ORC_D + c] = (uint16_t)orc_chain_code(C->svc[s * ORC_D + c], L->bits, L->shift_mode);
+        L->vm[dst * 2] = orc_chain_range(C->svm[s * 2], L->bits, L->shift_mode);
+        L->vm[dst * 2 + 1] = C->svm[s * 2 + 1];
+      }
+    }
+  L->n += ORC_KBLOCK;
+}
+
+/* Append n tokens (same arguments as orc_layer_append).  Returns 1 when the
+ * progressive cache could not hold the blocks completed by the call at Fbit
+ * (nothing written). */
+int orc_clayer_append(orc_clayer* C, const float* k, const float* v, int n, const float* lambda) {
+  orc_layer* L = &C->main;
+  if (n < 0) return -1;
+  if (((int64_t)C->n + n) / ORC_KBLOCK * ORC_KBLOCK > (int64_t)L->n_f) return 1;
+  float x[ORC_D];
+  for (int i = 0; i < n; i++) {
+    int t = C->n;
+    for (int bb = 0; bb < L->batch; bb++)
+      for (int h = 0; h < L->kv_heads; h++) {
+        size_t in = (((size_t)bb * n + i) * L->kv_heads + h) * ORC_D;
+        size_t s = orc_cstage(C, bb, h, t % ORC_KBLOCK);
+        for (int c = 0; c < ORC_D; c++)
+          x[c] = lambda ? orc_migrate(k[in + c], lambda[h * ORC_D + c]) : k[in + c];
+        orc_quantize_group(x, ORC_D, 16, C->skc + s * ORC_D, C->skm + s * 2, C->skm + s * 2 + 1);
+        orc_quantize_group(v + in, ORC_D, 16, C->svc + s * ORC_D, C->svm + s * 2, C->svm + s * 2 + 1);
+      }
+    C->n++;
+    if (C->n % ORC_KBLOCK == 0) orc_clayer_move_block(C);
+  }
+  return 0;
+}
+
+/* Decode attention over a block with per-channel Key groups: the progressive
+ * cache (Key channel c of token t dequantized with its block's (R_c, Z_c))
+ * and the staged tokens at INT16, every token attended in fp64. */
+int orc_cattention(const orc_clayer* C, const float* q, int q_heads, const float* lambda, double sm_scale,
+                   double* out) {
+  const orc_layer* L = &C->main;
+  if (C->n <= 0 || q_heads % L->kv_heads) return -1;
+  int g = q_heads / L->kv_heads;
+  int T = C->n; /* main tokens 0 .. L->n - 1, then the staged ones */
+  double* s = (double*)malloc(sizeof(double) * (size_t)T);
+  double qp[ORC_D];
+  if (!s) return -2;
+  for (int bb = 0; bb < L->batch; bb++)
+    for (int hq = 0; hq < q_heads; hq++) {
+      int h = hq / g;
+      const float* qq = q + ((size_t)bb * q_heads + hq) * ORC_D;
+      for (int c = 0; c < ORC_D; c++)
+        qp[c] = (double)qq[c] * (lambda ? (double)lambda[h * ORC_D + c] : 1.0);
+      double mx = -INFINITY;
+      for (int t = 0; t < T; t++) {
+        double acc = 0.0;
+        if (t < L->n) {
+          size_t slot = orc_slot(L, bb, h, t);
+          for (int c = 0; c < ORC_D; c++) {
+            size_t mi = orc_ckm(C, bb, h, t / ORC_KBLOCK, c);
+            acc += qp[c] * orc_dequant(L->kc[slot * ORC_D + c], C->kmc[mi], C->kmc[mi + 1], L->bits);
+          }
+        } else {
+          size_t st = orc_cstage(C, bb, h, t % ORC_KBLOCK);
+          for (int c = 0; c < ORC_D; c++)
+            acc += qp[c] * orc_dequant(C->skc[st * ORC_D + c], C->skm[st * 2], C->skm[st * 2 + 1], 16);
+        }
+        s[t] = sm_scale * acc;
+        if (s[t] > mx) mx = s[t];
+      }
+      double den = 0.0;
+      for (int t = 0; t < T; t++) {
+        s[t] = exp(s[t] - mx);
+        den += s[t];
+      }
+      double* o = out + ((size_t)bb * q_heads + hq) * ORC_D;
+      for (int c = 0; c < ORC_D; c++) o[c] = 0.0;
+      for (int t = 0; t < T; t++) {
+        const uint16_t *vc, *vm;
+        int bits;
+        if (t < L->n) {
+          size_t slot = orc_slot(L, bb, h, t);
+          vc = L->vc + slot * ORC_D, vm = L->vm + slot * 2, bits = L->bits;
+        } else {
+          size_t st = orc_cstage(C, bb, h, t % ORC_KBLOCK);
+          vc = C->svc + st * ORC_D, vm = C->svm + st * 2, bits = 16;
+        }
+        double p = s[t] / den;
+        for (int c = 0; c < ORC_D; c++) o[c] += p * orc_dequant(vc[c], vm[0], vm[1], bits);
+      }
+    }
+  free(s);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Decode attention over the quantized cache, fp64.                          */
 /* q: [batch][q_heads][128] (fp32 values of the bf16 queries).               */
 /* lambda: [kv_heads][128] or NULL.  out: [batch][q_heads][128].             */

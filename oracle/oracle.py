@@ -59,7 +59,16 @@ class _WLayer(C.Structure):
     ]
 
 
+class _CLayer(C.Structure):
+    _fields_ = [
+        ("main", _Layer), ("kmc", C.POINTER(C.c_uint16)), ("n", C.c_int),
+        ("skc", C.POINTER(C.c_uint16)), ("svc", C.POINTER(C.c_uint16)),
+        ("skm", C.POINTER(C.c_uint16)), ("svm", C.POINTER(C.c_uint16)),
+    ]
+
+
 WINDOW = 128
+KBLOCK = 128
 
 
 def lib():
@@ -107,8 +116,16 @@ def lib():
         L.orc_attention.argtypes = [P, P, C.c_int, P, C.c_double, P]
         L.orc_attention_dense.argtypes = [P, P, P, C.c_int, C.c_int, C.c_int, C.c_int,
                                           C.c_double, P]
+        L.orc_clayer_sizeof.restype = C.c_size_t
+        L.orc_clayer_init.argtypes = [P, C.c_int, C.c_int, C.c_int, C.c_int]
+        L.orc_clayer_free.argtypes = [P]
+        L.orc_clayer_append.argtypes = [P, P, P, C.c_int, P]
+        L.orc_cattention.argtypes = [P, P, C.c_int, P, C.c_double, P]
+        L.orc_int16_value.argtypes = [C.c_uint16, C.c_uint16, C.c_uint16]
+        L.orc_int16_value.restype = C.c_float
         assert L.orc_layer_sizeof() == C.sizeof(_Layer)
         assert L.orc_wlayer_sizeof() == C.sizeof(_WLayer)
+        assert L.orc_clayer_sizeof() == C.sizeof(_CLayer)
     return _lib
 
 
@@ -407,4 +424,87 @@ class WLayer:
         rc = lib().orc_wattention(C.byref(self._s), _ptr(q), q.shape[1], lp, float(sm_scale), _ptr(out))
         if rc != 0:
             raise ValueError(f"orc_wattention failed ({rc})")
+        return out
+
+
+def int16_value(code: int, r_bits: int, z_bits: int) -> float:
+    """fp32 value of an INT16 record: Z + code * (R / 65535), three RN steps
+    (how a staged Key re-enters the quantizer of a per-channel block)."""
+    return lib().orc_int16_value(int(code), int(r_bits), int(z_bits))
+
+
+class CLayer:
+    """A block whose Keys are grouped per channel over blocks of 128 tokens
+    (KIVI's axis, the other reading of the PM-KVQ note's group size 128);
+    Values per token.  The block being filled is staged at INT16; complete
+    blocks live in the progressive cache (`main`, a Layer view whose Key meta
+    is unused: the per-channel ranges are in `k_meta_channel`)."""
+
+    def __init__(self, batch: int, kv_heads: int, n_f: int, fbit: int):
+        self._s = _CLayer()
+        rc = lib().orc_clayer_init(C.byref(self._s), batch, kv_heads, n_f, fbit)
+        if rc != 0:
+            raise ValueError(f"orc_clayer_init failed ({rc})")
+        self.batch, self.kv_heads, self.n_f, self.fbit = batch, kv_heads, n_f, fbit
+        self.main = Layer.__new__(Layer)
+        self.main._s = self._s.main
+        self.main.batch, self.main.kv_heads, self.main.n_f, self.main.fbit = batch, kv_heads, n_f, fbit
+        self.main._view = True
+
+    def __del__(self):
+        try:
+            lib().orc_clayer_free(C.byref(self._s))
+        except Exception:
+            pass
+
+    @property
+    def n(self) -> int:
+        return self._s.n
+
+    @property
+    def n_staged(self) -> int:
+        return self._s.n - self._s.main.n
+
+    def set_shift_mode(self, mode: int) -> int:
+        return lib().orc_layer_set_shift_mode(C.byref(self._s.main), int(mode))
+
+    def append(self, k: np.ndarray, v: np.ndarray, lam: np.ndarray | None) -> int:
+        k = np.ascontiguousarray(k, dtype=np.float32)
+        v = np.ascontiguousarray(v, dtype=np.float32)
+        assert k.shape == v.shape and k.shape[0] == self.batch and k.shape[2] == self.kv_heads
+        lp = None
+        if lam is not None:
+            lam = np.ascontiguousarray(lam, dtype=np.float32)
+            lp = _ptr(lam)
+        return lib().orc_clayer_append(C.byref(self._s), _ptr(k), _ptr(v), k.shape[1], lp)
+
+    def k_meta_channel(self):
+        """[batch][kv_heads][blocks][128][2] uint16: (R bits, Z bits) of each
+        Key channel of each complete block."""
+        nb = self.n_f // KBLOCK
+        shape = (self.batch, self.kv_heads, nb, HEAD_DIM, 2)
+        a = np.ctypeslib.as_array(self._s.kmc, shape=(int(np.prod(shape)),)).reshape(shape)
+        return a[:, :, : self._s.main.n // KBLOCK].copy()
+
+    def staged_codes(self):
+        """(k codes, v codes, k meta, v meta) of the staged tokens at INT16,
+        oldest first: [batch][kv_heads][n_staged][...]."""
+        ns = self.n_staged
+        out = []
+        for p, d in ((self._s.skc, HEAD_DIM), (self._s.svc, HEAD_DIM), (self._s.skm, 2), (self._s.svm, 2)):
+            shape = (self.batch, self.kv_heads, KBLOCK, d)
+            a = np.ctypeslib.as_array(p, shape=(int(np.prod(shape)),)).reshape(shape)
+            out.append(a[:, :, :ns].copy())
+        return tuple(out)
+
+    def attention(self, q: np.ndarray, lam: np.ndarray | None, sm_scale: float) -> np.ndarray:
+        q = np.ascontiguousarray(q, dtype=np.float32)
+        out = np.empty(q.shape, np.float64)
+        lp = None
+        if lam is not None:
+            lam = np.ascontiguousarray(lam, dtype=np.float32)
+            lp = _ptr(lam)
+        rc = lib().orc_cattention(C.byref(self._s), _ptr(q), q.shape[1], lp, float(sm_scale), _ptr(out))
+        if rc != 0:
+            raise ValueError(f"orc_cattention failed ({rc})")
         return out

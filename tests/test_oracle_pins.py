@@ -475,6 +475,184 @@ def test_window_budget(orc):
     assert W.append(k[:, -1:], v[:, -1:], None) == 1 and W.n == 512 + 129
 
 
+# ------------------------------- per-channel Key groups over 128-token blocks
+
+def _int16_records(orc, x):
+    """INT16 per-token records of rows x [T][128] (the quantizer pinned above)."""
+    codes, meta = [], []
+    for row in x:
+        c, r, z = orc.quantize_group(row, 16)
+        codes.append(c)
+        meta.append((r, z))
+    return np.array(codes), np.array(meta)
+
+
+def test_channel_int16_value_is_three_fp32_steps(orc):
+    """A staged Key re-enters the quantizer as Z + code * (R / 65535) in fp32,
+    one IEEE round-to-nearest per step (numpy's float32 arithmetic here)."""
+    rng = np.random.default_rng(20)
+    f32 = np.float32
+    for _ in range(3000):
+        r = int(orc.f16_from_f64(float(rng.uniform(0.01, 40.0)), 1))
+        z = int(orc.f16_from_f64(float(rng.uniform(-20.0, 5.0)), -1))
+        code = int(rng.integers(0, 65536))
+        rf, zf = f32(orc.f16_to_f64(r)), f32(orc.f16_to_f64(z))
+        want = zf + f32(code) * (rf / f32(65535.0))
+        assert orc.int16_value(code, r, z) == want
+    assert orc.int16_value(0, r, z) == f32(orc.f16_to_f64(z))
+
+
+def test_channel_short_block_is_all_int16(orc):
+    """Fewer than 128 tokens: everything is staged at INT16, so codes and
+    attention equal those of a 16-bit per-token block of the same tokens."""
+    k, v = _cfg0_inputs(127, seed=21)
+    Cl = orc.CLayer(1, 2, 1024, 4)
+    P = orc.Layer(1, 2, 1024, 16)
+    assert Cl.append(k, v, None) == 0 and P.append(k, v, None) == 0
+    assert Cl.main.n == 0 and Cl.n_staged == 127
+    kc, vc, km, vm = Cl.staged_codes()
+    assert np.array_equal(kc, P.k_codes()) and np.array_equal(km, P.k_meta())
+    assert np.array_equal(vc, P.v_codes()) and np.array_equal(vm, P.v_meta())
+    q = torch.randn(1, 4, 128, generator=torch.Generator().manual_seed(22)).numpy()
+    np.testing.assert_allclose(Cl.attention(q, None, 0.1), P.attention(q, None, 0.1), rtol=1e-13, atol=1e-13)
+
+
+def test_channel_ramp_block_codes_run_along_tokens(orc):
+    """Keys that rise linearly along the tokens in every channel (each channel
+    with its own offset and slope): per-channel groups over the block put the
+    first token at code 0 and the last at 2^b - 1 in every channel and the
+    codes never fall along the tokens; a per-token (transposed) grouping
+    would not.  Z <= the channel's smallest INT16 value, Z + R >= its largest,
+    and every code is within half a step of it."""
+    t = np.arange(128, dtype=np.float64)[:, None]
+    a = np.linspace(-3.0, 2.0, 128)[None, :]
+    d = np.linspace(0.002, 0.05, 128)[None, :]
+    x = (a + d * t).astype(np.float32)  # [token][channel]
+    k = np.stack([x, x[:, ::-1]], axis=1)[None]  # [1][128][2 heads][128]
+    v = np.zeros_like(k)
+    for bits in (4, 2):
+        Cl = orc.CLayer(1, 2, 2048 if bits == 2 else 1024, bits)
+        # fill until the cache has shrunk to `bits`, then check the latest block
+        while Cl.main.bits != bits or Cl.main.n == 0:
+            assert Cl.append(k, v, None) == 0
+        blk = Cl.main.n // 128 - 1
+        kc = Cl.main.k_codes()[0, :, 128 * blk:]
+        kmc = Cl.k_meta_channel()[0, :, blk]
+        for h in range(2):
+            codes16, meta16 = _int16_records(orc, k[0, :, h])
+            xv = np.array([[orc.int16_value(int(codes16[i, c]), int(meta16[i, 0]), int(meta16[i, 1]))
+                            for c in range(128)] for i in range(128)], dtype=np.float64)
+            assert (kc[h, 0] == 0).all() and (kc[h, -1] == (1 << bits) - 1).all()
+            assert (np.diff(kc[h].astype(np.int64), axis=0) >= 0).all()
+            R = np.array([orc.f16_to_f64(int(r)) for r in kmc[h, :, 0]])
+            Z = np.array([orc.f16_to_f64(int(z)) for z in kmc[h, :, 1]])
+            assert (Z <= xv.min(axis=0)).all() and (Z + R >= xv.max(axis=0)).all()
+            S = R / ((1 << bits) - 1)
+            err = np.abs(xv - (Z[None] + kc[h] * S[None]))
+            assert (err <= S[None] / 2 * (1 + 1e-3) + 1e-6).all()
+            # the quantizer of the column, applied here to the same values
+            for c in (0, 37, 127):
+                want, r, z = orc.quantize_group(xv[:, c].astype(np.float32), bits)
+                assert np.array_equal(kc[h, :, c], want) and (r, z) == tuple(kmc[h, c])
+
+
+def test_channel_constant_channel(orc):
+    """Keys constant over a block (every INT16 record then has range 0 and
+    zero 1.25, so each channel's staged values are exactly 1.25): every
+    channel gets range 0, zero 1.25 and all codes 0."""
+    k, v = _cfg0_inputs(128, seed=23)
+    k[:] = 1.25
+    Cl = orc.CLayer(1, 2, 1024, 4)
+    assert Cl.append(k, v, None) == 0 and Cl.main.n == 128
+    kmc = Cl.k_meta_channel()[0, :, 0]
+    assert (kmc[..., 0] == 0).all() and (Cl.main.k_codes() == 0).all()
+    assert all(orc.f16_to_f64(int(z)) == 1.25 for z in kmc[..., 1].ravel())
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_channel_schedule_values_and_shifted_blocks(orc, mode):
+    """N = 1024 tokens at Fbit 2 (128 at 16 bits): the progressive cache
+    shrinks when the 2nd, 3rd and 5th blocks arrive (at 128, 256, 512
+    tokens), the 9th block is refused.  Values are the shift chain of their
+    INT16 codes (range chained under the direct shift, Z kept); the first
+    block's Keys are its 16-bit per-channel codes shifted down with the block
+    (ranges kept, or chained under the direct shift)."""
+    k, v = _cfg0_inputs(1152, seed=24)
+    Cl = orc.CLayer(1, 2, 1024, 2)
+    assert Cl.set_shift_mode(mode) == 0
+    assert Cl.append(k[:, :1151], v[:, :1151], None) == 0
+    m = Cl.main
+    assert (m.n, m.bits, m.shrink_at, Cl.n_staged) == (1024, 2, [128, 256, 512], 127)
+    assert Cl.append(k[:, 1151:], v[:, 1151:], None) == 1 and Cl.n == 1151
+    for h in range(2):
+        vc16, vm16 = _int16_records(orc, v[0, :1024, h])
+        assert np.array_equal(m.v_codes()[0, h], _chain(orc, vc16, 2, mode))
+        assert np.array_equal(m.v_meta()[0, h, :, 1], vm16[:, 1])
+        rr = vm16[:, 0].astype(np.int64)
+        if mode:
+            for b in (8, 4, 2):
+                rr = np.vectorize(lambda r, b=b: orc.drs_range(int(r), b))(rr)
+        assert np.array_equal(m.v_meta()[0, h, :, 0], rr)
+        # block 0 entered at 16 bits
+        kc16, km16 = _int16_records(orc, k[0, :128, h])
+        xv = np.array([[orc.int16_value(int(kc16[i, c]), int(km16[i, 0]), int(km16[i, 1]))
+                        for c in range(128)] for i in range(128)], dtype=np.float32)
+        for c in (0, 64, 127):
+            c16, r, z = orc.quantize_group(xv[:, c], 16)
+            assert np.array_equal(m.k_codes()[0, h, :128, c], _chain(orc, c16, 2, mode))
+            rw = r
+            if mode:
+                for b in (8, 4, 2):
+                    rw = orc.drs_range(rw, b)
+            assert tuple(Cl.k_meta_channel()[0, h, 0, c]) == (rw, z)
+
+
+def test_channel_capacity_must_be_whole_blocks(orc):
+    with pytest.raises(ValueError):
+        orc.CLayer(1, 2, 512, 2)  # 64 tokens at 16 bits: not a whole block
+    orc.CLayer(1, 2, 512, 4)
+
+
+def test_channel_chunked_equals_token_by_token(orc):
+    k, v = _cfg0_inputs(700, seed=25)
+    lam = np.exp(np.random.default_rng(6).uniform(0, 1.5, (2, 128))).astype(np.float32)
+    A = orc.CLayer(1, 2, 1024, 4)
+    B = orc.CLayer(1, 2, 1024, 4)
+    for t in range(700):
+        assert A.append(k[:, t:t + 1], v[:, t:t + 1], lam) == 0
+    for t0 in range(0, 700, 97):
+        assert B.append(k[:, t0:t0 + 97], v[:, t0:t0 + 97], lam) == 0
+    assert A.main.n_shrinks == B.main.n_shrinks == 2 and A.main.n == 640
+    for x, y in zip(A.staged_codes() + (A.main.k_codes(), A.main.v_codes(), A.main.v_meta(), A.k_meta_channel()),
+                    B.staged_codes() + (B.main.k_codes(), B.main.v_codes(), B.main.v_meta(), B.k_meta_channel())):
+        assert np.array_equal(x, y)
+
+
+def test_channel_attention_over_two_segments(orc):
+    """Attention = dense fp64 attention over the progressive cache (each Key
+    channel dequantized with its block's range and zero) and the staged INT16
+    tokens, assembled here."""
+    k, v = _cfg0_inputs(600, seed=26)
+    lam = np.exp(np.random.default_rng(7).uniform(0, 1.0, (2, 128))).astype(np.float32)
+    Cl = orc.CLayer(1, 2, 1024, 4)
+    Cl.append(k, v, lam)
+    m = Cl.main
+    nb = m.n // 128
+    kmc = Cl.k_meta_channel()[0]  # [2][nb][128][2]
+    R = np.vectorize(orc.f16_to_f64)(kmc[..., 0].astype(np.int64))
+    Z = np.vectorize(orc.f16_to_f64)(kmc[..., 1].astype(np.int64))
+    blk = np.repeat(np.arange(nb), 128)
+    Km = Z[:, blk] + m.k_codes()[0] * (R[:, blk] / ((1 << m.bits) - 1))
+    sk, sv, skm, svm = Cl.staged_codes()
+    K = np.concatenate([Km, orc.dequant_array(sk, skm, 16)[0]], axis=1)
+    V = np.concatenate([orc.dequant_array(m.v_codes(), m.v_meta(), m.bits)[0], orc.dequant_array(sv, svm, 16)[0]],
+                       axis=1)
+    q = torch.randn(1, 4, 128, generator=torch.Generator().manual_seed(27)).numpy()
+    qp = q[0].astype(np.float64) * np.repeat(lam.astype(np.float64), 2, axis=0)
+    want = orc.attention_dense(qp, K.transpose(1, 0, 2), V.transpose(1, 0, 2), 0.1)
+    np.testing.assert_allclose(Cl.attention(q, lam, 0.1)[0], want, rtol=1e-11, atol=1e-12)
+
+
 # ---------------------------------------------------------------- attention
 
 def _small_layer(orc, T, bits_target=4, seed=0, lam=None):
