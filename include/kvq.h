@@ -84,7 +84,31 @@ size_t kvq_pool_bytes(int layers, int batch, int kv_heads, int head_dim, size_t 
  *     progressive cache (tokens 1 .. n-129) and kvq_export_window the sink
  *     and the window; kvq_shrink needs the progressive cache full;
  *     attention covers all three. */
-enum { KVQ_OPT_SINK_WINDOW = 1 };
+/*   KVQ_OPT_KEY_CHANNEL  Key groups along the tokens (KIVI's per-channel Key,
+ *     per-token Value split, which the pages' comparison with KIVI names; the
+ *     pages' "group size 128" names no axis): a Key group is one channel of one
+ *     KV head over a block of 128 consecutive tokens.  The block being filled
+ *     (the latest n mod 128 tokens) is staged at 16 bits, each token quantized
+ *     per token as the pages store recent tokens at INT16.  When a block's
+ *     128th token arrives the block enters the progressive cache at its
+ *     current width: every staged Key is read back in fp32 as
+ *     Z + code * (R / 65535) (one division, one multiply, one add, each
+ *     round-to-nearest) and each channel's 128 values are quantized directly
+ *     at that width with the quantizer of this file; every staged Value moves
+ *     by the block's shift chain 16 -> ... -> b (R and Z kept; R rescaled
+ *     under KVQ_SHIFT_DIRECT).  A shrink treats the per-channel Key ranges as
+ *     the per-token ones.  N is a multiple of 1024 (so the progressive cache
+ *     takes whole blocks at every width); the staging adds 5 tiles of 16 KiB
+ *     plus 1,280 bytes of meta per (sequence, KV head) and block to the pool,
+ *     outside the budget, and the per-channel Key meta takes the place of the
+ *     per-token Key meta in the budget.  With the option: kvq_query reports
+ *     every token (tokens) and capacity + 127; kvq_max_tokens is N + 127;
+ *     kvq_export returns the progressive cache (tokens 0 .. n - (n mod 128) - 1)
+ *     with k_meta[2 (128 k + c) + {0, 1}] = (R, Z) of Key channel c of block
+ *     k; kvq_export_window returns the staged tokens; kvq_shrink needs the
+ *     progressive cache full; kvq_append_decode runs the two calls.  Not
+ *     combinable with KVQ_OPT_SINK_WINDOW. */
+enum { KVQ_OPT_SINK_WINDOW = 1, KVQ_OPT_KEY_CHANNEL = 2 };
 size_t kvq_pool_bytes_ex(int layers, int batch, int kv_heads, int head_dim, size_t budget_bytes,
                          const int* fbit, int options);
 
@@ -212,8 +236,10 @@ kvq_status kvq_export(const kvq_cache* c, int layer, int b, int j, uint16_t* k_c
  * KVQ_OPT_SINK_WINDOW), oldest first: token 0, then the latest min(n - 1,
  * 128) tokens, at 16 bits:
  *   k_codes, v_codes: host uint16 [129][128]; k_meta, v_meta: host uint16 [129][2]
- * (buffers for 129 tokens; the first *n_tokens rows are written).  Any of
- * the four may be NULL.  Synchronous.  Errors: INVALID (no window, stream). */
+ * (buffers for 129 tokens; the first *n_tokens rows are written).  With
+ * KVQ_OPT_KEY_CHANNEL: the staged tokens of the block being filled (n mod
+ * 128 of them), oldest first, in the same buffers.  Any of the four may be
+ * NULL.  Synchronous.  Errors: INVALID (neither option, stream). */
 kvq_status kvq_export_window(const kvq_cache* c, int layer, int b, int j, uint16_t* k_codes,
                              uint16_t* v_codes, uint16_t* k_meta, uint16_t* v_meta, int* n_tokens,
                              kvq_stream_t stream);

@@ -15,8 +15,8 @@ from typing import Optional, Sequence
 import numpy as np
 import torch
 
-from ._lib import (KVQ_DTYPE_BF16, KVQ_DTYPE_F32, KVQ_OPT_SINK_WINDOW, KVQ_SHIFT_DIRECT,  # noqa: F401
-                   KVQ_SHIFT_EQUIVALENT, WINDOW_TOKENS, KVQError, check, load)
+from ._lib import (KVQ_DTYPE_BF16, KVQ_DTYPE_F32, KVQ_OPT_KEY_CHANNEL, KVQ_OPT_SINK_WINDOW, KVQ_SHIFT_DIRECT,  # noqa: F401
+                   KVQ_SHIFT_EQUIVALENT, KEY_BLOCK, WINDOW_TOKENS, KVQError, check, load)
 
 HEAD_DIM = 128
 
@@ -167,13 +167,18 @@ def kvq_max_tokens(cache) -> int:
     return load().kvq_max_tokens(cache)
 
 
-def kvq_export(cache, layer: int, b: int, j: int, stream=None, sink_window: bool = False):
+def kvq_export(cache, layer: int, b: int, j: int, stream=None, sink_window: bool = False,
+               key_channel: bool = False):
     """-> (k_codes [T][128], v_codes [T][128], k_meta [T][2], v_meta [T][2]) uint16 numpy.
     With the sink + window option (sink_window=True) T counts the
-    progressive cache only: tokens 1 .. n - 129."""
+    progressive cache only: tokens 1 .. n - 129.  With per-channel Key
+    groups (key_channel=True) T counts the progressive cache (whole blocks of
+    128) and k_meta row 128 k + c is Key channel c of block k."""
     T = kvq_query(cache, layer)["tokens"]
     if sink_window:
         T = max(0, T - WINDOW_TOKENS - 1)
+    if key_channel:
+        T = T // KEY_BLOCK * KEY_BLOCK
     kc = np.zeros((T, HEAD_DIM), np.uint16)
     vc = np.zeros((T, HEAD_DIM), np.uint16)
     km = np.zeros((T, 2), np.uint16)
@@ -185,7 +190,8 @@ def kvq_export(cache, layer: int, b: int, j: int, stream=None, sink_window: bool
 
 def kvq_export_window(cache, layer: int, b: int, j: int, stream=None):
     """-> (k_codes [n][128], v_codes, k_meta [n][2], v_meta) uint16 numpy: the
-    sink and window tokens at 16 bits, oldest first."""
+    sink and window tokens (or, with per-channel Key groups, the staged
+    tokens) at 16 bits, oldest first."""
     n1 = WINDOW_TOKENS + 1
     kc = np.zeros((n1, HEAD_DIM), np.uint16)
     vc = np.zeros((n1, HEAD_DIM), np.uint16)
@@ -236,12 +242,14 @@ class KVQCache:
     the call (pinned memory makes the copy asynchronous)."""
 
     def __init__(self, layers: int, batch: int, kv_heads: int, budget_bytes: int,
-                 fbit: Sequence[int], head_dim: int = HEAD_DIM, device=None, sink_window: bool = False):
+                 fbit: Sequence[int], head_dim: int = HEAD_DIM, device=None, sink_window: bool = False,
+                 key_channel: bool = False):
         self.layers, self.batch, self.kv_heads = layers, batch, kv_heads
         self.fbit = list(fbit)
         self.device = torch.device(device if device is not None else "cuda")
         self.sink_window = sink_window
-        options = KVQ_OPT_SINK_WINDOW if sink_window else 0
+        self.key_channel = key_channel
+        options = (KVQ_OPT_SINK_WINDOW if sink_window else 0) | (KVQ_OPT_KEY_CHANNEL if key_channel else 0)
         nbytes = kvq_pool_bytes_ex(layers, batch, kv_heads, head_dim, budget_bytes, fbit, options)
         if nbytes == 0:
             raise KVQError(1, "invalid cache parameters or budget too small")
@@ -310,7 +318,7 @@ class KVQCache:
         return kvq_max_tokens(self.handle)
 
     def export(self, layer: int, b: int, j: int, stream=None):
-        return kvq_export(self.handle, layer, b, j, stream, self.sink_window)
+        return kvq_export(self.handle, layer, b, j, stream, self.sink_window, self.key_channel)
 
     def export_window(self, layer: int, b: int, j: int, stream=None):
         return kvq_export_window(self.handle, layer, b, j, stream)

@@ -27,6 +27,8 @@ KVQ_DTYPE_F32 = 1
 KVQ_SHIFT_EQUIVALENT = 0
 KVQ_SHIFT_DIRECT = 1
 KVQ_OPT_SINK_WINDOW = 1
+KVQ_OPT_KEY_CHANNEL = 2
+KEY_BLOCK = 128
 WINDOW_TOKENS = 128
 
 # name -> (restype, argtypes); the exported symbols of include/kvq.h

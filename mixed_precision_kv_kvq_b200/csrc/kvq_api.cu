@@ -77,6 +77,10 @@ struct LayerState {
   bool window;
   long long n_all;
   size_t off_wcodes, off_wmeta;
+  // per-channel Key groups (uses the window storage for the staged block):
+  // n counts the progressive cache (whole blocks), n_all every token
+  bool chan;
+  size_t off_kmc;
   bool lambda_set;
 };
 
@@ -92,8 +96,12 @@ bool make_plan(int layers, int batch, int kv_heads, int head_dim, size_t budget,
   *why = KVQ_ERR_INVALID;
   if (layers < 1 || batch < 1 || kv_heads < 1 || head_dim != kHeadDim || !fbit) return false;
   if (batch > 65535 || kv_heads > 4096) return false;  // kernel grid limits
-  if (options & ~KVQ_OPT_SINK_WINDOW) return false;
+  if (options & ~(KVQ_OPT_SINK_WINDOW | KVQ_OPT_KEY_CHANNEL)) return false;
+  const bool chan = (options & KVQ_OPT_KEY_CHANNEL) != 0;
+  if (chan && (options & KVQ_OPT_SINK_WINDOW)) return false;
   const bool window = (options & KVQ_OPT_SINK_WINDOW) != 0;
+  // whole 128-token blocks at every width: N * Fbit / 16 divisible by 128
+  const long long round = chan ? 2 * kTokenRound : kTokenRound;
   unsigned long long per_token = 0;  // bytes per token over all blocks
   const unsigned long long streams = (unsigned long long)batch * kv_heads * 2;
   for (int l = 0; l < layers; l++) {
@@ -101,8 +109,8 @@ bool make_plan(int layers, int batch, int kv_heads, int head_dim, size_t budget,
     per_token += streams * (16ull * fbit[l] + 4ull);
   }
   const unsigned long long n_raw = budget / per_token;
-  const long long n_f = (long long)(n_raw / kTokenRound) * kTokenRound;
-  if (n_f < kTokenRound || n_f > (1ll << 30)) {
+  const long long n_f = (long long)(n_raw / round) * round;
+  if (n_f < round || n_f > (1ll << 30)) {
     *why = KVQ_ERR_BUDGET;
     return false;
   }
@@ -133,9 +141,14 @@ bool make_plan(int layers, int batch, int kv_heads, int head_dim, size_t budget,
     L.off_meta = off;
     off += align_up(n_streams * (size_t)L.nt * L.pf * 8);
     L.window = window;
+    L.chan = chan;
     L.n_all = 0;
-    L.off_wcodes = L.off_wmeta = 0;
-    if (window) {  // token 0 and the latest 128 tokens at 16 bits, outside the budget rule
+    L.off_wcodes = L.off_wmeta = L.off_kmc = 0;
+    if (chan) {  // per-channel Key meta: (R, Z) of 128 channels per block of 128 tokens
+      L.off_kmc = off;
+      off += align_up(n_streams * (size_t)n_f * 4);
+    }
+    if (window || chan) {  // window: token 0 and the latest 128 tokens at 16 bits; chan: the staged block
       L.off_wcodes = off;
       off += align_up(n_streams * (size_t)kWindowTiles * kTileBytes);
       L.off_wmeta = off;
@@ -187,6 +200,8 @@ struct kvq_cache {
   uint32_t* meta(int l) { return reinterpret_cast<uint32_t*>(pool + L[l].off_meta); }
   uint8_t* wcodes(int l) { return pool + L[l].off_wcodes; }
   uint32_t* wmeta(int l) { return reinterpret_cast<uint32_t*>(pool + L[l].off_wmeta); }
+  uint32_t* kmc(int l) { return reinterpret_cast<uint32_t*>(pool + L[l].off_kmc); }
+  int blocks_max() const { return (int)(n_f / kKeyBlock); }
   float* lam(int l) { return reinterpret_cast<float*>(pool + L[l].off_lam); }
   float* lam_inv(int l) { return reinterpret_cast<float*>(pool + L[l].off_lam_inv); }
   int* counters(int l) { return reinterpret_cast<int*>(pool + L[l].off_counters); }
@@ -230,6 +245,10 @@ ShrinkArgs shrink_args(kvq_cache* c, int layer) {
   sa.meta = c->meta(layer);
   sa.pf = L.pf;
   sa.p_from = slots_per_tile(L.bits);
+  if (L.chan) {
+    sa.kmc = c->kmc(layer);
+    sa.kmc_words = (long long)c->batch * c->kv_heads * c->blocks_max() * kHeadDim;
+  }
   return sa;
 }
 
@@ -257,12 +276,18 @@ DecodePlan plan_decode(kvq_cache* c, const LayerState& L) {
   if (L.n > 0) {
     d.fill = make_fill(L.bits, L.nt, L.pf, L.n_shrinks, L.n);
     d.splits = decode_splits(c->sms(), n_streams, d.fill.gps);
+    if (L.chan) d.splits = (int)std::min<long long>(d.splits, d.fill.gps / 8);  // whole blocks per CTA
+  }
+  if (L.chan && L.n_all > L.n) {  // the staged block at 16 bits, token t in slot t mod 128
+    d.wfill = make_fill(16, kWindowTiles, slots_per_tile(16), 0, L.n_all - L.n);
+    d.wsplits = (int)std::min<long long>(3, d.wfill.gps);
+    if (d.splits > kMaxSplits - 3) d.splits = kMaxSplits - 3;
   }
   if (L.window) {
     d.wfill = make_fill(16, kWindowTiles, slots_per_tile(16), 0, std::min<long long>(L.n_all, kWindowTokens + 1));
     // up to 9 16-bit groups: 3 CTAs so the window's copies overlap; every CTA gets a group
     d.wsplits = (int)std::min<long long>(3, d.wfill.gps);
-    if (d.splits > kMaxSplits - 1) d.splits = kMaxSplits - 1;
+    if (d.splits > kMaxSplits - 3) d.splits = kMaxSplits - 3;
   }
   d.nparts = d.splits + d.wsplits;
   return d;
@@ -304,7 +329,13 @@ cudaError_t enqueue_decode(kvq_cache* c, int layer, const DecodePlan& d, const v
     a.fill = d.fill;
     a.splits = d.splits;
     a.part_base = 0;
-    a.safe = stable_groups(L, d.fill);
+    a.safe = L.chan ? 0 : stable_groups(L, d.fill);  // the block-move kernel may still run: no early copies
+    if (L.chan) {
+      a.chan = true;
+      a.kmc = c->kmc(layer);
+      a.blocks_max = c->blocks_max();
+      a.ep = make_epochs(L.nt, L.n_shrinks);
+    }
     a.trigger_early = d.wsplits > 0;
     if (app.group >= 0) {  // this launch writes the new token itself: keep the pre-wait copies clear of it
       a.app_group = app.group;
@@ -322,6 +353,7 @@ cudaError_t enqueue_decode(kvq_cache* c, int layer, const DecodePlan& d, const v
   }
   if (d.wsplits) {
     DecodeArgs w = a;
+    w.chan = false;
     w.codes = c->wcodes(layer);
     w.meta = c->wmeta(layer);
     w.fill = d.wfill;
@@ -332,6 +364,69 @@ cudaError_t enqueue_decode(kvq_cache* c, int layer, const DecodePlan& d, const v
     if (cudaError_t e = launch_decode(w, s)) return e;
   }
   return cudaSuccess;
+}
+
+// Per-channel Key groups: append into the staged block (16 bits, slot
+// t mod 128); each completed block enters the progressive cache, which is
+// shrunk first when the block does not fit at its width.
+kvq_status append_chan(kvq_cache* c, int layer, const void* k, const void* v, int dtype, int n_tokens,
+                       cudaStream_t s) {
+  LayerState& L = c->L[layer];
+  int off = 0;
+  while (off < n_tokens) {
+    const int staged = (int)(L.n_all - L.n);
+    const int cnt = std::min(n_tokens - off, kKeyBlock - staged);
+    AppendArgs a{};
+    a.k = k;
+    a.v = v;
+    a.dtype = dtype;
+    a.n_call = n_tokens;
+    a.tok_off = off;
+    a.cnt = cnt;
+    a.n0 = L.n;
+    a.bits = L.bits;
+    a.nt = L.nt;
+    a.pf = L.pf;
+    a.batch = c->batch;
+    a.kv_heads = c->kv_heads;
+    a.codes = c->codes(layer);
+    a.meta = c->meta(layer);
+    a.lam_inv = L.lambda_set ? c->lam_inv(layer) : nullptr;
+    a.window = true;
+    a.stage = true;
+    a.direct = L.shift_mode == KVQ_SHIFT_DIRECT;
+    a.t0 = L.n_all;
+    a.wcodes = c->wcodes(layer);
+    a.wmeta = c->wmeta(layer);
+    if (cudaError_t e = launch_append(a, s)) return cuda_fail(e, "append launch");
+    L.n_all += cnt;
+    off += cnt;
+    if (L.n_all - L.n < kKeyBlock) continue;
+    // the block is complete: make room at the current width, then move it
+    while (L.n + kKeyBlock > capacity(L, c->n_f, L.bits)) {  // the budget check keeps bits > fbit here
+      const ShrinkArgs sa = shrink_args(c, layer);
+      if (cudaError_t e = launch_shrink(sa, s)) return cuda_fail(e, "shrink launch");
+      L.bits /= 2;
+      L.n_shrinks++;
+    }
+    BlockMoveArgs m{};
+    m.wcodes = c->wcodes(layer);
+    m.wmeta = c->wmeta(layer);
+    m.codes = c->codes(layer);
+    m.meta = c->meta(layer);
+    m.kmc = c->kmc(layer);
+    m.blocks_max = c->blocks_max();
+    m.blk = (int)(L.n / kKeyBlock);
+    m.nt = L.nt;
+    m.pf = L.pf;
+    m.bits = L.bits;
+    m.direct = L.shift_mode == KVQ_SHIFT_DIRECT;
+    for (int gi = 0; gi < kKeyBlock / kGroupTokens; gi++) slot_of(L, L.n + kGroupTokens * gi, &m.g_tile[gi], &m.g_slot[gi]);
+    if (cudaError_t e = launch_block_move(m, c->batch * c->kv_heads, s)) return cuda_fail(e, "block move launch");
+    L.n += kKeyBlock;
+    L.n_stable = L.n;
+  }
+  return KVQ_OK;
 }
 
 uint32_t rd32(const uint8_t* p) {
@@ -433,6 +528,14 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* k, const void* v, int
     return fail(KVQ_ERR_INVALID, "k and v must be 16-byte aligned");
   LayerState& L = c->L[layer];
   const long long W1 = kWindowTokens + 1;  // sink + window
+  if (L.chan) {
+    if ((L.n_all + n_tokens) / kKeyBlock * kKeyBlock > c->n_f)
+      return fail(KVQ_ERR_BUDGET, "layer %d holds %lld tokens (%lld staged); %d more complete blocks that do not fit at "
+                  "Fbit %d", layer, L.n_all, L.n_all - L.n, n_tokens, L.fbit);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaError_t e = c->ensure_err(s)) return cuda_fail(e, "error flag reset");
+    return append_chan(c, layer, k, v, dtype, n_tokens, s);
+  }
   if (!L.window && L.n + n_tokens > c->n_f)
     return fail(KVQ_ERR_BUDGET, "layer %d holds %lld of %lld tokens at Fbit %d; %d more do not fit", layer, L.n, c->n_f,
                 L.fbit, n_tokens);
@@ -550,7 +653,7 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, 
   if ((reinterpret_cast<uintptr_t>(q) % 16) || (reinterpret_cast<uintptr_t>(out) % 4))
     return fail(KVQ_ERR_INVALID, "q must be 16-byte aligned and out 4-byte aligned");
   LayerState& L = c->L[layer];
-  if ((L.window ? L.n_all : L.n) <= 0) return fail(KVQ_ERR_STATE, "layer %d is empty", layer);
+  if ((L.window || L.chan ? L.n_all : L.n) <= 0) return fail(KVQ_ERR_STATE, "layer %d is empty", layer);
   const int n_streams = c->batch * c->kv_heads;
   const size_t need = decode_parts_bytes(n_streams, G);
   if (!workspace || ws_bytes < need)
@@ -573,7 +676,7 @@ kvq_status kvq_append_decode(kvq_cache* c, int layer, const void* k, const void*
                              kvq_stream_t stream) {
   if (kvq_status s = check_layer(c, layer)) return s;
   LayerState& L = c->L[layer];
-  if (L.window) {  // the window's moves need the append kernel: the two calls
+  if (L.window || L.chan) {  // the window's moves and the staged blocks need the append kernels: the two calls
     if (kvq_status st = kvq_append(c, layer, k, v, dtype, 1, stream)) return st;
     return kvq_decode_attn(c, layer, q, q_heads, sm_scale, out, workspace, ws_bytes, stream);
   }
@@ -679,7 +782,7 @@ kvq_status kvq_decode_attn_noalloc(kvq_cache* c, int layer, const void* q, int q
   if ((reinterpret_cast<uintptr_t>(q) % 16) || (reinterpret_cast<uintptr_t>(out) % 4))
     return fail(KVQ_ERR_INVALID, "q must be 16-byte aligned and out 4-byte aligned");
   LayerState& L = c->L[layer];
-  if ((L.window ? L.n_all : L.n) <= 0) return fail(KVQ_ERR_STATE, "layer %d is empty", layer);
+  if ((L.window || L.chan ? L.n_all : L.n) <= 0) return fail(KVQ_ERR_STATE, "layer %d is empty", layer);
   const int n_streams = c->batch * c->kv_heads;
   const DecodePlan d = plan_decode(c, L);
   const size_t need = decode_parts_used(n_streams, d.nparts);
@@ -706,8 +809,8 @@ kvq_status kvq_decode_attn_noalloc(kvq_cache* c, int layer, const void* q, int q
 kvq_status kvq_query(const kvq_cache* c, int layer, int* tokens, int* bits, int* cap, int* n_shrinks) {
   if (kvq_status s = check_layer(c, layer)) return s;
   const LayerState& L = c->L[layer];
-  const int w = L.window ? kWindowTokens + 1 : 0;
-  if (tokens) *tokens = (int)(L.window ? L.n_all : L.n);
+  const int w = L.window ? kWindowTokens + 1 : (L.chan ? kKeyBlock - 1 : 0);
+  if (tokens) *tokens = (int)(L.window || L.chan ? L.n_all : L.n);
   if (bits) *bits = L.bits;
   if (cap) *cap = (int)capacity(L, c->n_f, L.bits) + w;
   if (n_shrinks) *n_shrinks = L.n_shrinks;
@@ -716,6 +819,7 @@ kvq_status kvq_query(const kvq_cache* c, int layer, int* tokens, int* bits, int*
 
 int kvq_max_tokens(const kvq_cache* c) {
   if (!c) return 0;
+  if (c->layers > 0 && c->L[0].chan) return (int)c->n_f + kKeyBlock - 1;
   return (int)c->n_f + (c->layers > 0 && c->L[0].window ? kWindowTokens + 1 : 0);
 }
 
@@ -737,6 +841,14 @@ kvq_status kvq_export(const kvq_cache* c, int layer, int b, int j, uint16_t* k_c
   if (e != cudaSuccess) return cuda_fail(e, "export copy");
   const int bits = L.bits, ppw = 16 / bits;
   const uint32_t mask = bits == 16 ? 0xffffu : ((1u << bits) - 1u);
+  std::vector<uint32_t> kw;  // per-channel Key meta of the stream's blocks
+  if (L.chan && k_meta && L.n > 0) {
+    kw.resize((size_t)L.n);  // (L.n / 128) blocks of 128 words
+    const size_t base = st * (size_t)c->blocks_max() * kHeadDim;
+    e = cudaMemcpyAsync(kw.data(), m->kmc(layer) + base, kw.size() * 4, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "export copy");
+  }
   for (long long i = 0; i < L.n; i++) {
     int tile, slot;
     slot_of(L, i, &tile, &slot);
@@ -770,9 +882,10 @@ kvq_status kvq_export(const kvq_cache* c, int layer, int b, int j, uint16_t* k_c
       }
     }
     const size_t mi = ((size_t)tile * L.pf + slot) * 2;
-    if (k_meta) {
-      k_meta[2 * i] = (uint16_t)(mw[mi] & 0xffffu);
-      k_meta[2 * i + 1] = (uint16_t)(mw[mi] >> 16);
+    if (k_meta) {  // per-channel Key groups: entry 128 k + c is channel c of block k
+      const uint32_t w = L.chan ? kw[i] : mw[mi];
+      k_meta[2 * i] = (uint16_t)(w & 0xffffu);
+      k_meta[2 * i + 1] = (uint16_t)(w >> 16);
     }
     if (v_meta) {
       v_meta[2 * i] = (uint16_t)(mw[mi + 1] & 0xffffu);
@@ -788,7 +901,8 @@ kvq_status kvq_export_window(const kvq_cache* c, int layer, int b, int j, uint16
   if (b < 0 || b >= c->batch || j < 0 || j >= c->kv_heads)
     return fail(KVQ_ERR_INVALID, "stream (%d, %d) out of range", b, j);
   const LayerState& L = c->L[layer];
-  if (!L.window) return fail(KVQ_ERR_INVALID, "the cache was made without KVQ_OPT_SINK_WINDOW");
+  if (!L.window && !L.chan)
+    return fail(KVQ_ERR_INVALID, "the cache was made without KVQ_OPT_SINK_WINDOW or KVQ_OPT_KEY_CHANNEL");
   kvq_cache* m = const_cast<kvq_cache*>(c);
   constexpr int P16 = slots_per_tile(16);
   const size_t code_bytes = (size_t)kWindowTiles * kTileBytes, meta_words = (size_t)kWindowTiles * P16 * 2;
@@ -800,14 +914,19 @@ kvq_status kvq_export_window(const kvq_cache* c, int layer, int b, int j, uint16
   if (e == cudaSuccess) e = cudaMemcpyAsync(mw.data(), m->wmeta(layer) + st * meta_words, meta_words * 4, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "export copy");
-  // tokens held: 0, then max(1, n - 128) .. n - 1; token t >= 1 sits in slot 1 + (t - 1) mod 128
+  // window: tokens 0, then max(1, n - 128) .. n - 1; token t >= 1 sits in slot 1 + (t - 1) mod 128.
+  // per-channel Key groups: the staged tokens, token t in slot t mod 128.
   std::vector<long long> toks;
-  if (L.n_all > 0) toks.push_back(0);
-  for (long long t = std::max(1LL, L.n_all - kWindowTokens); t < L.n_all; t++) toks.push_back(t);
+  if (L.chan) {
+    for (long long t = L.n; t < L.n_all; t++) toks.push_back(t);
+  } else {
+    if (L.n_all > 0) toks.push_back(0);
+    for (long long t = std::max(1LL, L.n_all - kWindowTokens); t < L.n_all; t++) toks.push_back(t);
+  }
   constexpr int kUnit = 8 * 16;  // unit bytes at 16 bits
   for (size_t i = 0; i < toks.size(); i++) {
     const long long t = toks[i];
-    const int rs = t == 0 ? 0 : 1 + (int)((t - 1) % kWindowTokens);
+    const int rs = L.chan ? (int)(t % kKeyBlock) : (t == 0 ? 0 : 1 + (int)((t - 1) % kWindowTokens));
     const int tile = rs / P16, slot = rs % P16, grp = slot >> 4, tok = slot & 15;
     const size_t gbase = (size_t)tile * kTileBytes + (size_t)grp * group_bytes(16);
     if (k_codes) {

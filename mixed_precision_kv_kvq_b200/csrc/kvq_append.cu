@@ -100,13 +100,14 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs 
     int wtok = 0;
     if (a.window) {
       const long long t = a.t0 + tkn;
-      const int rs = t == 0 ? 0 : 1 + (int)((unsigned long long)(t - 1) & (kWindowTokens - 1));
+      const int rs = a.stage ? (int)((unsigned long long)t & (kKeyBlock - 1))
+                             : (t == 0 ? 0 : 1 + (int)((unsigned long long)(t - 1) & (kWindowTokens - 1)));
       const int wtile = rs / slots_per_tile(16), wslot = rs % slots_per_tile(16);
       wtok = wslot & 15;
       wg = a.wcodes + (stream * kWindowTiles + wtile) * (size_t)kTileBytes + (size_t)(wslot >> 4) * group_bytes(16) +
            (size_t)kv * part_bytes(16);
       wmi = ((stream * kWindowTiles + wtile) * (size_t)slots_per_tile(16) + wslot) * 2 + kv;
-      if (t >= kWindowTokens + 1) {
+      if (!a.stage && t >= kWindowTokens + 1) {
         // token t - 128 leaves the window: its INT16 codes go to the progressive
         // cache at the current width (index t - 129) by the block's shift chain
         unpack_codes16(wg, wtok, kv, sc, lane);
@@ -145,7 +146,101 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs 
   }
 }
 
+// Per-channel Key groups (KIVI's axis): the staged block of 128 tokens of
+// one stream enters the progressive cache at width BITS.  Keys: every staged
+// INT16 Key is read back in fp32 as Z + code * (R / 65535) and each channel's
+// 128 values go through the quantizer of kvq_quant.cuh (thread c owns
+// channel c); Values: each token's INT16 codes take the block's shift chain,
+// R and Z kept (R rescaled by the direct shift).  128 threads, one CTA per
+// stream.
+template <int BITS>
+__global__ void __launch_bounds__(kKeyBlock) block_move_kernel(BlockMoveArgs a) {
+  __shared__ uint16_t kc_sh[kKeyBlock][kHeadDim];  // [token][channel]: INT16 codes, then the new codes
+  __shared__ uint32_t km_sh[kKeyBlock];           // staged Key meta words
+  __shared__ uint16_t vc_sh[kKeyBlock / 32][kHeadDim];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const size_t stream = blockIdx.x;
+  constexpr int P16 = slots_per_tile(16);
+  auto staged = [&](int t, int kv) {  // group part holding staged token t
+    return a.wcodes + (stream * kWindowTiles + t / P16) * (size_t)kTileBytes +
+           (size_t)((t % P16) >> 4) * group_bytes(16) + (size_t)kv * part_bytes(16);
+  };
+  auto staged_meta = [&](int t, int kv) {
+    return ((stream * kWindowTiles + t / P16) * (size_t)P16 + t % P16) * 2 + kv;
+  };
+  for (int t = warp; t < kKeyBlock; t += kKeyBlock / 32) {
+    unpack_codes16(staged(t, 0), t & 15, 0, kc_sh[t], lane);
+    if (lane == 0) km_sh[t] = a.wmeta[staged_meta(t, 0)];
+  }
+  __syncthreads();
+  {
+    const int c = threadIdx.x;  // one channel per thread
+    auto value = [&](int t) {
+      const uint32_t w = km_sh[t];
+      const float r = __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
+      const float z = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+      return __fadd_rn(z, __fmul_rn((float)kc_sh[t][c], __fdiv_rn(r, 65535.0f)));
+    };
+    float mn = value(0), mx = mn;
+    for (int t = 1; t < kKeyBlock; t++) {
+      const float x = value(t);
+      mn = fminf(mn, x);
+      mx = fmaxf(mx, x);
+    }
+    const __half zh = __float2half_rd(mn);
+    const float z = __half2float(zh);
+    const __half rh = __float2half_ru(__fsub_rn(mx, z));
+    const float r = __half2float(rh);
+    constexpr unsigned qmax = BITS == 16 ? 65535u : (1u << BITS) - 1u;
+    const float inv = r == 0.0f ? 0.0f : __fdiv_rn((float)qmax, r);
+    for (int t = 0; t < kKeyBlock; t++) {
+      uint16_t q = 0;
+      if (r != 0.0f) {
+        const float y = __fadd_rn(__fmul_rn(__fsub_rn(value(t), z), inv), 0.5f);
+        q = (uint16_t)min(__float2uint_rd(y), qmax);
+      }
+      kc_sh[t][c] = q;  // only this thread reads or writes column c
+    }
+    a.kmc[(stream * a.blocks_max + a.blk) * kHeadDim + c] =
+        (uint32_t)__half_as_ushort(rh) | ((uint32_t)__half_as_ushort(zh) << 16);
+  }
+  __syncthreads();
+  uint16_t* sc = vc_sh[warp];
+  for (int t = warp; t < kKeyBlock; t += kKeyBlock / 32) {
+    const int gi = t >> 4, slot = a.g_slot[gi] + (t & 15);
+    const size_t tile = stream * a.nt + a.g_tile[gi];
+    uint8_t* gbase = a.codes + tile * kTileBytes + (size_t)(slot >> 4) * group_bytes(BITS);
+    pack_codes<BITS>(gbase, slot & 15, 0, kc_sh[t], lane);
+    unpack_codes16(staged(t, 1), t & 15, 1, sc, lane);
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; i++) sc[4 * lane + i] = (uint16_t)shift_chain<BITS>(sc[4 * lane + i], a.direct);
+    __syncwarp();
+    pack_codes<BITS>(gbase + part_bytes(BITS), slot & 15, 1, sc, lane);
+    if (lane == 0) {
+      const uint32_t old = a.wmeta[staged_meta(t, 1)];
+      a.meta[(tile * a.pf + slot) * 2 + 1] =
+          (uint32_t)range_chain<BITS>((uint16_t)(old & 0xffffu), a.direct) | (old & 0xffff0000u);
+    }
+    __syncwarp();  // sc is rewritten by the next token
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_block_move(const BlockMoveArgs& a, int n_streams, cudaStream_t s) {
+  if (n_streams <= 0) return cudaSuccess;
+  const dim3 grid((unsigned)n_streams), block(kKeyBlock);
+  switch (a.bits) {
+    case 16: return launch_pdl(block_move_kernel<16>, grid, block, 0, s, a);
+    case 8: return launch_pdl(block_move_kernel<8>, grid, block, 0, s, a);
+    case 4: return launch_pdl(block_move_kernel<4>, grid, block, 0, s, a);
+    case 2: return launch_pdl(block_move_kernel<2>, grid, block, 0, s, a);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
   const long long warps = ((long long)a.cnt + kTokensPerWarp - 1) / kTokensPerWarp * a.kv_heads * 2;  // per sequence

@@ -53,6 +53,10 @@ constexpr int kCtasPerSm = 4;
 constexpr int kQfBytes = 4 * 32 * 16;      // q' B fragments: [k-block][lane] x (hi b0, hi b1, lo b0, lo b1)
 constexpr int kSmemBytes = kWarps * kWarpSmem + kQfBytes + 3 * kWarps * kMaxGroup * 4 +
                            kWarps * kStages * 8 + kWarps * kStages * 8 + 16;
+// Per-channel Key groups: q' = q lambda qscale in fp32 for the whole kernel,
+// and per warp the int16 B fragments, scales and zero terms of its block.
+constexpr int kChanSmem = kMaxGroup * kHeadDim * 4 + kWarps * kQfBytes + kWarps * kQfBytes / 2 + 2 * kWarps * kMaxGroup * 4;
+static_assert(kSmemBytes % 16 == 0, "the channel area starts 16-byte aligned");
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
 constexpr int kPartFloats = 2 * kMaxGroup + kHeadDim * kMaxGroup;  // one CTA's partial record
 // Scratch of the fused append in a warp's second code stage (unused until the
@@ -259,9 +263,46 @@ __device__ __forceinline__ uint32_t quad_reg(const uint32_t* u) {
 // and q'_int = 256 hi + lo the per-head int16 query (hi: s8, lo: u8); every
 // product and sum is exact in int32.  The k-block loop is outermost so each
 // q' fragment is loaded once for all groups.
-template <int BITS, int NG>
-__device__ __forceinline__ void qk_groups(const uint32_t* const (&ku)[NG], const uint4* qfl, float (&d)[NG][4]) {
-  if constexpr (BITS == 16) {
+// QP = 3 (per-channel Key groups): the query operand is a 24-bit integer
+// 65536 hi + 256 mid + lo (hi s8; mid, lo u8 in qfl3), three MMAs per A.
+template <int BITS, int NG, int QP>
+__device__ __forceinline__ void qk_groups(const uint32_t* const (&ku)[NG], const uint4* qfl, const uint2* qfl3,
+                                          float (&d)[NG][4]) {
+  if constexpr (BITS == 16 && QP == 3) {
+    int hh[NG][4], hm[NG][4], hl[NG][4], lh[NG][4], lm[NG][4], ll[NG][4];
+#pragma unroll
+    for (int n = 0; n < NG; n++)
+#pragma unroll
+      for (int e = 0; e < 4; e++) hh[n][e] = hm[n][e] = hl[n][e] = lh[n][e] = lm[n][e] = ll[n][e] = 0;
+#pragma unroll
+    for (int sb = 0; sb < 4; sb++) {
+      const uint4 q4 = qfl[32 * sb];
+      const uint2 q2 = qfl3[32 * sb];
+#pragma unroll
+      for (int n = 0; n < NG; n++) {
+        const uint2 w00 = *reinterpret_cast<const uint2*>(ku[n] + 4 * sb);
+        const uint2 w01 = *reinterpret_cast<const uint2*>(ku[n] + 4 * sb + 2);
+        const uint2 w10 = *reinterpret_cast<const uint2*>(ku[n] + 16 + 4 * sb);
+        const uint2 w11 = *reinterpret_cast<const uint2*>(ku[n] + 16 + 4 * sb + 2);
+        const uint32_t l0 = __byte_perm(w00.x, w00.y, 0x6420), h0 = __byte_perm(w00.x, w00.y, 0x7531);
+        const uint32_t l1 = __byte_perm(w10.x, w10.y, 0x6420), h1 = __byte_perm(w10.x, w10.y, 0x7531);
+        const uint32_t l2 = __byte_perm(w01.x, w01.y, 0x6420), h2 = __byte_perm(w01.x, w01.y, 0x7531);
+        const uint32_t l3 = __byte_perm(w11.x, w11.y, 0x6420), h3 = __byte_perm(w11.x, w11.y, 0x7531);
+        imma_s8(hh[n], h0, h1, h2, h3, q4.x, q4.y);
+        imma_u8(hm[n], h0, h1, h2, h3, q4.z, q4.w);
+        imma_u8(hl[n], h0, h1, h2, h3, q2.x, q2.y);
+        imma_s8(lh[n], l0, l1, l2, l3, q4.x, q4.y);
+        imma_u8(lm[n], l0, l1, l2, l3, q4.z, q4.w);
+        imma_u8(ll[n], l0, l1, l2, l3, q2.x, q2.y);
+      }
+    }
+#pragma unroll
+    for (int n = 0; n < NG; n++)
+#pragma unroll
+      for (int e = 0; e < 4; e++)
+        d[n][e] = 256.0f * ((float)hh[n][e] * 65536.0f + (float)hm[n][e] * 256.0f + (float)hl[n][e]) +
+                  ((float)lh[n][e] * 65536.0f + (float)lm[n][e] * 256.0f + (float)ll[n][e]);
+  } else if constexpr (BITS == 16) {
     int hh[NG][4], hl[NG][4], lh[NG][4], ll[NG][4];
 #pragma unroll
     for (int n = 0; n < NG; n++)
@@ -302,19 +343,29 @@ __device__ __forceinline__ void qk_groups(const uint32_t* const (&ku)[NG], const
         u[n][i] = w4.x; u[n][i + 1] = w4.y; u[n][i + 2] = w4.z; u[n][i + 3] = w4.w;
       }
     }
-    int ah[NG][4], al[NG][4];
+    int ah[NG][4], al[NG][4], a3[QP == 3 ? NG : 1][4];
 #pragma unroll
     for (int n = 0; n < NG; n++)
 #pragma unroll
       for (int e = 0; e < 4; e++) ah[n][e] = al[n][e] = 0;
+    if constexpr (QP == 3) {
+#pragma unroll
+      for (int n = 0; n < NG; n++)
+#pragma unroll
+        for (int e = 0; e < 4; e++) a3[n][e] = 0;
+    }
 #define KVQ_QK(S)                                                                                    \
   {                                                                                                  \
     const uint4 q4 = qfl[32 * S];                                                                    \
     _Pragma("unroll") for (int n = 0; n < NG; n++) {                                                \
       const uint32_t a0 = quad_reg<BITS, S, 0, 0>(u[n]), a1 = quad_reg<BITS, S, 1, 0>(u[n]);         \
-      const uint32_t a2 = quad_reg<BITS, S, 0, 1>(u[n]), a3 = quad_reg<BITS, S, 1, 1>(u[n]);         \
-      imma_s8(ah[n], a0, a1, a2, a3, q4.x, q4.y);                                                    \
-      imma_u8(al[n], a0, a1, a2, a3, q4.z, q4.w);                                                    \
+      const uint32_t a2 = quad_reg<BITS, S, 0, 1>(u[n]), a3r = quad_reg<BITS, S, 1, 1>(u[n]);        \
+      imma_s8(ah[n], a0, a1, a2, a3r, q4.x, q4.y);                                                   \
+      imma_u8(al[n], a0, a1, a2, a3r, q4.z, q4.w);                                                   \
+      if constexpr (QP == 3) {                                                                       \
+        const uint2 q2 = qfl3[32 * S];                                                               \
+        imma_u8(a3[n], a0, a1, a2, a3r, q2.x, q2.y);                                                 \
+      }                                                                                              \
     }                                                                                                \
   }
     KVQ_QK(0) KVQ_QK(1) KVQ_QK(2) KVQ_QK(3)
@@ -322,7 +373,12 @@ __device__ __forceinline__ void qk_groups(const uint32_t* const (&ku)[NG], const
 #pragma unroll
     for (int n = 0; n < NG; n++)
 #pragma unroll
-      for (int e = 0; e < 4; e++) d[n][e] = (float)(ah[n][e] * 256 + al[n][e]);
+      for (int e = 0; e < 4; e++) {
+        if constexpr (QP == 3)
+          d[n][e] = (float)ah[n][e] * 65536.0f + (float)al[n][e] * 256.0f + (float)a3[n][e];
+        else
+          d[n][e] = (float)(ah[n][e] * 256 + al[n][e]);
+      }
   }
 }
 
@@ -379,10 +435,10 @@ struct Soft {
 // NG consecutive groups of one stage (cs, ms point at the first): scores,
 // one shared running-max update, probabilities, then P V.  valid0: valid
 // tokens from the first group on (FULL: all NG groups are full).
-template <int BITS, int NG, bool FULL>
+template <int BITS, int NG, bool FULL, bool CHAN>
 __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* ms, int valid0, int lane,
-                                               const uint4* qfl, float ks0, float ks1, float sig0, float sig1,
-                                               Soft& st) {
+                                               const uint4* qfl, const uint2* qfl3, float ks0, float ks1, float sig0,
+                                               float sig1, Soft& st) {
   constexpr int kGroupBytes = 512 * BITS, kPart = 256 * BITS;
   constexpr float kVMid = (float)(1u << (BITS - 1)) / (float)((1u << BITS) - 1u);
   const int g = lane >> 2;
@@ -394,9 +450,11 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
     vu[n] = reinterpret_cast<const uint32_t*>(cs + n * kGroupBytes + kPart + lane * unit_bytes(BITS));
   }
   float d[NG][4];
-  qk_groups<BITS, NG>(ku, qfl, d);
+  qk_groups<BITS, NG, CHAN ? 3 : 2>(ku, qfl, qfl3, d);
   // Scores relative to the running max: x = R ks_h d + (Z sum(q'_h) - m),
-  // ks_h = (q' scale of head h) / (code scale).
+  // ks_h = (q' scale of head h) / (code scale).  Per-channel Key groups: the
+  // block's ranges are inside the query operand and its zeros in sig, so
+  // x = ks_h d + sig_h - m (R and Z of the token read as 1).
   // Before the first group m is -inf; scores are then taken relative to 0.
   const float me0 = st.m0 == -INFINITY ? 0.f : st.m0, me1 = st.m1 == -INFINITY ? 0.f : st.m1;
   float x[NG][4], zv[NG][2];
@@ -404,8 +462,8 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
 #pragma unroll
   for (int n = 0; n < NG; n++) {
     const uint2 mga = ms[n * 16 + g], mgb = ms[n * 16 + g + 8];
-    const float2 ka = __half22float2(*reinterpret_cast<const __half2*>(&mga.x));
-    const float2 kb = __half22float2(*reinterpret_cast<const __half2*>(&mgb.x));
+    const float2 ka = CHAN ? make_float2(1.f, 1.f) : __half22float2(*reinterpret_cast<const __half2*>(&mga.x));
+    const float2 kb = CHAN ? make_float2(1.f, 1.f) : __half22float2(*reinterpret_cast<const __half2*>(&mgb.x));
     x[n][0] = fmaf(ka.x * ks0, d[n][0], fmaf(ka.y, sig0, -me0));  // token g,   head 2t
     x[n][1] = fmaf(ka.x * ks1, d[n][1], fmaf(ka.y, sig1, -me1));  // token g,   head 2t+1
     x[n][2] = fmaf(kb.x * ks0, d[n][2], fmaf(kb.y, sig0, -me0));  // token g+8, head 2t
@@ -487,6 +545,80 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
   pv_groups<BITS, NG>(vu, b0, b1, st.o);
 }
 
+// Per-channel Key groups: the query operand of one 128-token block.  The
+// block's Key channel c is Z_c + code R_c / (2^b - 1), so
+//   q'.k^_t = sum_c q'_c Z_c + sum_c (q'_c R_c / (2^b - 1)) code_t,c
+// and w_c = q'_c R_c / (2^b - 1) takes the place of q' as an exact per-head
+// 24-bit integer (scale max|w| / (2^23 - 1)); the first sum is the head's
+// zero term.  24 bits, not the 16 of the per-token operand: w carries both
+// the migrated query's outlier channels and the same channels' wider ranges,
+// so its largest entry is far above the typical one and 16 bits left the
+// ordinary channels too coarse (2.4e-3 output error on 2-bit blocks).  The
+// warp writes its own B fragments (hi and mid bytes in the per-token layout,
+// lo bytes in qfw3), and per head the score scale ks (w scale times the code
+// scale of the A operand) and the zero term.  km: the block's 128 (R, Z) words.
+template <int BITS>
+__device__ __noinline__ void chan_block(const float* s_qp, const uint32_t* km, uint4* qfw, uint2* qfw3, float* wks,
+                                        float* wsig, int lane) {
+  constexpr float kInvQ = 1.0f / (float)((1u << BITS) - 1u);
+  constexpr float kA = BITS >= 8 ? 1.0f : 1.0f / (float)(1 << (8 - BITS));  // A = c 2^(8 - BITS) at b <= 8
+  const int tq = (lane >> 2) & 3, sq = lane & 3, hsel = lane >> 4;
+  // this lane's channels: 32 sq + 16 hf + 4 tq + i
+  float R[2][4], Z[2][4];
+#pragma unroll
+  for (int hf = 0; hf < 2; hf++) {
+    const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(km + 32 * sq + 16 * hf + 4 * tq));
+    const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      R[hf][i] = __half2float(__ushort_as_half((unsigned short)(w[i] & 0xffffu))) * kInvQ;
+      Z[hf][i] = __half2float(__ushort_as_half((unsigned short)(w[i] >> 16)));
+    }
+  }
+#pragma unroll 1
+  for (int hp = 0; hp < kMaxGroup / 2; hp++) {
+    const int gq = 2 * hp + hsel;  // the 16 lanes of a head cover its 128 channels
+    float v[2][4];
+    float m = 0.f, zs = 0.f;
+#pragma unroll
+    for (int hf = 0; hf < 2; hf++) {
+      const float4 q4 = *reinterpret_cast<const float4*>(s_qp + gq * kHeadDim + 32 * sq + 16 * hf + 4 * tq);
+      const float q[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        v[hf][i] = q[i] * R[hf][i];
+        m = fmaxf(m, fabsf(v[hf][i]));
+        zs = fmaf(q[i], Z[hf][i], zs);
+      }
+    }
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) {
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      zs += __shfl_xor_sync(0xffffffffu, zs, o);
+    }
+    constexpr float kQMax = 8388607.0f;  // 2^23 - 1
+    const float inv = m > 0.f ? kQMax / m : 0.f;
+    uint32_t hb[2] = {0u, 0u}, mb[2] = {0u, 0u}, lb[2] = {0u, 0u};
+#pragma unroll
+    for (int hf = 0; hf < 2; hf++) {
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const int qi = max(-8388607, min(8388607, __float2int_rn(v[hf][i] * inv)));
+        hb[hf] |= (uint32_t)((qi >> 16) & 0xff) << (8 * i);  // arithmetic shift: s8
+        mb[hf] |= (uint32_t)((qi >> 8) & 0xff) << (8 * i);
+        lb[hf] |= (uint32_t)(qi & 0xff) << (8 * i);
+      }
+    }
+    qfw[sq * 32 + 4 * gq + tq] = make_uint4(hb[0], hb[1], mb[0], mb[1]);
+    qfw3[sq * 32 + 4 * gq + tq] = make_uint2(lb[0], lb[1]);
+    if ((lane & 15) == 0) {
+      wks[gq] = m / kQMax * kA;
+      wsig[gq] = zs;
+    }
+  }
+  __syncwarp();
+}
+
 // ------------------------------------------------------------------ kernel
 
 struct WarpSmem {
@@ -494,7 +626,7 @@ struct WarpSmem {
   uint8_t meta[kStages][kStageMeta];
 };
 
-template <int BITS>
+template <int BITS, bool CHAN>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   WarpSmem* ws = reinterpret_cast<WarpSmem*>(smem);
@@ -505,6 +637,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   uint64_t* bars = reinterpret_cast<uint64_t*>(w_pz + kWarps * kMaxGroup);  // [warps][stages]
   int2* desc = reinterpret_cast<int2*>(bars + kWarps * kStages);              // [warps][stages] (ng, valid0)
   volatile int* flags = reinterpret_cast<volatile int*>(desc + kWarps * kStages);  // [0] abort, [1] last
+  // per-channel Key groups only (the launch sizes the area): q' [8][128],
+  // per-warp B fragments [warps][4][32], scales and zero terms [warps][8]
+  float* s_qp = reinterpret_cast<float*>(smem + kSmemBytes);
+  uint4* qfw = reinterpret_cast<uint4*>(s_qp + kMaxGroup * kHeadDim);
+  uint2* qfw3 = reinterpret_cast<uint2*>(qfw + kWarps * 4 * 32);
+  float* w_ks = reinterpret_cast<float*>(qfw3 + kWarps * 4 * 32);
+  float* w_sig = w_ks + kWarps * kMaxGroup;
 
   constexpr int kGroupBytes = 512 * BITS;
   constexpr bool kWide = BITS == 16;            // a 16-bit group (8 KiB) takes every code stage
@@ -519,8 +658,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   const int g = lane >> 2, t = lane & 3;
   const int G = a.group;
   const int s = blockIdx.x / a.splits, split = blockIdx.x - s * a.splits;
-  const long long ca = f.gps * split / a.splits, cb = f.gps * (split + 1) / a.splits;
-  const long long wa = ca + (cb - ca) * warp / kWarps, wb = ca + (cb - ca) * (warp + 1) / kWarps;
+  // Per-channel Key groups split the stream by whole 128-token blocks (8 groups).
+  const long long units = CHAN ? f.gps / 8 : f.gps, per = CHAN ? 8 : 1;
+  const long long ca = units * split / a.splits, cb = units * (split + 1) / a.splits;
+  const long long wa = per * (ca + (cb - ca) * warp / kWarps), wb = per * (ca + (cb - ca) * (warp + 1) / kWarps);
   WarpSmem& my = ws[warp];
   const uint32_t bar0 = smem_u32(bars + warp * kStages);
   int2* mydesc = desc + warp * kStages;
@@ -548,7 +689,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   // copies; everyone reads the per-stage descriptors (groups, valid tokens) ----
   int left = (int)(wb - wa);  // groups this warp still has to issue
   int it_tile = 0, it_grp = 0, it_tgroups = 0, it_tvalid = 0;
-  if (left > 0) {
+  long long v_next = wa;  // per-channel Key groups: next group in logical order
+  if (!CHAN && left > 0) {
     const GroupLoc loc = locate_group(f, wa);
     it_tile = loc.tile;
     it_grp = loc.grp;
@@ -560,6 +702,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   auto issue = [&](int st) {  // lane 0 only: next chunk of this warp into stage st
     if (left <= 0) {
       mydesc[st] = make_int2(0, 0);
+      return;
+    }
+    if constexpr (CHAN) {
+      // logical order: group v holds tokens 16v .. 16v+15, which arrived in
+      // epoch e and sit in slots [h_e, h_e + ee_e) of tile (16v - start_e) / ee_e;
+      // a chunk stays inside one tile's run of the epoch (and so inside one
+      // 128-token block: runs and epoch starts are whole blocks or divide one)
+      const long long i = 16 * v_next;
+      int e = 0;
+      while (e + 1 < a.ep.n && i >= a.ep.start[e + 1]) e++;
+      const long long m = i - a.ep.start[e];
+      const int ee = a.ep.ee[e];
+      const int tile = (int)(m / ee), off = (int)(m - (long long)tile * ee);
+      const int grp = (a.ep.h[e] + off) >> 4;
+      int ng = (ee - off) >> 4;
+      ng = ng < kChunkGroups ? ng : kChunkGroups;
+      ng = ng < left ? ng : left;
+      mydesc[st] = make_int2(ng, (int)(v_next >> 3));  // groups, block
+      const uint32_t cbytes = (uint32_t)ng * kGroupBytes, mbytes = (uint32_t)ng * 128u;
+      const uint32_t bar = bar0 + 8 * st;
+      mbar_expect_tx(bar, cbytes + mbytes);
+      bulk_g2s(smem_u32(my.code[st]), sbase + (size_t)tile * kTileBytes + (size_t)grp * kGroupBytes, cbytes, bar);
+      bulk_g2s(smem_u32(my.meta[st]), mbase + ((size_t)tile * f.pf + (size_t)grp * 16) * 2, mbytes, bar);
+      left -= ng;
+      v_next += ng;
       return;
     }
     int ng = it_tgroups - it_grp;
@@ -585,7 +752,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   // be writing (a.safe: before the slots of the most recent append) is
   // fetched before waiting for the previous kernel.
   bool pre = false;
-  if constexpr (!kWide) {
+  if constexpr (!kWide && !CHAN) {
     if (lane == 0 && left > 0) {
       const int ng0 = min(min(it_tgroups - it_grp, kChunkGroups), left);
       if (wa + ng0 <= a.safe) {
@@ -607,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   // ---- fused single-token append: the warp whose range holds the new
   // token's group quantizes and writes the token (K, then V) before it
   // copies any group (a.safe kept the pre-wait copy away from that group) ----
-  if (a.app_group >= 0 && wa <= a.app_group && a.app_group < wb) {  // warp-uniform
+  if (!CHAN && a.app_group >= 0 && wa <= a.app_group && a.app_group < wb) {  // warp-uniform
     uint16_t* sc = reinterpret_cast<uint16_t*>(ws[warp].code[kStages - 1] + kAppScratch);
     const size_t tile = (size_t)s * f.nt + a.app_tile;
 #pragma unroll 1
@@ -658,7 +825,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   int* s_isum = reinterpret_cast<int*>(w_l);             // [8] sum of q_int
   reinterpret_cast<uint4*>(s_q)[threadIdx.x] = qv;  // heads >= G are zero
   __syncthreads();
-  {
+  if constexpr (CHAN) {  // q' in fp32 for the per-block operands
+    for (int idx = threadIdx.x; idx < kMaxGroup * kHeadDim; idx += kThreads)
+      s_qp[idx] = __bfloat162float(s_q[idx]) * a.qscale * s_lam[idx & (kHeadDim - 1)];
+  } else {
     // Warp w quantizes heads 2w and 2w+1: lane L takes head gq = 2w + L/16
     // and writes the B fragment of k-block sq = L%4 for MMA lane 4 gq + tq,
     // tq = (L/4)%4: channels 32 sq + 16 hf + 4 tq + i (hf = 0..1, i = 0..3).
@@ -699,15 +869,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     }
   }
   __syncthreads();
-  float ks0, ks1, sig0, sig1;  // heads 2t, 2t+1
-  {
+  float ks0 = 0.f, ks1 = 0.f, sig0 = 0.f, sig1 = 0.f;  // heads 2t, 2t+1 (per block with per-channel Keys)
+  if constexpr (!CHAN) {
     const float s0 = __uint_as_float(s_amax[2 * t]) / 32767.0f, s1 = __uint_as_float(s_amax[2 * t + 1]) / 32767.0f;
     ks0 = s0 * kKCode;
     ks1 = s1 * kKCode;
     sig0 = s0 * (float)s_isum[2 * t];
     sig1 = s1 * (float)s_isum[2 * t + 1];
   }
-  const uint4* qfl = qf + lane;
+  const uint4* qfl = CHAN ? qfw + warp * 4 * 32 + lane : qf + lane;
+  const uint2* qfl3 = qfw3 + warp * 4 * 32 + lane;  // per-channel Key groups only
+  int cur_blk = -1;  // per-channel Key groups: the block whose operand is in qfw
   __syncthreads();  // w_m / w_l are reused by the merge
   // The staging areas (second code stages) are refilled by bulk copies from
   // the first loop iteration on: order the generic accesses before them.
@@ -730,18 +902,39 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     if (!mbar_wait(bar0 + 8 * st, parity, a.err, flags)) break;
     const uint8_t* cs = my.code[st];
     const uint2* ms = reinterpret_cast<const uint2*>(my.meta[st]);
-    if (dsc.x == kChunkGroups && dsc.y >= 16 * kChunkGroups) {
+    if constexpr (CHAN) {  // every group full; dsc.y is the chunk's 128-token block
+      if (dsc.y != cur_blk) {
+        cur_blk = dsc.y;
+        float* wks = w_ks + warp * kMaxGroup;
+        float* wsig = w_sig + warp * kMaxGroup;
+        chan_block<BITS>(s_qp, a.kmc + ((size_t)s * a.blocks_max + (size_t)cur_blk) * kHeadDim,
+                         qfw + warp * 4 * 32, qfw3 + warp * 4 * 32, wks, wsig, lane);
+        ks0 = wks[2 * t];
+        ks1 = wks[2 * t + 1];
+        sig0 = wsig[2 * t];
+        sig1 = wsig[2 * t + 1];
+      }
+      int gi = 0;
+      if constexpr (kChunkGroups >= 2) {
+        for (; gi + 2 <= dsc.x; gi += 2)
+          process_groups<BITS, 2, true, true>(cs + gi * kGroupBytes, ms + gi * 16, 32, lane, qfl, qfl3, ks0, ks1, sig0,
+                                              sig1, sm);
+      }
+      if (gi < dsc.x)
+        process_groups<BITS, 1, true, true>(cs + gi * kGroupBytes, ms + gi * 16, 16, lane, qfl, qfl3, ks0, ks1, sig0,
+                                            sig1, sm);
+    } else if (dsc.x == kChunkGroups && dsc.y >= 16 * kChunkGroups) {
       // full chunk: fixed offsets, no masking
       // unrolled: one pair's P V and the next pair's QK share a basic block
       constexpr int kNG = kChunkGroups >= 2 ? 2 : 1;
 #pragma unroll
       for (int gi = 0; gi < kChunkGroups; gi += kNG)
-        process_groups<BITS, kNG, true>(cs + gi * kGroupBytes, ms + gi * 16, 16 * kNG, lane, qfl, ks0, ks1, sig0,
+        process_groups<BITS, kNG, true, false>(cs + gi * kGroupBytes, ms + gi * 16, 16 * kNG, lane, qfl, qfl3, ks0, ks1, sig0,
                                         sig1, sm);
     } else {
       for (int gi = 0; gi < dsc.x; gi++)
-        process_groups<BITS, 1, false>(cs + gi * kGroupBytes, ms + gi * 16, dsc.y - 16 * gi, lane, qfl, ks0, ks1,
-                                       sig0, sig1, sm);
+        process_groups<BITS, 1, false, false>(cs + gi * kGroupBytes, ms + gi * 16, dsc.y - 16 * gi, lane, qfl, qfl3, ks0,
+                                       ks1, sig0, sig1, sm);
     }
     __syncwarp();  // every lane is done with this stage before lane 0 refills it
   }
@@ -911,19 +1104,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   if (threadIdx.x == 0) a.counters[s] = 0;
 }
 
-template <int BITS>
+template <int BITS, bool CHAN>
 cudaError_t launch_bits(const DecodeArgs& a, cudaStream_t s) {
-  static bool attr_set = false;  // per process; set before the first launch
+  constexpr int kBytes = kSmemBytes + (CHAN ? kChanSmem : 0);
+  static bool attr_set = false;  // per process and kernel; set before the first launch
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, CHAN>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(decode_kernel<BITS>, cudaFuncAttributePreferredSharedMemoryCarveout,
+      e = cudaFuncSetAttribute(decode_kernel<BITS, CHAN>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const unsigned grid = (unsigned)(a.batch * a.kv_heads) * (unsigned)a.splits;
-  return launch_pdl(decode_kernel<BITS>, dim3(grid), dim3(kThreads), kSmemBytes, s, a);
+  return launch_pdl(decode_kernel<BITS, CHAN>, dim3(grid), dim3(kThreads), kBytes, s, a);
+}
+
+template <bool CHAN>
+cudaError_t launch_width(const DecodeArgs& a, cudaStream_t s) {
+  switch (a.fill.bits) {
+    case 2: return launch_bits<2, CHAN>(a, s);
+    case 4: return launch_bits<4, CHAN>(a, s);
+    case 8: return launch_bits<8, CHAN>(a, s);
+    case 16: return launch_bits<16, CHAN>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
@@ -963,13 +1168,9 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   if (a.group < 1 || a.group > kMaxGroup || a.splits < 1 || a.nparts > kMaxSplits || a.part_base < 0 ||
       a.part_base + a.splits > a.nparts)
     return cudaErrorInvalidValue;
-  switch (a.fill.bits) {
-    case 2: return launch_bits<2>(a, s);
-    case 4: return launch_bits<4>(a, s);
-    case 8: return launch_bits<8>(a, s);
-    case 16: return launch_bits<16>(a, s);
-    default: return cudaErrorInvalidValue;
-  }
+  if (a.chan && (!a.kmc || a.blocks_max < 1 || a.fill.gps % 8 != 0 || a.splits > a.fill.gps / 8))
+    return cudaErrorInvalidValue;
+  return a.chan ? launch_width<true>(a, s) : launch_width<false>(a, s);
 }
 
 }  // namespace kvq

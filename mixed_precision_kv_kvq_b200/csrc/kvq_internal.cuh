@@ -159,6 +159,7 @@ struct AppendArgs {
   const float* lam_inv;  // [kv_heads][128] or null
   // sink + window (the block keeps token 0 and the latest kWindowTokens at 16 bits)
   bool window;           // tokens enter the window; n0/bits/h/e/nt describe the progressive cache
+  bool stage;            // with window: per-channel Key staging -- token t takes slot t mod 128, nothing leaves
   bool direct;           // the block shrinks with the Direct Right Shift
   long long t0;          // token index (all tokens) of the first token of this launch
   uint8_t* wcodes;       // window codes: [batch][kv_heads][kWindowTiles][16 KiB]
@@ -173,7 +174,44 @@ struct ShrinkArgs {
   uint32_t* meta;     // layer base of the meta (used when direct)
   int pf;             // meta slots per tile
   int p_from;         // valid slots per tile before the shrink (the tile is full)
+  uint32_t* kmc;      // per-channel Key meta words rescaled too when direct, or null
+  long long kmc_words;
 };
+
+// Per-channel Key groups: a full staged block of 128 tokens enters the
+// progressive cache (one CTA per stream).
+constexpr int kKeyBlock = 128;
+struct BlockMoveArgs {
+  const uint8_t* wcodes;  // staging codes: [streams][kWindowTiles][16 KiB], token t of the block in slot t
+  const uint32_t* wmeta;  // staging meta:  [streams][kWindowTiles][32][2]
+  uint8_t* codes;         // progressive cache (layer base)
+  uint32_t* meta;
+  uint32_t* kmc;          // per-channel Key meta: [streams][blocks_max][128] words (R low, Z high)
+  int blocks_max, blk;    // blocks per stream; the block being moved
+  int nt, pf, bits;       // progressive cache: tiles per stream, meta slots per tile, current width
+  bool direct;            // the block shrinks with the Direct Right Shift
+  int g_tile[kKeyBlock / kGroupTokens], g_slot[kKeyBlock / kGroupTokens];  // where its 8 groups go
+};
+
+// Logical order of a block's progressive cache, epoch by epoch: tokens
+// [start_e, start_{e+1}) arrived at width 16 >> e and sit in slots
+// [h_e, h_e + ee_e) of tiles 0, 1, ... (ee_e per tile).
+struct Epochs {
+  int n;                  // epochs so far (shrinks + 1)
+  long long start[4];
+  int h[4], ee[4];
+};
+inline Epochs make_epochs(int nt, int n_shrinks) {
+  Epochs ep{};
+  ep.n = n_shrinks + 1;
+  for (int e = 0; e < ep.n && e < 4; e++) {
+    const int p = slots_per_tile(16 >> e);
+    ep.h[e] = e > 0 ? p / 2 : 0;
+    ep.ee[e] = p - ep.h[e];
+    ep.start[e] = (long long)nt * ep.h[e];
+  }
+  return ep;
+}
 
 struct DecodeArgs {
   uint8_t* codes;       // the block's (or window's) codes; written only by a fused append
@@ -202,6 +240,12 @@ struct DecodeArgs {
   const void* av;        // new Values
   int adtype;            // 0 bf16, 1 f32
   const float* lam_inv;  // [kv_heads][128] or null
+  // per-channel Key groups: groups are walked in logical order (ep) and
+  // each 128-token block's Key ranges and zeros come from kmc
+  bool chan;
+  const uint32_t* kmc;   // [streams][blocks_max][128]
+  int blocks_max;
+  Epochs ep;
 };
 
 // CTAs per stream for a launch over n_streams streams on num_sms SMs.
@@ -235,6 +279,7 @@ inline cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem,
 }
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
+cudaError_t launch_block_move(const BlockMoveArgs& a, int n_streams, cudaStream_t s);
 cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 

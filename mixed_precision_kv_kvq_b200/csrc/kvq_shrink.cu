@@ -118,7 +118,8 @@ __device__ __forceinline__ uint32_t drs_meta(uint32_t w) {
 }
 
 template <int BTO, class Op>
-__global__ void __launch_bounds__(kShrinkThreads) shrink_kernel(uint8_t* codes, uint32_t* meta, int pf, int p_from) {
+__global__ void __launch_bounds__(kShrinkThreads) shrink_kernel(uint8_t* codes, uint32_t* meta, int pf, int p_from,
+                                                               uint32_t* kmc, long long kmc_words) {
   // Tile = 1024 uint4 in, 512 uint4 out.  Thread i produces output uint4
   // u = i and u = i + 256 from input uint4 2u and 2u + 1.
   uint4* tile = reinterpret_cast<uint4*>(codes + (size_t)blockIdx.x * kTileBytes);
@@ -140,15 +141,19 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_kernel(uint8_t* codes, 
     // the tile's p_from slots (all valid: a shrink needs a full block), K and V words
     uint32_t* mt = meta + (size_t)blockIdx.x * pf * 2;
     for (int w = i; w < 2 * p_from; w += kShrinkThreads) mt[w] = drs_meta<BTO>(mt[w]);
+    // per-channel Key ranges (blocks with per-channel Key groups)
+    for (long long w = (long long)blockIdx.x * kShrinkThreads + i; w < kmc_words;
+         w += (long long)gridDim.x * kShrinkThreads)
+      kmc[w] = drs_meta<BTO>(kmc[w]);
   }
 }
 
 template <int BTO>
 cudaError_t launch_to(const ShrinkArgs& a, unsigned grid, cudaStream_t s) {
   if (a.direct)
-    shrink_kernel<BTO, Drs><<<grid, kShrinkThreads, 0, s>>>(a.codes, a.meta, a.pf, a.p_from);
+    shrink_kernel<BTO, Drs><<<grid, kShrinkThreads, 0, s>>>(a.codes, a.meta, a.pf, a.p_from, a.kmc, a.kmc_words);
   else
-    shrink_kernel<BTO, Ers><<<grid, kShrinkThreads, 0, s>>>(a.codes, a.meta, a.pf, a.p_from);
+    shrink_kernel<BTO, Ers><<<grid, kShrinkThreads, 0, s>>>(a.codes, a.meta, a.pf, a.p_from, nullptr, 0);
   return cudaGetLastError();
 }
 

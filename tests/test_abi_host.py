@@ -173,11 +173,11 @@ def test_window_option_host_side(kvq):
     per_block = 2 * 3 * (5 * 16384 + 5 * 32 * 8)
     assert plain < win <= plain + 2 * (per_block + 2 * 256)
     assert kvq.kvq_pool_bytes_ex(2, 2, 3, 128, budget, [2, 4], 0) == plain
-    assert kvq.kvq_pool_bytes_ex(2, 2, 3, 128, budget, [2, 4], 2) == 0
+    assert kvq.kvq_pool_bytes_ex(2, 2, 3, 128, budget, [2, 4], 4) == 0
     pool = HostPool(win)
     h = C.c_void_p()
     fb = (C.c_int * 2)(2, 4)
-    assert lib.kvq_alloc_ex(C.byref(h), 2, 2, 3, 128, budget, fb, pool.ptr, win, 2) == 1
+    assert lib.kvq_alloc_ex(C.byref(h), 2, 2, 3, 128, budget, fb, pool.ptr, win, 4) == 1
     assert lib.kvq_alloc_ex(C.byref(h), 2, 2, 3, 128, budget, fb, pool.ptr, plain, 1) == 1  # pool too small
     assert lib.kvq_alloc_ex(C.byref(h), 2, 2, 3, 128, budget, fb, pool.ptr, win, 1) == 0
     try:
@@ -193,3 +193,31 @@ def test_window_option_host_side(kvq):
         assert lib.kvq_export_window(h2, 0, 0, 0, None, None, None, None, C.byref(n), None) == 1  # no window
     finally:
         kvq.kvq_free(h2)
+
+
+def test_key_channel_option_host_side(kvq):
+    """Per-channel Key groups: N rounds down to a multiple of 1024, the pool
+    adds the staging (the window storage) and one (R, Z) word per Key channel
+    and 128-token block per stream; the option does not combine with the sink
+    + window; capacity and max tokens count the staged block (127 more)."""
+    lib = kvq.load()
+    budget = 4096 * _per_token(2, 3, [2, 4])
+    plain = kvq.kvq_pool_bytes(2, 2, 3, 128, budget, [2, 4])
+    win = kvq.kvq_pool_bytes_ex(2, 2, 3, 128, budget, [2, 4], kvq.KVQ_OPT_SINK_WINDOW)
+    ch = kvq.kvq_pool_bytes_ex(2, 2, 3, 128, budget, [2, 4], kvq.KVQ_OPT_KEY_CHANNEL)
+    kmc = 2 * 2 * 3 * 4096 * 4  # layers * streams * N words
+    assert ch == win + kmc or abs(ch - (win + kmc)) <= 2 * 256
+    assert kvq.kvq_pool_bytes_ex(2, 2, 3, 128, budget, [2, 4], 3) == 0
+    # 3584 tokens' budget: N = 3072 (a multiple of 1024), not 3584
+    b2 = 3584 * _per_token(2, 3, [2, 4])
+    pool = HostPool(kvq.kvq_pool_bytes_ex(2, 2, 3, 128, b2, [2, 4], kvq.KVQ_OPT_KEY_CHANNEL))
+    h = C.c_void_p()
+    fb = (C.c_int * 2)(2, 4)
+    assert lib.kvq_alloc_ex(C.byref(h), 2, 2, 3, 128, b2, fb, pool.ptr, pool.nbytes, kvq.KVQ_OPT_KEY_CHANNEL) == 0
+    try:
+        assert kvq.kvq_max_tokens(h) == 3072 + 127
+        assert kvq.kvq_query(h, 0) == {"tokens": 0, "bits": 16, "capacity": 3072 * 2 // 16 + 127, "n_shrinks": 0}
+        n = C.c_int()
+        assert lib.kvq_export_window(h, 0, 2, 0, None, None, None, None, C.byref(n), None) == 1  # stream
+    finally:
+        kvq.kvq_free(h)

@@ -330,6 +330,153 @@ def test_window_noalloc_matches_workspace_entry(kvq, orc):
     P.check_attention(q.cpu())
 
 
+# ------------------------------------------------ per-channel Key groups
+
+class CPair:
+    """A GPU cache with per-channel Key groups (KVQ_OPT_KEY_CHANNEL) and the
+    oracle's channel block, fed identically."""
+
+    def __init__(self, kvq, orc, batch, kv_heads, n_f, fbit, lam=None, shift_mode=0):
+        self.kvq = kvq
+        self.batch, self.kv_heads = batch, kv_heads
+        self.gpu = kvq.KVQCache(1, batch, kv_heads, n_f * per_token(batch, kv_heads, [fbit]), [fbit],
+                                key_channel=True)
+        assert self.gpu.max_tokens == n_f + 127
+        self.orc = orc.CLayer(batch, kv_heads, n_f, fbit)
+        self.lam = lam
+        if lam is not None:
+            self.gpu.set_lambda(0, lam)
+        if shift_mode:
+            self.gpu.set_shift_mode(0, shift_mode)
+            assert self.orc.set_shift_mode(shift_mode) == 0
+
+    def append(self, k, v):
+        self.gpu.append(0, k.cuda(), v.cuda())
+        assert self.orc.append(k.float().numpy(), v.float().numpy(), self.lam) == 0
+
+    def check_codes(self):
+        q = self.gpu.query(0)
+        m = self.orc.main
+        assert (q["tokens"], q["bits"], q["n_shrinks"]) == (self.orc.n, m.bits, m.n_shrinks), (q, m.shrink_at)
+        okc, ovc, ovm = m.k_codes(), m.v_codes(), m.v_meta()
+        okm = self.orc.k_meta_channel().reshape(self.batch, self.kv_heads, -1, 2)
+        skc, svc, skm, svm = self.orc.staged_codes()
+        for b in range(self.batch):
+            for j in range(self.kv_heads):
+                kc, vc, km, vm = self.gpu.export(0, b, j)
+                assert kc.shape[0] == m.n
+                for name, got, want in (("K", kc, okc[b, j]), ("V", vc, ovc[b, j]),
+                                        ("K channel meta", km, okm[b, j]), ("V meta", vm, ovm[b, j])):
+                    assert np.array_equal(got, want), (b, j, name, np.argwhere(got != want)[:4].tolist())
+                kc, vc, km, vm = self.gpu.export_window(0, b, j)
+                for name, got, want in (("staged K", kc, skc[b, j]), ("staged V", vc, svc[b, j]),
+                                        ("staged K meta", km, skm[b, j]), ("staged V meta", vm, svm[b, j])):
+                    assert np.array_equal(got, want), (b, j, name, np.argwhere(got != want)[:4].tolist())
+
+    def check_attention(self, q, sm_scale=1 / math.sqrt(128)):
+        out = self.gpu.decode_attn(0, q.cuda(), sm_scale).cpu().numpy().astype(np.float64)
+        torch.cuda.synchronize()
+        self.gpu.device_status()
+        ref = self.orc.attention(q.float().numpy(), self.lam, sm_scale)
+        err = np.abs(out - ref).max(axis=-1) / np.abs(ref).max(axis=-1)
+        assert np.isfinite(out).all()
+        assert err.max() <= TOL, f"max rel err {err.max():.3e} at {np.unravel_index(err.argmax(), err.shape)}"
+        return out
+
+
+def test_key_channel_tiny_one_by_one(kvq, orc):
+    """Token by token: the staged block alone, the first block entering the
+    progressive cache at 16 bits, and the cache shrinking as the 2nd, 3rd and
+    5th blocks arrive (N = 1024, Fbit 2), up to the last token that fits;
+    codes and meta bit-exact, attention within 2e-3."""
+    T = 1024 + 127
+    k, v = S.keys_values(11, 0, 1, T, 2, 0, 4, dtype=torch.float32)
+    lam = lam_for(k)
+    P = CPair(kvq, orc, 1, 2, 1024, 2, lam)
+    checkpoints = {1, 2, 127, 128, 129, 255, 256, 257, 384, 512, 513, 640, 1024, 1025, T}
+    for t in range(T):
+        P.append(k[:, t:t + 1], v[:, t:t + 1])
+        if t + 1 in checkpoints:
+            P.check_codes()
+            P.check_attention(S.queries(11, 0, t, 1, 4, t + 1, dtype=torch.bfloat16))
+    assert P.orc.main.shrink_at == [128, 256, 512]
+    with pytest.raises(kvq.KVQError) as e:  # the 9th block does not fit at Fbit
+        P.gpu.append(0, k[:, :1].cuda(), v[:, :1].cuda())
+    assert e.value.status == 2
+
+
+@pytest.mark.parametrize("fbit,mode", [(2, 0), (2, 1), (4, 0), (8, 1)])
+def test_key_channel_chunked_bf16(kvq, orc, fbit, mode):
+    """Chunks of 1 .. 700 tokens (launches are cut at block ends), batch 3,
+    4 KV heads, through every shrink of the block with either shift; then
+    the budget refuses a block that does not fit at Fbit."""
+    B, H, n_f = 3, 4, 2048
+    total = n_f + 127
+    k, v = S.keys_values(12, fbit, B, total, H, 0, 5, dtype=torch.bfloat16)
+    lam = lam_for(k)
+    P = CPair(kvq, orc, B, H, n_f, fbit, lam, shift_mode=mode)
+    pos = 0
+    for n in (1, 126, 1, 129, 300, 5, 700, total):
+        n = min(n, total - pos)
+        if n <= 0:
+            break
+        P.append(k[:, pos:pos + n], v[:, pos:pos + n])
+        pos += n
+        if pos in (1, 128, 257, 562):
+            P.check_codes()
+            P.check_attention(S.queries(12, fbit, pos, B, 4 * H, pos, dtype=torch.bfloat16))
+    assert pos == total and P.gpu.query(0)["bits"] == fbit
+    P.check_codes()
+    P.check_attention(S.queries(12, fbit, 0, B, 4 * H, total, dtype=torch.bfloat16))
+    with pytest.raises(kvq.KVQError) as e:
+        P.gpu.append(0, k[:, :1].cuda(), v[:, :1].cuda())
+    assert e.value.status == 2
+
+
+@pytest.mark.parametrize("G", [1, 5, 8])
+def test_key_channel_many_blocks_and_splits(kvq, orc, G):
+    """A longer block (N = 8192 at Fbit 2, every epoch present, several CTAs
+    per stream with warps on different blocks), GQA group sizes 1, 5, 8; the
+    no-workspace entry point gives the same output."""
+    B, H, n_f = 2, 2, 8192
+    T = n_f + 100
+    k, v = S.keys_values(13, G, B, T, H, 0, 3, dtype=torch.bfloat16)
+    P = CPair(kvq, orc, B, H, n_f, 2, lam_for(k))
+    for t0 in range(0, T, 4096):
+        P.append(k[:, t0:t0 + 4096], v[:, t0:t0 + 4096])
+    P.check_codes()
+    q = S.queries(13, G, 0, B, H * G, T, dtype=torch.bfloat16)
+    ref = P.check_attention(q)
+    out = torch.empty(B, H * G, 128, device="cuda")
+    kvq.kvq_decode_attn_noalloc(P.gpu.handle, 0, q.cuda(), 128 ** -0.5, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy().astype(np.float64), ref)
+
+
+def test_key_channel_append_decode_is_two_calls(kvq, orc):
+    """kvq_append_decode on a cache with per-channel Key groups runs the two
+    calls: same output and state as append then decode, across a block end."""
+    B, H, G, n_f = 2, 2, 4, 1024
+    t0, steps = 250, 10
+    k, v = S.keys_values(14, 0, B, t0 + steps, H, 0, 3, dtype=torch.bfloat16)
+    lam = lam_for(k)
+    P = CPair(kvq, orc, B, H, n_f, 4, lam)
+    F = kvq.KVQCache(1, B, H, n_f * per_token(B, H, [4]), [4], key_channel=True)
+    F.set_lambda(0, lam)
+    P.append(k[:, :t0], v[:, :t0])
+    F.append(0, k[:, :t0].cuda(), v[:, :t0].cuda())
+    for s_ in range(steps):
+        t = t0 + s_
+        q = S.queries(14, 0, s_, B, H * G, t + 1, dtype=torch.bfloat16)
+        P.append(k[:, t:t + 1], v[:, t:t + 1])
+        ref = P.check_attention(q)
+        out = F.append_decode(0, k[:, t:t + 1].cuda(), v[:, t:t + 1].cuda(), q.cuda())
+        torch.cuda.synchronize()
+        assert np.array_equal(out.cpu().numpy().astype(np.float64), ref)
+    assert F.query(0) == P.gpu.query(0)
+    F.free()
+
+
 # ------------------------------------------------ fused single-token append + decode
 
 @pytest.mark.parametrize("fbit,t0,steps", [(2, 509, 6), (2, 1021, 5), (4, 3000, 4), (16, 250, 4)])
