@@ -173,10 +173,11 @@ class ClockSampler:
 # ---------------------------------------------------------------- GPU arm
 
 def build_cache(kvq, dev, layers, batch, kv_heads, fbit, tokens, n_f, seed, n_out, chunk=4096, shift_mode=None,
-                sink_window=False):
+                sink_window=False, key_channel=False):
     budget = n_f * per_token_bytes(batch, kv_heads, fbit)
-    cache = kvq.KVQCache(layers, batch, kv_heads, budget, fbit, device=dev, sink_window=sink_window)
-    assert cache.max_tokens == n_f + (129 if sink_window else 0), (cache.max_tokens, n_f)
+    cache = kvq.KVQCache(layers, batch, kv_heads, budget, fbit, device=dev, sink_window=sink_window,
+                         key_channel=key_channel)
+    assert cache.max_tokens == n_f + (129 if sink_window else (127 if key_channel else 0)), (cache.max_tokens, n_f)
     if shift_mode is not None:
         for l in range(layers):
             cache.set_shift_mode(l, shift_mode)
@@ -296,11 +297,13 @@ def measure_decode_configs(kvq, dev, reps=20):
     cfgs = (("qwen7b", 16, 4, 28, 32768, 32768 + ROOM),
             ("qwen32b", 16, 8, 40, 32768, 55296),
             ("llama70b", 8, 8, 64, 131072, 131072))
-    runs = [(c, fbit, False) for c in cfgs for fbit in (2, 4)]
-    runs.append((("qwen7b_sink_window", 16, 4, 28, 32768 + 129, 32768), 2, True))
-    for (name, batch, kv_heads, q_heads, tokens, n_f), fbit, window in runs:
+    runs = [(c, fbit, "") for c in cfgs for fbit in (2, 4)]
+    runs.append((("qwen7b_sink_window", 16, 4, 28, 32768 + 129, 32768), 2, "window"))
+    runs += [(("qwen7b_key_channel", 16, 4, 28, 32768 + 100, 32768), fbit, "chan") for fbit in (2, 4)]
+    for (name, batch, kv_heads, q_heads, tokens, n_f), fbit, mode in runs:
+        window = mode == "window"
         cache = build_cache(kvq, dev, 1, batch, kv_heads, [fbit], tokens, n_f, SEED + 31, S.outliers_for(kv_heads),
-                            chunk=8192, sink_window=window)
+                            chunk=8192, sink_window=window, key_channel=mode == "chan")
         assert cache.query(0)["bits"] == fbit
         q = S.queries(SEED, 0, 0, batch, q_heads, tokens, dtype=torch.bfloat16, device=dev)
         out = torch.empty((batch, q_heads, HEAD_DIM), dtype=torch.float32, device=dev)
@@ -318,16 +321,58 @@ def measure_decode_configs(kvq, dev, reps=20):
         cache.device_status()
         us = e0.elapsed_time(e1) / reps * 1e3
         nb = decode_bytes(batch, kv_heads, q_heads, tokens, fbit)
-        if window:  # the sink and the window are read at 16 bits
-            nb = decode_bytes(batch, kv_heads, q_heads, tokens - 129, fbit) + \
-                decode_bytes(batch, kv_heads, q_heads, 129, 16) - batch * q_heads * HEAD_DIM * (2 + 4)
+        if window or mode == "chan":  # the sink and the window, or the staged tokens, are read at 16 bits
+            w = 129 if window else tokens % 128
+            nb = decode_bytes(batch, kv_heads, q_heads, tokens - w, fbit) + \
+                decode_bytes(batch, kv_heads, q_heads, w, 16) - batch * q_heads * HEAD_DIM * (2 + 4)
         res[f"{name}_{fbit}bit"] = {"us": round(us, 2), "gbs": round(nb / us / 1e3, 1), "bytes": nb,
                                     "batch": batch, "kv_heads": kv_heads, "q_heads": q_heads, "tokens": tokens}
         cache.free()
         del cache
     res["timing"] = (f"{reps} back-to-back calls on one block, CUDA events around the batch, mean per call "
-                     "(with the sink + window: two launches a call, the window at 16 bits and the rest)")
+                     "(with the sink + window or per-channel Key groups: two launches a call, the window or the "
+                     "staged block at 16 bits and the rest; per-channel Key groups count their (R, Z) per channel "
+                     "and 128-token block, the same bytes as per token)")
     return res
+
+
+def measure_block_append_key_channel(kvq, dev, reps=50):
+    """Per-channel Key groups: appends of 128 tokens that each complete a
+    block (staging at 16 bits, then the block move: Keys quantized per channel
+    over the block, Values shift-chained) on a 7B-shaped 2-bit block (batch
+    16, 4 KV heads) holding 16384 tokens; `reps` back-to-back calls, mean."""
+    import ctypes as C
+    lib = kvq.load()
+    stream = torch.cuda.current_stream(dev)
+    cache = build_cache(kvq, dev, 1, B7, HKV7, [2], 16384, 32768, SEED + 51, S.outliers_for(HKV7), chunk=8192,
+                        key_channel=True)
+    g = torch.Generator(device=dev)
+    g.manual_seed(SEED + 53)
+    kin = torch.randn((B7, 128, HKV7, HEAD_DIM), generator=g, device=dev).to(torch.bfloat16)
+    vin = torch.randn((B7, 128, HKV7, HEAD_DIM), generator=g, device=dev).to(torch.bfloat16)
+    sp = C.c_void_p(stream.cuda_stream)
+    args = (cache.handle, 0, C.c_void_p(kin.data_ptr()), C.c_void_p(vin.data_ptr()), kvq.KVQ_DTYPE_BF16, 128, sp)
+    for _ in range(3):
+        kvq.check(lib.kvq_append(*args))
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        lib.kvq_append(*args)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    cache.device_status()
+    us = e0.elapsed_time(e1) / reps * 1e3
+    st = cache.query(0)
+    assert st["tokens"] == 16384 + 128 * (reps + 3) and st["bits"] == 2
+    cache.free()
+    streams = B7 * HKV7
+    # bf16 in, INT16 staging written and read back, codes at 2 bits + meta out
+    nb = append_bytes(B7, HKV7, 128, 16) + streams * 128 * 2 * (2 * HEAD_DIM + 4) + append_bytes(B7, HKV7, 128, 2) \
+        - streams * 128 * 2 * HEAD_DIM * 2
+    return {"us": round(us, 2), "gbs": round(nb / us / 1e3, 1), "bytes": nb, "tokens": 128, "batch": B7,
+            "kv_heads": HKV7, "bits": 2, "timing": f"{reps} back-to-back 128-token appends (two launches each), "
+                                                   "CUDA events around the batch"}
 
 
 def measure_append_token(kvq, dev, reps=200, sink_window=False):
@@ -649,6 +694,7 @@ def run_gpu(args, rank, world):
         extra["append_token"] = measure_append_token(kvq, dev)
         extra["append_token_sink_window"] = measure_append_token(kvq, dev, sink_window=True)
         extra["decode_configs"] = measure_decode_configs(kvq, dev)
+        extra["block_append_key_channel"] = measure_block_append_key_channel(kvq, dev)
         extra["decode_graph"] = graph
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,

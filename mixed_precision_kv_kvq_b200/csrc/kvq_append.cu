@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs 
 template <int BITS>
 __global__ void __launch_bounds__(kKeyBlock) block_move_kernel(BlockMoveArgs a) {
   __shared__ uint16_t kc_sh[kKeyBlock][kHeadDim];  // [token][channel]: INT16 codes, then the new codes
-  __shared__ uint32_t km_sh[kKeyBlock];           // staged Key meta words
+  __shared__ float z_sh[kKeyBlock], step_sh[kKeyBlock];  // staged Keys: Z and R / 65535 of each token
   __shared__ uint16_t vc_sh[kKeyBlock / 32][kHeadDim];
   pdl_wait();
   pdl_launch_dependents();
@@ -172,17 +172,16 @@ __global__ void __launch_bounds__(kKeyBlock) block_move_kernel(BlockMoveArgs a) 
   };
   for (int t = warp; t < kKeyBlock; t += kKeyBlock / 32) {
     unpack_codes16(staged(t, 0), t & 15, 0, kc_sh[t], lane);
-    if (lane == 0) km_sh[t] = a.wmeta[staged_meta(t, 0)];
+    if (lane == 0) {
+      const uint32_t w = a.wmeta[staged_meta(t, 0)];
+      z_sh[t] = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+      step_sh[t] = __fdiv_rn(__half2float(__ushort_as_half((unsigned short)(w & 0xffffu))), 65535.0f);
+    }
   }
   __syncthreads();
   {
     const int c = threadIdx.x;  // one channel per thread
-    auto value = [&](int t) {
-      const uint32_t w = km_sh[t];
-      const float r = __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
-      const float z = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
-      return __fadd_rn(z, __fmul_rn((float)kc_sh[t][c], __fdiv_rn(r, 65535.0f)));
-    };
+    auto value = [&](int t) { return __fadd_rn(z_sh[t], __fmul_rn((float)kc_sh[t][c], step_sh[t])); };
     float mn = value(0), mx = mn;
     for (int t = 1; t < kKeyBlock; t++) {
       const float x = value(t);

@@ -57,6 +57,7 @@ constexpr int kSmemBytes = kWarps * kWarpSmem + kQfBytes + 3 * kWarps * kMaxGrou
 // and per warp the int16 B fragments, scales and zero terms of its block.
 constexpr int kChanSmem = kMaxGroup * kHeadDim * 4 + kWarps * kQfBytes + kWarps * kQfBytes / 2 + 2 * kWarps * kMaxGroup * 4;
 static_assert(kSmemBytes % 16 == 0, "the channel area starts 16-byte aligned");
+static_assert(kQfBytes >= kWarps * kHeadDim * 4, "per-warp block (R, Z) words fit the per-token fragment area");
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
 constexpr int kPartFloats = 2 * kMaxGroup + kHeadDim * kMaxGroup;  // one CTA's partial record
 // Scratch of the fused append in a warp's second code stage (unused until the
@@ -556,9 +557,10 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
 // ordinary channels too coarse (2.4e-3 output error on 2-bit blocks).  The
 // warp writes its own B fragments (hi and mid bytes in the per-token layout,
 // lo bytes in qfw3), and per head the score scale ks (w scale times the code
-// scale of the A operand) and the zero term.  km: the block's 128 (R, Z) words.
+// scale of the A operand) and the zero term.  km: the block's 128 (R, Z)
+// words, in shared memory.
 template <int BITS>
-__device__ __noinline__ void chan_block(const float* s_qp, const uint32_t* km, uint4* qfw, uint2* qfw3, float* wks,
+__device__ __forceinline__ void chan_block(const float* s_qp, const uint32_t* km, uint4* qfw, uint2* qfw3, float* wks,
                                         float* wsig, int lane) {
   constexpr float kInvQ = 1.0f / (float)((1u << BITS) - 1u);
   constexpr float kA = BITS >= 8 ? 1.0f : 1.0f / (float)(1 << (8 - BITS));  // A = c 2^(8 - BITS) at b <= 8
@@ -567,7 +569,7 @@ __device__ __noinline__ void chan_block(const float* s_qp, const uint32_t* km, u
   float R[2][4], Z[2][4];
 #pragma unroll
   for (int hf = 0; hf < 2; hf++) {
-    const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(km + 32 * sq + 16 * hf + 4 * tq));
+    const uint4 w4 = *reinterpret_cast<const uint4*>(km + 32 * sq + 16 * hf + 4 * tq);
     const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
     for (int i = 0; i < 4; i++) {
@@ -597,17 +599,21 @@ __device__ __noinline__ void chan_block(const float* s_qp, const uint32_t* km, u
       zs += __shfl_xor_sync(0xffffffffu, zs, o);
     }
     constexpr float kQMax = 8388607.0f;  // 2^23 - 1
-    const float inv = m > 0.f ? kQMax / m : 0.f;
-    uint32_t hb[2] = {0u, 0u}, mb[2] = {0u, 0u}, lb[2] = {0u, 0u};
+    // any inv close to kQMax / m works: the clamp keeps |qi| < 2^23 and the
+    // score scale below is the same m / kQMax the MMAs' integers are read with
+    // (qi / inv ~ w up to half a step, ks d = sum w c up to the rounding of inv)
+    const float inv = m > 0.f ? kQMax * __frcp_rn(m) : 0.f;
+    uint32_t hb[2], mb[2], lb[2];
 #pragma unroll
     for (int hf = 0; hf < 2; hf++) {
+      uint32_t q[4];
 #pragma unroll
-      for (int i = 0; i < 4; i++) {
-        const int qi = max(-8388607, min(8388607, __float2int_rn(v[hf][i] * inv)));
-        hb[hf] |= (uint32_t)((qi >> 16) & 0xff) << (8 * i);  // arithmetic shift: s8
-        mb[hf] |= (uint32_t)((qi >> 8) & 0xff) << (8 * i);
-        lb[hf] |= (uint32_t)(qi & 0xff) << (8 * i);
-      }
+      for (int i = 0; i < 4; i++) q[i] = (uint32_t)max(-8388607, min(8388607, __float2int_rn(v[hf][i] * inv)));
+      // bytes 0, 1, 2 of the four 24-bit two's-complement integers (byte 2 is the s8 high part)
+      const uint32_t ab = __byte_perm(q[0], q[1], 0x5140), cd = __byte_perm(q[2], q[3], 0x5140);
+      lb[hf] = __byte_perm(ab, cd, 0x5410);
+      mb[hf] = __byte_perm(ab, cd, 0x7632);
+      hb[hf] = __byte_perm(__byte_perm(q[0], q[1], 0x0062), __byte_perm(q[2], q[3], 0x0062), 0x5410);
     }
     qfw[sq * 32 + 4 * gq + tq] = make_uint4(hb[0], hb[1], mb[0], mb[1]);
     qfw3[sq * 32 + 4 * gq + tq] = make_uint2(lb[0], lb[1]);
@@ -665,6 +671,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   WarpSmem& my = ws[warp];
   const uint32_t bar0 = smem_u32(bars + warp * kStages);
   int2* mydesc = desc + warp * kStages;
+  // per-channel Key groups: this warp's copy of its block's (R, Z) words, in
+  // the per-token query fragments' area (unused then)
+  uint32_t* kmcb = reinterpret_cast<uint32_t*>(qf) + warp * kHeadDim;
 
   if (threadIdx.x == 0) {
     flags[0] = 0;
@@ -706,27 +715,49 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     }
     if constexpr (CHAN) {
       // logical order: group v holds tokens 16v .. 16v+15, which arrived in
-      // epoch e and sit in slots [h_e, h_e + ee_e) of tile (16v - start_e) / ee_e;
-      // a chunk stays inside one tile's run of the epoch (and so inside one
-      // 128-token block: runs and epoch starts are whole blocks or divide one)
-      const long long i = 16 * v_next;
-      int e = 0;
-      while (e + 1 < a.ep.n && i >= a.ep.start[e + 1]) e++;
-      const long long m = i - a.ep.start[e];
-      const int ee = a.ep.ee[e];
-      const int tile = (int)(m / ee), off = (int)(m - (long long)tile * ee);
-      const int grp = (a.ep.h[e] + off) >> 4;
-      int ng = (ee - off) >> 4;
-      ng = ng < kChunkGroups ? ng : kChunkGroups;
-      ng = ng < left ? ng : left;
-      mydesc[st] = make_int2(ng, (int)(v_next >> 3));  // groups, block
-      const uint32_t cbytes = (uint32_t)ng * kGroupBytes, mbytes = (uint32_t)ng * 128u;
+      // epoch e and sit in slots [h_e, h_e + ee_e) of tile (16v - start_e) / ee_e.
+      // A chunk gathers whole or partial runs (one tile's slots of an epoch,
+      // contiguous) up to kChunkGroups groups without leaving its 128-token
+      // block (runs never straddle blocks: epochs start on block boundaries
+      // and a run is 32, 64 or 128 tokens at a multiple of its length).  The
+      // first chunk of a block also fetches the block's Key (R, Z) words.
+      int rt[kChunkGroups], rg[kChunkGroups], rn[kChunkGroups];
+      int nr = 0, ng = 0;
+      const long long v0 = v_next;
+      while (ng < kChunkGroups && left > 0 && (ng == 0 || (v_next & 7) != 0)) {
+        const int i = 16 * (int)v_next;
+        int e = 0;
+        while (e + 1 < a.ep.n && i >= a.ep.start[e + 1]) e++;
+        const int m = i - a.ep.start[e], lg = a.ep.lg_ee[e];
+        const int tile = m >> lg, off = m & ((1 << lg) - 1);
+        int take = ((1 << lg) - off) >> 4;
+        take = take < kChunkGroups - ng ? take : kChunkGroups - ng;
+        take = take < left ? take : left;
+        const int to_end = 8 - (int)(v_next & 7);  // stay inside the block
+        take = take < to_end ? take : to_end;
+        rt[nr] = tile;
+        rg[nr] = (a.ep.h[e] + off) >> 4;
+        rn[nr] = take;
+        nr++;
+        ng += take;
+        left -= take;
+        v_next += take;
+      }
+      const int blk = (int)(v0 >> 3);
+      const bool first = (v0 & 7) == 0;
+      mydesc[st] = make_int2(ng, blk);  // groups, block
       const uint32_t bar = bar0 + 8 * st;
-      mbar_expect_tx(bar, cbytes + mbytes);
-      bulk_g2s(smem_u32(my.code[st]), sbase + (size_t)tile * kTileBytes + (size_t)grp * kGroupBytes, cbytes, bar);
-      bulk_g2s(smem_u32(my.meta[st]), mbase + ((size_t)tile * f.pf + (size_t)grp * 16) * 2, mbytes, bar);
-      left -= ng;
-      v_next += ng;
+      mbar_expect_tx(bar, (uint32_t)ng * (kGroupBytes + 128u) + (first ? 4u * kHeadDim : 0u));
+      int done = 0;
+      for (int r = 0; r < nr; r++) {
+        bulk_g2s(smem_u32(my.code[st] + done * kGroupBytes), sbase + (size_t)rt[r] * kTileBytes + (size_t)rg[r] * kGroupBytes,
+                 (uint32_t)rn[r] * kGroupBytes, bar);
+        bulk_g2s(smem_u32(my.meta[st] + done * 128), mbase + ((size_t)rt[r] * f.pf + (size_t)rg[r] * 16) * 2,
+                 (uint32_t)rn[r] * 128u, bar);
+        done += rn[r];
+      }
+      if (first)  // one buffer per warp: a block spans at least two chunks, so the previous block's words are used
+        bulk_g2s(smem_u32(kmcb), a.kmc + ((size_t)s * a.blocks_max + (size_t)blk) * kHeadDim, 4u * kHeadDim, bar);
       return;
     }
     int ng = it_tgroups - it_grp;
@@ -907,8 +938,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
         cur_blk = dsc.y;
         float* wks = w_ks + warp * kMaxGroup;
         float* wsig = w_sig + warp * kMaxGroup;
-        chan_block<BITS>(s_qp, a.kmc + ((size_t)s * a.blocks_max + (size_t)cur_blk) * kHeadDim,
-                         qfw + warp * 4 * 32, qfw3 + warp * 4 * 32, wks, wsig, lane);
+        chan_block<BITS>(s_qp, kmcb, qfw + warp * 4 * 32, qfw3 + warp * 4 * 32, wks, wsig, lane);
         ks0 = wks[2 * t];
         ks1 = wks[2 * t + 1];
         sig0 = wsig[2 * t];

@@ -198,8 +198,8 @@ struct BlockMoveArgs {
 // [h_e, h_e + ee_e) of tiles 0, 1, ... (ee_e per tile).
 struct Epochs {
   int n;                  // epochs so far (shrinks + 1)
-  long long start[4];
-  int h[4], ee[4];
+  int start[4];           // tokens per stream stay below 2^30
+  int h[4], lg_ee[4];     // ee_e = 1 << lg_ee[e] (32, 32, 64, 128 slots)
 };
 inline Epochs make_epochs(int nt, int n_shrinks) {
   Epochs ep{};
@@ -207,8 +207,10 @@ inline Epochs make_epochs(int nt, int n_shrinks) {
   for (int e = 0; e < ep.n && e < 4; e++) {
     const int p = slots_per_tile(16 >> e);
     ep.h[e] = e > 0 ? p / 2 : 0;
-    ep.ee[e] = p - ep.h[e];
-    ep.start[e] = (long long)nt * ep.h[e];
+    int lg = 0;
+    while ((1 << lg) < p - ep.h[e]) lg++;
+    ep.lg_ee[e] = lg;
+    ep.start[e] = nt * ep.h[e];
   }
   return ep;
 }

@@ -56,15 +56,16 @@ class Sampled:
     """A full-size GPU block plus oracle replays of a few of its streams."""
 
     def __init__(self, kvq, orc, batch, kv_heads, n_f, fbit, streams, layer, seed=SEED, shift_mode=0,
-                 window=False):
+                 window=False, chan=False):
         self.kvq, self.orc_mod = kvq, orc
         self.batch, self.kv_heads, self.n_f, self.fbit = batch, kv_heads, n_f, fbit
         self.streams, self.layer, self.seed = streams, layer, seed
-        self.window = window
+        self.window, self.chan = window, chan
         self.gpu = kvq.KVQCache(1, batch, kv_heads, n_f * per_token(batch, kv_heads, fbit), [fbit],
-                                sink_window=window)
-        assert self.gpu.max_tokens == n_f + (129 if window else 0)
-        self.orc = {s: (orc.WLayer if window else orc.Layer)(1, 1, n_f, fbit) for s in streams}
+                                sink_window=window, key_channel=chan)
+        assert self.gpu.max_tokens == n_f + (129 if window else (127 if chan else 0))
+        cls = orc.WLayer if window else (orc.CLayer if chan else orc.Layer)
+        self.orc = {s: cls(1, 1, n_f, fbit) for s in streams}
         self.lam = None
         self.pos = 0
         self.n_out = S.outliers_for(kv_heads)
@@ -113,19 +114,21 @@ class Sampled:
     def check_state(self):
         st = self.gpu.query(0)
         for o in self.orc.values():
-            m = o.main if self.window else o
+            m = o.main if self.window or self.chan else o
             assert (st["tokens"], st["bits"], st["n_shrinks"]) == (o.n, m.bits, m.n_shrinks), (st, m.shrink_at)
         return st
 
     def check_codes(self):
         for (b, j), w in self.orc.items():
-            o = w.main if self.window else w
-            if self.window:
+            o = w.main if self.window or self.chan else w
+            if self.window or self.chan:
                 got = self.gpu.export_window(0, b, j)
-                for name, x, y in zip(("wK", "wV", "wKm", "wVm"), got, w.window_codes()):
+                want = w.window_codes() if self.window else w.staged_codes()
+                for name, x, y in zip(("wK", "wV", "wKm", "wVm"), got, want):
                     assert np.array_equal(x, y[0, 0]), (b, j, name)
             kc, vc, km, vm = self.gpu.export(0, b, j)
-            assert np.array_equal(km, o.k_meta()[0, 0]), (b, j, "K meta")
+            want_km = w.k_meta_channel()[0, 0].reshape(-1, 2) if self.chan else o.k_meta()[0, 0]
+            assert np.array_equal(km, want_km), (b, j, "K meta")
             assert np.array_equal(vm, o.v_meta()[0, 0]), (b, j, "V meta")
             for name, got, want in (("K", kc, o.k_codes()[0, 0]), ("V", vc, o.v_codes()[0, 0])):
                 if not np.array_equal(got, want):
@@ -252,6 +255,22 @@ def test_7b_decode_sink_window_fullsize(kvq, orc):
     assert st["bits"] == 2 and st["tokens"] == T
     x.check_codes()
     x.check_attention(HQ)
+    x.free()
+
+
+@pytest.mark.parametrize("fbit,layer", [(2, 5), (4, 0)])
+def test_7b_decode_key_channel_fullsize(kvq, orc, fbit, layer):
+    """The 7B block with per-channel Key groups: 32768 + 100 tokens (the last
+    100 staged at INT16), built from empty through the shrinks, sampled
+    streams bit-exact and within 2e-3."""
+    B, H, HQ, T = 16, 4, 28, 32768 + 100
+    x = Sampled(kvq, orc, B, H, 32768, fbit, corners(B, H), layer, chan=True)
+    x.fill(T, chunk=4096)
+    st = x.check_state()
+    assert st["bits"] == fbit and st["tokens"] == T
+    x.check_codes()
+    x.check_attention(HQ)
+    x.check_attention(HQ, step=1)
     x.free()
 
 
