@@ -149,15 +149,19 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs 
 // Per-channel Key groups (KIVI's axis): the staged block of 128 tokens of
 // one stream enters the progressive cache at width BITS.  Keys: every staged
 // INT16 Key is read back in fp32 as Z + code * (R / 65535) and each channel's
-// 128 values go through the quantizer of kvq_quant.cuh (thread c owns
-// channel c); Values: each token's INT16 codes take the block's shift chain,
-// R and Z kept (R rescaled by the direct shift).  128 threads, one CTA per
-// stream.
+// 128 values go through the quantizer of kvq_quant.cuh; Values: each token's
+// INT16 codes take the block's shift chain, R and Z kept (R rescaled by the
+// direct shift).  One CTA of 512 threads per stream: warps unpack and pack 8
+// tokens each; for the channels, thread (quarter, c) covers tokens
+// 32 quarter .. +31 of channel c and the quarters combine their min / max.
+constexpr int kMoveThreads = 512;
+constexpr int kMoveWarps = kMoveThreads / 32;
 template <int BITS>
-__global__ void __launch_bounds__(kKeyBlock) block_move_kernel(BlockMoveArgs a) {
+__global__ void __launch_bounds__(kMoveThreads) block_move_kernel(BlockMoveArgs a) {
   __shared__ uint16_t kc_sh[kKeyBlock][kHeadDim];  // [token][channel]: INT16 codes, then the new codes
   __shared__ float z_sh[kKeyBlock], step_sh[kKeyBlock];  // staged Keys: Z and R / 65535 of each token
-  __shared__ uint16_t vc_sh[kKeyBlock / 32][kHeadDim];
+  __shared__ float mn_sh[4][kHeadDim], mx_sh[4][kHeadDim];
+  __shared__ uint16_t vc_sh[kMoveWarps][kHeadDim];
   pdl_wait();
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -170,7 +174,7 @@ __global__ void __launch_bounds__(kKeyBlock) block_move_kernel(BlockMoveArgs a) 
   auto staged_meta = [&](int t, int kv) {
     return ((stream * kWindowTiles + t / P16) * (size_t)P16 + t % P16) * 2 + kv;
   };
-  for (int t = warp; t < kKeyBlock; t += kKeyBlock / 32) {
+  for (int t = warp; t < kKeyBlock; t += kMoveWarps) {
     unpack_codes16(staged(t, 0), t & 15, 0, kc_sh[t], lane);
     if (lane == 0) {
       const uint32_t w = a.wmeta[staged_meta(t, 0)];
@@ -180,34 +184,41 @@ __global__ void __launch_bounds__(kKeyBlock) block_move_kernel(BlockMoveArgs a) 
   }
   __syncthreads();
   {
-    const int c = threadIdx.x;  // one channel per thread
+    const int c = threadIdx.x & (kHeadDim - 1), qt = threadIdx.x >> 7;  // channel, token quarter
+    const int t0 = 32 * qt;
     auto value = [&](int t) { return __fadd_rn(z_sh[t], __fmul_rn((float)kc_sh[t][c], step_sh[t])); };
-    float mn = value(0), mx = mn;
-    for (int t = 1; t < kKeyBlock; t++) {
+    float mn = value(t0), mx = mn;
+    for (int t = t0 + 1; t < t0 + 32; t++) {
       const float x = value(t);
       mn = fminf(mn, x);
       mx = fmaxf(mx, x);
     }
+    mn_sh[qt][c] = mn;
+    mx_sh[qt][c] = mx;
+    __syncthreads();
+    mn = fminf(fminf(mn_sh[0][c], mn_sh[1][c]), fminf(mn_sh[2][c], mn_sh[3][c]));
+    mx = fmaxf(fmaxf(mx_sh[0][c], mx_sh[1][c]), fmaxf(mx_sh[2][c], mx_sh[3][c]));
     const __half zh = __float2half_rd(mn);
     const float z = __half2float(zh);
     const __half rh = __float2half_ru(__fsub_rn(mx, z));
     const float r = __half2float(rh);
     constexpr unsigned qmax = BITS == 16 ? 65535u : (1u << BITS) - 1u;
     const float inv = r == 0.0f ? 0.0f : __fdiv_rn((float)qmax, r);
-    for (int t = 0; t < kKeyBlock; t++) {
+    for (int t = t0; t < t0 + 32; t++) {
       uint16_t q = 0;
       if (r != 0.0f) {
         const float y = __fadd_rn(__fmul_rn(__fsub_rn(value(t), z), inv), 0.5f);
         q = (uint16_t)min(__float2uint_rd(y), qmax);
       }
-      kc_sh[t][c] = q;  // only this thread reads or writes column c
+      kc_sh[t][c] = q;  // only this thread reads or writes this token's channel c
     }
-    a.kmc[(stream * a.blocks_max + a.blk) * kHeadDim + c] =
-        (uint32_t)__half_as_ushort(rh) | ((uint32_t)__half_as_ushort(zh) << 16);
+    if (qt == 0)
+      a.kmc[(stream * a.blocks_max + a.blk) * kHeadDim + c] =
+          (uint32_t)__half_as_ushort(rh) | ((uint32_t)__half_as_ushort(zh) << 16);
   }
   __syncthreads();
   uint16_t* sc = vc_sh[warp];
-  for (int t = warp; t < kKeyBlock; t += kKeyBlock / 32) {
+  for (int t = warp; t < kKeyBlock; t += kMoveWarps) {
     const int gi = t >> 4, slot = a.g_slot[gi] + (t & 15);
     const size_t tile = stream * a.nt + a.g_tile[gi];
     uint8_t* gbase = a.codes + tile * kTileBytes + (size_t)(slot >> 4) * group_bytes(BITS);
@@ -231,7 +242,7 @@ __global__ void __launch_bounds__(kKeyBlock) block_move_kernel(BlockMoveArgs a) 
 
 cudaError_t launch_block_move(const BlockMoveArgs& a, int n_streams, cudaStream_t s) {
   if (n_streams <= 0) return cudaSuccess;
-  const dim3 grid((unsigned)n_streams), block(kKeyBlock);
+  const dim3 grid((unsigned)n_streams), block(kMoveThreads);
   switch (a.bits) {
     case 16: return launch_pdl(block_move_kernel<16>, grid, block, 0, s, a);
     case 8: return launch_pdl(block_move_kernel<8>, grid, block, 0, s, a);
