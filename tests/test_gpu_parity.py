@@ -453,6 +453,29 @@ def test_key_channel_many_blocks_and_splits(kvq, orc, G):
     assert np.array_equal(out.cpu().numpy().astype(np.float64), ref)
 
 
+@pytest.mark.parametrize("mode", [0, 1])
+def test_key_channel_explicit_shrink(kvq, orc, mode):
+    """kvq_shrink on a full progressive cache with per-channel Key groups (the
+    step the next block would take; the direct shift also rescales the
+    per-channel ranges): after the next block the cache equals the oracle's,
+    which shrinks when that block arrives; a shrink of a cache that is not
+    full, or at Fbit, is refused."""
+    B, H = 2, 2
+    k, v = S.keys_values(15, mode, B, 400, H, 0, 3, dtype=torch.bfloat16)
+    P = CPair(kvq, orc, B, H, 1024, 2, lam_for(k), shift_mode=mode)  # 128 tokens at 16 bits
+    P.append(k[:, :100], v[:, :100])
+    with pytest.raises(kvq.KVQError) as e:  # the progressive cache is empty, not full
+        P.gpu.shrink(0)
+    assert e.value.status == 3
+    P.append(k[:, 100:200], v[:, 100:200])  # block 0 in the cache: full at 16 bits
+    P.gpu.shrink(0)
+    assert P.gpu.query(0)["bits"] == 8 and P.orc.main.bits == 16
+    P.append(k[:, 200:300], v[:, 200:300])  # block 1 completes at 256: no second shrink on the GPU
+    assert P.gpu.query(0)["n_shrinks"] == 1 and P.orc.main.n_shrinks == 1
+    P.check_codes()
+    P.check_attention(S.queries(15, mode, 0, B, 4 * H, 300, dtype=torch.bfloat16))
+
+
 def test_key_channel_append_decode_is_two_calls(kvq, orc):
     """kvq_append_decode on a cache with per-channel Key groups runs the two
     calls: same output and state as append then decode, across a block end."""
