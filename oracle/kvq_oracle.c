@@ -21,7 +21,7 @@
  * And the ChanMix note on the same site, key design 1: an asymmetric
  * quantizer has scale S = (Cmax - Cmin) / (2^b - 1) and worst-case error S/2.
  *
- * Readings where the pages are silent (each one is restated in the design doc):
+ * Readings where the pages are silent:
  *   - One group = one token's 128 channels of one KV head (K and V alike).
  *   - Dequantisation is  x^ = Z + S * q  with Z a real-valued zero (the group
  *     minimum rounded down to binary16), which is what keeps Z_b = Z_{2b}
