@@ -500,6 +500,28 @@ def test_key_channel_append_decode_is_two_calls(kvq, orc):
     F.free()
 
 
+# ------------------------------------------------ one stream: the most CTAs per stream
+
+@pytest.mark.parametrize("mode", ["plain", "window", "chan"])
+def test_single_stream_most_splits(kvq, orc, mode):
+    """Batch 1 and one KV head: a long block is cut into the largest number
+    of CTAs per stream (64 partials, or 61 plus the window's or staged
+    block's 3), and the merge over all of them matches the oracle."""
+    B, H, G, n_f, fbit = 1, 1, 8, 65536, 4  # 4096 groups at 4 bits: the split model wants more than 64
+    T = n_f + (100 if mode == "chan" else (129 if mode == "window" else 0))
+    k, v = S.keys_values(16, 1, B, T, H, 0, 2, dtype=torch.bfloat16)
+    lam = lam_for(k)
+    if mode == "window":
+        P = WPair(kvq, orc, B, H, n_f, fbit, lam)
+    elif mode == "chan":
+        P = CPair(kvq, orc, B, H, n_f, fbit, lam)
+    else:
+        P = Pair(kvq, orc, B, H, n_f, fbit, lam)
+    for t0 in range(0, T, 8192):
+        P.append(k[:, t0:t0 + 8192], v[:, t0:t0 + 8192])
+    P.check_attention(S.queries(16, 1, 0, B, H * G, T, dtype=torch.bfloat16))
+
+
 # ------------------------------------------------ fused single-token append + decode
 
 @pytest.mark.parametrize("fbit,t0,steps", [(2, 509, 6), (2, 1021, 5), (4, 3000, 4), (16, 250, 4)])
