@@ -10,6 +10,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <algorithm>
+
 #include "kvq_quant.cuh"
 
 namespace kvq {
@@ -146,6 +148,135 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs 
   }
 }
 
+// Group mode (chunked appends at b <= 8 bits): one warp quantizes the 16
+// tokens of one slot group (one KV head, K or V) with the same quantizer,
+// keeps their codes in shared memory as bytes, token-major, and then writes
+// the group part lane unit by lane unit: lane L builds unit L's 2b words
+// from byte quads (Keys) or token pairs (Values) and stores them with 16-byte
+// stores -- instead of every token scattering its codes with shuffles and
+// 4- or 2-byte stores.  The group's 16 tokens are consecutive in the call
+// and fill the group (the host cuts a chunk at 16-token boundaries).
+constexpr int kGroupWarps = 4;
+constexpr int kRowBytes = 144;  // 128 codes + pad: quad reads of lanes (g, t) hit 32 distinct banks
+template <int BITS>
+__global__ void __launch_bounds__(kGroupWarps * 32) append_group_kernel(AppendArgs a) {
+  static_assert(BITS <= 8, "16-bit codes take the per-token path");
+  __shared__ __align__(16) uint8_t cs[kGroupWarps][kGroupTokens][kRowBytes];
+  __shared__ uint32_t ms[kGroupWarps][kGroupTokens];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const unsigned ngroups = (unsigned)a.cnt / kGroupTokens;
+  const unsigned w = blockIdx.x * kGroupWarps + wib;
+  if (w >= ngroups * (unsigned)a.kv_heads * 2u) return;  // warp-uniform
+  const int b = blockIdx.y;
+  const int kv = (int)(w & 1u);
+  const unsigned rest = w >> 1;
+  const int gi = (int)(rest / (unsigned)a.kv_heads);
+  const int j = (int)(rest - (unsigned)gi * (unsigned)a.kv_heads);
+  const size_t stream = (size_t)b * a.kv_heads + j;
+  const int tk0 = gi * kGroupTokens;  // first token of the group within this launch
+  constexpr unsigned qmax = (1u << BITS) - 1u;
+
+  // ---- quantize the 16 tokens (8 at a time: their loads are issued together) ----
+  const void* src = kv ? a.v : a.k;
+  float4 li = make_float4(1.f, 1.f, 1.f, 1.f);
+  const bool mig = kv == 0 && a.lam_inv;
+  if (mig) li = *reinterpret_cast<const float4*>(a.lam_inv + (size_t)j * kHeadDim + 4 * lane);
+#pragma unroll 1
+  for (int half = 0; half < 2; half++) {
+    float4 xv[8];
+#pragma unroll
+    for (int tt = 0; tt < 8; tt++) {
+      const size_t in_off =
+          (((size_t)b * a.n_call + (size_t)(a.tok_off + tk0 + 8 * half + tt)) * a.kv_heads + j) * kHeadDim + 4 * lane;
+      if (a.dtype == 1) {
+        xv[tt] = *reinterpret_cast<const float4*>(static_cast<const float*>(src) + in_off);
+      } else {
+        const uint2 raw = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(src) + in_off);
+        xv[tt] = make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u),
+                             __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xffff0000u));
+      }
+    }
+#pragma unroll
+    for (int tt = 0; tt < 8; tt++) {
+      float x[4] = {xv[tt].x, xv[tt].y, xv[tt].z, xv[tt].w};
+      if (mig) {
+        x[0] = __fmul_rn(x[0], li.x); x[1] = __fmul_rn(x[1], li.y);
+        x[2] = __fmul_rn(x[2], li.z); x[3] = __fmul_rn(x[3], li.w);
+      }
+      // the quantizer of kvq_quant.cuh, codes kept in registers
+      float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
+      float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+      mn = warp_min(mn);
+      mx = warp_max(mx);
+      const __half zh = __float2half_rd(mn);
+      const float z = __half2float(zh);
+      const __half rh = __float2half_ru(__fsub_rn(mx, z));
+      const float r = __half2float(rh);
+      uint32_t quad = 0;
+      if (r != 0.0f) {
+        const float inv = __fdiv_rn((float)qmax, r);
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+          const float y = __fadd_rn(__fmul_rn(__fsub_rn(x[i], z), inv), 0.5f);
+          quad |= min(__float2uint_rd(y), qmax) << (8 * i);
+        }
+      }
+      const int tok = 8 * half + tt;
+      *reinterpret_cast<uint32_t*>(&cs[wib][tok][4 * lane]) = quad;  // channels 4 lane .. 4 lane + 3, one per byte
+      if (lane == 0) ms[wib][tok] = (uint32_t)__half_as_ushort(rh) | ((uint32_t)__half_as_ushort(zh) << 16);
+    }
+  }
+  __syncwarp();
+
+  // ---- the group part, lane unit L = 4g + t ----
+  const unsigned m = (unsigned)(a.n0 + tk0 - (long long)a.nt * a.h);  // the group's first token, this epoch
+  const int tile = (int)(m / (unsigned)a.e);
+  const int slot0 = a.h + (int)(m - (unsigned)tile * (unsigned)a.e);  // a multiple of 16
+  const size_t tl = stream * a.nt + tile;
+  uint8_t* gbase = a.codes + tl * kTileBytes + (size_t)(slot0 >> 4) * group_bytes(BITS) + (size_t)kv * part_bytes(BITS);
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t wd[2 * BITS];
+  if (kv == 0) {
+    // word x b + jw holds quads p = jw (8/b) + k (field k) of token g + 8x:
+    // channels 32 (p/2) + 16 (p%2) + 4t + i, member i in byte i
+#pragma unroll
+    for (int x = 0; x < 2; x++)
+#pragma unroll
+      for (int jw = 0; jw < BITS; jw++) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int k = 0; k < 8 / BITS; k++) {
+          const int p = jw * (8 / BITS) + k;
+          word |= *reinterpret_cast<const uint32_t*>(&cs[wib][g + 8 * x][32 * (p >> 1) + 16 * (p & 1) + 4 * t])
+                  << (BITS * k);
+        }
+        wd[x * BITS + jw] = word;
+      }
+  } else {
+    // word u b + jw holds pairs p = jw (16/b) + k (field k): channel
+    // 16 (p/2) + g + 8 (p%2) of tokens 2t + 8u (low half) and 2t + 8u + 1 (high half)
+#pragma unroll
+    for (int u = 0; u < 2; u++)
+#pragma unroll
+      for (int jw = 0; jw < BITS; jw++) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int k = 0; k < 16 / BITS; k++) {
+          const int p = jw * (16 / BITS) + k;
+          const int ch = 16 * (p >> 1) + g + 8 * (p & 1);
+          word |= ((uint32_t)cs[wib][2 * t + 8 * u][ch] | ((uint32_t)cs[wib][2 * t + 8 * u + 1][ch] << 16)) << (BITS * k);
+        }
+        wd[u * BITS + jw] = word;
+      }
+  }
+  uint4* dst = reinterpret_cast<uint4*>(gbase + (size_t)lane * unit_bytes(BITS));
+#pragma unroll
+  for (int i = 0; i < BITS / 2; i++) dst[i] = make_uint4(wd[4 * i], wd[4 * i + 1], wd[4 * i + 2], wd[4 * i + 3]);
+  if (lane < kGroupTokens) a.meta[(tl * a.pf + slot0 + lane) * 2 + kv] = ms[wib][lane];
+}
+
 // Per-channel Key groups (KIVI's axis): the staged block of 128 tokens of
 // one stream enters the progressive cache at width BITS.  Keys: every staged
 // INT16 Key is read back in fp32 as Z + code * (R / 65535) and each channel's
@@ -253,6 +384,40 @@ cudaError_t launch_block_move(const BlockMoveArgs& a, int n_streams, cudaStream_
 }
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
+  // A chunk of a per-token cache at b <= 8 bits: its whole 16-token groups
+  // go through the group mode, the tokens before the first and after the
+  // last whole group through the per-token path (three launches at most,
+  // disjoint slots).
+  if (!a.window && a.bits <= 8 && a.cnt >= kGroupTokens) {
+    const int head = std::min(a.cnt, (int)((kGroupTokens - a.n0 % kGroupTokens) % kGroupTokens));
+    const int body = (a.cnt - head) / kGroupTokens * kGroupTokens;
+    if (body > 0) {
+      AppendArgs p = a;
+      p.cnt = head;
+      if (head > 0)
+        if (cudaError_t e = launch_append(p, s)) return e;
+      p = a;
+      p.tok_off = a.tok_off + head;
+      p.n0 = a.n0 + head;
+      p.cnt = body;
+      const long long gw = (long long)(body / kGroupTokens) * a.kv_heads * 2;  // warps per sequence
+      if (gw >= (1ll << 31) || a.batch > 65535) return cudaErrorInvalidValue;
+      const dim3 grid((unsigned)((gw + kGroupWarps - 1) / kGroupWarps), (unsigned)a.batch), block(kGroupWarps * 32);
+      cudaError_t e = cudaSuccess;
+      switch (a.bits) {
+        case 8: e = launch_pdl(append_group_kernel<8>, grid, block, 0, s, p); break;
+        case 4: e = launch_pdl(append_group_kernel<4>, grid, block, 0, s, p); break;
+        case 2: e = launch_pdl(append_group_kernel<2>, grid, block, 0, s, p); break;
+        default: return cudaErrorInvalidValue;
+      }
+      if (e != cudaSuccess) return e;
+      p = a;
+      p.tok_off = a.tok_off + head + body;
+      p.n0 = a.n0 + head + body;
+      p.cnt = a.cnt - head - body;
+      return p.cnt > 0 ? launch_append(p, s) : cudaSuccess;
+    }
+  }
   const long long warps = ((long long)a.cnt + kTokensPerWarp - 1) / kTokensPerWarp * a.kv_heads * 2;  // per sequence
   if (warps <= 0 || a.batch <= 0) return cudaSuccess;
   if (warps >= (1ll << 31) || a.batch > 65535) return cudaErrorInvalidValue;
