@@ -520,7 +520,6 @@ def run_gpu(args, rank, world):
     # ---- per-launch decode durations: the same step again, K more times,
     # with CUDA events on the launch stream around every decode launch ----
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(layers)] for _ in range(K)]
-    t1_tokens = cache.query(0)["tokens"]
     torch.cuda.synchronize(dev)
     r_start, r_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     r_start.record(stream)
@@ -531,9 +530,7 @@ def run_gpu(args, rank, world):
     cache.device_status()
     dec_ms = sum(evs[i][l][0].elapsed_time(evs[i][l][1]) for i in range(K) for l in range(layers))
     dec_ms_bits = {}
-    dec_bytes = 0
     for i in range(K):
-        dec_bytes += bytes_of_step(t1_tokens + i)[0]  # the fused launch: attention + the new token
         for l in range(layers):
             dec_ms_bits.setdefault(fbit[l], []).append(evs[i][l][0].elapsed_time(evs[i][l][1]))
     ev_step_ms = r_start.elapsed_time(r_end) / K
@@ -668,19 +665,31 @@ def run_gpu(args, rank, world):
                    "d2h_bytes_per_step": layers * out[0].numel() * 4, "steps": E}
 
     # ---- roofline of the decode kernel ----
+    # Every launch of the timed region is this kernel (kvq_append_decode: one
+    # launch per block, no shrink in the timed steps), so its average launch
+    # duration over the timed region is the region's time over its launches.
+    # The event pass above brackets each launch instead; its events break the
+    # dependent-launch overlap of consecutive launches, so it is reported as a
+    # breakdown by width, not as the kernel's duration.
     peak, peak_kind = peaks()
-    achieved = dec_bytes / (dec_ms / 1e3) / 1e9
     n_dec = K * layers
+    avg_ms = total_ms / n_dec
+    bytes_per_launch = tot_bytes / n_dec
+    achieved = bytes_per_launch / (avg_ms / 1e3) / 1e9
     traffic, traffic_src = decode_traffic(fbit)
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs (copy)",
             "traffic": traffic, "traffic_source": traffic_src,
             "kernel": "decode_kernel (kvq_append_decode: the step's new token and the attention)",
-            "avg_launch_us": round(dec_ms * 1e3 / n_dec, 2),
-            "bytes_per_launch": int(dec_bytes / n_dec),
-            "per_bits_us": {f"{b}bit": round(statistics.mean(v) * 1e3, 2) for b, v in sorted(dec_ms_bits.items())},
-            "timing": f"CUDA events around each of {n_dec} decode launches ({K} more steps after the timed "
-                      f"ones; {ev_step_ms:.4f} ms/step with the events)"}
+            "avg_launch_us": round(avg_ms * 1e3, 2),
+            "bytes_per_launch": int(bytes_per_launch),
+            "timing": f"CUDA events around the timed region, whose {n_dec} launches are all this kernel "
+                      "(slowest rank): region time / launches",
+            "per_launch_events": {
+                "avg_launch_us": round(dec_ms * 1e3 / n_dec, 2),
+                "per_bits_us": {f"{b}bit": round(statistics.mean(v) * 1e3, 2) for b, v in sorted(dec_ms_bits.items())},
+                "what": f"CUDA events around each of {n_dec} launches in {K} more steps ({ev_step_ms:.4f} ms/step "
+                        "with the events, which serialise the launches)"}}
 
     extra = {}
     if not args.no_shrink and rank == 0:
