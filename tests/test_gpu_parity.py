@@ -135,6 +135,29 @@ def test_chunked_append_bit_exact(kvq, orc, fbit, chunks):
     P.check_codes()
 
 
+@pytest.mark.parametrize("fbit", [2, 4, 8])
+def test_chunked_append_fp32_group_mode(kvq, orc, fbit):
+    """fp32 inputs with lambda in chunks whose whole 16-token groups take the
+    group-mode append at 8, 4 and 2 bits (and whose unaligned heads and tails
+    take the per-token path): codes and meta bit-exact, attention within 2e-3."""
+    B, H, n_f = 2, 3, 4096
+    cap16 = n_f * fbit // 16
+    k, v = S.keys_values(17, fbit, B, n_f, H, 0, 4, dtype=torch.float32)
+    lam = lam_for(k)
+    P = Pair(kvq, orc, B, H, n_f, fbit, lam)
+    pos = 0
+    for n in (cap16, 5, 250, 37, 1000, 333, n_f):
+        n = min(n, n_f - pos)
+        if n <= 0:
+            break
+        P.append(k[:, pos:pos + n], v[:, pos:pos + n])
+        pos += n
+        P.check_codes(streams=[(0, 0), (1, 2)])
+    assert pos == n_f and P.gpu.query(0)["bits"] == fbit
+    P.check_codes()
+    P.check_attention(S.queries(17, fbit, 0, B, 4 * H, n_f, dtype=torch.bfloat16))
+
+
 @pytest.mark.parametrize("G", [1, 2, 3, 5, 7, 8])
 @pytest.mark.parametrize("T,fbit", [(1, 2), (17, 2), (300, 4), (1500, 4), (3000, 2), (4096, 2)])
 def test_decode_attention(kvq, orc, G, T, fbit):
