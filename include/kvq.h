@@ -248,6 +248,14 @@ kvq_status kvq_export_window(const kvq_cache* c, int layer, int b, int j, uint16
  * bounded wait (KVQ_ERR_TIMEOUT) since the last check; clears the flag. */
 kvq_status kvq_device_status(kvq_cache* c, kvq_stream_t stream);
 
+/* Self-test of that path: enqueues a one-warp kernel whose bulk-copy barrier
+ * waits for bytes no copy will bring, with the attention kernel's bounded
+ * wait; after its time limit (2 s) the wait gives up, raises the cache's
+ * error flag and the kernel returns normally (nothing faults, no copy is in
+ * flight).  The next kvq_device_status then reports KVQ_ERR_TIMEOUT and the
+ * cache stays usable.  Asynchronous.  Errors: INVALID, CUDA. */
+kvq_status kvq_selftest_timeout(kvq_cache* c, kvq_stream_t stream);
+
 /* Block-wise bit allocation (key design 2): choose one width per block from
  * the candidate widths bits[0..n_opts) (each 2, 4, 8 or 16, distinct;
  * n_opts <= 4) minimising  sum_i sens[i][o_i]  subject to the cache's budget

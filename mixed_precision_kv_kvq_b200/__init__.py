@@ -24,7 +24,7 @@ __all__ = [
     "KVQCache", "KVQError", "load",
     "kvq_pool_bytes", "kvq_pool_bytes_ex", "kvq_alloc", "kvq_alloc_ex", "kvq_export_window", "kvq_set_lambda", "kvq_append", "kvq_shrink", "kvq_set_shift_mode",
     "kvq_decode_workspace", "kvq_decode_attn", "kvq_decode_attn_noalloc", "kvq_append_decode", "kvq_query", "kvq_max_tokens", "kvq_export",
-    "kvq_device_status", "kvq_last_error", "kvq_free", "kvq_allocate_bits",
+    "kvq_device_status", "kvq_selftest_timeout", "kvq_last_error", "kvq_free", "kvq_allocate_bits",
 ]
 
 
@@ -205,6 +205,10 @@ def kvq_export_window(cache, layer: int, b: int, j: int, stream=None):
 
 def kvq_device_status(cache, stream=None) -> None:
     check(load().kvq_device_status(cache, _stream_ptr(stream)))
+
+
+def kvq_selftest_timeout(cache, stream=None) -> None:
+    check(load().kvq_selftest_timeout(cache, _stream_ptr(stream)))
 
 
 def kvq_allocate_bits(sens, bits: Sequence[int], batch: int, kv_heads: int, max_tokens: int,

@@ -53,6 +53,7 @@ SIGNATURES = {
     "kvq_export": (I, [P, I, I, I, P, P, P, P, P]),
     "kvq_export_window": (I, [P, I, I, I, P, P, P, P, P, P]),
     "kvq_device_status": (I, [P, P]),
+    "kvq_selftest_timeout": (I, [P, P]),
     "kvq_allocate_bits": (I, [I, I, P, P, I, I, I, C.c_longlong, SZ, P, P]),
     "kvq_last_error": (C.c_char_p, []),
     "kvq_free": (None, [P]),

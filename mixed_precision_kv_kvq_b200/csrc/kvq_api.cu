@@ -1006,6 +1006,14 @@ kvq_status kvq_device_status(kvq_cache* c, kvq_stream_t stream) {
   return KVQ_OK;
 }
 
+kvq_status kvq_selftest_timeout(kvq_cache* c, kvq_stream_t stream) {
+  if (!c) return fail(KVQ_ERR_INVALID, "cache is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaError_t e = c->ensure_err(s)) return cuda_fail(e, "error flag reset");
+  if (cudaError_t e = launch_wait_probe(c->err(), s)) return cuda_fail(e, "wait probe launch");
+  return KVQ_OK;
+}
+
 const char* kvq_last_error(void) { return g_last_error.c_str(); }
 
 void kvq_free(kvq_cache* c) {

@@ -1161,7 +1161,28 @@ cudaError_t launch_width(const DecodeArgs& a, cudaStream_t s) {
   }
 }
 
+// Self-test of the bounded wait: a barrier that expects 16 bytes no copy will
+// bring.  The decode kernel's own wait gives up after its time limit, raises
+// the device error flag and the kernel returns normally; no copy is in flight,
+// so nothing touches shared memory after the kernel ends.
+__global__ void wait_probe_kernel(int* err) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_expect_tx(smem_u32(&bar), 16u);
+    (void)mbar_wait(smem_u32(&bar), 0, err, &abort_flag);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_wait_probe(int* err, cudaStream_t s) {
+  wait_probe_kernel<<<1, 32, 0, s>>>(err);
+  return cudaGetLastError();
+}
 
 int decode_splits(int num_sms, int n_streams, long long gps) {
   // Smallest modelled makespan  waves(s) * (gps / s + c0)  over

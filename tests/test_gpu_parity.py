@@ -185,6 +185,24 @@ def test_forced_shrink_matches_oracle(kvq, orc):
     P.check_attention(S.queries(3, 0, 0, B, 4, 512))
 
 
+def test_bounded_wait_gives_up_and_reports(kvq, orc):
+    """The decode kernel's bounded wait, run on a barrier no copy completes
+    (kvq_selftest_timeout): after its time limit the kernel returns, the
+    next device status is KVQ_ERR_TIMEOUT, and the cache keeps working."""
+    import time
+    P = Pair(kvq, orc, 1, 2, 4096, 4, None)
+    k, v = S.keys_values(18, 0, 1, 300, 2, 0, 2, dtype=torch.bfloat16)
+    P.append(k, v)
+    t0 = time.time()
+    kvq.kvq_selftest_timeout(P.gpu.handle)
+    with pytest.raises(kvq.KVQError) as e:
+        P.gpu.device_status()
+    assert e.value.status == 7 and time.time() - t0 >= 1.5
+    P.gpu.device_status()  # cleared
+    P.check_codes()
+    P.check_attention(S.queries(18, 0, 0, 1, 4, 300, dtype=torch.bfloat16))
+
+
 def test_decode_rejects_small_workspace(kvq, orc):
     P = Pair(kvq, orc, 1, 2, 4096, 4, None)
     k, v = S.keys_values(4, 0, 1, 10, 2, 0, 1, dtype=torch.float32)
