@@ -149,7 +149,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs 
 }
 
 // Group mode (chunked appends at b <= 8 bits): one warp quantizes the 16
-// tokens of one slot group (one KV head, K or V) with the same quantizer,
+// tokens of one slot group (one KV head, K or V) with the same quantizer
+// (four tokens at a time, 8 lanes each),
 // keeps their codes in shared memory as bytes, token-major, and then writes
 // the group part lane unit by lane unit: lane L builds unit L's 2b words
 // from byte quads (Keys) or token pairs (Values) and stores them with 16-byte
@@ -178,55 +179,88 @@ __global__ void __launch_bounds__(kGroupWarps * 32) append_group_kernel(AppendAr
   const int tk0 = gi * kGroupTokens;  // first token of the group within this launch
   constexpr unsigned qmax = (1u << BITS) - 1u;
 
-  // ---- quantize the 16 tokens (8 at a time: their loads are issued together) ----
+  // ---- quantize the 16 tokens, four at a time: lane L takes token 4 step + L / 8
+  // and its channels 16 (L % 8) .. + 15, so a token's min / max needs three
+  // shuffle levels over its 8 lanes and one division serves 16 values ----
   const void* src = kv ? a.v : a.k;
-  float4 li = make_float4(1.f, 1.f, 1.f, 1.f);
+  const int sub = lane & 7, tq = lane >> 3;
   const bool mig = kv == 0 && a.lam_inv;
-  if (mig) li = *reinterpret_cast<const float4*>(a.lam_inv + (size_t)j * kHeadDim + 4 * lane);
-#pragma unroll 1
-  for (int half = 0; half < 2; half++) {
-    float4 xv[8];
+  float li[16];
 #pragma unroll
-    for (int tt = 0; tt < 8; tt++) {
-      const size_t in_off =
-          (((size_t)b * a.n_call + (size_t)(a.tok_off + tk0 + 8 * half + tt)) * a.kv_heads + j) * kHeadDim + 4 * lane;
-      if (a.dtype == 1) {
-        xv[tt] = *reinterpret_cast<const float4*>(static_cast<const float*>(src) + in_off);
-      } else {
-        const uint2 raw = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(src) + in_off);
-        xv[tt] = make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u),
-                             __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xffff0000u));
-      }
+  for (int c = 0; c < 16; c++) li[c] = 1.0f;
+  if (mig) {
+#pragma unroll
+    for (int c4 = 0; c4 < 4; c4++) {
+      const float4 l4 = *reinterpret_cast<const float4*>(a.lam_inv + (size_t)j * kHeadDim + 16 * sub + 4 * c4);
+      li[4 * c4] = l4.x; li[4 * c4 + 1] = l4.y; li[4 * c4 + 2] = l4.z; li[4 * c4 + 3] = l4.w;
     }
+  }
+  uint4 rawb[kGroupTokens / 4][2];  // bf16 inputs of every step, loaded before any is used
+  if (a.dtype != 1) {
 #pragma unroll
-    for (int tt = 0; tt < 8; tt++) {
-      float x[4] = {xv[tt].x, xv[tt].y, xv[tt].z, xv[tt].w};
-      if (mig) {
-        x[0] = __fmul_rn(x[0], li.x); x[1] = __fmul_rn(x[1], li.y);
-        x[2] = __fmul_rn(x[2], li.z); x[3] = __fmul_rn(x[3], li.w);
+    for (int step = 0; step < kGroupTokens / 4; step++) {
+      const size_t off = (((size_t)b * a.n_call + (size_t)(a.tok_off + tk0 + 4 * step + tq)) * a.kv_heads + j) *
+                         kHeadDim + 16 * sub;
+#pragma unroll
+      for (int c8 = 0; c8 < 2; c8++)
+        rawb[step][c8] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(src) + off + 8 * c8);
+    }
+  }
+#pragma unroll
+  for (int step = 0; step < kGroupTokens / 4; step++) {
+    const int tok = 4 * step + tq;
+    const size_t in_off =
+        (((size_t)b * a.n_call + (size_t)(a.tok_off + tk0 + tok)) * a.kv_heads + j) * kHeadDim + 16 * sub;
+    float x[16];
+    if (a.dtype == 1) {
+#pragma unroll
+      for (int c4 = 0; c4 < 4; c4++) {
+        const float4 f4 = *reinterpret_cast<const float4*>(static_cast<const float*>(src) + in_off + 4 * c4);
+        x[4 * c4] = f4.x; x[4 * c4 + 1] = f4.y; x[4 * c4 + 2] = f4.z; x[4 * c4 + 3] = f4.w;
       }
-      // the quantizer of kvq_quant.cuh, codes kept in registers
-      float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
-      float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-      mn = warp_min(mn);
-      mx = warp_max(mx);
-      const __half zh = __float2half_rd(mn);
-      const float z = __half2float(zh);
-      const __half rh = __float2half_ru(__fsub_rn(mx, z));
-      const float r = __half2float(rh);
-      uint32_t quad = 0;
-      if (r != 0.0f) {
-        const float inv = __fdiv_rn((float)qmax, r);
+    } else {
 #pragma unroll
-        for (int i = 0; i < 4; i++) {
-          const float y = __fadd_rn(__fmul_rn(__fsub_rn(x[i], z), inv), 0.5f);
-          quad |= min(__float2uint_rd(y), qmax) << (8 * i);
+      for (int c8 = 0; c8 < 2; c8++) {
+        const uint4 raw = rawb[step][c8];
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+          x[8 * c8 + 2 * q] = __uint_as_float(w[q] << 16);
+          x[8 * c8 + 2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
         }
       }
-      const int tok = 8 * half + tt;
-      *reinterpret_cast<uint32_t*>(&cs[wib][tok][4 * lane]) = quad;  // channels 4 lane .. 4 lane + 3, one per byte
-      if (lane == 0) ms[wib][tok] = (uint32_t)__half_as_ushort(rh) | ((uint32_t)__half_as_ushort(zh) << 16);
     }
+    if (mig) {
+#pragma unroll
+      for (int c = 0; c < 16; c++) x[c] = __fmul_rn(x[c], li[c]);
+    }
+    // the quantizer of kvq_quant.cuh over the token's 8 lanes, codes kept in registers
+    float mn = x[0], mx = x[0];
+#pragma unroll
+    for (int c = 1; c < 16; c++) {
+      mn = fminf(mn, x[c]);
+      mx = fmaxf(mx, x[c]);
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    const __half zh = __float2half_rd(mn);
+    const float z = __half2float(zh);
+    const __half rh = __float2half_ru(__fsub_rn(mx, z));
+    const float r = __half2float(rh);
+    uint32_t wq[4] = {0u, 0u, 0u, 0u};
+    if (r != 0.0f) {
+      const float inv = __fdiv_rn((float)qmax, r);
+#pragma unroll
+      for (int c = 0; c < 16; c++) {
+        const float y = __fadd_rn(__fmul_rn(__fsub_rn(x[c], z), inv), 0.5f);
+        wq[c >> 2] |= min(__float2uint_rd(y), qmax) << (8 * (c & 3));
+      }
+    }
+    *reinterpret_cast<uint4*>(&cs[wib][tok][16 * sub]) = make_uint4(wq[0], wq[1], wq[2], wq[3]);  // one byte per channel
+    if (sub == 0) ms[wib][tok] = (uint32_t)__half_as_ushort(rh) | ((uint32_t)__half_as_ushort(zh) << 16);
   }
   __syncwarp();
 
