@@ -565,13 +565,16 @@ def test_single_stream_most_splits(kvq, orc, mode):
 
 # ------------------------------------------------ fused single-token append + decode
 
-@pytest.mark.parametrize("fbit,t0,steps", [(2, 509, 6), (2, 1021, 5), (4, 3000, 4), (16, 250, 4)])
-def test_append_decode_equals_two_calls(kvq, orc, fbit, t0, steps):
+@pytest.mark.parametrize("fbit,t0,steps,dtype", [(2, 509, 6, torch.bfloat16), (2, 1021, 5, torch.bfloat16),
+                                                 (4, 3000, 4, torch.bfloat16), (16, 250, 4, torch.bfloat16),
+                                                 (4, 1020, 6, torch.float32)])
+def test_append_decode_equals_two_calls(kvq, orc, fbit, t0, steps, dtype):
     """kvq_append_decode (one launch: the decode kernel writes the new token)
     gives the same codes, meta and output, bit for bit, as kvq_append then
-    kvq_decode_attn -- including across a shrink -- and matches the oracle."""
+    kvq_decode_attn -- including across a shrink, for bf16 and fp32 inputs --
+    and matches the oracle."""
     B, H, G, n_f = 2, 3, 4, 4096
-    k, v = S.keys_values(10, fbit, B, t0 + steps, H, 0, 3, dtype=torch.bfloat16)
+    k, v = S.keys_values(10, fbit, B, t0 + steps, H, 0, 3, dtype=dtype)
     lam = lam_for(k)
     P = Pair(kvq, orc, B, H, n_f, fbit, lam)  # separate calls, and the oracle
     F = kvq.KVQCache(1, B, H, n_f * per_token(B, H, [fbit]), [fbit])
