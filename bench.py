@@ -77,14 +77,46 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def code_tokens(text):
+    """C/CUDA source with comments removed and whitespace runs collapsed, so
+    that an edit to comments or layout leaves the digest unchanged.  String
+    and character literals are kept verbatim."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+            out.append(" ")
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif c.isspace():
+            while i < n and text[i].isspace():
+                i += 1
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_digest():
-    """sha256 of the decode kernel's sources: ncu counters stay valid only
-    while it matches the digest recorded with them."""
+    """sha256 of the decode kernel's code (kvq_decode.cu + kvq_internal.cuh,
+    comments and whitespace removed): ncu counters stay valid only while it
+    matches the digest recorded with them."""
     import hashlib
     h = hashlib.sha256()
     for name in ("kvq_decode.cu", "kvq_internal.cuh"):
-        with open(os.path.join(ROOT, "mixed_precision_kv_kvq_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "mixed_precision_kv_kvq_b200", "csrc", name)) as f:
+            h.update(code_tokens(f.read()).encode())
     return h.hexdigest()[:16]
 
 

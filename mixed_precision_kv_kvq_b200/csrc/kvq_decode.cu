@@ -34,6 +34,13 @@
 // to finish the stream (atomic ticket, no waiting) merges them with
 // log-sum-exp weights.  Every mbarrier wait is bounded in time; a kernel that
 // gives up sets the cache's error flag and returns normally.
+//
+// Per-channel Key groups (CHAN = true): a Key's range and zero belong to a
+// channel of a 128-token block, so they move from the token side of the dot
+// product to the query side.  Warps take whole blocks and walk them in
+// logical order; per block a warp rebuilds the query operand (a 24-bit
+// integer per head, see chan_block) from the block's (R, Z) words, which the
+// block's first chunk brings along with its codes.  Values are unchanged.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 

@@ -1,0 +1,36 @@
+"""Host-side pieces of bench.py that need no GPU."""
+import os
+import sys
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+import bench  # noqa: E402
+
+
+def test_code_tokens_drops_comments_and_layout_only():
+    a = "int f(int x) {  // twice\n  return x * 2; /* doubled */\n}\n"
+    b = "int f(int x)\n{\n    return x * 2;\n}"
+    assert bench.code_tokens(a) == bench.code_tokens(b)
+    assert bench.code_tokens(a) != bench.code_tokens(a.replace("2;", "3;"))
+
+
+def test_code_tokens_keeps_literals():
+    s = 'asm("mov.u32 %0, 1; // not a comment" : "=r"(x)); char c = \'"\';'
+    t = bench.code_tokens(s)
+    assert "// not a comment" in t
+    assert "'\"'" in t
+    assert bench.code_tokens('p = "a\\"//b";') == 'p = "a\\"//b";'
+
+
+def test_recorded_traffic_follows_kernel_code():
+    """The committed decode profile's counters are used only while its
+    recorded digest matches the kernel code in the tree."""
+    import json
+    path = os.path.join(bench.ROOT, "profiles", "decode_kernel_7b_b16_t32k.md")
+    with open(path) as f:
+        rec = json.loads(next(l for l in f if l.startswith("traffic-json: "))[14:])
+    bytes_, src = bench.decode_traffic([2, 4])
+    if rec["source_digest"] == bench.source_digest():
+        per = rec["bytes_per_launch"]
+        assert bytes_ == (per["2bit"] + per["4bit"]) // 2
+    else:
+        assert bytes_ is None and "changed" in src
