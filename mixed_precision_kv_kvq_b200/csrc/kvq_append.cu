@@ -159,6 +159,24 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) append_kernel(AppendArgs 
 // and fill the group (the host cuts a chunk at 16-token boundaries).
 constexpr int kGroupWarps = 4;
 constexpr int kRowBytes = 144;  // 128 codes + pad: quad reads of lanes (g, t) hit 32 distinct banks
+// Three-input min / max (one instruction on sm_100), same result as two
+// nested two-input ones.
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// floor(y) for 0 <= y < 2^23 in the low bits of the result: y + 2^23 rounded
+// down is exactly 2^23 + floor(y), since the spacing of floats in
+// [2^23, 2^24) is 1.
+__device__ __forceinline__ uint32_t floor_bits(float y) {
+  return __float_as_uint(__fadd_rd(y, 8388608.0f));
+}
 template <int BITS>
 __global__ void __launch_bounds__(kGroupWarps * 32) append_group_kernel(AppendArgs a) {
   static_assert(BITS <= 8, "16-bit codes take the per-token path");
@@ -235,12 +253,10 @@ __global__ void __launch_bounds__(kGroupWarps * 32) append_group_kernel(AppendAr
       for (int c = 0; c < 16; c++) x[c] = __fmul_rn(x[c], li[c]);
     }
     // the quantizer of kvq_quant.cuh over the token's 8 lanes, codes kept in registers
-    float mn = x[0], mx = x[0];
-#pragma unroll
-    for (int c = 1; c < 16; c++) {
-      mn = fminf(mn, x[c]);
-      mx = fmaxf(mx, x[c]);
-    }
+    float mn = fminf(fmin3(fmin3(x[0], x[1], x[2]), fmin3(x[3], x[4], x[5]), fmin3(x[6], x[7], x[8])),
+                     fmin3(fmin3(x[9], x[10], x[11]), fmin3(x[12], x[13], x[14]), x[15]));
+    float mx = fmaxf(fmax3(fmax3(x[0], x[1], x[2]), fmax3(x[3], x[4], x[5]), fmax3(x[6], x[7], x[8])),
+                     fmax3(fmax3(x[9], x[10], x[11]), fmax3(x[12], x[13], x[14]), x[15]));
 #pragma unroll
     for (int o = 1; o < 8; o <<= 1) {
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
@@ -253,11 +269,19 @@ __global__ void __launch_bounds__(kGroupWarps * 32) append_group_kernel(AppendAr
     uint32_t wq[4] = {0u, 0u, 0u, 0u};
     if (r != 0.0f) {
       const float inv = __fdiv_rn((float)qmax, r);
+      // code = min(floor(y), qmax) = floor(min(y, qmax + 1/2)); y >= 1/2 as x >= Z.
+      // The code is the low byte of floor_bits; four bytes go into a word by
+      // byte permutes.
+      uint32_t fb[16];
 #pragma unroll
       for (int c = 0; c < 16; c++) {
         const float y = __fadd_rn(__fmul_rn(__fsub_rn(x[c], z), inv), 0.5f);
-        wq[c >> 2] |= min(__float2uint_rd(y), qmax) << (8 * (c & 3));
+        fb[c] = floor_bits(fminf(y, (float)qmax + 0.5f));
       }
+#pragma unroll
+      for (int c4 = 0; c4 < 4; c4++)
+        wq[c4] = __byte_perm(__byte_perm(fb[4 * c4], fb[4 * c4 + 1], 0x0040),
+                             __byte_perm(fb[4 * c4 + 2], fb[4 * c4 + 3], 0x0040), 0x5410);
     }
     *reinterpret_cast<uint4*>(&cs[wib][tok][16 * sub]) = make_uint4(wq[0], wq[1], wq[2], wq[3]);  // one byte per channel
     if (sub == 0) ms[wib][tok] = (uint32_t)__half_as_ushort(rh) | ((uint32_t)__half_as_ushort(zh) << 16);

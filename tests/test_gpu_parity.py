@@ -215,6 +215,49 @@ def test_decode_rejects_small_workspace(kvq, orc):
     assert e.value.status == 6
 
 
+def test_empty_block_and_full_budget_edges(kvq, orc):
+    """Empty block: decode is refused (STATE) and writes nothing; a zero-token
+    append is a no-op.  A block filled to exactly its Fbit capacity matches the
+    oracle (two shrinks on the way); one token more -- alone or fused with a
+    decode -- is refused (BUDGET) and changes neither codes, meta nor state."""
+    n_f, B, H, Hq = 1024, 2, 2, 6
+    P = Pair(kvq, orc, B, H, n_f, 4, None)
+    q = S.queries(21, 0, 0, B, Hq, n_f, dtype=torch.bfloat16)
+    out = torch.full((B, Hq, 128), 7.0, device="cuda")
+    with pytest.raises(kvq.KVQError) as e:
+        P.gpu.decode_attn(0, q.cuda(), out=out)
+    assert e.value.status == 3
+    torch.cuda.synchronize()
+    assert bool((out == 7.0).all())
+    empty = torch.empty(B, 0, H, 128, dtype=torch.bfloat16, device="cuda")
+    P.gpu.append(0, empty, empty)
+    assert P.gpu.query(0)["tokens"] == 0
+    k, v = S.keys_values(21, 0, B, n_f + 1, H, 0, 3, dtype=torch.bfloat16)
+    for a0, a1 in [(0, 200), (200, 300), (300, 550), (550, n_f)]:
+        P.append(k[:, a0:a1], v[:, a0:a1])
+    assert P.orc.shrink_at == [256, 512]  # a chunk is split where the next token would not fit
+    P.check_codes()
+    P.check_attention(q)
+    before = [P.gpu.export(0, b, j) for b in range(B) for j in range(H)]
+    assert P.orc.append(k[:, n_f:].float().numpy(), v[:, n_f:].float().numpy(), None) == 1
+    with pytest.raises(kvq.KVQError) as e:
+        P.gpu.append(0, k[:, n_f:].cuda(), v[:, n_f:].cuda())
+    assert e.value.status == 2
+    with pytest.raises(kvq.KVQError) as e:
+        P.gpu.append_decode(0, k[:, n_f:, :, :].cuda(), v[:, n_f:].cuda(), q.cuda(), out=out)
+    assert e.value.status == 2
+    torch.cuda.synchronize()
+    assert bool((out == 7.0).all())
+    qs = P.gpu.query(0)
+    assert qs["tokens"] == n_f and qs["bits"] == 4 and qs["n_shrinks"] == 2
+    after = [P.gpu.export(0, b, j) for b in range(B) for j in range(H)]
+    for x, y in zip(before, after):
+        for a, b in zip(x, y):
+            assert np.array_equal(a, b)
+    P.check_codes()
+    P.check_attention(q)
+
+
 # ---------------------------------------------------- Direct Right Shift (ablation)
 
 def test_direct_shift_tiny_config_one_by_one(kvq, orc):
