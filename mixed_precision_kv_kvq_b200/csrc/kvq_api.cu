@@ -262,9 +262,10 @@ long long stable_groups(const LayerState& L, const Fill& f) {
 }
 
 // The decode launches of one call: the progressive cache (if it holds
-// tokens) and, with the sink + window option, the window (one CTA per
-// stream, 16 bits); every CTA leaves one partial and the last to finish a
-// stream merges them all.
+// tokens) and, with the sink + window option, the window, or with
+// per-channel Key groups the staged block (up to three CTAs per stream, 16
+// bits); every CTA leaves one partial and the last to finish a stream merges
+// them all.
 struct DecodePlan {
   Fill fill, wfill;
   int splits = 0, wsplits = 0, nparts = 0;
