@@ -775,13 +775,13 @@ def oracle_sample(tokens, fbit=2, g=HQ7 // HKV7, seed=SEED):
     return L, q, lam
 
 
-def host_cores(cap=64):
+def host_cores(cap=64, cpu_max="/sys/fs/cgroup/cpu.max"):
     """CPUs this process may run on: its affinity set, capped by a cgroup v2
-    CPU quota when one is set, and at `cap` (one oracle stream, ~17 MB, per
-    thread)."""
+    CPU quota when one is set ("quota period" in `cpu_max`, "max" for none),
+    and at `cap` (one oracle stream, ~17 MB, per thread)."""
     n = min(cap, len(os.sched_getaffinity(0)))
     try:
-        with open("/sys/fs/cgroup/cpu.max") as f:
+        with open(cpu_max) as f:
             quota, period = f.read().split()[:2]
         if quota != "max":
             n = min(n, max(1, math.ceil(int(quota) / int(period))))

@@ -34,3 +34,13 @@ def test_recorded_traffic_follows_kernel_code():
         assert bytes_ == (per["2bit"] + per["4bit"]) // 2
     else:
         assert bytes_ is None and "changed" in src
+
+
+def test_host_cores_respects_quota_and_cap(tmp_path):
+    f = tmp_path / "cpu.max"
+    avail = len(os.sched_getaffinity(0))
+    f.write_text("max 100000\n")
+    assert bench.host_cores(cap=1000, cpu_max=str(f)) == avail
+    f.write_text("150000 100000\n")  # 1.5 CPUs of quota -> 2 threads
+    assert bench.host_cores(cap=1000, cpu_max=str(f)) == min(avail, 2)
+    assert bench.host_cores(cap=1, cpu_max=str(tmp_path / "absent")) == 1
