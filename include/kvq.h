@@ -138,7 +138,10 @@ kvq_status kvq_set_lambda(kvq_cache* c, int layer, const float* lambda_host);
 /* Quantize-on-append (key design 1): append n_tokens tokens to every
  * sequence of the batch.  k, v: device [batch][n_tokens][kv_heads][128],
  * dtype KVQ_DTYPE_BF16 or KVQ_DTYPE_F32, 16-byte aligned, every value
- * finite (the codes of a non-finite value are unspecified).  Each token is
+ * finite (the codes of a non-finite value are unspecified).  A group's
+ * minimum and range must fit binary16 (magnitudes up to 65,504): beyond that
+ * Z or R overflows to infinity, the group's codes are 0 and attention over it
+ * is undefined (not checked, as on the oracle).  Each token is
  * quantized at the block's current width; when the block is full the block
  * is first shrunk one level (never below its Fbit).  n tokens behave exactly
  * like n single-token appends.  Errors: BUDGET when the block cannot hold
