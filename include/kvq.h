@@ -140,8 +140,8 @@ kvq_status kvq_set_lambda(kvq_cache* c, int layer, const float* lambda_host);
  * dtype KVQ_DTYPE_BF16 or KVQ_DTYPE_F32, 16-byte aligned, every value
  * finite (the codes of a non-finite value are unspecified).  A group's
  * minimum and range must fit binary16 (magnitudes up to 65,504): beyond that
- * Z or R overflows to infinity, the group's codes are 0 and attention over it
- * is undefined (not checked, as on the oracle).  Each token is
+ * Z or R overflows to infinity, and the group's codes and attention over it
+ * are unspecified (not checked, as on the oracle).  Each token is
  * quantized at the block's current width; when the block is full the block
  * is first shrunk one level (never below its Fbit).  n tokens behave exactly
  * like n single-token appends.  Errors: BUDGET when the block cannot hold
