@@ -269,15 +269,14 @@ __global__ void __launch_bounds__(kGroupWarps * 32) append_group_kernel(AppendAr
     uint32_t wq[4] = {0u, 0u, 0u, 0u};
     if (r != 0.0f) {
       const float inv = __fdiv_rn((float)qmax, r);
-      // code = min(floor(y), qmax) = floor(min(y, qmax + 1/2)); y >= 1/2 as x >= Z.
-      // The code is the low byte of floor_bits; four bytes go into a word by
-      // byte permutes.
+      // code = clamp(floor(y), 0, qmax), and the clamp never binds here:
+      // y >= 1/2 as x >= Z, and fl(x - Z) <= fl(max - Z) <= R, inv <= (qmax /
+      // R)(1 + 2^-24), so y < qmax (1 + 2^-24)^3 + 1/2 < qmax + 1 for qmax <
+      // 2^16.  The code is the low byte of floor_bits; four bytes go into a
+      // word by byte permutes.
       uint32_t fb[16];
 #pragma unroll
-      for (int c = 0; c < 16; c++) {
-        const float y = __fadd_rn(__fmul_rn(__fsub_rn(x[c], z), inv), 0.5f);
-        fb[c] = floor_bits(fminf(y, (float)qmax + 0.5f));
-      }
+      for (int c = 0; c < 16; c++) fb[c] = floor_bits(__fadd_rn(__fmul_rn(__fsub_rn(x[c], z), inv), 0.5f));
 #pragma unroll
       for (int c4 = 0; c4 < 4; c4++)
         wq[c4] = __byte_perm(__byte_perm(fb[4 * c4], fb[4 * c4 + 1], 0x0040),
