@@ -47,6 +47,12 @@ SEED = 0
 L7, HQ7, HKV7, B7, T7 = 28, 28, 4, 16, 32768
 FBIT7 = [4 if (l == 0 or l >= L7 - 8) else 2 for l in range(L7)]
 ROOM = 4096  # tokens of head-room for the appended decode tokens
+# Llama-70B long-CoT workload
+L70, HQ70, HKV70, B70, T70 = 80, 64, 8, 8, 131072
+FBIT70 = [4 if l % 4 == 0 else 2 for l in range(L70)]
+ROOM70 = 512
+WORKLOAD70 = ("Llama-70B-shape long-CoT decode: 80 layers, 64 Q / 8 KV heads, head_dim 128, batch 8, context 131072, "
+              "Fbit 4 for every 4th layer (0, 4, ...) else 2; one decode step = append + attention per layer")
 WORKLOAD = ("DeepSeek-R1-Distill-Qwen-7B-shape decode: 28 layers, 28 Q / 4 KV heads, head_dim 128, "
             "batch 16, context 32768, Fbit 4 for layer 0 and the last 8 layers else 2; one decode step "
             "= append + attention per layer")
@@ -120,23 +126,24 @@ def source_digest():
     return h.hexdigest()[:16]
 
 
-def decode_traffic(fbit):
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
+
+
+def decode_traffic(fbit, path=TRAFFIC_FILE):
     """DRAM bytes per decode launch (ncu dram__bytes_read.sum +
     dram__bytes_write.sum, averaged over the layers' bit widths) from the
-    committed profile summary, or None when the kernel changed since."""
-    path = os.path.join(ROOT, "profiles", "decode_kernel_7b_b16_t32k.md")
+    committed traffic record, or None when the kernel changed since."""
     try:
         with open(path) as f:
-            line = next(l for l in f if l.startswith("traffic-json: "))
-        rec = json.loads(line[len("traffic-json: "):])
-    except (OSError, StopIteration, ValueError):
-        return None, "no ncu summary"
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None, "no ncu traffic record"
     if rec.get("source_digest") != source_digest():
         return None, "kernel changed since the ncu capture"
-    per = rec["bytes_per_launch"]
+    per = rec.get("bytes_per_launch", {})
     if not all(f"{b}bit" in per for b in fbit):
         return None, "no capture for some bit width"
-    return int(sum(per[f"{b}bit"] for b in fbit) / len(fbit)), "profiles/decode_kernel_7b_b16_t32k.md"
+    return int(sum(per[f"{b}bit"] for b in fbit) / len(fbit)), "profiles/decode_traffic.json"
 
 
 def calib_lambda(k):
@@ -230,47 +237,53 @@ def flush_l2(buf):
     buf.add_(1)
 
 
-def measure_shrink(kvq, dev, flush_buf, reps=3):
-    """Shrink kernel GB/s (algorithmic: whole region read, half written; the
-    Direct Right Shift also reads and rewrites the meta of every token).
+def measure_shrink(kvq, dev, flush_buf, blocks_7b=20, blocks_70b=3):
+    """Shrink kernel GB/s (algorithmic: the block's code region read, half of
+    it written; the Direct Right Shift also reads and rewrites the meta of
+    every token).  Each event is timed on several blocks of one cache, each
+    filled to the point where its next token would shrink it: the blocks are
+    shrunk back to back (one launch each, every launch on a block no other
+    launch touches) with CUDA events around the batch after an L2 flush, and
+    the time per launch is the batch time over the blocks.
     (a) Llama-70B-shape layer (batch 8, 8 KV heads), Fbit 2, a block full with
     131072 tokens at 4 bits shrinking to 2 bits, with either shift.  (b) the
     7B progressive stream (batch 8, 4 KV heads, 32768 tokens at Fbit 2):
     events 16->8 at 4096, 8->4 at 8192, 4->2 at 16384 tokens."""
     res = {}
+    stream = torch.cuda.current_stream(dev)
 
-    def one(batch, kv_heads, n_f, fbit, fill_tokens, tag, direct=False):
-        times = []
-        nbytes = None
-        for r in range(reps):
-            cache = build_cache(kvq, dev, 1, batch, kv_heads, [fbit], fill_tokens, n_f, SEED + 17 + r, 10,
-                                chunk=8192, shift_mode=kvq.KVQ_SHIFT_DIRECT if direct else None)
-            st = cache.query(0)
-            assert st["tokens"] == st["capacity"], st
-            region = batch * kv_heads * 2 * n_f * 16 * fbit  # code bytes of the block
-            nbytes = region + region // 2
-            if direct:  # the meta of every stored token is read and rewritten too
-                nbytes += 2 * batch * kv_heads * st["tokens"] * 2 * 4
-            flush_l2(flush_buf)
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record()
-            cache.shrink(0)
-            e1.record()
-            torch.cuda.synchronize(dev)
-            cache.device_status()
-            times.append(e0.elapsed_time(e1) / 1e3)
-            bits_from = st["bits"]
-            cache.free()
-            del cache
-        t = statistics.median(times)
-        res[tag] = {"gbs": nbytes / t / 1e9, "us": t * 1e6, "bytes": nbytes, "bits": f"{bits_from}->{bits_from // 2}",
-                    "reps": reps}
+    def one(batch, kv_heads, n_f, fbit, fill_tokens, tag, blocks, direct=False):
+        cache = build_cache(kvq, dev, blocks, batch, kv_heads, [fbit] * blocks, fill_tokens, n_f, SEED + 17, 10,
+                            chunk=8192, shift_mode=kvq.KVQ_SHIFT_DIRECT if direct else None)
+        st = [cache.query(l) for l in range(blocks)]
+        assert all(x["tokens"] == x["capacity"] == fill_tokens for x in st), st
+        region = batch * kv_heads * 2 * n_f * 16 * fbit  # code bytes of one block
+        nbytes = region + region // 2
+        if direct:  # the meta of every stored token is read and rewritten too
+            nbytes += 2 * batch * kv_heads * fill_tokens * 2 * 4
+        flush_l2(flush_buf)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for l in range(blocks):
+            cache.shrink(l)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        cache.device_status()
+        t = e0.elapsed_time(e1) / 1e3 / blocks
+        bits_from = st[0]["bits"]
+        assert all(cache.query(l)["bits"] == bits_from // 2 for l in range(blocks))
+        cache.free()
+        del cache
+        res[tag] = {"gbs": round(nbytes / t / 1e9, 1), "us": round(t * 1e6, 2), "bytes": nbytes,
+                    "bits": f"{bits_from}->{bits_from // 2}", "launches": blocks,
+                    "timing": f"{blocks} blocks shrunk back to back after an L2 flush, CUDA events around the "
+                              "batch, time per launch"}
 
-    one(8, 8, 262144, 2, 131072, "llama70b_128k_4to2")
-    one(8, 8, 262144, 2, 131072, "llama70b_128k_4to2_direct_shift", direct=True)
+    one(8, 8, 262144, 2, 131072, "llama70b_128k_4to2", blocks_70b)
+    one(8, 8, 262144, 2, 131072, "llama70b_128k_4to2_direct_shift", blocks_70b, direct=True)
     for tokens, tag in ((4096, "qwen7b_16to8"), (8192, "qwen7b_8to4"), (16384, "qwen7b_4to2")):
-        one(8, 4, 32768, 2, tokens, tag)
+        one(8, 4, 32768, 2, tokens, tag, blocks_7b)
     return res
 
 
@@ -439,6 +452,154 @@ def measure_append_token(kvq, dev, reps=200, sink_window=False):
     return {"us": round(us, 2), "gbs": round(nb / us / 1e3, 2), "bytes": nb, "batch": B7, "kv_heads": HKV7,
             "bits": 2, "timing": f"{reps} back-to-back single-token appends, CUDA events around the batch; "
                                  "launch-latency bound"}
+
+
+def serve_steps(cache, kh, vh, qh, oh, sm_scale, dev, stream):
+    """A serving loop's decode steps through the public API, end to end:
+    step i's K, V, Q (kh[i], vh[i], qh[i]: pinned host [layers][...]) go to
+    the device, every block runs KVQCache.append_decode on device views, and
+    the step's outputs come back to pinned host memory (oh).  Double-buffered
+    on a copy stream: step i+1's inputs arrive and step i-1's outputs leave
+    while step i computes.  Returns the device time in ms of all the steps,
+    every copy included (CUDA events on `stream`)."""
+    E, layers = kh.shape[0], kh.shape[1]
+    cs = torch.cuda.Stream(dev)
+    bufs = [(torch.empty(kh.shape[1:], dtype=kh.dtype, device=dev), torch.empty(vh.shape[1:], dtype=vh.dtype, device=dev),
+             torch.empty(qh.shape[1:], dtype=qh.dtype, device=dev), torch.empty(oh.shape, dtype=oh.dtype, device=dev))
+            for _ in range(2)]
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]      # step's compute finished (inputs read, output written)
+    drained = [torch.cuda.Event() for _ in range(2)]   # step's output copied out
+
+    def fetch(i):
+        b = i % 2
+        with torch.cuda.stream(cs):
+            if i >= 2:
+                cs.wait_event(done[b])  # the step that last read these buffers
+            kd, vd, qd, _ = bufs[b]
+            kd.copy_(kh[i], non_blocking=True)
+            vd.copy_(vh[i], non_blocking=True)
+            qd.copy_(qh[i], non_blocking=True)
+            in_ready[b].record(cs)
+
+    torch.cuda.synchronize(dev)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    cs.wait_event(f0)
+    fetch(0)
+    for i in range(E):
+        b = i % 2
+        if i + 1 < E:
+            fetch(i + 1)
+        kd, vd, qd, od = bufs[b]
+        stream.wait_event(in_ready[b])
+        if i >= 2:
+            stream.wait_event(drained[b])  # output buffer b copied out by then
+        for l in range(layers):
+            cache.append_decode(l, kd[l], vd[l], qd[l], sm_scale, out=od[l])
+        done[b].record(stream)
+        with torch.cuda.stream(cs):
+            cs.wait_event(done[b])
+            oh.copy_(od, non_blocking=True)
+            drained[b].record(cs)
+    stream.wait_stream(cs)
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    return f0.elapsed_time(f1)
+
+
+def measure_step_70b(kvq, dev, K, W, E, cpu=True, peak=None):
+    """The Llama-70B long-CoT decode step as a whole: 80 blocks (every 4th at
+    4 bits, the rest at 2), batch 8, 64 query / 8 KV heads, 131072 cached
+    tokens per sequence (the cache holds 59 GB), one kvq_append_decode per
+    block.  W warm-up steps, then K steps with CUDA events around the region
+    only; E more steps end to end through the public API with host buffers
+    (serve_steps); the CPU oracle on 70B-shaped streams beside it."""
+    import ctypes as C
+    lib = kvq.load()
+    stream = torch.cuda.current_stream(dev)
+    layers = L70
+    n_f = T70 + ROOM70
+    if K + W + E > ROOM70:
+        raise SystemExit(f"70B step: steps + warm-up + e2e steps must be <= {ROOM70}")
+    t_build = time.perf_counter()
+    cache = build_cache(kvq, dev, layers, B70, HKV70, FBIT70, T70, n_f, SEED + 70, S.outliers_for(HKV70), chunk=8192)
+    t_build = time.perf_counter() - t_build
+    for l in range(layers):
+        assert cache.query(l)["bits"] == FBIT70[l]
+    sm_scale = HEAD_DIM ** -0.5
+    nsteps = W + K + E
+    g = torch.Generator(device=dev)
+    g.manual_seed(SEED + 71)
+    kin = torch.randn((nsteps, layers, B70, 1, HKV70, HEAD_DIM), generator=g, device=dev).to(torch.bfloat16)
+    vin = torch.randn((nsteps, layers, B70, 1, HKV70, HEAD_DIM), generator=g, device=dev).to(torch.bfloat16)
+    qin = torch.randn((nsteps, layers, B70, HQ70, HEAD_DIM), generator=g, device=dev).to(torch.bfloat16)
+    out = torch.empty((layers, B70, HQ70, HEAD_DIM), dtype=torch.float32, device=dev)
+    ws = [cache.workspace(l, HQ70) for l in range(layers)]
+    sp = C.c_void_p(stream.cuda_stream)
+    h = cache.handle
+    scale_c = C.c_float(sm_scale)
+    args = [[(h, l, C.c_void_p(kin[i, l].data_ptr()), C.c_void_p(vin[i, l].data_ptr()), kvq.KVQ_DTYPE_BF16,
+              C.c_void_p(qin[i, l].data_ptr()), HQ70, scale_c, C.c_void_p(out[l].data_ptr()),
+              C.c_void_p(ws[l].data_ptr()), ws[l].numel() * 4, sp) for l in range(layers)] for i in range(W + K)]
+
+    def step(i):
+        for l in range(layers):
+            st = lib.kvq_append_decode(*args[i][l])
+            if st:
+                kvq.check(st)
+
+    def step_bytes(t_before):
+        return sum(append_bytes(B70, HKV70, 1, FBIT70[l]) + decode_bytes(B70, HKV70, HQ70, t_before + 1, FBIT70[l])
+                   for l in range(layers))
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize(dev)
+    t0 = cache.query(0)["tokens"]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        e0.record(stream)
+        for i in range(K):
+            step(W + i)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    cache.device_status()
+    ms = e0.elapsed_time(e1)
+    nb = sum(step_bytes(t0 + i) for i in range(K))
+    value = nb / (ms / 1e3) / 1e9
+    if peak is None:
+        peak = peaks()[0]
+    n_dec = K * layers
+    res = {"value": round(value, 1), "unit": "GB/s", "ms_per_step": round(ms / K, 4), "steps": K, "warmup": W,
+           "config": {"workload": WORKLOAD70, "layers": layers, "batch": B70, "q_heads": HQ70, "kv_heads": HKV70,
+                      "head_dim": HEAD_DIM, "context": T70, "fbit": "4 if layer % 4 == 0 else 2",
+                      "cache_gb": round(cache.pool.numel() / 1e9, 2), "build_s": round(t_build, 1),
+                      "l2": "no flush: every block's cache read (0.6-1.1 GB) exceeds the 126 MB L2"},
+           "roofline": {"bound": "hbm", "achieved": round(value, 1), "peak": peak, "unit": "GB/s",
+                        "frac": round(value / peak, 4), "kernel": "decode_kernel (kvq_append_decode)",
+                        "avg_launch_us": round(ms * 1e3 / n_dec, 2), "bytes_per_launch": int(nb / n_dec),
+                        "timing": f"CUDA events around the {n_dec} launches of the timed region, all this kernel"},
+           "gpu_launches": n_dec, "clocks": clk.summary()}
+    if E > 0:
+        kh = kin[W + K:].cpu().pin_memory()
+        vh = vin[W + K:].cpu().pin_memory()
+        qh = qin[W + K:].cpu().pin_memory()
+        oh = torch.empty((layers, B70, HQ70, HEAD_DIM), dtype=torch.float32).pin_memory()
+        t1 = cache.query(0)["tokens"]
+        e2e_ms = serve_steps(cache, kh, vh, qh, oh, sm_scale, dev, stream)
+        cache.device_status()
+        eb = sum(step_bytes(t1 + i) for i in range(E))
+        res["e2e"] = {"value": round(eb / (e2e_ms / 1e3) / 1e9, 1), "unit": "GB/s",
+                      "h2d_bytes_per_step": layers * (2 * kin[0, 0].numel() * 2 + qin[0, 0].numel() * 2),
+                      "d2h_bytes_per_step": layers * out[0].numel() * 4, "steps": E}
+    cache.free()
+    del cache, kin, vin, qin, args
+    torch.cuda.empty_cache()
+    if cpu:
+        res["cpu_baseline"] = cpu_baseline(tokens=T70, g=HQ70 // HKV70, n_out=S.outliers_for(HKV70),
+                                           budget_s=12.0, single_s=4.0, max_threads=16)
+    return res
 
 
 def run_gpu(args, rank, world):
@@ -642,51 +803,7 @@ def run_gpu(args, rank, world):
             torch.cuda.synchronize(dev)
             if world > 1:
                 torch.distributed.barrier()
-            # A serving loop's steps, double-buffered: a copy stream brings step
-            # i+1's K, V, Q in and takes step i-1's outputs out while step i runs
-            # (the public API per block, on device views).  Every copy of every
-            # step is inside the timed region.
-            cs = torch.cuda.Stream(dev)
-            bufs = [(torch.empty_like(kin[0]), torch.empty_like(vin[0]), torch.empty_like(qin[0]), torch.empty_like(out))
-                    for _ in range(2)]
-            in_ready = [torch.cuda.Event() for _ in range(2)]
-            done = [torch.cuda.Event() for _ in range(2)]      # step's compute finished (inputs read, output written)
-            drained = [torch.cuda.Event() for _ in range(2)]   # step's output copied out
-
-            def fetch(i):
-                b = i % 2
-                with torch.cuda.stream(cs):
-                    if i >= 2:
-                        cs.wait_event(done[b])  # the step that last read these buffers
-                    kd, vd, qd, _ = bufs[b]
-                    kd.copy_(kh[i], non_blocking=True)
-                    vd.copy_(vh[i], non_blocking=True)
-                    qd.copy_(qh[i], non_blocking=True)
-                    in_ready[b].record(cs)
-
-            f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            f0.record(stream)
-            cs.wait_event(f0)
-            fetch(0)
-            for i in range(E):
-                b = i % 2
-                if i + 1 < E:
-                    fetch(i + 1)
-                kd, vd, qd, od = bufs[b]
-                stream.wait_event(in_ready[b])
-                if i >= 2:
-                    stream.wait_event(drained[b])  # output buffer b copied out by then
-                for l in range(layers):
-                    cache.append_decode(l, kd[l], vd[l], qd[l], sm_scale, out=od[l])
-                done[b].record(stream)
-                with torch.cuda.stream(cs):
-                    cs.wait_event(done[b])
-                    oh.copy_(od, non_blocking=True)
-                    drained[b].record(cs)
-            stream.wait_stream(cs)
-            f1.record(stream)
-            torch.cuda.synchronize(dev)
-            e2e_ms = f0.elapsed_time(f1)
+            e2e_ms = serve_steps(cache, kh[:E], vh[:E], qh[:E], oh, sm_scale, dev, stream)
             e2e_ms = max_over_ranks(e2e_ms, world, dev)
             eb = 0
             t1 = cache.query(0)["tokens"] - E
@@ -737,6 +854,16 @@ def run_gpu(args, rank, world):
         extra["decode_configs"] = measure_decode_configs(kvq, dev)
         extra["block_append_key_channel"] = measure_block_append_key_channel(kvq, dev)
         extra["decode_graph"] = graph
+    if not args.no_70b and rank == 0:
+        if not args.no_shrink:
+            del flush
+        else:
+            cache.free()
+            del cache, kin, vin, qin
+        torch.cuda.empty_cache()
+        k70 = min(K, 100)
+        extra["llama70b_step"] = measure_step_70b(kvq, dev, k70, 3, 0 if args.no_e2e else min(k70, 20),
+                                                  cpu=world == 1 and not args.no_cpu)
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(total_ms / K, 4), "higher_is_better": True, "scaling": "weak",
@@ -754,11 +881,13 @@ def run_gpu(args, rank, world):
 
 # ---------------------------------------------------------------- CPU oracle
 
-def oracle_sample(tokens, fbit=2, g=HQ7 // HKV7, seed=SEED):
-    """One (sequence, KV head) stream of a 7B-shape block, replayed through
-    the oracle's progressive cache; returns (layer, q, lam)."""
+def oracle_sample(tokens, fbit=2, g=HQ7 // HKV7, seed=SEED, n_out=None):
+    """One (sequence, KV head) stream of a model-shaped block, replayed
+    through the oracle's progressive cache; returns (layer, q, lam)."""
     from oracle import oracle as orc
 
+    if n_out is None:
+        n_out = S.outliers_for(HKV7)
     # a block sized for exactly `tokens` (a multiple of 512) ends full at its Fbit
     tokens = (tokens + 511) // 512 * 512
     L = orc.Layer(1, 1, tokens, fbit)
@@ -766,7 +895,7 @@ def oracle_sample(tokens, fbit=2, g=HQ7 // HKV7, seed=SEED):
     pos = 0
     while pos < tokens:
         n = min(4096, tokens - pos)
-        k, v = S.keys_values(seed, 1, 1, n, 1, pos, S.outliers_for(HKV7), dtype=torch.bfloat16)
+        k, v = S.keys_values(seed, 1, 1, n, 1, pos, n_out, dtype=torch.bfloat16)
         if lam is None:
             lam = calib_lambda(k).numpy().reshape(1, HEAD_DIM).astype(np.float32)
         assert L.append(k.float().numpy(), v.float().numpy(), lam) == 0
@@ -790,7 +919,7 @@ def host_cores(cap=64, cpu_max="/sys/fs/cgroup/cpu.max"):
     return n
 
 
-def oracle_threads(threads, tokens, warmup, run):
+def oracle_threads(threads, tokens, warmup, run, g=HQ7 // HKV7, n_out=None):
     """Run the oracle's fp64 attention on `threads` threads at once, each over
     its own stream sample (the oracle's C code runs without the Python lock
     and keeps no global state).  After `warmup` calls per thread and a
@@ -801,7 +930,7 @@ def oracle_threads(threads, tokens, warmup, run):
     barrier = threading.Barrier(threads)
 
     def one(i):
-        L, q, lam = oracle_sample(tokens, seed=SEED + i)
+        L, q, lam = oracle_sample(tokens, g=g, seed=SEED + i, n_out=n_out)
         assert L.bits == 2, "the sample block ends full at its Fbit of 2"
         call = lambda: L.attention(q, lam, HEAD_DIM ** -0.5)  # noqa: E731
         for _ in range(warmup):
@@ -814,31 +943,36 @@ def oracle_threads(threads, tokens, warmup, run):
     return sum(r[0] for r in res), max(r[1] for r in res)
 
 
-def cpu_baseline(budget_s=15.0):
-    """The oracle's fp64 attention over sampled streams of a 7B 2-bit block at
-    the full context, on every host core at once (one stream per thread)."""
-    cores = host_cores()
+def cpu_baseline(budget_s=15.0, single_s=5.0, tokens=T7, g=HQ7 // HKV7, n_out=None, max_threads=64):
+    """The oracle's fp64 attention over sampled (sequence, KV head) streams of
+    a 2-bit block at the full context (7B shape by default): on one thread,
+    then on every host core at once (one stream per thread)."""
+    cores = min(host_cores(), max_threads)
 
-    def run(call):
-        t0 = time.perf_counter()
-        n = 0
-        while True:
-            call()
-            n += 1
-            if time.perf_counter() - t0 > budget_s:
-                return n, time.perf_counter() - t0
+    def timed(budget):
+        def run(call):
+            t0 = time.perf_counter()
+            n = 0
+            while True:
+                call()
+                n += 1
+                if time.perf_counter() - t0 > budget:
+                    return n, time.perf_counter() - t0
+        return run
 
-    n, dt = oracle_threads(cores, T7, 0, run)
-    nb = decode_bytes(1, 1, HQ7 // HKV7, T7, 2)
+    nb = decode_bytes(1, 1, g, tokens, 2)
+    n1, dt1 = oracle_threads(1, tokens, 0, timed(single_s), g=g, n_out=n_out)
+    n, dt = oracle_threads(cores, tokens, 0, timed(budget_s), g=g, n_out=n_out)
     return {"value": round(n * nb / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} x one (sequence, KV head) stream of a 2-bit 7B-shape block, {T7} tokens, "
-                      f"{HQ7 // HKV7} query heads, fp64 attention, {cores} threads each on its own stream; "
-                      f"{dt:.1f} s"}
+            "sample": f"{n} x one (sequence, KV head) stream of a 2-bit block, {tokens} tokens, "
+                      f"{g} query heads, fp64 attention, {cores} threads each on its own stream; {dt:.1f} s",
+            "single_thread": {"value": round(n1 * nb / dt1 / 1e9, 5), "unit": "GB/s", "cores": 1,
+                              "sample": f"{n1} x the same stream on one thread; {dt1:.1f} s"}}
 
 
 def run_reference(args, world=1):
     K, W = args.steps, args.warmup
-    tokens = T7 if K + W <= 20 else max(1024, (T7 * 20 // (K + W)) // 512 * 512)
+    tokens = T7  # the GPU arm's context; a step is one call per thread
     cores = host_cores()
 
     def run(call):
@@ -862,6 +996,25 @@ def run_reference(args, world=1):
             "e2e": {"value": round(v, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_part(args):
+    """One measurement alone on cuda:0 (for profiling): the shrink events, or
+    the Llama-70B step (args.steps timed steps, no end-to-end pass)."""
+    from mixed_precision_kv_kvq_b200 import build as kbuild
+
+    kbuild.build()
+    import mixed_precision_kv_kvq_b200 as kvq
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if args.part == "shrink":
+        flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        n = args.shrink_blocks
+        return {"part": "shrink", **measure_shrink(kvq, dev, flush, blocks_7b=n or 20, blocks_70b=n or 3)}
+    return {"part": "step70b",
+            **measure_step_70b(kvq, dev, args.steps, args.warmup, 0 if args.no_e2e else min(args.steps, 20),
+                               cpu=not args.no_cpu)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -872,6 +1025,11 @@ def main():
     ap.add_argument("--no-shrink", action="store_true", help="skip the separate shrink/append measurements")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--no-70b", action="store_true", help="skip the Llama-70B decode step")
+    ap.add_argument("--part", choices=["all", "shrink", "step70b"], default="all",
+                    help="run one measurement alone (profiling cases): the shrink events or the 70B step")
+    ap.add_argument("--shrink-blocks", type=int, default=0,
+                    help="with --part shrink: blocks per event (0: 20 for the 7B events, 3 for the 70B ones)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "kvq":
         print("note: warm-up raised to 3", file=sys.stderr)
@@ -882,6 +1040,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args, world)), flush=True)
+        return
+    if args.part != "all":
+        if rank == 0:
+            print(json.dumps(run_part(args)), flush=True)
         return
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))

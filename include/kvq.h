@@ -208,14 +208,17 @@ kvq_status kvq_append_decode(kvq_cache* c, int layer, const void* k, const void*
  * no counterpart to this call: it exists for callers that cannot allocate device
  * memory where they run decode (an allocator owned by a host framework, a
  * serving loop that must not allocate after start-up, a host that only hands
- * out inputs and outputs).  The split partials go to a 24 MiB buffer that is
- * part of the library: every GPU that loads the library holds it until the
- * process exits.  A block whose batch * kv_heads streams need more than that
- * is rejected with KVQ_ERR_WORKSPACE (use kvq_decode_attn).  The first call
- * on a device looks up the buffer's device address (a CUDA runtime query,
- * no allocation); make that first call before any stream capture.  All calls
- * on one device share the buffer, so calls that can overlap on the GPU
- * (different streams, or different caches) race: serialise them. */
+ * out inputs and outputs).  When a stream of the block is cut into several
+ * slices, their partials go to a 24 MiB buffer that is part of the library:
+ * every GPU that loads the library holds it until the process exits.  A
+ * block whose batch * kv_heads streams need more than that is rejected with
+ * KVQ_ERR_WORKSPACE (use kvq_decode_attn); a block whose streams take one
+ * slice each needs no scratch at all.  Each call looks up the buffer's
+ * device address on the current device (a CUDA runtime query, no
+ * allocation); the first call on a device may also load the library's
+ * device code there, so make that first call before any stream capture.
+ * All calls on one device share the buffer, so calls that can overlap on
+ * the GPU (different streams, or different caches) race: serialise them. */
 kvq_status kvq_decode_attn_noalloc(kvq_cache* c, int layer, const void* q, int q_heads, float sm_scale,
                                    float* out, kvq_stream_t stream);
 

@@ -7,13 +7,14 @@
 // The host keeps every counter, so deciding to shrink never reads device
 // memory and nothing synchronises.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
-#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -39,6 +40,23 @@ kvq_status fail(kvq_status s, const char* fmt, ...) {
 }
 kvq_status cuda_fail(cudaError_t e, const char* what) {
   return fail(KVQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// NVTX range around one entry point (a profiler's timeline shows the calls
+// around their kernels; with no tool attached a push and a pop cost a few ns).
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range&) = delete;
+  Range& operator=(const Range&) = delete;
+};
+
+// Host-side fault injection: with KVQ_FAULT_ALLOC set to anything but "" or
+// "0", the library's own device allocation reports failure without calling
+// CUDA, so the out-of-memory path can be tested on any machine.
+bool fault_alloc() {
+  const char* f = getenv("KVQ_FAULT_ALLOC");
+  return f && *f && strcmp(f, "0") != 0;
 }
 
 }  // namespace
@@ -508,6 +526,10 @@ kvq_status kvq_alloc_ex(kvq_cache** out, int layers, int batch, int kv_heads, in
     c->pool = static_cast<uint8_t*>(dev_pool);
     c->owns_pool = false;
   } else {
+    if (fault_alloc()) {
+      delete c;
+      return fail(KVQ_ERR_OOM, "cudaMalloc(%zu): injected failure (KVQ_FAULT_ALLOC)", p.bytes);
+    }
     void* ptr = nullptr;
     cudaError_t e = cudaMalloc(&ptr, p.bytes);
     if (e != cudaSuccess) {
@@ -548,6 +570,7 @@ kvq_status kvq_set_lambda(kvq_cache* c, int layer, const float* lambda_host) {
 
 kvq_status kvq_append(kvq_cache* c, int layer, const void* k, const void* v, int dtype, int n_tokens,
                       kvq_stream_t stream) {
+  const Range range("kvq_append");
   if (kvq_status s = check_layer(c, layer)) return s;
   if (n_tokens < 0) return fail(KVQ_ERR_INVALID, "n_tokens %d < 0", n_tokens);
   if (n_tokens == 0) return KVQ_OK;
@@ -637,6 +660,7 @@ kvq_status kvq_append(kvq_cache* c, int layer, const void* k, const void* v, int
 }
 
 kvq_status kvq_shrink(kvq_cache* c, int layer, kvq_stream_t stream) {
+  const Range range("kvq_shrink");
   if (kvq_status s = check_layer(c, layer)) return s;
   LayerState& L = c->L[layer];
   if (L.bits <= L.fbit) return fail(KVQ_ERR_STATE, "layer %d is at its Fbit %d", layer, L.fbit);
@@ -672,6 +696,7 @@ size_t kvq_decode_workspace(const kvq_cache* c, int layer, int q_heads) {
 
 kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, float sm_scale, float* out,
                            void* workspace, size_t ws_bytes, kvq_stream_t stream) {
+  const Range range("kvq_decode_attn");
   if (kvq_status s = check_layer(c, layer)) return s;
   if (!q || !out) return fail(KVQ_ERR_INVALID, "q or out is NULL");
   if (q_heads <= 0 || q_heads % c->kv_heads)
@@ -703,6 +728,7 @@ kvq_status kvq_decode_attn(kvq_cache* c, int layer, const void* q, int q_heads, 
 kvq_status kvq_append_decode(kvq_cache* c, int layer, const void* k, const void* v, int dtype, const void* q,
                              int q_heads, float sm_scale, float* out, void* workspace, size_t ws_bytes,
                              kvq_stream_t stream) {
+  const Range range("kvq_append_decode");
   if (kvq_status s = check_layer(c, layer)) return s;
   LayerState& L = c->L[layer];
   if (L.window || L.chan) {  // the window's moves and the staged blocks need the append kernels: the two calls
@@ -775,32 +801,20 @@ constexpr size_t kNoAllocScratchBytes = (size_t)24 << 20;  // 24 MiB per device
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
 
 namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};
-
 // Device address of the scratch buffer on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// with the device current, on every call: a runtime query that allocates
+// nothing, and that stays right after a device reset or a new context (which
+// may load the library's device code at another address).
 cudaError_t noalloc_scratch(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
-  return cudaSuccess;
+  *out = nullptr;
+  return cudaGetSymbolAddress(out, g_noalloc_scratch);
 }
 }  // namespace
 
 kvq_status kvq_decode_attn_noalloc(kvq_cache* c, int layer, const void* q, int q_heads, float sm_scale,
                                    float* out, kvq_stream_t stream) {
+  const Range range("kvq_decode_attn_noalloc");
   if (kvq_status s = check_layer(c, layer)) return s;
   if (!q || !out) return fail(KVQ_ERR_INVALID, "q or out is NULL");
   if (q_heads <= 0 || q_heads % c->kv_heads)
@@ -814,7 +828,9 @@ kvq_status kvq_decode_attn_noalloc(kvq_cache* c, int layer, const void* q, int q
   if ((L.window || L.chan ? L.n_all : L.n) <= 0) return fail(KVQ_ERR_STATE, "layer %d is empty", layer);
   const int n_streams = c->batch * c->kv_heads;
   const DecodePlan d = plan_decode(c, L);
-  const size_t need = decode_parts_used(n_streams, d.nparts);
+  // A single partial per stream goes straight to `out`: the scratch is used
+  // only when a stream is cut into several.
+  const size_t need = d.nparts > 1 ? decode_parts_used(n_streams, d.nparts) : 0;
   if (need > kNoAllocScratchBytes)
     return fail(KVQ_ERR_WORKSPACE,
                 "this block needs %zu bytes of scratch (batch*kv_heads=%d x %d splits); the built-in buffer holds "

@@ -269,18 +269,24 @@ __global__ void __launch_bounds__(kGroupWarps * 32) append_group_kernel(AppendAr
     uint32_t wq[4] = {0u, 0u, 0u, 0u};
     if (r != 0.0f) {
       const float inv = __fdiv_rn((float)qmax, r);
-      // code = clamp(floor(y), 0, qmax), and the clamp never binds here:
-      // y >= 1/2 as x >= Z, and fl(x - Z) <= fl(max - Z) <= R, inv <= (qmax /
-      // R)(1 + 2^-24), so y < qmax (1 + 2^-24)^3 + 1/2 < qmax + 1 for qmax <
-      // 2^16.  The code is the low byte of floor_bits; four bytes go into a
-      // word by byte permutes.
+      // code = clamp(floor(y), 0, qmax), and for finite groups within
+      // binary16 range the clamp never binds: y >= 1/2 as x >= Z, and
+      // fl(x - Z) <= fl(max - Z) <= R, inv <= (qmax / R)(1 + 2^-24), so
+      // y < qmax (1 + 2^-24)^3 + 1/2 < qmax + 1 for qmax < 2^16.  The code is
+      // the low byte of floor_bits; four bytes go into a word by byte
+      // permutes.  A group outside that contract (an infinite Value gives
+      // R = inf, inv = 0 and inf * 0 = NaN; a minimum below -65504 gives
+      // Z = -inf) can yield NaN, whose low byte is 0xff: the mask keeps every
+      // byte inside its b-bit field, so such a group's codes, unspecified as
+      // they are, never reach the fields of the tokens packed beside them.
       uint32_t fb[16];
 #pragma unroll
       for (int c = 0; c < 16; c++) fb[c] = floor_bits(__fadd_rn(__fmul_rn(__fsub_rn(x[c], z), inv), 0.5f));
 #pragma unroll
       for (int c4 = 0; c4 < 4; c4++)
         wq[c4] = __byte_perm(__byte_perm(fb[4 * c4], fb[4 * c4 + 1], 0x0040),
-                             __byte_perm(fb[4 * c4 + 2], fb[4 * c4 + 3], 0x0040), 0x5410);
+                             __byte_perm(fb[4 * c4 + 2], fb[4 * c4 + 3], 0x0040), 0x5410) &
+                 (qmax * 0x01010101u);
     }
     *reinterpret_cast<uint4*>(&cs[wib][tok][16 * sub]) = make_uint4(wq[0], wq[1], wq[2], wq[3]);  // one byte per channel
     if (sub == 0) ms[wib][tok] = (uint32_t)__half_as_ushort(rh) | ((uint32_t)__half_as_ushort(zh) << 16);

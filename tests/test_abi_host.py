@@ -221,3 +221,26 @@ def test_key_channel_option_host_side(kvq):
         assert lib.kvq_export_window(h, 0, 2, 0, None, None, None, None, C.byref(n), None) == 1  # stream
     finally:
         kvq.kvq_free(h)
+
+
+def test_injected_allocation_failure(kvq, monkeypatch):
+    """KVQ_FAULT_ALLOC makes the library's own pool allocation fail on the
+    host, before any CUDA call: kvq_alloc returns KVQ_ERR_OOM, hands back no
+    cache and says the failure was injected; a caller-owned pool is not
+    affected (the library allocates nothing then), and "0" turns it off."""
+    lib = kvq.load()
+    fb = (C.c_int * 1)(4)
+    monkeypatch.setenv("KVQ_FAULT_ALLOC", "1")
+    h = C.c_void_p(1234)
+    assert lib.kvq_alloc(C.byref(h), 1, 1, 2, 128, 1_114_112, fb, None, 0) == 4
+    assert h.value is None
+    msg = kvq.kvq_last_error()
+    assert "injected" in msg and "KVQ_FAULT_ALLOC" in msg
+    hc, pool = _host_cache(kvq)  # caller pool: succeeds with the hook set
+    kvq.kvq_free(hc)
+    monkeypatch.setenv("KVQ_FAULT_ALLOC", "0")
+    st = lib.kvq_alloc(C.byref(h), 1, 1, 2, 128, 1_114_112, fb, None, 0)
+    if st == 0:  # a GPU is present: the real allocation went through
+        kvq.kvq_free(h)
+    else:
+        assert st == 4 and "injected" not in kvq.kvq_last_error()

@@ -22,18 +22,28 @@ def test_code_tokens_keeps_literals():
 
 
 def test_recorded_traffic_follows_kernel_code():
-    """The committed decode profile's counters are used only while its
-    recorded digest matches the kernel code in the tree."""
+    """The committed decode traffic record is used only while its recorded
+    digest matches the kernel code in the tree."""
     import json
-    path = os.path.join(bench.ROOT, "profiles", "decode_kernel_7b_b16_t32k.md")
-    with open(path) as f:
-        rec = json.loads(next(l for l in f if l.startswith("traffic-json: "))[14:])
+    with open(bench.TRAFFIC_FILE) as f:
+        rec = json.load(f)
     bytes_, src = bench.decode_traffic([2, 4])
     if rec["source_digest"] == bench.source_digest():
         per = rec["bytes_per_launch"]
         assert bytes_ == (per["2bit"] + per["4bit"]) // 2
     else:
         assert bytes_ is None and "changed" in src
+
+
+def test_traffic_record_missing_or_other_kernel(tmp_path):
+    import json
+    assert bench.decode_traffic([2], path=str(tmp_path / "absent.json"))[0] is None
+    p = tmp_path / "t.json"
+    p.write_text(json.dumps({"source_digest": bench.source_digest(), "bytes_per_launch": {"2bit": 10, "4bit": 30}}))
+    assert bench.decode_traffic([2, 4, 4], path=str(p)) == (23, "profiles/decode_traffic.json")
+    assert bench.decode_traffic([8], path=str(p))[0] is None
+    p.write_text(json.dumps({"source_digest": "0" * 16, "bytes_per_launch": {"2bit": 10}}))
+    assert bench.decode_traffic([2], path=str(p))[0] is None
 
 
 def test_host_cores_respects_quota_and_cap(tmp_path):

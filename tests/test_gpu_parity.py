@@ -258,6 +258,49 @@ def test_empty_block_and_full_budget_edges(kvq, orc):
     P.check_attention(q)
 
 
+@pytest.mark.parametrize("fbit", [2, 4])
+@pytest.mark.parametrize("bad", [float("inf"), -70000.0])
+def test_group_append_contains_a_non_finite_group(kvq, orc, fbit, bad):
+    """A chunk taken in group mode holds groups outside the append contract:
+    a Value with an infinite channel (R = inf, NaN scaled values) or a minimum
+    below -65504 (Z = -inf), and a Key with an infinite channel.  Their own
+    codes are unspecified; every other token's codes and meta must equal the
+    oracle's (fed the finite originals) and a one-token-at-a-time append of the
+    same chunk."""
+    B, H, n_f = 1, 2, 4096
+    pre = n_f // 2  # the capacity at 2 * fbit bits: the chunk shrinks the block to fbit first
+    k, v = S.keys_values(23, fbit, B, pre + 48, H, 0, 3, dtype=torch.float32)
+    P = Pair(kvq, orc, B, H, n_f, fbit, None)
+    one = kvq.KVQCache(1, B, H, n_f * per_token(B, H, [fbit]), [fbit])
+    P.append(k[:, :pre], v[:, :pre])
+    one.append(0, k[:, :pre].cuda(), v[:, :pre].cuda())
+    kb, vb = k[:, pre:].clone(), v[:, pre:].clone()
+    bad_v, bad_k = 21, 30  # tokens of the chunk; the V of token 21 shares its words with token 20's
+    vb[0, bad_v, 1, 9] = bad
+    kb[0, bad_k, 0, 3] = float("inf")
+    P.gpu.append(0, kb.cuda(), vb.cuda())  # the non-finite chunk goes to the GPU only
+    assert P.orc.append(k[:, pre:].numpy(), v[:, pre:].numpy(), None) == 0
+    for t in range(48):
+        one.append(0, kb[:, t:t + 1].cuda(), vb[:, t:t + 1].cuda())
+    torch.cuda.synchronize()
+    assert P.gpu.query(0)["bits"] == fbit and P.gpu.query(0)["tokens"] == pre + 48
+    okc, ovc, okm, ovm = P.orc.k_codes(), P.orc.v_codes(), P.orc.k_meta(), P.orc.v_meta()
+    for j in range(H):
+        kc, vc, km, vm = P.gpu.export(0, 0, j)
+        kc1, vc1, km1, vm1 = one.export(0, 0, j)
+        keep_k = np.ones(pre + 48, bool)
+        keep_v = np.ones(pre + 48, bool)
+        if j == 0:
+            keep_k[pre + bad_k] = False
+        if j == 1:
+            keep_v[pre + bad_v] = False
+        for got, ref, keep in ((kc, okc[0, j], keep_k), (km, okm[0, j], keep_k), (vc, ovc[0, j], keep_v),
+                               (vm, ovm[0, j], keep_v), (kc1, okc[0, j], keep_k), (vc1, ovc[0, j], keep_v)):
+            assert np.array_equal(got[keep], ref[keep])
+        assert int(vc[~keep_v].max(initial=0)) < (1 << fbit) and int(kc[~keep_k].max(initial=0)) < (1 << fbit)
+    one.free()
+
+
 # ---------------------------------------------------- Direct Right Shift (ablation)
 
 def test_direct_shift_tiny_config_one_by_one(kvq, orc):
