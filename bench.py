@@ -115,12 +115,12 @@ def code_tokens(text):
 
 
 def source_digest():
-    """sha256 of the decode kernel's code (kvq_decode.cu + kvq_internal.cuh,
-    comments and whitespace removed): ncu counters stay valid only while it
+    """sha256 of the decode kernel's code (kvq_decode.cu, kvq_decode_common.cuh
+    and kvq_internal.cuh, comments and whitespace removed): ncu counters stay valid only while it
     matches the digest recorded with them."""
     import hashlib
     h = hashlib.sha256()
-    for name in ("kvq_decode.cu", "kvq_internal.cuh"):
+    for name in ("kvq_decode.cu", "kvq_decode_common.cuh", "kvq_internal.cuh"):
         with open(os.path.join(ROOT, "mixed_precision_kv_kvq_b200", "csrc", name)) as f:
             h.update(code_tokens(f.read()).encode())
     return h.hexdigest()[:16]

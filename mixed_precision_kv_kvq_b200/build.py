@@ -28,7 +28,7 @@ def _nvcc() -> str:
 
 def build(force: bool = False, verbose: bool = False) -> Path:
     srcs = [CSRC / s for s in SOURCES]
-    deps = srcs + [CSRC / "kvq_internal.cuh", CSRC / "kvq_quant.cuh", ROOT / "include" / "kvq.h"]
+    deps = srcs + [CSRC / "kvq_internal.cuh", CSRC / "kvq_quant.cuh", CSRC / "kvq_decode_common.cuh", ROOT / "include" / "kvq.h"]
     if not force and LIB.exists() and all(LIB.stat().st_mtime >= d.stat().st_mtime for d in deps):
         return LIB
     tmp = LIB.with_suffix(f".so.{os.getpid()}")

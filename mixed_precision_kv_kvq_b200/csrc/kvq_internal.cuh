@@ -284,6 +284,7 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 cudaError_t launch_block_move(const BlockMoveArgs& a, int n_streams, cudaStream_t s);
 cudaError_t launch_shrink(const ShrinkArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+
 cudaError_t launch_wait_probe(int* err, cudaStream_t s);
 
 }  // namespace kvq
