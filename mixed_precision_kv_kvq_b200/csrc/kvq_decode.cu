@@ -243,7 +243,8 @@ __device__ __forceinline__ void pv_groups(const uint32_t* const (&vu)[NG], const
 
 // Online-softmax state of one warp for the heads 2t, 2t+1 of its lanes.
 struct Soft {
-  float m0, m1, l0, l1, pz0, pz1;
+  float m0, m1;
+  float2 l, pz;  // heads 2t, 2t+1
   float o[8][4];
 };
 
@@ -274,20 +275,23 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
   const float me0 = st.m0 == -INFINITY ? 0.f : st.m0, me1 = st.m1 == -INFINITY ? 0.f : st.m1;
   float x[NG][4], zv[NG][2];
   uint32_t rv2[NG][2];  // (R^V, R^V) of tokens g and g+8 as half2
+  const float2 ks = make_float2(ks0, ks1), sg = make_float2(sig0, sig1), nme = make_float2(-me0, -me1);
 #pragma unroll
   for (int n = 0; n < NG; n++) {
     const uint2 mga = ms[n * 16 + g], mgb = ms[n * 16 + g + 8];
     const float2 ka = CHAN ? make_float2(1.f, 1.f) : __half22float2(*reinterpret_cast<const __half2*>(&mga.x));
     const float2 kb = CHAN ? make_float2(1.f, 1.f) : __half22float2(*reinterpret_cast<const __half2*>(&mgb.x));
-    x[n][0] = fmaf(ka.x * ks0, d[n][0], fmaf(ka.y, sig0, -me0));  // token g,   head 2t
-    x[n][1] = fmaf(ka.x * ks1, d[n][1], fmaf(ka.y, sig1, -me1));  // token g,   head 2t+1
-    x[n][2] = fmaf(kb.x * ks0, d[n][2], fmaf(kb.y, sig0, -me0));  // token g+8, head 2t
-    x[n][3] = fmaf(kb.x * ks1, d[n][3], fmaf(kb.y, sig1, -me1));  // token g+8, head 2t+1
-    // Value zero moved by the centring of the codes: Z + R 2^(b-1) / (2^b - 1)
+    // heads 2t, 2t+1 at once: x = (R ks) d + (Z sig - m), the same IEEE steps as one head at a time
+    const float2 xa = fma2(mul2(splat2(ka.x), ks), make_float2(d[n][0], d[n][1]), fma2(splat2(ka.y), sg, nme));  // token g
+    const float2 xb = fma2(mul2(splat2(kb.x), ks), make_float2(d[n][2], d[n][3]), fma2(splat2(kb.y), sg, nme));  // token g+8
+    x[n][0] = xa.x; x[n][1] = xa.y;
+    x[n][2] = xb.x; x[n][3] = xb.y;
+    // Value zero moved by the centring of the codes: Z + R 2^(b-1) / (2^b - 1), both tokens at once
     const float2 va = __half22float2(*reinterpret_cast<const __half2*>(&mga.y));
     const float2 vb = __half22float2(*reinterpret_cast<const __half2*>(&mgb.y));
-    zv[n][0] = fmaf(va.x, kVMid, va.y);
-    zv[n][1] = fmaf(vb.x, kVMid, vb.y);
+    const float2 z2 = fma2(make_float2(va.x, vb.x), splat2(kVMid), make_float2(va.y, vb.y));
+    zv[n][0] = z2.x;
+    zv[n][1] = z2.y;
     rv2[n][0] = __byte_perm(mga.y, 0, 0x1010);  // low half twice
     rv2[n][1] = __byte_perm(mgb.y, 0, 0x1010);
   }
@@ -334,8 +338,8 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
       st.o[sb][0] *= a0; st.o[sb][2] *= a0;
       st.o[sb][1] *= a1; st.o[sb][3] *= a1;
     }
-    st.l0 *= a0; st.pz0 *= a0;
-    st.l1 *= a1; st.pz1 *= a1;
+    st.l = mul2(st.l, make_float2(a0, a1));
+    st.pz = mul2(st.pz, make_float2(a0, a1));
     st.m0 = me0 + d0;
     st.m1 = me1 + d1;
 #pragma unroll
@@ -349,10 +353,9 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
   for (int n = 0; n < NG; n++) {
     const float p00 = ex2(x[n][0]), p01 = ex2(x[n][1]);
     const float p10 = ex2(x[n][2]), p11 = ex2(x[n][3]);
-    st.l0 += p00 + p10;
-    st.l1 += p01 + p11;
-    st.pz0 = fmaf(p00, zv[n][0], fmaf(p10, zv[n][1], st.pz0));
-    st.pz1 = fmaf(p01, zv[n][0], fmaf(p11, zv[n][1], st.pz1));
+    const float2 pa = make_float2(p00, p01), pb = make_float2(p10, p11);  // tokens g, g+8
+    st.l = add2(st.l, add2(pa, pb));
+    st.pz = fma2(pa, splat2(zv[n][0]), fma2(pb, splat2(zv[n][1]), st.pz));
     // P = p R^V in fp16, transposed to the B fragment (tokens 2t, 2t+1 / 2t+8, 2t+9 of head g)
     b0[n] = movmatrix_t(hmul2_u(pack_h2(p00, p01), rv2[n][0]));
     b1[n] = movmatrix_t(hmul2_u(pack_h2(p10, p11), rv2[n][1]));
@@ -732,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
 
   Soft sm;
   sm.m0 = sm.m1 = -INFINITY;
-  sm.l0 = sm.l1 = sm.pz0 = sm.pz1 = 0.f;
+  sm.l = sm.pz = make_float2(0.f, 0.f);
 #pragma unroll
   for (int sb = 0; sb < 8; sb++) sm.o[sb][0] = sm.o[sb][1] = sm.o[sb][2] = sm.o[sb][3] = 0.f;
 
@@ -782,7 +785,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     }
     __syncwarp();  // every lane is done with this stage before lane 0 refills it
   }
-  float m0 = sm.m0, m1 = sm.m1, l0 = sm.l0, l1 = sm.l1, pz0 = sm.pz0, pz1 = sm.pz1;
+  float m0 = sm.m0, m1 = sm.m1, l0 = sm.l.x, l1 = sm.l.y, pz0 = sm.pz.x, pz1 = sm.pz.y;
   float (&o)[8][4] = sm.o;
 
   if (!a.trigger_early) pdl_launch_dependents();  // the next kernel may start to launch while this one merges

@@ -190,6 +190,27 @@ __device__ __forceinline__ uint32_t pair_at(const uint32_t* u, const uint32_t* u
   return widen<BITS, p % ppw>(u[wi], u8[wi]);
 }
 
+// Packed fp32 pairs (add / mul / fma .f32x2): one instruction for the two
+// heads a lane holds, each lane an ordinary IEEE round-to-nearest operation.
+__device__ __forceinline__ unsigned long long f2_bits(float2 v) { return *reinterpret_cast<unsigned long long*>(&v); }
+__device__ __forceinline__ float2 f2_from(unsigned long long b) { return *reinterpret_cast<float2*>(&b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_from(d);
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_from(d);
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return f2_from(d);
+}
+__device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
+
 // Key quads.  A quad is the 4 codes of one token at 4 consecutive Key
 // positions, one int8 A-fragment register of mma.m16n8k32; member i sits in
 // byte i of its word at the quad's field (kvq_internal.cuh).  quad_reg gives

@@ -124,6 +124,10 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_kernel(uint8_t* codes, 
   // u = i and u = i + 256 from input uint4 2u and 2u + 1.
   uint4* tile = reinterpret_cast<uint4*>(codes + (size_t)blockIdx.x * kTileBytes);
   const int i = threadIdx.x;
+  // Launched with programmatic dependent launch so its launch overlaps the
+  // previous kernel's tail; it waits for that kernel before touching the
+  // block, and never triggers its dependents early (they start when it ends).
+  pdl_wait();
   uint4 in[4];
   in[0] = __ldcs(tile + 2 * i);
   in[1] = __ldcs(tile + 2 * i + 1);
@@ -150,11 +154,9 @@ __global__ void __launch_bounds__(kShrinkThreads) shrink_kernel(uint8_t* codes, 
 
 template <int BTO>
 cudaError_t launch_to(const ShrinkArgs& a, unsigned grid, cudaStream_t s) {
-  if (a.direct)
-    shrink_kernel<BTO, Drs><<<grid, kShrinkThreads, 0, s>>>(a.codes, a.meta, a.pf, a.p_from, a.kmc, a.kmc_words);
-  else
-    shrink_kernel<BTO, Ers><<<grid, kShrinkThreads, 0, s>>>(a.codes, a.meta, a.pf, a.p_from, nullptr, 0);
-  return cudaGetLastError();
+  const dim3 g(grid), blk(kShrinkThreads);
+  if (a.direct) return launch_pdl(shrink_kernel<BTO, Drs>, g, blk, 0, s, a.codes, a.meta, a.pf, a.p_from, a.kmc, a.kmc_words);
+  return launch_pdl(shrink_kernel<BTO, Ers>, g, blk, 0, s, a.codes, a.meta, a.pf, a.p_from, (uint32_t*)nullptr, 0LL);
 }
 
 }  // namespace
