@@ -177,6 +177,30 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 __device__ __forceinline__ uint32_t floor_bits(float y) {
   return __float_as_uint(__fadd_rd(y, 8388608.0f));
 }
+// Packed fp32 pairs: one instruction for two values, each lane the IEEE
+// operation with the named rounding (round-to-nearest, or down for add2f_rd).
+__device__ __forceinline__ unsigned long long f2u(float2 v) { return *reinterpret_cast<unsigned long long*>(&v); }
+__device__ __forceinline__ float2 u2f(unsigned long long b) { return *reinterpret_cast<float2*>(&b); }
+__device__ __forceinline__ float2 sub2f(float2 a, float2 b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
+  return u2f(d);
+}
+__device__ __forceinline__ float2 mul2f(float2 a, float2 b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
+  return u2f(d);
+}
+__device__ __forceinline__ float2 add2f(float2 a, float2 b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
+  return u2f(d);
+}
+__device__ __forceinline__ float2 add2f_rd(float2 a, float2 b) {
+  unsigned long long d;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
+  return u2f(d);
+}
 template <int BITS>
 __global__ void __launch_bounds__(kGroupWarps * 32) append_group_kernel(AppendArgs a) {
   static_assert(BITS <= 8, "16-bit codes take the per-token path");
@@ -248,9 +272,13 @@ __global__ void __launch_bounds__(kGroupWarps * 32) append_group_kernel(AppendAr
         }
       }
     }
-    if (mig) {
+    if (mig) {  // channel pairs at once: each an IEEE fp32 product, as x * lambda^-1 alone
 #pragma unroll
-      for (int c = 0; c < 16; c++) x[c] = __fmul_rn(x[c], li[c]);
+      for (int c = 0; c < 16; c += 2) {
+        const float2 y = mul2f(make_float2(x[c], x[c + 1]), make_float2(li[c], li[c + 1]));
+        x[c] = y.x;
+        x[c + 1] = y.y;
+      }
     }
     // the quantizer of kvq_quant.cuh over the token's 8 lanes, codes kept in registers
     float mn = fminf(fmin3(fmin3(x[0], x[1], x[2]), fmin3(x[3], x[4], x[5]), fmin3(x[6], x[7], x[8])),
@@ -279,9 +307,16 @@ __global__ void __launch_bounds__(kGroupWarps * 32) append_group_kernel(AppendAr
       // Z = -inf) can yield NaN, whose low byte is 0xff: the mask keeps every
       // byte inside its b-bit field, so such a group's codes, unspecified as
       // they are, never reach the fields of the tokens packed beside them.
+      // channel pairs at once (packed f32x2): the same four IEEE steps per value
       uint32_t fb[16];
+      const float2 z2 = make_float2(z, z), inv2 = make_float2(inv, inv);
 #pragma unroll
-      for (int c = 0; c < 16; c++) fb[c] = floor_bits(__fadd_rn(__fmul_rn(__fsub_rn(x[c], z), inv), 0.5f));
+      for (int c = 0; c < 16; c += 2) {
+        const float2 y = add2f(mul2f(sub2f(make_float2(x[c], x[c + 1]), z2), inv2), make_float2(0.5f, 0.5f));
+        const float2 fl = add2f_rd(y, make_float2(8388608.0f, 8388608.0f));
+        fb[c] = __float_as_uint(fl.x);
+        fb[c + 1] = __float_as_uint(fl.y);
+      }
 #pragma unroll
       for (int c4 = 0; c4 < 4; c4++)
         wq[c4] = __byte_perm(__byte_perm(fb[4 * c4], fb[4 * c4 + 1], 0x0040),
