@@ -264,11 +264,13 @@ def measure_shrink(kvq, dev, flush_buf, blocks_7b=20, blocks_70b=3):
         flush_l2(flush_buf)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.nvtx.range_push("timed")
         e0.record(stream)
         for l in range(blocks):
             cache.shrink(l)
         e1.record(stream)
         torch.cuda.synchronize(dev)
+        torch.cuda.nvtx.range_pop()
         cache.device_status()
         t = e0.elapsed_time(e1) / 1e3 / blocks
         bits_from = st[0]["bits"]
@@ -287,28 +289,39 @@ def measure_shrink(kvq, dev, flush_buf, blocks_7b=20, blocks_70b=3):
     return res
 
 
-def measure_append_chunk(kvq, dev, flush_buf, reps=3):
-    """Chunked append of 4096 tokens (7B shape, batch 8) at 2 bits."""
-    batch, kv_heads, n_f = 8, 4, 65536
-    # past the 4 -> 2 shrink at 32768 tokens, with room for the timed chunks
-    cache = build_cache(kvq, dev, 1, batch, kv_heads, [2], 40960, n_f, SEED + 5, 5, chunk=8192)
+def measure_append_chunk(kvq, dev, flush_buf, reps=15):
+    """Chunked appends of 4096 tokens (7B shape, batch 8, 4 KV heads) into a
+    2-bit block: `reps` back-to-back calls, each with its own input chunk (so
+    every input is read from HBM), CUDA events around the batch after an L2
+    flush; time per call."""
+    batch, kv_heads, n = 8, 4, 4096
+    n_f = 131072
+    pre = n_f // 2 + n  # past the 4 -> 2 shrink at n_f / 2 tokens
+    assert pre + reps * n <= n_f
+    cache = build_cache(kvq, dev, 1, batch, kv_heads, [2], pre, n_f, SEED + 5, 5, chunk=8192)
     st = cache.query(0)
-    k, v = S.keys_values(SEED, 99, batch, 4096, kv_heads, 0, 5, dtype=torch.bfloat16, device=dev)
-    times = []
-    for r in range(reps):
-        flush_l2(flush_buf)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
+    assert st["bits"] == 2
+    chunks = [S.keys_values(SEED, 99, batch, n, kv_heads, pre + r * n, 5, dtype=torch.bfloat16, device=dev)
+              for r in range(reps)]
+    torch.cuda.synchronize(dev)
+    flush_l2(flush_buf)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("timed")
+    e0.record(stream)
+    for k, v in chunks:
         cache.append(0, k, v)
-        e1.record()
-        torch.cuda.synchronize(dev)
-        times.append(e0.elapsed_time(e1) / 1e3)
-    bits = cache.query(0)["bits"]
-    assert bits == st["bits"]
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    torch.cuda.nvtx.range_pop()
+    cache.device_status()
+    assert cache.query(0)["bits"] == 2 and cache.query(0)["tokens"] == pre + reps * n
     cache.free()
-    nb = append_bytes(batch, kv_heads, 4096, bits)
-    t = statistics.median(times)
-    return {"gbs": nb / t / 1e9, "us": t * 1e6, "bytes": nb, "bits": bits, "tokens": 4096, "batch": batch}
+    nb = append_bytes(batch, kv_heads, n, 2)
+    t = e0.elapsed_time(e1) / 1e3 / reps
+    return {"gbs": round(nb / t / 1e9, 1), "us": round(t * 1e6, 2), "bytes": nb, "bits": 2, "tokens": n,
+            "batch": batch, "timing": f"{reps} back-to-back appends of distinct chunks after an L2 flush, CUDA events "
+                                      "around the batch, time per call"}
 
 
 def max_over_ranks(ms: float, world: int, device) -> float:
@@ -1006,6 +1019,9 @@ def run_part(args):
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
+    if args.part == "append":
+        flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        return {"part": "append", **measure_append_chunk(kvq, dev, flush)}
     if args.part == "shrink":
         flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
         n = args.shrink_blocks
@@ -1026,8 +1042,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--no-70b", action="store_true", help="skip the Llama-70B decode step")
-    ap.add_argument("--part", choices=["all", "shrink", "step70b"], default="all",
-                    help="run one measurement alone (profiling cases): the shrink events or the 70B step")
+    ap.add_argument("--part", choices=["all", "shrink", "append", "step70b"], default="all",
+                    help="run one measurement alone (profiling cases): the shrink events, the chunked append or "
+                         "the 70B step")
     ap.add_argument("--shrink-blocks", type=int, default=0,
                     help="with --part shrink: blocks per event (0: 20 for the 7B events, 3 for the 70B ones)")
     args = ap.parse_args()

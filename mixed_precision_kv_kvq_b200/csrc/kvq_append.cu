@@ -177,30 +177,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 __device__ __forceinline__ uint32_t floor_bits(float y) {
   return __float_as_uint(__fadd_rd(y, 8388608.0f));
 }
-// Packed fp32 pairs: one instruction for two values, each lane the IEEE
-// operation with the named rounding (round-to-nearest, or down for add2f_rd).
-__device__ __forceinline__ unsigned long long f2u(float2 v) { return *reinterpret_cast<unsigned long long*>(&v); }
-__device__ __forceinline__ float2 u2f(unsigned long long b) { return *reinterpret_cast<float2*>(&b); }
-__device__ __forceinline__ float2 sub2f(float2 a, float2 b) {
-  unsigned long long d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
-  return u2f(d);
-}
-__device__ __forceinline__ float2 mul2f(float2 a, float2 b) {
-  unsigned long long d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
-  return u2f(d);
-}
-__device__ __forceinline__ float2 add2f(float2 a, float2 b) {
-  unsigned long long d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
-  return u2f(d);
-}
-__device__ __forceinline__ float2 add2f_rd(float2 a, float2 b) {
-  unsigned long long d;
-  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
-  return u2f(d);
-}
 template <int BITS>
 __global__ void __launch_bounds__(kGroupWarps * 32) append_group_kernel(AppendArgs a) {
   static_assert(BITS <= 8, "16-bit codes take the per-token path");
@@ -272,13 +248,9 @@ __global__ void __launch_bounds__(kGroupWarps * 32) append_group_kernel(AppendAr
         }
       }
     }
-    if (mig) {  // channel pairs at once: each an IEEE fp32 product, as x * lambda^-1 alone
+    if (mig) {
 #pragma unroll
-      for (int c = 0; c < 16; c += 2) {
-        const float2 y = mul2f(make_float2(x[c], x[c + 1]), make_float2(li[c], li[c + 1]));
-        x[c] = y.x;
-        x[c + 1] = y.y;
-      }
+      for (int c = 0; c < 16; c++) x[c] = __fmul_rn(x[c], li[c]);
     }
     // the quantizer of kvq_quant.cuh over the token's 8 lanes, codes kept in registers
     float mn = fminf(fmin3(fmin3(x[0], x[1], x[2]), fmin3(x[3], x[4], x[5]), fmin3(x[6], x[7], x[8])),
@@ -307,16 +279,9 @@ __global__ void __launch_bounds__(kGroupWarps * 32) append_group_kernel(AppendAr
       // Z = -inf) can yield NaN, whose low byte is 0xff: the mask keeps every
       // byte inside its b-bit field, so such a group's codes, unspecified as
       // they are, never reach the fields of the tokens packed beside them.
-      // channel pairs at once (packed f32x2): the same four IEEE steps per value
       uint32_t fb[16];
-      const float2 z2 = make_float2(z, z), inv2 = make_float2(inv, inv);
 #pragma unroll
-      for (int c = 0; c < 16; c += 2) {
-        const float2 y = add2f(mul2f(sub2f(make_float2(x[c], x[c + 1]), z2), inv2), make_float2(0.5f, 0.5f));
-        const float2 fl = add2f_rd(y, make_float2(8388608.0f, 8388608.0f));
-        fb[c] = __float_as_uint(fl.x);
-        fb[c + 1] = __float_as_uint(fl.y);
-      }
+      for (int c = 0; c < 16; c++) fb[c] = floor_bits(__fadd_rn(__fmul_rn(__fsub_rn(x[c], z), inv), 0.5f));
 #pragma unroll
       for (int c4 = 0; c4 < 4; c4++)
         wq[c4] = __byte_perm(__byte_perm(fb[4 * c4], fb[4 * c4 + 1], 0x0040),
@@ -380,21 +345,29 @@ __global__ void __launch_bounds__(kGroupWarps * 32) append_group_kernel(AppendAr
 // INT16 Key is read back in fp32 as Z + code * (R / 65535) and each channel's
 // 128 values go through the quantizer of kvq_quant.cuh; Values: each token's
 // INT16 codes take the block's shift chain, R and Z kept (R rescaled by the
-// direct shift).  One CTA of 512 threads per stream: warps unpack and pack 8
-// tokens each; for the channels, thread (quarter, c) covers tokens
-// 32 quarter .. +31 of channel c and the quarters combine their min / max.
-constexpr int kMoveThreads = 512;
+// direct shift).  Six CTAs of 256 threads per stream: two take the Keys of
+// one half of the channels each (a half's codes fill whole words of the
+// packed layout at every width, so the two never write the same word), four
+// take the Values of 32 tokens each.  In a Key CTA thread (quarter, c) finds
+// channel c's min / max over tokens 32 quarter .. +31 and the quarters
+// combine them.
+constexpr int kMoveThreads = 256;
 constexpr int kMoveWarps = kMoveThreads / 32;
+constexpr int kMoveRoles = 6;  // 2 Key halves, 4 Value quarters
+constexpr int kHalf = kHeadDim / 2;
+struct MoveKeySmem {
+  uint16_t kc[kKeyBlock][kHalf];       // [token][channel of the half]: INT16 codes, then the new codes
+  float z[kKeyBlock], step[kKeyBlock];  // staged Keys: Z and R / 65535 of each token
+  float mn[4][kHalf], mx[4][kHalf];
+};
 template <int BITS>
 __global__ void __launch_bounds__(kMoveThreads) block_move_kernel(BlockMoveArgs a) {
-  __shared__ uint16_t kc_sh[kKeyBlock][kHeadDim];  // [token][channel]: INT16 codes, then the new codes
-  __shared__ float z_sh[kKeyBlock], step_sh[kKeyBlock];  // staged Keys: Z and R / 65535 of each token
-  __shared__ float mn_sh[4][kHeadDim], mx_sh[4][kHeadDim];
-  __shared__ uint16_t vc_sh[kMoveWarps][kHeadDim];
+  __shared__ __align__(16) uint8_t sm_raw[sizeof(MoveKeySmem)];
   pdl_wait();
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const size_t stream = blockIdx.x;
+  const size_t stream = blockIdx.x / kMoveRoles;
+  const int role = (int)(blockIdx.x % kMoveRoles);
   constexpr int P16 = slots_per_tile(16);
   auto staged = [&](int t, int kv) {  // group part holding staged token t
     return a.wcodes + (stream * kWindowTiles + t / P16) * (size_t)kTileBytes +
@@ -403,30 +376,63 @@ __global__ void __launch_bounds__(kMoveThreads) block_move_kernel(BlockMoveArgs 
   auto staged_meta = [&](int t, int kv) {
     return ((stream * kWindowTiles + t / P16) * (size_t)P16 + t % P16) * 2 + kv;
   };
-  for (int t = warp; t < kKeyBlock; t += kMoveWarps) {
-    unpack_codes16(staged(t, 0), t & 15, 0, kc_sh[t], lane);
-    if (lane == 0) {
-      const uint32_t w = a.wmeta[staged_meta(t, 0)];
-      z_sh[t] = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
-      step_sh[t] = __fdiv_rn(__half2float(__ushort_as_half((unsigned short)(w & 0xffffu))), 65535.0f);
+  if (role >= 2) {  // ---- Values of tokens 32 q .. 32 q + 31 ----
+    uint16_t* sc = reinterpret_cast<uint16_t*>(sm_raw) + warp * kHeadDim;
+    const int q = role - 2;
+    for (int t = 32 * q + warp; t < 32 * q + 32; t += kMoveWarps) {
+      const int gi = t >> 4, slot = a.g_slot[gi] + (t & 15);
+      const size_t tile = stream * a.nt + a.g_tile[gi];
+      uint8_t* gbase = a.codes + tile * kTileBytes + (size_t)(slot >> 4) * group_bytes(BITS);
+      unpack_codes16(staged(t, 1), t & 15, 1, sc, lane);
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 4; i++) sc[4 * lane + i] = (uint16_t)shift_chain<BITS>(sc[4 * lane + i], a.direct);
+      __syncwarp();
+      pack_codes<BITS>(gbase + part_bytes(BITS), slot & 15, 1, sc, lane);
+      if (lane == 0) {
+        const uint32_t old = a.wmeta[staged_meta(t, 1)];
+        a.meta[(tile * a.pf + slot) * 2 + 1] =
+            (uint32_t)range_chain<BITS>((uint16_t)(old & 0xffffu), a.direct) | (old & 0xffff0000u);
+      }
+      __syncwarp();  // sc is rewritten by the next token
     }
+    return;
+  }
+  // ---- Keys of channels 64 h .. 64 h + 63 ----
+  MoveKeySmem& sh = *reinterpret_cast<MoveKeySmem*>(sm_raw);
+  const int h = role;
+  // staged INT16 Key codes of the half: channel ch of token t is member i = ch % 4
+  // of quad p = 2 (ch / 32) + (ch / 16) % 2 in unit 4 (t % 8) + (ch / 4) % 4, word
+  // 16 x + 2 p + i / 2 (x = (t % 16) / 8), half-word i % 2 (the 16-bit layout)
+  for (int e = threadIdx.x; e < kKeyBlock * kHalf; e += kMoveThreads) {
+    const int t = e / kHalf, cc = e % kHalf, ch = kHalf * h + cc;
+    const int tok = t & 15, g = tok & 7, x = tok >> 3;
+    const int p = 2 * (ch >> 5) + ((ch >> 4) & 1), tt = (ch >> 2) & 3, mi = ch & 3;
+    const uint16_t* u16 = reinterpret_cast<const uint16_t*>(staged(t, 0));
+    sh.kc[t][cc] = u16[(4 * g + tt) * (unit_bytes(16) / 2) + 2 * (x * 16 + 2 * p + (mi >> 1)) + (mi & 1)];
+  }
+  if (threadIdx.x < kKeyBlock) {
+    const int t = threadIdx.x;
+    const uint32_t w = a.wmeta[staged_meta(t, 0)];
+    sh.z[t] = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+    sh.step[t] = __fdiv_rn(__half2float(__ushort_as_half((unsigned short)(w & 0xffffu))), 65535.0f);
   }
   __syncthreads();
   {
-    const int c = threadIdx.x & (kHeadDim - 1), qt = threadIdx.x >> 7;  // channel, token quarter
+    const int cc = threadIdx.x & (kHalf - 1), qt = threadIdx.x / kHalf;  // channel of the half, token quarter
     const int t0 = 32 * qt;
-    auto value = [&](int t) { return __fadd_rn(z_sh[t], __fmul_rn((float)kc_sh[t][c], step_sh[t])); };
+    auto value = [&](int t) { return __fadd_rn(sh.z[t], __fmul_rn((float)sh.kc[t][cc], sh.step[t])); };
     float mn = value(t0), mx = mn;
     for (int t = t0 + 1; t < t0 + 32; t++) {
       const float x = value(t);
       mn = fminf(mn, x);
       mx = fmaxf(mx, x);
     }
-    mn_sh[qt][c] = mn;
-    mx_sh[qt][c] = mx;
+    sh.mn[qt][cc] = mn;
+    sh.mx[qt][cc] = mx;
     __syncthreads();
-    mn = fminf(fminf(mn_sh[0][c], mn_sh[1][c]), fminf(mn_sh[2][c], mn_sh[3][c]));
-    mx = fmaxf(fmaxf(mx_sh[0][c], mx_sh[1][c]), fmaxf(mx_sh[2][c], mx_sh[3][c]));
+    mn = fminf(fminf(sh.mn[0][cc], sh.mn[1][cc]), fminf(sh.mn[2][cc], sh.mn[3][cc]));
+    mx = fmaxf(fmaxf(sh.mx[0][cc], sh.mx[1][cc]), fmaxf(sh.mx[2][cc], sh.mx[3][cc]));
     const __half zh = __float2half_rd(mn);
     const float z = __half2float(zh);
     const __half rh = __float2half_ru(__fsub_rn(mx, z));
@@ -439,31 +445,44 @@ __global__ void __launch_bounds__(kMoveThreads) block_move_kernel(BlockMoveArgs 
         const float y = __fadd_rn(__fmul_rn(__fsub_rn(value(t), z), inv), 0.5f);
         q = (uint16_t)min(__float2uint_rd(y), qmax);
       }
-      kc_sh[t][c] = q;  // only this thread reads or writes this token's channel c
+      sh.kc[t][cc] = q;  // only this thread reads or writes this token's channel cc
     }
     if (qt == 0)
-      a.kmc[(stream * a.blocks_max + a.blk) * kHeadDim + c] =
+      a.kmc[(stream * a.blocks_max + a.blk) * kHeadDim + kHalf * h + cc] =
           (uint32_t)__half_as_ushort(rh) | ((uint32_t)__half_as_ushort(zh) << 16);
   }
   __syncthreads();
-  uint16_t* sc = vc_sh[warp];
-  for (int t = warp; t < kKeyBlock; t += kMoveWarps) {
+  // the half's Key words of every token: unit 4 g + t4 of the token's group,
+  // words x b + jw for jw in [h b / 2, (h + 1) b / 2) (b <= 8; at 16 bits the
+  // half's quads 4h .. 4h + 3 fill words 8h .. 8h + 7); word x b + jw holds quads
+  // p = jw (8/b) + k at field k, member i (channel 32 (p/2) + 16 (p%2) + 4 t4 + i) in byte i
+  constexpr int kWords = BITS == 16 ? 8 : BITS / 2;  // per (token, unit) and half
+  for (int e = threadIdx.x; e < kKeyBlock * 4 * kWords; e += kMoveThreads) {
+    const int t = e / (4 * kWords), t4 = (e / kWords) % 4, wl = e % kWords;
     const int gi = t >> 4, slot = a.g_slot[gi] + (t & 15);
     const size_t tile = stream * a.nt + a.g_tile[gi];
-    uint8_t* gbase = a.codes + tile * kTileBytes + (size_t)(slot >> 4) * group_bytes(BITS);
-    pack_codes<BITS>(gbase, slot & 15, 0, kc_sh[t], lane);
-    unpack_codes16(staged(t, 1), t & 15, 1, sc, lane);
-    __syncwarp();
+    const int tok = slot & 15, g = tok & 7, x = tok >> 3;
+    uint32_t* unit = reinterpret_cast<uint32_t*>(a.codes + tile * kTileBytes + (size_t)(slot >> 4) * group_bytes(BITS) +
+                                                 (size_t)(4 * g + t4) * unit_bytes(BITS));
+    uint32_t word = 0;
+    int widx;
+    if constexpr (BITS == 16) {
+      const int wi = 8 * h + wl, p = wi >> 1, mi0 = 2 * (wi & 1);  // members mi0, mi0 + 1 as half-words
+      const int cb = 32 * (p >> 1) + 16 * (p & 1) + 4 * t4 - kHalf * h;
+      word = (uint32_t)sh.kc[t][cb + mi0] | ((uint32_t)sh.kc[t][cb + mi0 + 1] << 16);
+      widx = x * 16 + wi;
+    } else {
+      const int jw = h * (BITS / 2) + wl;
 #pragma unroll
-    for (int i = 0; i < 4; i++) sc[4 * lane + i] = (uint16_t)shift_chain<BITS>(sc[4 * lane + i], a.direct);
-    __syncwarp();
-    pack_codes<BITS>(gbase + part_bytes(BITS), slot & 15, 1, sc, lane);
-    if (lane == 0) {
-      const uint32_t old = a.wmeta[staged_meta(t, 1)];
-      a.meta[(tile * a.pf + slot) * 2 + 1] =
-          (uint32_t)range_chain<BITS>((uint16_t)(old & 0xffffu), a.direct) | (old & 0xffff0000u);
+      for (int k = 0; k < 8 / BITS; k++) {
+        const int p = jw * (8 / BITS) + k;
+        const int cb = 32 * (p >> 1) + 16 * (p & 1) + 4 * t4 - kHalf * h;
+#pragma unroll
+        for (int i = 0; i < 4; i++) word |= (uint32_t)sh.kc[t][cb + i] << (8 * i + BITS * k);
+      }
+      widx = x * BITS + jw;
     }
-    __syncwarp();  // sc is rewritten by the next token
+    unit[widx] = word;
   }
 }
 
@@ -471,7 +490,8 @@ __global__ void __launch_bounds__(kMoveThreads) block_move_kernel(BlockMoveArgs 
 
 cudaError_t launch_block_move(const BlockMoveArgs& a, int n_streams, cudaStream_t s) {
   if (n_streams <= 0) return cudaSuccess;
-  const dim3 grid((unsigned)n_streams), block(kMoveThreads);
+  if ((long long)n_streams * kMoveRoles > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const dim3 grid((unsigned)n_streams * kMoveRoles), block(kMoveThreads);
   switch (a.bits) {
     case 16: return launch_pdl(block_move_kernel<16>, grid, block, 0, s, a);
     case 8: return launch_pdl(block_move_kernel<8>, grid, block, 0, s, a);
