@@ -9,17 +9,18 @@
 // query).  Dequantisation is folded out of the inner loop:
 //   q'.k^_t = (R_t / (2^b-1)) (q'.c_t) + Z_t sum(q'),
 //   sum_t p_t v^_t = (sum_t p_t R_t (c_t - h)) / (2^b-1) + sum_t p_t Z'_t,
-//   h = 2^(b-1), Z'_t = Z_t + R_t h / (2^b-1)  (codes centred),
+//   h = 2^(b-1), Z'_t = Z_t + R_t h / (2^b-1)  (codes centred: the MMAs sum
+//   P_t c_t and the h sum_t P_t over the same fp16 P_t is taken off in fp32),
 // so the raw codes go straight into tensor-core operands:
 //   QK^T: int8 mma.sync.m16n8k32, A = 16 tokens x 32 Key channels of codes
 //   (byte quads, each code moved to the top of its byte: c 2^(8-b), exact in
 //   u8), B = the query as an exact per-head int16, q' = s_h (256 hi + lo)
 //   with hi s8 and lo u8, two MMAs on the same A registers, int32
 //   accumulation (no rounding until one int -> float conversion per score);
-//   PV: fp16 mma.sync.m16n8k16, A = 16 channels x 16 tokens of V codes
-//   widened in registers with the 0x6400 exponent trick (integer c in the
-//   low mantissa bits of 1024.0; one lop3 + one sub.f16x2 per code pair,
-//   which also subtracts h),
+//   PV: fp16 mma.sync.m16n8k16, A = 16 channels x 16 tokens of V codes,
+//   each pair masked in place by one AND and read as binary16 subnormals
+//   (c 2^(e-24): the code bits are the mantissa of a number whose exponent
+//   field is zero),
 //   B = p R (transposed from the score fragment with movmatrix).
 // 16-bit codes go in as two bytes (Keys) or two fp16 halves (Values).
 
@@ -250,8 +251,10 @@ struct Soft {
 
 // NG consecutive groups of one stage (cs, ms point at the first): scores,
 // one shared running-max update, probabilities, then P V.  valid0: valid
-// tokens from the first group on (FULL: all NG groups are full).
-template <int BITS, int NG, bool FULL, bool CHAN>
+// tokens from the first group on (FULL: all NG groups are full).  FIRST: the
+// warp's first group (no running max yet: scores are taken relative to 0 and
+// the max is set from them; o, l and pz are still zero).
+template <int BITS, int NG, bool FULL, bool CHAN, bool FIRST = false>
 __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* ms, int valid0, int lane,
                                                const uint4* qfl, const uint2* qfl3, float ks0, float ks1, float sig0,
                                                float sig1, Soft& st) {
@@ -271,8 +274,8 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
   // ks_h = (q' scale of head h) / (code scale).  Per-channel Key groups: the
   // block's ranges are inside the query operand and its zeros in sig, so
   // x = ks_h d + sig_h - m (R and Z of the token read as 1).
-  // Before the first group m is -inf; scores are then taken relative to 0.
-  const float me0 = st.m0 == -INFINITY ? 0.f : st.m0, me1 = st.m1 == -INFINITY ? 0.f : st.m1;
+  // The warp's first group takes its scores relative to 0.
+  const float me0 = FIRST ? 0.f : st.m0, me1 = FIRST ? 0.f : st.m1;
   float x[NG][4], zv[NG][2];
   uint32_t rv2[NG][2];  // (R^V, R^V) of tokens g and g+8 as half2
   const float2 ks = make_float2(ks0, ks1), sg = make_float2(sig0, sig1), nme = make_float2(-me0, -me1);
@@ -286,7 +289,7 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
     const float2 xb = fma2(mul2(splat2(kb.x), ks), make_float2(d[n][2], d[n][3]), fma2(splat2(kb.y), sg, nme));  // token g+8
     x[n][0] = xa.x; x[n][1] = xa.y;
     x[n][2] = xb.x; x[n][3] = xb.y;
-    // Value zero moved by the centring of the codes: Z + R 2^(b-1) / (2^b - 1), both tokens at once
+    // Value zero of tokens g, g+8 for centred codes: Z + R 2^(b-1) / (2^b - 1)
     const float2 va = __half22float2(*reinterpret_cast<const __half2*>(&mga.y));
     const float2 vb = __half22float2(*reinterpret_cast<const __half2*>(&mgb.y));
     const float2 z2 = fma2(make_float2(va.x, vb.x), splat2(kVMid), make_float2(va.y, vb.y));
@@ -323,23 +326,25 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
   // than kRebase (log2 units), so p = 2^(s - m) <= 2^kRebase.  Whether any
   // lane needs it is one vote; the maxima over the tokens are only formed
   // when it does.
-  if (__any_sync(0xffffffffu, (fmaxf(mx0, mx1) > kRebase) | (st.m0 == -INFINITY))) {
+  if (FIRST || __any_sync(0xffffffffu, fmaxf(mx0, mx1) > kRebase)) {
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
     }
-    // new max = old max + shift (exact for the first group: relative to 0)
-    const float d0 = st.m0 == -INFINITY ? mx0 : fmaxf(mx0, 0.f);
-    const float d1 = st.m1 == -INFINITY ? mx1 : fmaxf(mx1, 0.f);
-    const float a0 = ex2(-d0), a1 = ex2(-d1);  // 0 when the old max was -inf (o, l, pz are 0 then)
+    // new max = old max + shift (the first group: its own max, relative to 0)
+    const float d0 = FIRST ? mx0 : fmaxf(mx0, 0.f);
+    const float d1 = FIRST ? mx1 : fmaxf(mx1, 0.f);
+    if constexpr (!FIRST) {
+      const float a0 = ex2(-d0), a1 = ex2(-d1);  // in (0, 1]
 #pragma unroll
-    for (int sb = 0; sb < 8; sb++) {
-      st.o[sb][0] *= a0; st.o[sb][2] *= a0;
-      st.o[sb][1] *= a1; st.o[sb][3] *= a1;
+      for (int sb = 0; sb < 8; sb++) {
+        st.o[sb][0] *= a0; st.o[sb][2] *= a0;
+        st.o[sb][1] *= a1; st.o[sb][3] *= a1;
+      }
+      st.l = mul2(st.l, make_float2(a0, a1));
+      st.pz = mul2(st.pz, make_float2(a0, a1));
     }
-    st.l = mul2(st.l, make_float2(a0, a1));
-    st.pz = mul2(st.pz, make_float2(a0, a1));
     st.m0 = me0 + d0;
     st.m1 = me1 + d1;
 #pragma unroll
@@ -357,8 +362,16 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
     st.l = add2(st.l, add2(pa, pb));
     st.pz = fma2(pa, splat2(zv[n][0]), fma2(pb, splat2(zv[n][1]), st.pz));
     // P = p R^V in fp16, transposed to the B fragment (tokens 2t, 2t+1 / 2t+8, 2t+9 of head g)
-    b0[n] = movmatrix_t(hmul2_u(pack_h2(p00, p01), rv2[n][0]));
-    b1[n] = movmatrix_t(hmul2_u(pack_h2(p10, p11), rv2[n][1]));
+    const uint32_t Pa = hmul2_u(pack_h2(p00, p01), rv2[n][0]), Pb = hmul2_u(pack_h2(p10, p11), rv2[n][1]);
+    if constexpr (BITS <= 8) {
+      // the P V MMAs take the codes uncentred: sum_t P_t (c_t - h) = sum_t P_t c_t
+      // - h sum_t P_t, the second sum over the same fp16 P
+      const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&Pa));
+      const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&Pb));
+      st.pz = fma2(add2(fa, fb), splat2(-kVMid), st.pz);
+    }
+    b0[n] = movmatrix_t(Pa);
+    b1[n] = movmatrix_t(Pb);
   }
   pv_groups<BITS, NG>(vu, b0, b1, st.o);
 }
@@ -750,6 +763,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     if (!mbar_wait(bar0 + 8 * st, parity, a.err, flags)) break;
     const uint8_t* cs = my.code[st];
     const uint2* ms = reinterpret_cast<const uint2*>(my.meta[st]);
+    // the warp's first group (chunk 0 holds at least one) sets the running max
+    const int gi0 = ci == 0 ? 1 : 0;
     if constexpr (CHAN) {  // every group full; dsc.y is the chunk's 128-token block
       if (dsc.y != cur_blk) {
         cur_blk = dsc.y;
@@ -761,7 +776,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
         sig0 = wsig[2 * t];
         sig1 = wsig[2 * t + 1];
       }
-      int gi = 0;
+      if (ci == 0)
+        process_groups<BITS, 1, true, true, true>(cs, ms, 16, lane, qfl, qfl3, ks0, ks1, sig0, sig1, sm);
+      int gi = gi0;
       if constexpr (kChunkGroups >= 2) {
         for (; gi + 2 <= dsc.x; gi += 2)
           process_groups<BITS, 2, true, true>(cs + gi * kGroupBytes, ms + gi * 16, 32, lane, qfl, qfl3, ks0, ks1, sig0,
@@ -770,7 +787,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
       if (gi < dsc.x)
         process_groups<BITS, 1, true, true>(cs + gi * kGroupBytes, ms + gi * 16, 16, lane, qfl, qfl3, ks0, ks1, sig0,
                                             sig1, sm);
-    } else if (dsc.x == kChunkGroups && dsc.y >= 16 * kChunkGroups) {
+    } else if (ci > 0 && dsc.x == kChunkGroups && dsc.y >= 16 * kChunkGroups) {
       // full chunk: fixed offsets, no masking
       // unrolled: one pair's P V and the next pair's QK share a basic block
       constexpr int kNG = kChunkGroups >= 2 ? 2 : 1;
@@ -779,7 +796,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
         process_groups<BITS, kNG, true, false>(cs + gi * kGroupBytes, ms + gi * 16, 16 * kNG, lane, qfl, qfl3, ks0, ks1, sig0,
                                         sig1, sm);
     } else {
-      for (int gi = 0; gi < dsc.x; gi++)
+      if (ci == 0)
+        process_groups<BITS, 1, false, false, true>(cs, ms, dsc.y, lane, qfl, qfl3, ks0, ks1, sig0, sig1, sm);
+      for (int gi = gi0; gi < dsc.x; gi++)
         process_groups<BITS, 1, false, false>(cs + gi * kGroupBytes, ms + gi * 16, dsc.y - 16 * gi, lane, qfl, qfl3, ks0,
                                        ks1, sig0, sig1, sm);
     }
@@ -817,38 +836,49 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     float* ob = reinterpret_cast<float*>(my.code[0]);  // this warp's scaled o: [8][128]
 #pragma unroll
     for (int sb = 0; sb < 8; sb++) {
-      // rows 16sb+g (pair 2sb) and 16sb+g+8 (pair 2sb+1) carry 2^field_shift
-      const float r0 = 1.0f / (float)(1 << pair_shift<BITS>(2 * sb));
-      const float r1 = 1.0f / (float)(1 << pair_shift<BITS>(2 * sb + 1));
+      // rows 16sb+g (pair 2sb) and 16sb+g+8 (pair 2sb+1) carry 2^(field_shift - 24) at BITS <= 8
+      const float r0 = BITS == 16 ? 1.0f : (float)(1 << (24 - pair_shift<BITS>(2 * sb)));
+      const float r1 = BITS == 16 ? 1.0f : (float)(1 << (24 - pair_shift<BITS>(2 * sb + 1)));
       ob[(2 * t) * kHeadDim + 16 * sb + g] = sc0 * r0 * o[sb][0];
       ob[(2 * t + 1) * kHeadDim + 16 * sb + g] = sc1 * r0 * o[sb][1];
       ob[(2 * t) * kHeadDim + 16 * sb + g + 8] = sc0 * r1 * o[sb][2];
       ob[(2 * t + 1) * kHeadDim + 16 * sb + g + 8] = sc1 * r1 * o[sb][3];
     }
   }
-  __syncthreads();
-  // Final state of this CTA for every head h < G and channel c = thread:
-  //   M = max over warps, L and PZ = e^(m_w - M)-weighted sums, O = sum of the
-  //   warps' scaled rows (times 2^-e and 1/(2^b-1)) + PZ  (unnormalised).
-  const int c = threadIdx.x;  // one channel per thread
-  static_assert(kThreads == kHeadDim, "one channel per thread");
-  float Oc[kMaxGroup], Mh[kMaxGroup], Lh[kMaxGroup];
-#pragma unroll
-  for (int h = 0; h < kMaxGroup; h++) {
+  // Per head h (thread h): the CTA's max M over its warps and the
+  // e^(m_w - M)-weighted sums L and PZ, in warp 0's free second stage.
+  float* fin = reinterpret_cast<float*>(ws[0].code[1]);  // M[8], L[8], PZ[8]
+  if (threadIdx.x < kMaxGroup) {
+    const int h = threadIdx.x;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kWarps; w++) M = fmaxf(M, w_m[w * kMaxGroup + h]);
-    float L = 0.f, PZ = 0.f, O = 0.f;
+    float L = 0.f, PZ = 0.f;
 #pragma unroll
     for (int w = 0; w < kWarps; w++) {
       const float e = ex2(w_m[w * kMaxGroup + h] - M);
       L += e * w_l[w * kMaxGroup + h];
       PZ += e * w_pz[w * kMaxGroup + h];
-      O += reinterpret_cast<const float*>(ws[w].code[0])[h * kHeadDim + c];
     }
-    Oc[h] = O * kCScale + PZ;
-    Mh[h] = M;
-    Lh[h] = L;
+    fin[h] = M;
+    fin[kMaxGroup + h] = L;
+    fin[2 * kMaxGroup + h] = PZ;
+  }
+  __syncthreads();
+  // Final state of this CTA for every head h < G and channel c = thread:
+  //   O = sum of the warps' scaled rows (times 2^-e and 1/(2^b-1)) + PZ
+  //   (unnormalised), with the head's M and L.
+  const int c = threadIdx.x;  // one channel per thread
+  static_assert(kThreads == kHeadDim, "one channel per thread");
+  float Oc[kMaxGroup], Mh[kMaxGroup], Lh[kMaxGroup];
+#pragma unroll
+  for (int h = 0; h < kMaxGroup; h++) {
+    float O = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; w++) O += reinterpret_cast<const float*>(ws[w].code[0])[h * kHeadDim + c];
+    Oc[h] = O * kCScale + fin[2 * kMaxGroup + h];
+    Mh[h] = fin[h];
+    Lh[h] = fin[kMaxGroup + h];
   }
   finish_stream(a, s, split, Oc, Mh, Lh, flags, reinterpret_cast<float*>(ws[0].code[0]));
 }

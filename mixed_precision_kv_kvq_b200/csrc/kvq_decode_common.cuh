@@ -146,26 +146,22 @@ __host__ __device__ constexpr int field_shift() {
   return BITS * ((POS % (16 / BITS)) % (8 / BITS));
 }
 // Pair at field position POS: the two codes sit at bits [BITS*POS, +BITS) of
-// each half-word.  Result: half2 ((c0 - 2^(BITS-1)) 2^e, (c1 - 2^(BITS-1)) 2^e),
-// exact, with e = field_shift: (0x6400 | c << e) is the fp16 number
-// 1024 + c 2^e, and subtracting the integer 1024 + 2^(BITS-1+e) is exact.
-// Centring the codes keeps the P V sum and the Z sum small (both near the
-// output instead of two large terms that cancel), so the fp32 accumulation
-// of the MMAs loses nothing to cancellation; the 2^(BITS-1) R / (2^BITS - 1)
-// taken out here is added to each token's zero.  The 2^e is undone outside
-// the inner loop, in the output rows.
+// each half-word.  Result: half2 (c0 2^(e-24), c1 2^(e-24)), exact, with
+// e = field_shift: the code bits, masked in place, are the mantissa of a
+// binary16 subnormal (exponent field zero: the value is the 10-bit mantissa
+// times 2^-24), which the fp16 MMA takes as it is.  One AND per pair; the
+// 2^(e-24) is undone outside the inner loop, in the output rows.  The legacy
+// MMA rounds products with a subnormal operand (up to ~2^-12.5 of the sum of
+// the terms' sizes, measured), the same order as the fp16 rounding of P; the
+// caller centres the codes afterwards (sum_t P_t (c_t - h) = sum_t P_t c_t -
+// h sum_t P_t) so neither error is weighted by the uncentred code.
 template <int BITS, int POS>
 __device__ __forceinline__ uint32_t widen(uint32_t w, uint32_t w8) {
   constexpr int kPerByte = 8 / BITS;
   constexpr int e = field_shift<BITS, POS>();
   constexpr uint32_t m = (1u << BITS) - 1u;
-  constexpr uint32_t mask = (m << e) | (m << (16 + e));
-  constexpr uint32_t off = (0x6400u + (1u << (BITS - 1 + e))) * 0x00010001u;
-  static_assert((1u << (BITS - 1 + e)) < 1024u, "the offset is an integer below 2048");
-  const uint32_t x = lop_and_or((POS % (16 / BITS)) >= kPerByte ? w8 : w, mask, 0x64006400u);
-  uint32_t d;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(x), "r"(off));
-  return d;
+  static_assert(((m << e) >> 10) == 0u, "the code lies in the mantissa field");
+  return ((POS % (16 / BITS)) >= kPerByte ? w8 : w) & ((m << e) | (m << (16 + e)));
 }
 // field_shift of pair p (any p in 0..15) at BITS <= 8.
 template <int BITS>
@@ -173,7 +169,9 @@ __host__ __device__ constexpr int pair_shift(int p) {
   return BITS >= 16 ? 0 : BITS * ((p % (16 / BITS)) % (8 / BITS));
 }
 // 16-bit codes: the whole word is the pair; split each code into high and low
-// byte, c - 2^15 = 256 (hi - 128) + lo (centred as above).
+// byte, c - 2^15 = 256 (hi - 128) + lo.  Each byte x goes in as the binary16
+// 1024 + x (0x6400 | x), and one fma.f16x2 takes the offset off exactly; the
+// codes are centred so the high-byte MMA sum stays near the output.
 __device__ __forceinline__ uint32_t widen16_hi(uint32_t w) {
   return hfma2_u(lop_and_or(w >> 8, 0x00ff00ffu, 0x64006400u), 0x3c003c00u, 0xe480e480u);  // - 1152
 }
