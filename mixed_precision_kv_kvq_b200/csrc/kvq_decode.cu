@@ -524,8 +524,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
                             : make_float4(1.f, 1.f, 1.f, 1.f);
     reinterpret_cast<float4*>(s_lam)[lane] = lv;
   }
-  // ---- chunk iterator: lane 0 walks its groups tile by tile and issues the
-  // copies; everyone reads the per-stage descriptors (groups, valid tokens) ----
+  // ---- chunk iterator: the warp walks its groups tile by tile (per-channel
+  // Key groups: lane 0, in logical order, publishing per-stage descriptors) ----
   int left = (int)(wb - wa);  // groups this warp still has to issue
   int it_tile = 0, it_grp = 0, it_tgroups = 0, it_tvalid = 0;
   long long v_next = wa;  // per-channel Key groups: next group in logical order
@@ -538,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   }
   const uint8_t* sbase = a.codes + (size_t)s * f.nt * kTileBytes;
   const uint32_t* mbase = a.meta + (size_t)s * f.nt * f.pf * 2;
-  auto issue = [&](int st) {  // lane 0 only: next chunk of this warp into stage st
+  auto issue = [&](int st) {  // per-channel Key groups, lane 0 only: next chunk of this warp into stage st
     if (left <= 0) {
       mydesc[st] = make_int2(0, 0);
       return;
@@ -590,15 +590,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
         bulk_g2s(smem_u32(kmcb), a.kmc + ((size_t)s * a.blocks_max + (size_t)blk) * kHeadDim, 4u * kHeadDim, bar);
       return;
     }
-    int ng = it_tgroups - it_grp;
-    ng = ng < kChunkGroups ? ng : kChunkGroups;
-    ng = ng < left ? ng : left;
-    mydesc[st] = make_int2(ng, it_tvalid - 16 * it_grp);
-    const uint32_t cbytes = (uint32_t)ng * kGroupBytes, mbytes = (uint32_t)ng * 128u;
-    const uint32_t bar = bar0 + 8 * st;
-    mbar_expect_tx(bar, cbytes + mbytes);
-    bulk_g2s(smem_u32(my.code[st]), sbase + (size_t)it_tile * kTileBytes + (size_t)it_grp * kGroupBytes, cbytes, bar);
-    bulk_g2s(smem_u32(my.meta[st]), mbase + ((size_t)it_tile * f.pf + (size_t)it_grp * 16) * 2, mbytes, bar);
+  };
+  // Every other layout: all lanes step the same iterator (the values are
+  // warp-uniform) and lane 0 alone issues the copies.  A chunk is up to
+  // kChunkGroups groups of one tile; x = groups, y = valid tokens from its
+  // first group; coff, moff: its code byte and meta word offsets in the stream.
+  auto next_chunk = [&](size_t& coff, size_t& moff) -> int2 {
+    if (left <= 0) return make_int2(0, 0);
+    const int ng = min(min(it_tgroups - it_grp, kChunkGroups), left);
+    const int2 d = make_int2(ng, it_tvalid - 16 * it_grp);
+    coff = (size_t)it_tile * kTileBytes + (size_t)it_grp * kGroupBytes;
+    moff = ((size_t)it_tile * f.pf + (size_t)it_grp * 16) * 2;
     left -= ng;
     it_grp += ng;
     if (it_grp == it_tgroups) {  // next tile: full, the partial tile k, or a base tile
@@ -607,19 +609,29 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
       it_tgroups = it_tile < f.k ? f.gpt : (it_tile == f.k ? f.gk : f.gh);
       it_tvalid = it_tile < f.k ? f.p : (it_tile == f.k ? f.h + f.r : f.h);
     }
+    return d;
+  };
+  auto copy_chunk = [&](int st, int2 d, size_t coff, size_t moff) {
+    if (lane == 0 && d.x > 0) {
+      const uint32_t cbytes = (uint32_t)d.x * kGroupBytes, mbytes = (uint32_t)d.x * 128u;
+      const uint32_t bar = bar0 + 8 * st;
+      mbar_expect_tx(bar, cbytes + mbytes);
+      bulk_g2s(smem_u32(my.code[st]), sbase + coff, cbytes, bar);
+      bulk_g2s(smem_u32(my.meta[st]), mbase + moff, mbytes, bar);
+    }
   };
 
   // A first chunk that lies wholly in groups no kernel still in flight can
   // be writing (a.safe: before the slots of the most recent append) is
   // fetched before waiting for the previous kernel.
   bool pre = false;
+  int2 d0 = make_int2(0, 0);  // the first chunk (double-buffered layouts)
+  size_t c0 = 0, m0off = 0;
   if constexpr (!kWide && !CHAN) {
-    if (lane == 0 && left > 0) {
-      const int ng0 = min(min(it_tgroups - it_grp, kChunkGroups), left);
-      if (wa + ng0 <= a.safe) {
-        issue(0);
-        pre = true;
-      }
+    d0 = next_chunk(c0, m0off);
+    if (d0.x > 0 && wa + d0.x <= a.safe) {
+      copy_chunk(0, d0, c0, m0off);
+      pre = true;
     }
   }
   // the rest of the cache, q and the counters may be written by earlier
@@ -669,9 +681,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   }
 
   // start streaming before the q' set-up so DRAM latency overlaps it
-  if (lane == 0 && !pre) {
-#pragma unroll
-    for (int i = 0; i < kS - 1; i++) issue(i);
+  if constexpr (CHAN) {
+    if (!kWide && lane == 0) issue(0);
+  } else if constexpr (!kWide) {
+    if (!pre) copy_chunk(0, d0, c0, m0off);
   }
   __syncwarp();
 
@@ -752,14 +765,27 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
 #pragma unroll
   for (int sb = 0; sb < 8; sb++) sm.o[sb][0] = sm.o[sb][1] = sm.o[sb][2] = sm.o[sb][3] = 0.f;
 
+  int2 dA = d0, dB = make_int2(0, 0);  // chunks in stages 0 and 1 (not per-channel Key groups)
   for (int ci = 0;; ci++) {
-    const int st = kWide ? 0 : ci % kS;
-    if (!kWide && lane == 0) issue((ci + kS - 1) % kS);  // refills the stage used by chunk ci-1
-    if (kWide && lane == 0) issue(0);
-    __syncwarp();
-    const int2 dsc = mydesc[st];
+    const int st = kWide ? 0 : (ci & 1);
+    int2 dsc;
+    if constexpr (CHAN) {
+      if (lane == 0) issue(kWide ? 0 : st ^ 1);  // refills the stage used by chunk ci-1 (one stage: this chunk)
+      __syncwarp();
+      dsc = mydesc[st];
+    } else if constexpr (kWide) {  // one stage: the chunk is fetched and waited for in turn
+      size_t co = 0, mo = 0;
+      dsc = next_chunk(co, mo);
+      copy_chunk(0, dsc, co, mo);
+    } else {  // chunk ci+1 into the stage chunk ci-1 used
+      size_t co = 0, mo = 0;
+      const int2 dn = next_chunk(co, mo);
+      copy_chunk(st ^ 1, dn, co, mo);
+      dsc = st ? dB : dA;
+      if (st) dA = dn; else dB = dn;
+    }
     if (dsc.x == 0) break;
-    const uint32_t parity = kWide ? (ci & 1) : ((ci / kS) & 1);
+    const uint32_t parity = kWide ? (ci & 1) : ((ci >> 1) & 1);
     if (!mbar_wait(bar0 + 8 * st, parity, a.err, flags)) break;
     const uint8_t* cs = my.code[st];
     const uint2* ms = reinterpret_cast<const uint2*>(my.meta[st]);
