@@ -396,9 +396,11 @@ def measure_decode_configs(kvq, dev, reps=20):
 
 def measure_block_append_key_channel(kvq, dev, reps=50):
     """Per-channel Key groups: appends of 128 tokens that each complete a
-    block (staging at 16 bits, then the block move: Keys quantized per channel
-    over the block, Values shift-chained) on a 7B-shaped 2-bit block (batch
-    16, 4 KV heads) holding 16384 tokens; `reps` back-to-back calls, mean."""
+    block with nothing staged, so the block goes from the input straight into
+    the progressive cache in one launch (each token quantized to INT16 as the
+    staging would hold it, then Keys quantized per channel over the block and
+    Values shift-chained) on a 7B-shaped 2-bit block (batch 16, 4 KV heads)
+    holding 16384 tokens; `reps` back-to-back calls, mean."""
     import ctypes as C
     lib = kvq.load()
     stream = torch.cuda.current_stream(dev)
@@ -425,12 +427,12 @@ def measure_block_append_key_channel(kvq, dev, reps=50):
     assert st["tokens"] == 16384 + 128 * (reps + 3) and st["bits"] == 2
     cache.free()
     streams = B7 * HKV7
-    # bf16 in, INT16 staging written and read back, codes at 2 bits + meta out
-    nb = append_bytes(B7, HKV7, 128, 16) + streams * 128 * 2 * (2 * HEAD_DIM + 4) + append_bytes(B7, HKV7, 128, 2) \
-        - streams * 128 * 2 * HEAD_DIM * 2
+    # bf16 K/V in, codes at 2 bits + meta out (per-token Value meta; the Keys'
+    # per-channel meta is one word per channel of the block, as many bytes)
+    nb = append_bytes(B7, HKV7, 128, 2)
     return {"us": round(us, 2), "gbs": round(nb / us / 1e3, 1), "bytes": nb, "tokens": 128, "batch": B7,
-            "kv_heads": HKV7, "bits": 2, "timing": f"{reps} back-to-back 128-token appends (two launches each), "
-                                                   "CUDA events around the batch"}
+            "kv_heads": HKV7, "bits": 2, "streams": streams,
+            "timing": f"{reps} back-to-back 128-token appends (one launch each), CUDA events around the batch"}
 
 
 def measure_append_token(kvq, dev, reps=200, sink_window=False):

@@ -423,29 +423,35 @@ kvq_status append_chan(kvq_cache* c, int layer, const void* k, const void* v, in
   while (off < n_tokens) {
     const int staged = (int)(L.n_all - L.n);
     const int cnt = std::min(n_tokens - off, kKeyBlock - staged);
-    AppendArgs a{};
-    a.k = k;
-    a.v = v;
-    a.dtype = dtype;
-    a.n_call = n_tokens;
-    a.tok_off = off;
-    a.cnt = cnt;
-    a.n0 = L.n;
-    a.bits = L.bits;
-    a.nt = L.nt;
-    a.pf = L.pf;
-    a.batch = c->batch;
-    a.kv_heads = c->kv_heads;
-    a.codes = c->codes(layer);
-    a.meta = c->meta(layer);
-    a.lam_inv = L.lambda_set ? c->lam_inv(layer) : nullptr;
-    a.window = true;
-    a.stage = true;
-    a.direct = L.shift_mode == KVQ_SHIFT_DIRECT;
-    a.t0 = L.n_all;
-    a.wcodes = c->wcodes(layer);
-    a.wmeta = c->wmeta(layer);
-    if (cudaError_t e = launch_append(a, s)) return cuda_fail(e, "append launch");
+    // a whole block with nothing staged goes straight from the input into
+    // the progressive cache (the block move quantizes it as the append would
+    // have staged it); otherwise the tokens are staged first
+    const bool direct_block = staged == 0 && cnt == kKeyBlock;
+    if (!direct_block) {
+      AppendArgs a{};
+      a.k = k;
+      a.v = v;
+      a.dtype = dtype;
+      a.n_call = n_tokens;
+      a.tok_off = off;
+      a.cnt = cnt;
+      a.n0 = L.n;
+      a.bits = L.bits;
+      a.nt = L.nt;
+      a.pf = L.pf;
+      a.batch = c->batch;
+      a.kv_heads = c->kv_heads;
+      a.codes = c->codes(layer);
+      a.meta = c->meta(layer);
+      a.lam_inv = L.lambda_set ? c->lam_inv(layer) : nullptr;
+      a.window = true;
+      a.stage = true;
+      a.direct = L.shift_mode == KVQ_SHIFT_DIRECT;
+      a.t0 = L.n_all;
+      a.wcodes = c->wcodes(layer);
+      a.wmeta = c->wmeta(layer);
+      if (cudaError_t e = launch_append(a, s)) return cuda_fail(e, "append launch");
+    }
     L.n_all += cnt;
     off += cnt;
     if (L.n_all - L.n < kKeyBlock) continue;
@@ -468,6 +474,14 @@ kvq_status append_chan(kvq_cache* c, int layer, const void* k, const void* v, in
     m.pf = L.pf;
     m.bits = L.bits;
     m.direct = L.shift_mode == KVQ_SHIFT_DIRECT;
+    m.from_input = direct_block;
+    m.k = k;
+    m.v = v;
+    m.dtype = dtype;
+    m.n_call = n_tokens;
+    m.tok_off = off - cnt;
+    m.kv_heads = c->kv_heads;
+    m.lam_inv = L.lambda_set ? c->lam_inv(layer) : nullptr;
     for (int gi = 0; gi < kKeyBlock / kGroupTokens; gi++) slot_of(L, L.n + kGroupTokens * gi, &m.g_tile[gi], &m.g_slot[gi]);
     if (cudaError_t e = launch_block_move(m, c->batch * c->kv_heads, s)) return cuda_fail(e, "block move launch");
     L.n += kKeyBlock;

@@ -360,14 +360,79 @@ struct MoveKeySmem {
   float z[kKeyBlock], step[kKeyBlock];  // staged Keys: Z and R / 65535 of each token
   float mn[4][kHalf], mx[4][kHalf];
 };
+static_assert(kMoveWarps * 4 * (kHeadDim * 2 + 4) <= (int)sizeof(MoveKeySmem), "the Value rows fit the Key state");
 template <int BITS>
 __global__ void __launch_bounds__(kMoveThreads) block_move_kernel(BlockMoveArgs a) {
+  // the Key roles' state; the Value roles keep per warp their tokens' codes
+  // (and meta words) here instead
   __shared__ __align__(16) uint8_t sm_raw[sizeof(MoveKeySmem)];
   pdl_wait();
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const size_t stream = blockIdx.x / kMoveRoles;
   const int role = (int)(blockIdx.x % kMoveRoles);
+  // From the call's input, four tokens per warp step: lane L takes token
+  // 4 step + L / 8 of the warp's tokens and its channels 16 (L % 8) .. + 15,
+  // and each token gets the INT16 quantization the append would stage (Keys
+  // divided by lambda first; the steps of quantize_group, the min / max over
+  // the token's 8 lanes in three shuffle levels).
+  const int sub = lane & 7, tq = lane >> 3;
+  const int bq = (int)(stream / (size_t)a.kv_heads), jq = (int)(stream % (size_t)a.kv_heads);
+  auto in_ptr = [&](int t, int kv) {  // this lane's 16 values of token t
+    const size_t off = (((size_t)bq * a.n_call + (size_t)(a.tok_off + t)) * a.kv_heads + jq) * kHeadDim + 16 * sub;
+    return a.dtype == 1 ? static_cast<const void*>(static_cast<const float*>(kv ? a.v : a.k) + off)
+                        : static_cast<const void*>(static_cast<const __nv_bfloat16*>(kv ? a.v : a.k) + off);
+  };
+  auto widen_bf16 = [](const uint4 (&r)[2], float (&x)[16]) {
+#pragma unroll
+    for (int c8 = 0; c8 < 2; c8++) {
+      const uint32_t w[4] = {r[c8].x, r[c8].y, r[c8].z, r[c8].w};
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        x[8 * c8 + 2 * i] = __uint_as_float(w[i] << 16);
+        x[8 * c8 + 2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+      }
+    }
+  };
+  auto load_f32 = [](const void* p, float (&x)[16]) {
+#pragma unroll
+    for (int c4 = 0; c4 < 4; c4++) {
+      const float4 f4 = reinterpret_cast<const float4*>(p)[c4];
+      x[4 * c4] = f4.x; x[4 * c4 + 1] = f4.y; x[4 * c4 + 2] = f4.z; x[4 * c4 + 3] = f4.w;
+    }
+  };
+  auto quant16 = [&](float (&x)[16], int kv, uint16_t (&c)[16]) -> uint32_t {
+    if (kv == 0 && a.lam_inv) {
+      const float4* l4 = reinterpret_cast<const float4*>(a.lam_inv + (size_t)jq * kHeadDim + 16 * sub);
+#pragma unroll
+      for (int c4 = 0; c4 < 4; c4++) {
+        const float4 li = l4[c4];
+        x[4 * c4] = __fmul_rn(x[4 * c4], li.x); x[4 * c4 + 1] = __fmul_rn(x[4 * c4 + 1], li.y);
+        x[4 * c4 + 2] = __fmul_rn(x[4 * c4 + 2], li.z); x[4 * c4 + 3] = __fmul_rn(x[4 * c4 + 3], li.w);
+      }
+    }
+    float mn = x[0], mx = x[0];
+#pragma unroll
+    for (int i = 1; i < 16; i++) {
+      mn = fminf(mn, x[i]);
+      mx = fmaxf(mx, x[i]);
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    const __half zh = __float2half_rd(mn);
+    const float z = __half2float(zh);
+    const __half rh = __float2half_ru(__fsub_rn(mx, z));
+    const float r = __half2float(rh);
+    const float inv = r == 0.0f ? 0.0f : __fdiv_rn(65535.0f, r);
+#pragma unroll
+    for (int i = 0; i < 16; i++)
+      c[i] = r == 0.0f ? (uint16_t)0
+                       : (uint16_t)min(__float2uint_rd(__fadd_rn(__fmul_rn(__fsub_rn(x[i], z), inv), 0.5f)), 65535u);
+    return (uint32_t)__half_as_ushort(rh) | ((uint32_t)__half_as_ushort(zh) << 16);
+  };
   constexpr int P16 = slots_per_tile(16);
   auto staged = [&](int t, int kv) {  // group part holding staged token t
     return a.wcodes + (stream * kWindowTiles + t / P16) * (size_t)kTileBytes +
@@ -377,8 +442,38 @@ __global__ void __launch_bounds__(kMoveThreads) block_move_kernel(BlockMoveArgs 
     return ((stream * kWindowTiles + t / P16) * (size_t)P16 + t % P16) * 2 + kv;
   };
   if (role >= 2) {  // ---- Values of tokens 32 q .. 32 q + 31 ----
-    uint16_t* sc = reinterpret_cast<uint16_t*>(sm_raw) + warp * kHeadDim;
     const int q = role - 2;
+    if (a.from_input) {  // warp w: tokens 32 q + 4 w .. + 3, one step
+      uint16_t (*rows)[kHeadDim] = reinterpret_cast<uint16_t (*)[kHeadDim]>(sm_raw) + 4 * warp;  // [4][128]
+      uint32_t* wm = reinterpret_cast<uint32_t*>(sm_raw + kMoveWarps * 4 * kHeadDim * 2) + 4 * warp;
+      const int t0 = 32 * q + 4 * warp;
+      float x[16];
+      if (a.dtype == 1) {
+        load_f32(in_ptr(t0 + tq, 1), x);
+      } else {
+        const uint4* p = reinterpret_cast<const uint4*>(in_ptr(t0 + tq, 1));
+        const uint4 r[2] = {p[0], p[1]};
+        widen_bf16(r, x);
+      }
+      uint16_t c[16];
+      const uint32_t mw = quant16(x, 1, c);
+#pragma unroll
+      for (int i = 0; i < 16; i++) rows[tq][16 * sub + i] = (uint16_t)shift_chain<BITS>(c[i], a.direct);
+      if (sub == 0) wm[tq] = mw;
+      __syncwarp();
+#pragma unroll 1
+      for (int r = 0; r < 4; r++) {
+        const int t = t0 + r, gi = t >> 4, slot = a.g_slot[gi] + (t & 15);
+        const size_t tile = stream * a.nt + a.g_tile[gi];
+        uint8_t* gbase = a.codes + tile * kTileBytes + (size_t)(slot >> 4) * group_bytes(BITS);
+        pack_codes<BITS>(gbase + part_bytes(BITS), slot & 15, 1, rows[r], lane);
+        if (lane == 0)
+          a.meta[(tile * a.pf + slot) * 2 + 1] =
+              (uint32_t)range_chain<BITS>((uint16_t)(wm[r] & 0xffffu), a.direct) | (wm[r] & 0xffff0000u);
+      }
+      return;
+    }
+    uint16_t* sc = reinterpret_cast<uint16_t*>(sm_raw) + warp * kHeadDim;
     for (int t = 32 * q + warp; t < 32 * q + 32; t += kMoveWarps) {
       const int gi = t >> 4, slot = a.g_slot[gi] + (t & 15);
       const size_t tile = stream * a.nt + a.g_tile[gi];
@@ -404,18 +499,51 @@ __global__ void __launch_bounds__(kMoveThreads) block_move_kernel(BlockMoveArgs 
   // staged INT16 Key codes of the half: channel ch of token t is member i = ch % 4
   // of quad p = 2 (ch / 32) + (ch / 16) % 2 in unit 4 (t % 8) + (ch / 4) % 4, word
   // 16 x + 2 p + i / 2 (x = (t % 16) / 8), half-word i % 2 (the 16-bit layout)
-  for (int e = threadIdx.x; e < kKeyBlock * kHalf; e += kMoveThreads) {
-    const int t = e / kHalf, cc = e % kHalf, ch = kHalf * h + cc;
-    const int tok = t & 15, g = tok & 7, x = tok >> 3;
-    const int p = 2 * (ch >> 5) + ((ch >> 4) & 1), tt = (ch >> 2) & 3, mi = ch & 3;
-    const uint16_t* u16 = reinterpret_cast<const uint16_t*>(staged(t, 0));
-    sh.kc[t][cc] = u16[(4 * g + tt) * (unit_bytes(16) / 2) + 2 * (x * 16 + 2 * p + (mi >> 1)) + (mi & 1)];
-  }
-  if (threadIdx.x < kKeyBlock) {
-    const int t = threadIdx.x;
-    const uint32_t w = a.wmeta[staged_meta(t, 0)];
-    sh.z[t] = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
-    sh.step[t] = __fdiv_rn(__half2float(__ushort_as_half((unsigned short)(w & 0xffffu))), 65535.0f);
+  if (a.from_input) {  // warp w: tokens 16 w .. 16 w + 15, four steps, every load in flight first
+    const int t0 = 16 * warp;
+    uint4 raw[4][2];
+    if (a.dtype != 1) {
+#pragma unroll
+      for (int st = 0; st < 4; st++) {
+        const uint4* p = reinterpret_cast<const uint4*>(in_ptr(t0 + 4 * st + tq, 0));
+        raw[st][0] = p[0];
+        raw[st][1] = p[1];
+      }
+    }
+#pragma unroll
+    for (int st = 0; st < 4; st++) {
+      const int t = t0 + 4 * st + tq;
+      float x[16];
+      if (a.dtype == 1) load_f32(in_ptr(t, 0), x);
+      else widen_bf16(raw[st], x);
+      uint16_t c[16];
+      const uint32_t w = quant16(x, 0, c);
+      if ((sub >> 2) == h) {  // this lane's channels lie in the half
+        uint4* d = reinterpret_cast<uint4*>(&sh.kc[t][16 * (sub & 3)]);
+        d[0] = make_uint4(c[0] | ((uint32_t)c[1] << 16), c[2] | ((uint32_t)c[3] << 16), c[4] | ((uint32_t)c[5] << 16),
+                          c[6] | ((uint32_t)c[7] << 16));
+        d[1] = make_uint4(c[8] | ((uint32_t)c[9] << 16), c[10] | ((uint32_t)c[11] << 16),
+                          c[12] | ((uint32_t)c[13] << 16), c[14] | ((uint32_t)c[15] << 16));
+      }
+      if (sub == 0) {
+        sh.z[t] = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+        sh.step[t] = __fdiv_rn(__half2float(__ushort_as_half((unsigned short)(w & 0xffffu))), 65535.0f);
+      }
+    }
+  } else {
+    for (int e = threadIdx.x; e < kKeyBlock * kHalf; e += kMoveThreads) {
+      const int t = e / kHalf, cc = e % kHalf, ch = kHalf * h + cc;
+      const int tok = t & 15, g = tok & 7, x = tok >> 3;
+      const int p = 2 * (ch >> 5) + ((ch >> 4) & 1), tt = (ch >> 2) & 3, mi = ch & 3;
+      const uint16_t* u16 = reinterpret_cast<const uint16_t*>(staged(t, 0));
+      sh.kc[t][cc] = u16[(4 * g + tt) * (unit_bytes(16) / 2) + 2 * (x * 16 + 2 * p + (mi >> 1)) + (mi & 1)];
+    }
+    if (threadIdx.x < kKeyBlock) {
+      const int t = threadIdx.x;
+      const uint32_t w = a.wmeta[staged_meta(t, 0)];
+      sh.z[t] = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+      sh.step[t] = __fdiv_rn(__half2float(__ushort_as_half((unsigned short)(w & 0xffffu))), 65535.0f);
+    }
   }
   __syncthreads();
   {

@@ -191,6 +191,15 @@ struct BlockMoveArgs {
   int nt, pf, bits;       // progressive cache: tiles per stream, meta slots per tile, current width
   bool direct;            // the block shrinks with the Direct Right Shift
   int g_tile[kKeyBlock / kGroupTokens], g_slot[kKeyBlock / kGroupTokens];  // where its 8 groups go
+  // from_input: the block arrives whole in one append call with nothing
+  // staged, and is read from the call's k, v (as the append would stage it:
+  // Keys divided by lambda, each token quantized to INT16) instead of the
+  // staging area, which it never touches
+  bool from_input;
+  const void* k;
+  const void* v;
+  int dtype, n_call, tok_off, kv_heads;
+  const float* lam_inv;  // [kv_heads][128] or null
 };
 
 // Logical order of a block's progressive cache, epoch by epoch: tokens
