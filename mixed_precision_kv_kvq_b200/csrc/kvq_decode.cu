@@ -59,8 +59,7 @@ constexpr int kStageMeta = 512;            // meta bytes per stage (128 per grou
 constexpr int kWarpSmem = kStages * (kStageCode + kStageMeta);
 constexpr int kCtasPerSm = 4;
 constexpr int kQfBytes = 4 * 32 * 16;      // q' B fragments: [k-block][lane] x (hi b0, hi b1, lo b0, lo b1)
-constexpr int kSmemBytes = kWarps * kWarpSmem + kQfBytes + 3 * kWarps * kMaxGroup * 4 +
-                           kWarps * kStages * 8 + kWarps * kStages * 8 + 16;
+constexpr int kSmemBytes = kWarps * kWarpSmem + kQfBytes + 3 * kWarps * kMaxGroup * 4 + kWarps * kStages * 8 + 16;
 // Per-channel Key groups: q' = q lambda qscale in fp32 for the whole kernel,
 // and per warp the int16 B fragments, scales and zero terms of its block.
 constexpr int kChanSmem = kMaxGroup * kHeadDim * 4 + kWarps * kQfBytes + kWarps * kQfBytes / 2 + 2 * kWarps * kMaxGroup * 4;
@@ -380,7 +379,7 @@ __device__ __forceinline__ void process_groups(const uint8_t* cs, const uint2* m
 // block's Key channel c is Z_c + code R_c / (2^b - 1), so
 //   q'.k^_t = sum_c q'_c Z_c + sum_c (q'_c R_c / (2^b - 1)) code_t,c
 // and w_c = q'_c R_c / (2^b - 1) takes the place of q' as an exact per-head
-// 24-bit integer (scale max|w| / (2^23 - 1)); the first sum is the head's
+// 24-bit integer (scale max|w| / (2^22 - 2)); the first sum is the head's
 // zero term.  24 bits, not the 16 of the per-token operand: w carries both
 // the migrated query's outlier channels and the same channels' wider ranges,
 // so its largest entry is far above the typical one and 16 bits left the
@@ -428,17 +427,20 @@ __device__ __forceinline__ void chan_block(const float* s_qp, const uint32_t* km
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       zs += __shfl_xor_sync(0xffffffffu, zs, o);
     }
-    constexpr float kQMax = 8388607.0f;  // 2^23 - 1
-    // any inv close to kQMax / m works: the clamp keeps |qi| < 2^23 and the
-    // score scale below is the same m / kQMax the MMAs' integers are read with
-    // (qi / inv ~ w up to half a step, ks d = sum w c up to the rounding of inv)
+    constexpr float kQMax = 4194302.0f;  // 2^22 - 2
+    // any inv close to kQMax / m works: |w inv| < 2^22 - 1 then, and the score
+    // scale below is the same m / kQMax the MMAs' integers are read with
+    // (qi / inv ~ w up to half a step, ks d = sum w c up to the rounding of
+    // inv).  qi = w inv rounded to an integer by one fma with 1.5 * 2^23: the
+    // sum lies in [2^23, 2^24), where floats are the integers, and its bits
+    // minus those of 1.5 * 2^23 are qi as a 32-bit two's-complement integer.
     const float inv = m > 0.f ? kQMax * __frcp_rn(m) : 0.f;
     uint32_t hb[2], mb[2], lb[2];
 #pragma unroll
     for (int hf = 0; hf < 2; hf++) {
       uint32_t q[4];
 #pragma unroll
-      for (int i = 0; i < 4; i++) q[i] = (uint32_t)max(-8388607, min(8388607, __float2int_rn(v[hf][i] * inv)));
+      for (int i = 0; i < 4; i++) q[i] = __float_as_uint(fmaf(v[hf][i], inv, 12582912.0f)) - 0x4B400000u;
       // bytes 0, 1, 2 of the four 24-bit two's-complement integers (byte 2 is the s8 high part)
       const uint32_t ab = __byte_perm(q[0], q[1], 0x5140), cd = __byte_perm(q[2], q[3], 0x5140);
       lb[hf] = __byte_perm(ab, cd, 0x5410);
@@ -471,8 +473,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   float* w_l = w_m + kWarps * kMaxGroup;
   float* w_pz = w_l + kWarps * kMaxGroup;
   uint64_t* bars = reinterpret_cast<uint64_t*>(w_pz + kWarps * kMaxGroup);  // [warps][stages]
-  int2* desc = reinterpret_cast<int2*>(bars + kWarps * kStages);              // [warps][stages] (ng, valid0)
-  volatile int* flags = reinterpret_cast<volatile int*>(desc + kWarps * kStages);  // [0] abort, [1] last
+  volatile int* flags = reinterpret_cast<volatile int*>(bars + kWarps * kStages);  // [0] abort, [1] last
   // per-channel Key groups only (the launch sizes the area): q' [8][128],
   // per-warp B fragments [warps][4][32], scales and zero terms [warps][8]
   float* s_qp = reinterpret_cast<float*>(smem + kSmemBytes);
@@ -500,7 +501,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   const long long wa = per * (ca + (cb - ca) * warp / kWarps), wb = per * (ca + (cb - ca) * (warp + 1) / kWarps);
   WarpSmem& my = ws[warp];
   const uint32_t bar0 = smem_u32(bars + warp * kStages);
-  int2* mydesc = desc + warp * kStages;
   // per-channel Key groups: this warp's copy of its block's (R, Z) words, in
   // the per-token query fragments' area (unused then)
   uint32_t* kmcb = reinterpret_cast<uint32_t*>(qf) + warp * kHeadDim;
@@ -538,57 +538,61 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   }
   const uint8_t* sbase = a.codes + (size_t)s * f.nt * kTileBytes;
   const uint32_t* mbase = a.meta + (size_t)s * f.nt * f.pf * 2;
-  auto issue = [&](int st) {  // per-channel Key groups, lane 0 only: next chunk of this warp into stage st
-    if (left <= 0) {
-      mydesc[st] = make_int2(0, 0);
-      return;
-    }
-    if constexpr (CHAN) {
-      // logical order: group v holds tokens 16v .. 16v+15, which arrived in
-      // epoch e and sit in slots [h_e, h_e + ee_e) of tile (16v - start_e) / ee_e.
-      // A chunk gathers whole or partial runs (one tile's slots of an epoch,
-      // contiguous) up to kChunkGroups groups without leaving its 128-token
-      // block (runs never straddle blocks: epochs start on block boundaries
-      // and a run is 32, 64 or 128 tokens at a multiple of its length).  The
-      // first chunk of a block also fetches the block's Key (R, Z) words.
-      int rt[kChunkGroups], rg[kChunkGroups], rn[kChunkGroups];
-      int nr = 0, ng = 0;
-      const long long v0 = v_next;
-      while (ng < kChunkGroups && left > 0 && (ng == 0 || (v_next & 7) != 0)) {
+  // Per-channel Key groups: all lanes step the same iterator in logical order.
+  // Group v holds tokens 16v .. 16v+15, which arrived in epoch e and sit in
+  // slots [h_e, h_e + ee_e) of tile (16v - start_e) / ee_e.  A chunk gathers
+  // whole or partial runs (one tile's slots of an epoch, contiguous) up to
+  // kChunkGroups groups without leaving its 128-token block (runs never
+  // straddle blocks: epochs start on block boundaries and a run is 32, 64 or
+  // 128 tokens at a multiple of its length); x = groups, y = block, and
+  // `first` when it starts the block (it then also fetches the block's Key
+  // (R, Z) words).  ep_e, the epoch of v_next, only moves forward.
+  int ep_e = 0;
+  struct Runs {
+    uint32_t r[kChunkGroups];  // tile << 10 | first group << 4 | groups (tiles per stream < 2^22)
+    bool first;
+  };
+  auto next_chunk_chan = [&](Runs& ru) -> int2 {
+    int ng = 0;
+    const long long v0 = v_next;
+#pragma unroll
+    for (int r = 0; r < kChunkGroups; r++) {
+      ru.r[r] = 0u;
+      if (ng < kChunkGroups && left > 0 && (ng == 0 || (v_next & 7) != 0)) {
         const int i = 16 * (int)v_next;
-        int e = 0;
-        while (e + 1 < a.ep.n && i >= a.ep.start[e + 1]) e++;
-        const int m = i - a.ep.start[e], lg = a.ep.lg_ee[e];
+        while (ep_e + 1 < a.ep.n && i >= a.ep.start[ep_e + 1]) ep_e++;
+        const int m = i - a.ep.start[ep_e], lg = a.ep.lg_ee[ep_e];
         const int tile = m >> lg, off = m & ((1 << lg) - 1);
         int take = ((1 << lg) - off) >> 4;
-        take = take < kChunkGroups - ng ? take : kChunkGroups - ng;
-        take = take < left ? take : left;
-        const int to_end = 8 - (int)(v_next & 7);  // stay inside the block
-        take = take < to_end ? take : to_end;
-        rt[nr] = tile;
-        rg[nr] = (a.ep.h[e] + off) >> 4;
-        rn[nr] = take;
-        nr++;
+        take = min(min(take, kChunkGroups - ng), left);
+        take = min(take, 8 - (int)(v_next & 7));  // stay inside the block
+        ru.r[r] = ((uint32_t)tile << 10) | ((uint32_t)((a.ep.h[ep_e] + off) >> 4) << 4) | (uint32_t)take;
         ng += take;
         left -= take;
         v_next += take;
       }
-      const int blk = (int)(v0 >> 3);
-      const bool first = (v0 & 7) == 0;
-      mydesc[st] = make_int2(ng, blk);  // groups, block
+    }
+    ru.first = (v0 & 7) == 0;
+    return make_int2(ng, (int)(v0 >> 3));
+  };
+  auto copy_chunk_chan = [&](int st, int2 d, const Runs& ru) {
+    if (lane == 0 && d.x > 0) {
       const uint32_t bar = bar0 + 8 * st;
-      mbar_expect_tx(bar, (uint32_t)ng * (kGroupBytes + 128u) + (first ? 4u * kHeadDim : 0u));
+      mbar_expect_tx(bar, (uint32_t)d.x * (kGroupBytes + 128u) + (ru.first ? 4u * kHeadDim : 0u));
       int done = 0;
-      for (int r = 0; r < nr; r++) {
-        bulk_g2s(smem_u32(my.code[st] + done * kGroupBytes), sbase + (size_t)rt[r] * kTileBytes + (size_t)rg[r] * kGroupBytes,
-                 (uint32_t)rn[r] * kGroupBytes, bar);
-        bulk_g2s(smem_u32(my.meta[st] + done * 128), mbase + ((size_t)rt[r] * f.pf + (size_t)rg[r] * 16) * 2,
-                 (uint32_t)rn[r] * 128u, bar);
-        done += rn[r];
+#pragma unroll
+      for (int r = 0; r < kChunkGroups; r++) {
+        const uint32_t n = ru.r[r] & 15u, g = (ru.r[r] >> 4) & 63u;
+        const size_t tile = ru.r[r] >> 10;
+        if (n > 0) {
+          bulk_g2s(smem_u32(my.code[st] + done * kGroupBytes), sbase + tile * kTileBytes + (size_t)g * kGroupBytes,
+                   n * kGroupBytes, bar);
+          bulk_g2s(smem_u32(my.meta[st] + done * 128), mbase + (tile * f.pf + (size_t)g * 16) * 2, n * 128u, bar);
+          done += (int)n;
+        }
       }
-      if (first)  // one buffer per warp: a block spans at least two chunks, so the previous block's words are used
-        bulk_g2s(smem_u32(kmcb), a.kmc + ((size_t)s * a.blocks_max + (size_t)blk) * kHeadDim, 4u * kHeadDim, bar);
-      return;
+      if (ru.first)  // one buffer per warp: a block spans at least two chunks, so the previous block's words are used
+        bulk_g2s(smem_u32(kmcb), a.kmc + ((size_t)s * a.blocks_max + (size_t)d.y) * kHeadDim, 4u * kHeadDim, bar);
     }
   };
   // Every other layout: all lanes step the same iterator (the values are
@@ -682,7 +686,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
 
   // start streaming before the q' set-up so DRAM latency overlaps it
   if constexpr (CHAN) {
-    if (!kWide && lane == 0) issue(0);
+    if constexpr (!kWide) {
+      Runs ru;
+      d0 = next_chunk_chan(ru);
+      copy_chunk_chan(0, d0, ru);
+    }
   } else if constexpr (!kWide) {
     if (!pre) copy_chunk(0, d0, c0, m0off);
   }
@@ -770,9 +778,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     const int st = kWide ? 0 : (ci & 1);
     int2 dsc;
     if constexpr (CHAN) {
-      if (lane == 0) issue(kWide ? 0 : st ^ 1);  // refills the stage used by chunk ci-1 (one stage: this chunk)
-      __syncwarp();
-      dsc = mydesc[st];
+      Runs ru;
+      if constexpr (kWide) {  // one stage: the chunk is fetched and waited for in turn
+        dsc = next_chunk_chan(ru);
+        copy_chunk_chan(0, dsc, ru);
+      } else {  // chunk ci+1 into the stage chunk ci-1 used
+        const int2 dn = next_chunk_chan(ru);
+        copy_chunk_chan(st ^ 1, dn, ru);
+        dsc = st ? dB : dA;
+        if (st) dA = dn; else dB = dn;
+      }
     } else if constexpr (kWide) {  // one stage: the chunk is fetched and waited for in turn
       size_t co = 0, mo = 0;
       dsc = next_chunk(co, mo);
