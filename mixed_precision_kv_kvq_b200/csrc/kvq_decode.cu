@@ -921,6 +921,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     Mh[h] = fin[h];
     Lh[h] = fin[kMaxGroup + h];
   }
+  // warp 0's two code stages (free now; the merge weights above are in registers)
+  static_assert(kScratchFloats * 4 <= kStages * kStageCode, "the merge scratch fits");
   finish_stream(a, s, split, Oc, Mh, Lh, flags, reinterpret_cast<float*>(ws[0].code[0]));
 }
 

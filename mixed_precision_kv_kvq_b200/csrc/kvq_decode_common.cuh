@@ -232,7 +232,8 @@ __device__ __forceinline__ uint32_t quad_reg(const uint32_t* u) {
 // output; otherwise the CTA leaves a partial record (M[8], L[8], O[128][8])
 // and the CTA that takes the stream's last ticket (atomic, no waiting) merges
 // all partials with log-sum-exp weights.  flags[1]: CTA-shared scratch word;
-// scratch: 2 * kMaxSplits * kMaxGroup floats of free shared memory.
+// scratch: kScratchFloats floats of free shared memory.
+constexpr int kScratchFloats = 2 * kMaxSplits * kMaxGroup + 2 * kMaxGroup;
 __device__ __forceinline__ void finish_stream(const DecodeArgs& a, int s, int split, const float (&Oc)[kMaxGroup],
                                               const float (&Mh)[kMaxGroup], const float (&Lh)[kMaxGroup],
                                               volatile int* flags, float* scratch) {
@@ -258,15 +259,15 @@ __device__ __forceinline__ void finish_stream(const DecodeArgs& a, int s, int sp
   }
   *reinterpret_cast<float4*>(mypart + 2 * kMaxGroup + c * kMaxGroup) = make_float4(Oc[0], Oc[1], Oc[2], Oc[3]);
   *reinterpret_cast<float4*>(mypart + 2 * kMaxGroup + c * kMaxGroup + 4) = make_float4(Oc[4], Oc[5], Oc[6], Oc[7]);
-  // Ticket: after the CTA barrier one thread publishes the CTA's partial
-  // (fence, then the atomic); the CTA that takes the last ticket merges.
+  // Ticket: after the CTA barrier one thread takes it with an
+  // acquire-release atomic at GPU scope (it publishes the CTA's partial, which
+  // the barrier ordered before it, and the CTA that takes the last ticket sees
+  // every other partial); that CTA merges.
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
-    const int old = atomicAdd(a.counters + s, 1);
-    const int last = old == nparts - 1;
-    if (last) __threadfence();
-    flags[1] = last;
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(a.counters + s) : "memory");
+    flags[1] = old == nparts - 1;
   }
   __syncthreads();
   // A launch that skipped its dependency wait still completes only after the
@@ -297,31 +298,33 @@ __device__ __forceinline__ void finish_stream(const DecodeArgs& a, int s, int sp
     dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
   }
   __syncthreads();
-  // Every thread forms the log-sum-exp weights itself (broadcast reads):
-  // w_k = e^(M_k - M) for head h, out = sum_k w_k O_k / sum_k w_k L_k.
-  float Mx[kMaxGroup], Ls[kMaxGroup], acc[kMaxGroup];
+  // Log-sum-exp weights, formed once: thread h takes head h's max M over the
+  // partials, then thread (k, h) the weight w_k = e^(M_k - M) (in place of
+  // M_k), then thread h the sum of w_k L_k; out = sum_k w_k O_k / sum_k w_k L_k.
+  float* mxs = lk + kMaxSplits * kMaxGroup;  // [8] M, then [8] sum w L
+  if (threadIdx.x < kMaxGroup) {
+    float m = -INFINITY;
+    for (int k = 0; k < nparts; k++) m = fmaxf(m, wk[k * kMaxGroup + threadIdx.x]);
+    mxs[threadIdx.x] = m;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < nparts * kMaxGroup; i += kHeadDim) wk[i] = ex2(wk[i] - mxs[i % kMaxGroup]);
+  __syncthreads();
+  if (threadIdx.x < kMaxGroup) {
+    float l = 0.f;
+    for (int k = 0; k < nparts; k++) l = fmaf(wk[k * kMaxGroup + threadIdx.x], lk[k * kMaxGroup + threadIdx.x], l);
+    mxs[kMaxGroup + threadIdx.x] = l;
+  }
+  float acc[kMaxGroup];
 #pragma unroll
-  for (int h = 0; h < kMaxGroup; h++) {
-    Mx[h] = -INFINITY;
-    Ls[h] = 0.f;
-    acc[h] = 0.f;
-  }
-  for (int k = 0; k < nparts; k++) {
-    const float4 m0 = *reinterpret_cast<const float4*>(wk + k * kMaxGroup);
-    const float4 m1 = *reinterpret_cast<const float4*>(wk + k * kMaxGroup + 4);
-    Mx[0] = fmaxf(Mx[0], m0.x); Mx[1] = fmaxf(Mx[1], m0.y); Mx[2] = fmaxf(Mx[2], m0.z); Mx[3] = fmaxf(Mx[3], m0.w);
-    Mx[4] = fmaxf(Mx[4], m1.x); Mx[5] = fmaxf(Mx[5], m1.y); Mx[6] = fmaxf(Mx[6], m1.z); Mx[7] = fmaxf(Mx[7], m1.w);
-  }
+  for (int h = 0; h < kMaxGroup; h++) acc[h] = 0.f;
   auto add = [&](int k, const float4& o0, const float4& o1) {
-    const float* mk = wk + k * kMaxGroup;
-    const float* lkk = lk + k * kMaxGroup;
-    const float ov8[kMaxGroup] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; h++) {
-      const float e = ex2(mk[h] - Mx[h]);
-      Ls[h] = fmaf(e, lkk[h], Ls[h]);
-      acc[h] = fmaf(e, ov8[h], acc[h]);
-    }
+    const float4 w0 = *reinterpret_cast<const float4*>(wk + k * kMaxGroup);
+    const float4 w1 = *reinterpret_cast<const float4*>(wk + k * kMaxGroup + 4);
+    acc[0] = fmaf(w0.x, o0.x, acc[0]); acc[1] = fmaf(w0.y, o0.y, acc[1]);
+    acc[2] = fmaf(w0.z, o0.z, acc[2]); acc[3] = fmaf(w0.w, o0.w, acc[3]);
+    acc[4] = fmaf(w1.x, o1.x, acc[4]); acc[5] = fmaf(w1.y, o1.y, acc[5]);
+    acc[6] = fmaf(w1.z, o1.z, acc[6]); acc[7] = fmaf(w1.w, o1.w, acc[7]);
   };
 #pragma unroll
   for (int k = 0; k < kPre; k++)
@@ -332,11 +335,10 @@ __device__ __forceinline__ void finish_stream(const DecodeArgs& a, int s, int sp
     const float4 v1 = __ldcg(reinterpret_cast<const float4*>(oc + (size_t)k * kPartFloats + 4));
     add(k, v0, v1);
   }
-#pragma unroll
-  for (int h = 0; h < kMaxGroup; h++) acc[h] /= Ls[h];
+  __syncthreads();  // the sums of w L
 #pragma unroll
   for (int h = 0; h < kMaxGroup; h++)
-    if (h < G) outp[h * kHeadDim + c] = acc[h];
+    if (h < G) outp[h * kHeadDim + c] = acc[h] / mxs[kMaxGroup + h];
   if (threadIdx.x == 0) a.counters[s] = 0;
 }
 
