@@ -886,7 +886,10 @@ def run_gpu(args, rank, world):
         "config": {"workload": WORKLOAD, "layers": layers, "batch": B7, "q_heads": HQ7, "kv_heads": HKV7,
                    "head_dim": HEAD_DIM, "context": T7, "fbit": fbit, "parallelism": f"replicas x{world}",
                    "l2": "no flush: every block's cache read (151-285 MB) exceeds the 126 MB L2",
-                   "decode_ms_share": round(dec_ms / (ev_step_ms * K), 3)},
+                   "decode_ms_share": round(dec_ms / (ev_step_ms * K), 3),
+                   "headline": "the 7B-shape decode step, the model-shaped workload the metric is quoted on; the "
+                               "largest one-GPU workload (Llama-70B shape, 128K context) is measured the same way "
+                               "as the llama70b_step entry"},
         "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
         "two_call_step": two_calls,
         **extra,
