@@ -560,6 +560,29 @@ def test_key_channel_chunked_bf16(kvq, orc, fbit, mode):
     assert e.value.status == 2
 
 
+@pytest.mark.parametrize("mode", [0, 1])
+def test_key_channel_whole_blocks_fp32(kvq, orc, mode):
+    """fp32 inputs in calls of whole, aligned blocks (each block goes from the
+    input straight into the progressive cache, nothing staged), through the
+    shrinks of a Fbit-4 block with either shift, then a partial call that
+    stages tokens: codes, meta and staged records bit-exact, attention within
+    2e-3."""
+    B, H, n_f = 2, 3, 1024
+    T = n_f + 77
+    k, v = S.keys_values(21, mode, B, T, H, 0, 3, dtype=torch.float32)
+    P = CPair(kvq, orc, B, H, n_f, 4, lam_for(k), shift_mode=mode)
+    pos = 0
+    for n in (128, 256, 128, 512, 77):
+        P.append(k[:, pos:pos + n], v[:, pos:pos + n])
+        pos += n
+        if n != 512:
+            P.check_codes()
+            P.check_attention(S.queries(21, mode, pos, B, 2 * H, pos, dtype=torch.bfloat16))
+    assert pos == T and P.gpu.query(0)["bits"] == 4 and P.orc.main.shrink_at
+    P.check_codes()
+    P.check_attention(S.queries(21, mode, 0, B, 2 * H, T, dtype=torch.bfloat16))
+
+
 @pytest.mark.parametrize("G", [1, 5, 8])
 def test_key_channel_many_blocks_and_splits(kvq, orc, G):
     """A longer block (N = 8192 at Fbit 2, every epoch present, several CTAs
