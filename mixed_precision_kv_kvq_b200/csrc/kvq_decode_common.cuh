@@ -1,8 +1,7 @@
-// kvq_decode_common.cuh -- pieces shared by the two split-K GQA decode
-// kernels (kvq_decode.cu: legacy warp-level MMAs; kvq_decode_tc.cu: tcgen05
-// with operands in tensor memory): PTX wrappers, bounded mbarrier waits,
-// bulk copies, the widening of packed codes into MMA operands, and the
-// split merge that ends every CTA of a stream.
+// kvq_decode_common.cuh -- pieces of the split-K GQA decode kernel
+// (kvq_decode.cu) kept apart from its main loop: PTX wrappers, bounded
+// mbarrier waits, bulk copies, the widening of packed codes into MMA
+// operands, and the split merge that ends every CTA of a stream.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
