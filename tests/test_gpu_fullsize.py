@@ -1,11 +1,12 @@
 """GPU parity at the full sizes of the four model-shaped workloads, through
 the same C-ABI calls and launch configuration the benchmark times.
 
-The whole cache is built on the GPU; the oracle replays a few sampled
-(sequence, KV head) streams from the same inputs (copied to the host chunk
-by chunk) and checks, for each sampled stream: codes and meta bit-exact
-against kvq_export, the block's shrink schedule, and decode attention of
-every query head of that KV head within 2e-3 (max_c |o - o*| / max_c |o*|).
+The whole cache is built on the GPU; the oracle replays sampled (sequence,
+KV head) streams -- every stream of the 32B 2-bit and the 70B 4-bit blocks --
+from the same inputs (copied to the host chunk by chunk) and checks, for each
+replayed stream: codes and meta bit-exact against kvq_export, the block's
+shrink schedule, and decode attention of every query head of that KV head
+within 2e-3 (max_c |o - o*| / max_c |o*|).
 
 Workloads (synthetic RoPE'd bf16 K/V with x20 outlier Key channels on 1% of
 the layer's channels, lambda = sqrt(max |K|) from the first chunk):
@@ -22,6 +23,8 @@ the layer's channels, lambda = sqrt(max |K|) from the first chunk):
                  4 -> 2 shrink, then decode.
 """
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 import pytest
@@ -146,12 +149,16 @@ class Sampled:
         self.gpu.device_status()
         assert np.isfinite(out).all()
         qc = q.float().cpu().numpy()
-        worst = 0.0
-        for (b, j), o in self.orc.items():
+
+        def stream_err(item):
+            (b, j), o = item
             ref = o.attention(qc[b:b + 1, j * G:(j + 1) * G], self.lam[j:j + 1], sm)[0]
             got = out[b, j * G:(j + 1) * G]
-            err = np.abs(got - ref).max(axis=-1) / np.abs(ref).max(axis=-1)
-            worst = max(worst, float(err.max()))
+            return float((np.abs(got - ref).max(axis=-1) / np.abs(ref).max(axis=-1)).max())
+
+        # the oracle's C attention runs without the Python lock: many streams go in threads
+        with ThreadPoolExecutor(max_workers=min(len(self.orc), os.cpu_count() or 1)) as pool:
+            worst = max(pool.map(stream_err, self.orc.items()))
         assert worst <= TOL, f"max rel err {worst:.3e}"
         return worst
 
@@ -161,6 +168,10 @@ class Sampled:
 
 def corners(batch, kv_heads):
     return [(0, 0), (batch // 2, kv_heads // 2 - 1), (batch - 1, kv_heads - 1)]
+
+
+def every(batch, kv_heads):
+    return [(b, j) for b in range(batch) for j in range(kv_heads)]
 
 
 @pytest.mark.parametrize("fbit,layer", [(2, 1), (4, 0)])
@@ -192,8 +203,11 @@ def test_7b_progressive_one_token_per_step(kvq, orc, fbit, shrinks):
 
 @pytest.mark.parametrize("fbit,layer", [(2, 3), (4, 60)])
 def test_32b_decode_fullsize(kvq, orc, fbit, layer):
+    """At 2 bits every one of the 128 (sequence, KV head) streams is replayed
+    through the oracle (codes bit-exact, all 40 query heads within 2e-3);
+    at 4 bits three streams."""
     B, H, HQ, T = 16, 8, 40, 32768
-    x = Sampled(kvq, orc, B, H, 55296, fbit, corners(B, H), layer)
+    x = Sampled(kvq, orc, B, H, 55296, fbit, every(B, H) if fbit == 2 else corners(B, H), layer)
     x.fill(T, chunk=8192)
     st = x.check_state()
     assert st["bits"] == fbit
@@ -203,8 +217,10 @@ def test_32b_decode_fullsize(kvq, orc, fbit, layer):
 
 
 def test_70b_fbit4_decode_fullsize(kvq, orc):
+    """Every one of the 64 streams of the 128K-token block replayed through the
+    oracle: codes bit-exact, all 64 query heads (G = 8) within 2e-3."""
     B, H, HQ, T = 8, 8, 64, 131072
-    x = Sampled(kvq, orc, B, H, T, 4, corners(B, H), 0)
+    x = Sampled(kvq, orc, B, H, T, 4, every(B, H), 0)
     x.fill(T, chunk=8192)
     st = x.check_state()
     assert (st["bits"], st["capacity"]) == (4, T)
