@@ -59,7 +59,8 @@ constexpr int kStageMeta = 512;            // meta bytes per stage (128 per grou
 constexpr int kWarpSmem = kStages * (kStageCode + kStageMeta);
 constexpr int kCtasPerSm = 4;
 constexpr int kQfBytes = 4 * 32 * 16;      // q' B fragments: [k-block][lane] x (hi b0, hi b1, lo b0, lo b1)
-constexpr int kSmemBytes = kWarps * kWarpSmem + kQfBytes + 3 * kWarps * kMaxGroup * 4 + kWarps * kStages * 8 + 16;
+constexpr int kSmemBytes = kWarps * kWarpSmem + kQfBytes + 3 * kWarps * kMaxGroup * 4 + kWarps * kStages * 8 + 16 +
+                           2 * kMaxGroup * 4;
 // Per-channel Key groups: q' = q lambda qscale in fp32 for the whole kernel,
 // and per warp the int16 B fragments, scales and zero terms of its block.
 constexpr int kChanSmem = kMaxGroup * kHeadDim * 4 + kWarps * kQfBytes + kWarps * kQfBytes / 2 + 2 * kWarps * kMaxGroup * 4;
@@ -474,6 +475,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   float* w_pz = w_l + kWarps * kMaxGroup;
   uint64_t* bars = reinterpret_cast<uint64_t*>(w_pz + kWarps * kMaxGroup);  // [warps][stages]
   volatile int* flags = reinterpret_cast<volatile int*>(bars + kWarps * kStages);  // [0] abort, [1] last
+  unsigned* s_amax = reinterpret_cast<unsigned*>(const_cast<int*>(flags) + 4);  // [8] bits of max|q'| per head
+  int* s_isum = reinterpret_cast<int*>(s_amax + kMaxGroup);                     // [8] sum of q_int per head
   // per-channel Key groups only (the launch sizes the area): q' [8][128],
   // per-warp B fragments [warps][4][32], scales and zero terms [warps][8]
   float* s_qp = reinterpret_cast<float*>(smem + kSmemBytes);
@@ -513,16 +516,26 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     for (int i = 0; i < kS; i++) mbar_init(bar0 + 8 * i, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // q and lambda are staged in shared memory (in warp 0's second code stage,
-  // unused until the main loop starts).  lambda is fixed while kernels run on
-  // the block, so it is fetched before waiting for the previous kernel.
+  // lambda is fixed while kernels run on the block, so it is fetched before
+  // waiting for the previous kernel.  Per-channel Key groups stage q and
+  // lambda in shared memory (in warp 0's second code stage, unused until the
+  // main loop starts); otherwise each lane loads the channels it quantizes:
+  // head gq = 2 warp + lane / 16, channels 32 sq + 16 hf + 4 tq + i.
   const int b = s / a.kv_heads, j = s - b * a.kv_heads;
   __nv_bfloat16* s_q = reinterpret_cast<__nv_bfloat16*>(ws[0].code[kStages - 1]);  // [8][128]
   float* s_lam = reinterpret_cast<float*>(s_q + kMaxGroup * kHeadDim);               // [128]
-  if (warp == 1) {
-    const float4 lv = a.lam ? __ldg(reinterpret_cast<const float4*>(a.lam + (size_t)j * kHeadDim) + lane)
-                            : make_float4(1.f, 1.f, 1.f, 1.f);
-    reinterpret_cast<float4*>(s_lam)[lane] = lv;
+  const int gq = 2 * warp + (lane >> 4), tq = (lane >> 2) & 3, sq = lane & 3;
+  float4 lam4[2] = {make_float4(1.f, 1.f, 1.f, 1.f), make_float4(1.f, 1.f, 1.f, 1.f)};
+  if constexpr (CHAN) {
+    if (warp == 1) {
+      const float4 lv = a.lam ? __ldg(reinterpret_cast<const float4*>(a.lam + (size_t)j * kHeadDim) + lane)
+                              : make_float4(1.f, 1.f, 1.f, 1.f);
+      reinterpret_cast<float4*>(s_lam)[lane] = lv;
+    }
+  } else if (a.lam) {
+#pragma unroll
+    for (int hf = 0; hf < 2; hf++)
+      lam4[hf] = __ldg(reinterpret_cast<const float4*>(a.lam + (size_t)j * kHeadDim + 32 * sq + 16 * hf + 4 * tq));
   }
   // ---- chunk iterator: the warp walks its groups tile by tile (per-channel
   // Key groups: lane 0, in logical order, publishing per-stage descriptors) ----
@@ -645,8 +658,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   if (!a.after_decode) pdl_wait();
   if (a.trigger_early) pdl_launch_dependents();  // a window launch follows: let it fill free SMs now
   const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.q_heads + (size_t)j * G) * kHeadDim;
-  uint4 qv = make_uint4(0u, 0u, 0u, 0u);  // 8 bf16 of q: head threadIdx/16, channels 8 (threadIdx%16) ..
-  if ((int)threadIdx.x < G * (kHeadDim / 8)) qv = reinterpret_cast<const uint4*>(qb)[threadIdx.x];
+  uint4 qv = make_uint4(0u, 0u, 0u, 0u);  // per-channel Key groups: 8 bf16 of q, head threadIdx/16, channels 8 (threadIdx%16) ..
+  uint2 qv2[2] = {make_uint2(0u, 0u), make_uint2(0u, 0u)};  // otherwise this lane's channels of head gq
+  if constexpr (CHAN) {
+    if ((int)threadIdx.x < G * (kHeadDim / 8)) qv = reinterpret_cast<const uint4*>(qb)[threadIdx.x];
+  } else if (gq < G) {
+#pragma unroll
+    for (int hf = 0; hf < 2; hf++)
+      qv2[hf] = *reinterpret_cast<const uint2*>(qb + (size_t)gq * kHeadDim + 32 * sq + 16 * hf + 4 * tq);
+  }
 
   // ---- fused single-token append: the warp whose range holds the new
   // token's group quantizes and writes the token (K, then V) before it
@@ -703,11 +723,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   // is taken as s_h sum(q_int), over exactly the values the MMAs use, so
   // (R/(2^b-1)) q'.c + Z sum(q') is the dot product of s_h q_int with the
   // dequantised key.
-  unsigned* s_amax = reinterpret_cast<unsigned*>(w_m);  // [8] bits of max|q'| (w_m is free here)
-  int* s_isum = reinterpret_cast<int*>(w_l);             // [8] sum of q_int
-  reinterpret_cast<uint4*>(s_q)[threadIdx.x] = qv;  // heads >= G are zero
-  __syncthreads();
   if constexpr (CHAN) {  // q' in fp32 for the per-block operands
+    reinterpret_cast<uint4*>(s_q)[threadIdx.x] = qv;  // heads >= G are zero
+    __syncthreads();
     for (int idx = threadIdx.x; idx < kMaxGroup * kHeadDim; idx += kThreads)
       s_qp[idx] = __bfloat162float(s_q[idx]) * a.qscale * s_lam[idx & (kHeadDim - 1)];
   } else {
@@ -715,15 +733,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
     // and writes the B fragment of k-block sq = L%4 for MMA lane 4 gq + tq,
     // tq = (L/4)%4: channels 32 sq + 16 hf + 4 tq + i (hf = 0..1, i = 0..3).
     // The 16 lanes of a head cover its 128 channels.
-    const int gq = 2 * warp + (lane >> 4), tq = (lane >> 2) & 3, sq = lane & 3;
     float v[2][4];
     float m = 0.f;
 #pragma unroll
     for (int hf = 0; hf < 2; hf++) {
+      const float qx[4] = {__uint_as_float(qv2[hf].x << 16), __uint_as_float(qv2[hf].x & 0xffff0000u),
+                           __uint_as_float(qv2[hf].y << 16), __uint_as_float(qv2[hf].y & 0xffff0000u)};
+      const float lx[4] = {lam4[hf].x, lam4[hf].y, lam4[hf].z, lam4[hf].w};
 #pragma unroll
       for (int i = 0; i < 4; i++) {
-        const int ch = 32 * sq + 16 * hf + 4 * tq + i;
-        v[hf][i] = __bfloat162float(s_q[gq * kHeadDim + ch]) * a.qscale * s_lam[ch];
+        v[hf][i] = qx[i] * a.qscale * lx[i];
         m = fmaxf(m, fabsf(v[hf][i]));
       }
     }
@@ -762,7 +781,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   const uint4* qfl = CHAN ? qfw + warp * 4 * 32 + lane : qf + lane;
   const uint2* qfl3 = qfw3 + warp * 4 * 32 + lane;  // per-channel Key groups only
   int cur_blk = -1;  // per-channel Key groups: the block whose operand is in qfw
-  __syncthreads();  // w_m / w_l are reused by the merge
   // The staging areas (second code stages) are refilled by bulk copies from
   // the first loop iteration on: order the generic accesses before them.
   if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
