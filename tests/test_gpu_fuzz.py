@@ -3,6 +3,8 @@ and append schedules (single tokens, short runs, long chunks in any mix),
 each checked against the oracle -- codes and meta bit-exact, attention
 within 2e-3 -- at a random point on the way and at the end.  The fixed cases
 of test_gpu_parity.py cover one feature each; these mix them."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -12,7 +14,10 @@ from test_gpu_parity import CPair, Pair, WPair, kvq, lam_for  # noqa: F401  (kvq
 
 pytestmark = pytest.mark.gpu
 
-MODES = ("plain", "window", "chan", "direct") * 12
+MODES = ("plain", "window", "chan", "direct")
+# the case seeds: 7000 .. 7047 by default; KVQ_FUZZ_SEED and KVQ_FUZZ_CASES run others
+SEED0 = int(os.environ.get("KVQ_FUZZ_SEED", "7000"))
+CASES = int(os.environ.get("KVQ_FUZZ_CASES", "48"))
 
 
 def schedule(rng, total):
@@ -28,10 +33,10 @@ def schedule(rng, total):
     return sizes
 
 
-@pytest.mark.parametrize("case", range(len(MODES)))
+@pytest.mark.parametrize("case", range(CASES))
 def test_random_mix(kvq, orc, case):
-    rng = np.random.default_rng(7000 + case)
-    mode = MODES[case]
+    rng = np.random.default_rng(SEED0 + case)
+    mode = MODES[case % len(MODES)]
     B = int(rng.integers(1, 4))
     H = int(rng.choice([1, 2, 4]))
     G = int(rng.integers(1, 9))
@@ -44,7 +49,7 @@ def test_random_mix(kvq, orc, case):
         n_f = int(rng.choice([512, 1024, 2048]))
         cap = n_f + 129 if mode == "window" else n_f
     T = int(rng.integers(cap // 2, cap + 1))
-    seed = 300 + case
+    seed = 300 + SEED0 - 7000 + case
     k, v = S.keys_values(seed, fbit, B, T, H, 0, int(rng.integers(1, 6)), dtype=dtype)
     lam = lam_for(k) if rng.random() < 0.7 else None
     shift = kvq.KVQ_SHIFT_DIRECT if mode == "direct" else 0
