@@ -384,6 +384,7 @@ cudaError_t enqueue_decode(kvq_cache* c, int layer, const DecodePlan& d, const v
       a.ep = make_epochs(L.nt, L.n_shrinks);
     }
     a.trigger_early = d.wsplits > 0;
+    a.rank_sms = !L.chan && d.wsplits == 0 ? c->sms() : 0;  // the block's only launch: arrival-weighted slices
     if (app.group >= 0) {  // this launch writes the new token itself: keep the pre-wait copies clear of it
       a.app_group = app.group;
       a.app_tile = app.tile;
@@ -397,6 +398,7 @@ cudaError_t enqueue_decode(kvq_cache* c, int layer, const DecodePlan& d, const v
     if (cudaError_t e = launch_decode(a, s)) return e;
     a.trigger_early = false;
     a.app_group = -1;
+    a.rank_sms = 0;
   }
   if (d.wsplits) {
     DecodeArgs w = a;

@@ -407,7 +407,7 @@ __device__ __forceinline__ void chan_block(const float* s_qp, const uint32_t* km
       Z[hf][i] = __half2float(__ushort_as_half((unsigned short)(w[i] >> 16)));
     }
   }
-#pragma unroll 1
+#pragma unroll 2
   for (int hp = 0; hp < kMaxGroup / 2; hp++) {
     const int gq = 2 * hp + hsel;  // the 16 lanes of a head cover its 128 channels
     float v[2][4];
@@ -500,7 +500,26 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   const int s = blockIdx.x / a.splits, split = blockIdx.x - s * a.splits;
   // Per-channel Key groups split the stream by whole 128-token blocks (8 groups).
   const long long units = CHAN ? f.gps / 8 : f.gps, per = CHAN ? 8 : 1;
-  const long long ca = units * split / a.splits, cb = units * (split + 1) / a.splits;
+  // Slices are equal, or, in a one-wave launch (a.rank_sms > 0), weighted by
+  // the order in which the CTAs reach their SMs: CTA i is the (i / SMs)-th on
+  // its SM, and the warp schedulers favour older warps, so with equal slices an
+  // SM's first CTA ends its loop well before its fourth.  Weights 20 : 19 : 18 :
+  // 17 even that out; the host asks for them only with >= 2 units per CTA, so
+  // every slice still holds at least one.
+  long long ca, cb;
+  if (a.rank_sms > 0) {
+    long long wsum = 0, wpre = 0;
+    for (int k = 0; k < a.splits; k++) {
+      const int w = 20 - min(3, (s * a.splits + k) / a.rank_sms);
+      wpre += k < split ? w : 0;
+      wsum += w;
+    }
+    ca = units * wpre / wsum;
+    cb = units * (wpre + 20 - min(3, (int)blockIdx.x / a.rank_sms)) / wsum;
+  } else {
+    ca = units * split / a.splits;
+    cb = units * (split + 1) / a.splits;
+  }
   const long long wa = per * (ca + (cb - ca) * warp / kWarps), wb = per * (ca + (cb - ca) * (warp + 1) / kWarps);
   WarpSmem& my = ws[warp];
   const uint32_t bar0 = smem_u32(bars + warp * kStages);
@@ -1031,7 +1050,13 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
   if (a.chan && (!a.kmc || a.blocks_max < 1 || a.fill.gps % 8 != 0 || a.splits > a.fill.gps / 8))
     return cudaErrorInvalidValue;
-  return a.chan ? launch_width<true>(a, s) : launch_width<false>(a, s);
+  if (a.rank_sms < 0) return cudaErrorInvalidValue;
+  DecodeArgs b = a;
+  // weighted slices only where they are meant: one wave, >= 2 units per CTA
+  const long long units = a.chan ? a.fill.gps / 8 : a.fill.gps;
+  if ((long long)a.batch * a.kv_heads * a.splits > (long long)a.rank_sms * kCtasPerSm || units < 2LL * a.splits)
+    b.rank_sms = 0;
+  return b.chan ? launch_width<true>(b, s) : launch_width<false>(b, s);
 }
 
 }  // namespace kvq

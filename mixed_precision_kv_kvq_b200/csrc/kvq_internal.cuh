@@ -241,6 +241,7 @@ struct DecodeArgs {
   int part_base;        // index of this launch's first partial
   long long safe;       // groups [0, safe) of every stream are not written by kernels still in flight
   bool after_decode;    // launched right after another decode launch of the same call: no dependency wait
+  int rank_sms;         // > 0: the GPU's SM count, slices weighted by arrival order (one-wave launches); 0: equal
   bool trigger_early;   // another decode launch of the call follows: trigger it right after the wait
   // fused single-token append (kvq_append_decode): the warp whose groups
   // include group app_group writes the new token (slot app_slot of tile
