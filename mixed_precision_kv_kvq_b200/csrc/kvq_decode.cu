@@ -674,9 +674,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const Deco
   // kernels -- unless this launch directly follows another decode launch of
   // the same call, which triggers this one only after its own wait (then
   // everything before that launch is complete).
+  // q may be written by an earlier kernel, so it is read only after the wait;
+  // an L2 prefetch of its lines before the wait is a hint that reads nothing
+  // into registers (the loads after the wait see whatever q holds then).
+  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.q_heads + (size_t)j * G) * kHeadDim;
+  if (CHAN ? (int)threadIdx.x < G * (kHeadDim / 8) : gq < G)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(CHAN ? qb + 8 * threadIdx.x : qb + (size_t)gq * kHeadDim + 32 * sq + 4 * tq));
   if (!a.after_decode) pdl_wait();
   if (a.trigger_early) pdl_launch_dependents();  // a window launch follows: let it fill free SMs now
-  const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q) + ((size_t)b * a.q_heads + (size_t)j * G) * kHeadDim;
   uint4 qv = make_uint4(0u, 0u, 0u, 0u);  // per-channel Key groups: 8 bf16 of q, head threadIdx/16, channels 8 (threadIdx%16) ..
   uint2 qv2[2] = {make_uint2(0u, 0u), make_uint2(0u, 0u)};  // otherwise this lane's channels of head gq
   if constexpr (CHAN) {
