@@ -24,9 +24,9 @@
 //   B = p R (transposed from the score fragment with movmatrix).
 // 16-bit codes go in as two bytes (Keys) or two fp16 halves (Values).
 
-// Work split: each stream is cut into `splits` equal slices of 16-token
-// groups, one CTA per slice (the host picks `splits` so the grid fills the
-// GPU in whole waves).  The CTA's four warps take contiguous quarters of the
+// Work split: each stream is cut into `splits` slices of 16-token groups,
+// one CTA per slice (the host picks `splits` so the grid fills the GPU in
+// whole waves; the slices are equal, or weighted as described below).  The CTA's four warps take contiguous quarters of the
 // slice; each warp streams its quarter through its own ring of shared-memory
 // stages filled by cp.async.bulk (TMA bulk copies) on mbarriers, a few KiB
 // ahead of its math, and keeps its own online-softmax state.  The warps merge
